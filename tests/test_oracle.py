@@ -1,0 +1,296 @@
+"""Pins for the fp64 oracle, against things other than itself (CPU only).
+
+Each test ties the oracle to brute force, a closed form, a library routine, or an
+invariant that the DeepSeekMoE pages fix, so that a dropped term, a wrong sign or index,
+or a transposed operand in the oracle fails at least one of them.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+from oracle import moe_oracle as O
+from mixture_experts_layer_65_b200 import workloads as W
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "deepseekmoe_pages.json")
+
+
+def _small(seed, T=6, d=12, ks=1, nr=6, inter=8, k=2, bias=False, std_w=0.3):
+    rng = np.random.default_rng(seed)
+    g = ks + nr
+    return dict(
+        u=rng.standard_normal((T, d)),
+        centroids=rng.standard_normal((nr, d)) / math.sqrt(d),
+        w_gate=rng.standard_normal((g, inter, d)) * std_w,
+        w_up=rng.standard_normal((g, inter, d)) * std_w,
+        w_down=rng.standard_normal((g, d, inter)) * std_w,
+        n_shared=ks, top_k=k, alpha1=0.01,
+        bias=rng.standard_normal(nr) if bias else None,
+    )
+
+
+# ----------------------------------------------------------------- brute force
+@pytest.mark.parametrize("seed,ks,nr,k,bias", [
+    (0, 1, 6, 2, False), (1, 0, 5, 1, False), (2, 2, 8, 3, True), (3, 1, 4, 4, False),
+    (4, 0, 1, 1, False), (5, 3, 7, 5, True),
+])
+def test_vectorised_matches_brute_force(seed, ks, nr, k, bias):
+    a = _small(seed, ks=ks, nr=nr, k=k, bias=bias)
+    out = O.moe_forward(a["u"], a["centroids"], a["w_gate"], a["w_up"], a["w_down"],
+                        a["n_shared"], a["top_k"], a["alpha1"], bias=a["bias"])
+    H, IDX, Wt, counts, aux = O.brute_force_layer(
+        a["u"], a["centroids"], a["w_gate"], a["w_up"], a["w_down"], a["n_shared"],
+        a["top_k"], a["alpha1"], bias=a["bias"])
+    np.testing.assert_array_equal(out.routing.topk_idx, np.array(IDX))
+    np.testing.assert_allclose(out.routing.topk_w, np.array(Wt), rtol=1e-13, atol=0)
+    np.testing.assert_allclose(out.h, np.array(H), rtol=1e-12, atol=1e-13)
+    np.testing.assert_array_equal(out.counts, np.array(counts))
+    assert out.aux == pytest.approx(aux, rel=1e-13)
+
+
+# ----------------------------------------------------------------- library routines
+def test_softmax_matches_scipy():
+    rng = np.random.default_rng(7)
+    l = rng.standard_normal((50, 17)) * 5
+    np.testing.assert_allclose(O.affinity_softmax(l), scipy.special.softmax(l, axis=1),
+                               rtol=1e-14, atol=0)
+
+
+def _llama_mlp(x, wg, wu, wd):
+    """SwiGLU FFN as implemented by transformers' LlamaMLP (down(silu(gate x) * up x))."""
+    from transformers import LlamaConfig
+    from transformers.models.llama.modeling_llama import LlamaMLP
+    d, inter = wg.shape[1], wg.shape[0]
+    cfg = LlamaConfig(hidden_size=d, intermediate_size=inter, hidden_act="silu",
+                      mlp_bias=False, num_attention_heads=1, num_key_value_heads=1,
+                      head_dim=d)
+    mlp = LlamaMLP(cfg).double()
+    with torch.no_grad():
+        mlp.gate_proj.weight.copy_(torch.from_numpy(np.asarray(wg, dtype=np.float64)))
+        mlp.up_proj.weight.copy_(torch.from_numpy(np.asarray(wu, dtype=np.float64)))
+        mlp.down_proj.weight.copy_(torch.from_numpy(np.asarray(wd, dtype=np.float64)))
+        return mlp(torch.from_numpy(np.asarray(x, dtype=np.float64))).numpy()
+
+
+def test_swiglu_matches_llama_mlp():
+    a = _small(11, inter=9, d=13)
+    y = O.swiglu_ffn(a["u"], a["w_gate"][0], a["w_up"][0], a["w_down"][0])
+    ref = _llama_mlp(a["u"], a["w_gate"][0], a["w_up"][0], a["w_down"][0])
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-14)
+
+
+def test_single_expert_layer_is_dense_swiglu():
+    """N_r = 1, top-1, no shared expert: s = g = 1 and h = u + SwiGLU(u)."""
+    a = _small(12, ks=0, nr=1, k=1, d=10, inter=7)
+    out = O.moe_forward(a["u"], a["centroids"], a["w_gate"], a["w_up"], a["w_down"],
+                        0, 1, 0.01)
+    assert np.all(out.routing.topk_idx == 0)
+    np.testing.assert_allclose(out.routing.topk_w, 1.0, rtol=0, atol=1e-15)
+    ref = a["u"] + _llama_mlp(a["u"], a["w_gate"][0], a["w_up"][0], a["w_down"][0])
+    np.testing.assert_allclose(out.h, ref, rtol=1e-12, atol=1e-13)
+    # f = 1, P = 1 -> aux = alpha1
+    assert out.aux == pytest.approx(0.01, rel=1e-15)
+
+
+def test_shared_expert_has_gate_one():
+    """A shared copy of the single routed expert doubles the FFN term: h = u + 2 SwiGLU(u)."""
+    a = _small(13, ks=0, nr=1, k=1, d=10, inter=7)
+    wg = np.concatenate([a["w_gate"], a["w_gate"]])
+    wu = np.concatenate([a["w_up"], a["w_up"]])
+    wd = np.concatenate([a["w_down"], a["w_down"]])
+    out = O.moe_forward(a["u"], a["centroids"], wg, wu, wd, 1, 1, 0.01)
+    ref = a["u"] + 2.0 * _llama_mlp(a["u"], a["w_gate"][0], a["w_up"][0], a["w_down"][0])
+    np.testing.assert_allclose(out.h, ref, rtol=1e-12, atol=1e-13)
+
+
+def test_gate_is_unrenormalised_softmax():
+    """Two routed experts, top-1: the kept gate is sigmoid(l0 - l1), not 1."""
+    a = _small(14, ks=0, nr=2, k=1, d=8, inter=5)
+    out = O.moe_forward(a["u"], a["centroids"], a["w_gate"], a["w_up"], a["w_down"],
+                        0, 1, 0.01)
+    l = a["u"] @ a["centroids"].T
+    for t in range(a["u"].shape[0]):
+        e = int(np.argmax(l[t]))
+        g = scipy.special.expit(l[t, e] - l[t, 1 - e])
+        ref = a["u"][t] + g * _llama_mlp(a["u"][t:t + 1], a["w_gate"][e], a["w_up"][e],
+                                         a["w_down"][e])[0]
+        assert out.routing.topk_idx[t, 0] == e
+        assert out.routing.topk_w[t, 0] == pytest.approx(g, rel=1e-14)
+        np.testing.assert_allclose(out.h[t], ref, rtol=1e-12, atol=1e-13)
+
+
+# ----------------------------------------------------------------- closed forms / special cases
+def test_uniform_router_closed_form():
+    """All-zero centroids: s = 1/N_r everywhere, ties -> experts 0..K'-1, aux = a1*K'/N_r."""
+    a = _small(15, ks=1, nr=6, k=3)
+    cen = np.zeros_like(a["centroids"])
+    out = O.moe_forward(a["u"], cen, a["w_gate"], a["w_up"], a["w_down"], 1, 3, 0.01)
+    T = a["u"].shape[0]
+    np.testing.assert_array_equal(out.routing.topk_idx, np.tile(np.arange(3), (T, 1)))
+    np.testing.assert_allclose(out.routing.topk_w, 1.0 / 6.0, rtol=1e-15)
+    np.testing.assert_array_equal(out.counts, [T, T, T, 0, 0, 0])
+    np.testing.assert_allclose(out.P, 1.0 / 6.0, rtol=1e-15)
+    assert out.aux == pytest.approx(0.01 * 3 / 6, rel=1e-14)
+
+
+def test_zero_down_projection_leaves_residual():
+    a = _small(16, ks=2, nr=5, k=2)
+    out = O.moe_forward(a["u"], a["centroids"], a["w_gate"], a["w_up"],
+                        np.zeros_like(a["w_down"]), 2, 2, 0.01)
+    np.testing.assert_array_equal(out.h, a["u"])
+
+
+def test_zero_input_gives_zero_output():
+    a = _small(17, ks=1, nr=5, k=2)
+    z = np.zeros_like(a["u"])
+    out = O.moe_forward(z, a["centroids"], a["w_gate"], a["w_up"], a["w_down"], 1, 2, 0.01)
+    np.testing.assert_array_equal(out.h, 0.0)
+
+
+def test_tie_break_lower_index_wins():
+    """Duplicate centroids: equal logits; the stable order keeps the lower index first."""
+    rng = np.random.default_rng(18)
+    d = 8
+    cen = rng.standard_normal((5, d))
+    cen[3] = cen[1]
+    u = cen[1][None, :] * 3.0            # experts 1 and 3 tie for the largest logit
+    l = O.router_logits(u, cen)
+    assert l[0, 1] == l[0, 3] and np.argmax(l[0]) in (1, 3)
+    idx = O.select_topk(l, 1)
+    assert idx[0, 0] == 1
+    idx2 = O.select_topk(l, 2)
+    np.testing.assert_array_equal(idx2[0], [1, 3])
+
+
+def test_topk_equal_to_all_experts_gates_sum_to_one():
+    a = _small(19, ks=0, nr=5, k=5)
+    r = O.route(a["u"], a["centroids"], 5)
+    np.testing.assert_allclose(r.topk_w.sum(axis=1), 1.0, rtol=0, atol=1e-15)
+    for row in r.topk_idx:
+        assert sorted(row.tolist()) == list(range(5))
+
+
+# ----------------------------------------------------------------- invariants
+@pytest.mark.parametrize("name", ["tiny"])
+def test_routing_invariants_on_tiny_workload(name):
+    w = W.make_workload(name)
+    out = O.moe_forward(w.u, w.centroids, w.w_gate, w.w_up, w.w_down, w.n_shared,
+                        w.top_k, w.alpha1)
+    r = out.routing
+    # exactly K' distinct routed indices in [0, N_r)
+    assert r.topk_idx.shape == (w.T, w.top_k)
+    assert r.topk_idx.min() >= 0 and r.topk_idx.max() < w.n_routed
+    assert all(len(set(row)) == w.top_k for row in r.topk_idx.tolist())
+    # descending logit order
+    ls = np.take_along_axis(r.logits, r.topk_idx, axis=1)
+    assert np.all(np.diff(ls, axis=1) <= 0)
+    # gates = softmax mass of the selected experts, < 1 since K' < N_r
+    gsum = r.topk_w.sum(axis=1)
+    sel_mass = np.array([r.s[t, r.topk_idx[t]].sum() for t in range(w.T)])
+    np.testing.assert_allclose(gsum, sel_mass, rtol=1e-15)
+    assert np.all(gsum < 1.0)
+    # balance statistics
+    assert out.counts.sum() == w.T * w.top_k
+    np.testing.assert_allclose(out.P.sum(), 1.0, rtol=1e-14)
+    np.testing.assert_allclose(out.f, out.counts / w.T)
+    assert out.aux == pytest.approx(w.alpha1 * float(np.sum(out.f * out.P)), rel=1e-15)
+
+
+def test_balance_brute_recount():
+    a = _small(20, ks=0, nr=7, k=3, T=40)
+    out = O.moe_forward(a["u"], a["centroids"], a["w_gate"], a["w_up"], a["w_down"],
+                        0, 3, 0.01)
+    cnt = [0] * 7
+    for row in out.routing.topk_idx.tolist():
+        for e in row:
+            cnt[e] += 1
+    np.testing.assert_array_equal(out.counts, cnt)
+    P = [sum(out.routing.s[t, i] for t in range(40)) / 40 for i in range(7)]
+    np.testing.assert_allclose(out.P, P, rtol=1e-14)
+
+
+def test_fine_grained_segmentation_reproduces_unsplit_expert():
+    """Split one expert's intermediate dim into m = 4 pieces (rows of W_gate/W_up, columns
+    of W_down); the pieces, all routed together with the same gate, sum to the unsplit
+    expert.  Shown both on the FFN and at layer level with the pieces as shared experts
+    (gate 1), which also justifies running K_s shared experts as one wide group."""
+    a = _small(21, ks=1, nr=4, k=2, inter=16, d=10)
+    wg, wu, wd = a["w_gate"][0], a["w_up"][0], a["w_down"][0]
+    m = 4
+    x = a["u"]
+    whole = O.swiglu_ffn(x, wg, wu, wd)
+    parts = sum(O.swiglu_ffn(x, wg[p::m], wu[p::m], wd[:, p::m]) for p in range(m))
+    np.testing.assert_allclose(parts, whole, rtol=1e-13, atol=1e-15)
+    # layer level: 1 unsplit shared expert vs m pieces as shared experts
+    inter_p = wg.shape[0] // m
+    pg = np.stack([wg[p * inter_p:(p + 1) * inter_p] for p in range(m)])
+    pu = np.stack([wu[p * inter_p:(p + 1) * inter_p] for p in range(m)])
+    pd = np.stack([wd[:, p * inter_p:(p + 1) * inter_p] for p in range(m)])
+    # routed experts must share the pieces' width: give them width inter_p
+    rg, ru, rd = a["w_gate"][1:, :inter_p], a["w_up"][1:, :inter_p], a["w_down"][1:, :, :inter_p]
+    split = O.moe_forward(x, a["centroids"], np.concatenate([pg, rg]),
+                          np.concatenate([pu, ru]), np.concatenate([pd, rd]), m, 2, 0.01)
+    base = O.moe_forward(x, a["centroids"], rg, ru, rd, 0, 2, 0.01)
+    np.testing.assert_allclose(split.h - base.h, whole, rtol=1e-12, atol=1e-14)
+
+
+def test_rows_subset_matches_full():
+    a = _small(22, ks=1, nr=6, k=2, T=12)
+    full = O.moe_forward(a["u"], a["centroids"], a["w_gate"], a["w_up"], a["w_down"],
+                         1, 2, 0.01)
+    sub = O.moe_forward(a["u"], a["centroids"], a["w_gate"], a["w_up"], a["w_down"],
+                        1, 2, 0.01, rows=[0, 5, 11])
+    np.testing.assert_allclose(sub.h, full.h[[0, 5, 11]], rtol=1e-15, atol=0)
+    assert sub.aux == full.aux
+
+
+def test_near_tie_detection():
+    s = np.array([[0.5, 0.3, 0.3 - 5e-7, 0.1], [0.4, 0.3, 0.2, 0.1]])
+    np.testing.assert_array_equal(O.near_tie_tokens(s, 2), [True, False])
+    np.testing.assert_array_equal(O.near_tie_tokens(s, 4), [False, False])
+
+
+def test_bf16_bits_widen_exactly():
+    x = np.array([1.0, -2.5, 3.140625, 1e-3], dtype=np.float32)
+    bits = W.f32_to_bf16_bits(x)
+    ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(O.widen(bits), ref)
+
+
+# ----------------------------------------------------------------- numbers the pages print
+def test_configs_match_the_pages():
+    g = json.load(open(GOLDEN))
+    c16 = W.CONFIGS["16b_prefill"]
+    assert c16["d"] == g["config_16b"]["hidden"]
+    assert c16["n_shared"] == g["config_16b"]["n_shared"]
+    assert c16["n_routed"] == g["config_16b"]["n_routed"]
+    assert c16["top_k"] == g["config_16b"]["routed_active"]
+    assert c16["n_shared"] + c16["top_k"] == g["config_16b"]["expert_passes_per_token"]
+    c145 = W.CONFIGS["145b"]
+    assert (c145["n_shared"], c145["n_routed"], c145["top_k"]) == (
+        g["config_145b"]["n_shared"], g["config_145b"]["n_routed"], g["config_145b"]["routed_active"])
+    assert W.CONFIGS["2b"]["alpha1"] == g["alpha1"]["2b"]
+    assert c16["alpha1"] == g["alpha1"]["16b"]
+    # fine-grained segmentation: same total expert params and per-token FLOPs as GShard
+    c2, cg = W.CONFIGS["2b"], W.CONFIGS["gshard"]
+    assert (c2["n_shared"] + c2["n_routed"]) * c2["inter"] == cg["n_routed"] * cg["inter"]
+    assert (c2["n_shared"] + c2["top_k"]) * c2["inter"] == cg["top_k"] * cg["inter"]
+    assert math.comb(16, 2) == g["combinations"]["choose_2_of_16"]
+    assert math.comb(64, 8) == g["combinations"]["choose_8_of_64"]
+
+
+def test_workload_is_seeded_and_prefix_stable():
+    a = W.make_workload("tiny")
+    b = W.make_workload("tiny", T=64)
+    np.testing.assert_array_equal(a.u[:64], b.u)
+    np.testing.assert_array_equal(a.w_down, b.w_down)
+    c = W.make_workload("tiny", seed=1)
+    assert not np.array_equal(a.u, c.u)
+    z = W.make_workload("145b", T=4, d=64, inter=64, n_routed=16, n_shared=1, top_k=3)
+    assert z.logit_bias is not None and z.logit_bias.shape == (16,)
+    assert np.all(np.diff(z.logit_bias) < 0)
+    np.testing.assert_allclose(np.exp(z.logit_bias.astype(np.float64)).sum(), 1.0, rtol=1e-6)
