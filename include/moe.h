@@ -1,0 +1,150 @@
+/*
+ * moe.h -- C-ABI of the DeepSeekMoE layer forward pass for NVIDIA B200 (sm_100a).
+ *
+ * What is computed (per token t, hidden vector u_t of width d):
+ *   logit[t,i] = u_t . e_i + b_i                 for the N_r routed experts
+ *   s[t,:]     = softmax(logit[t,:])              over the routed experts only
+ *   sel[t]     = the top_k largest logits, lower expert index first on equal logits
+ *   g[t,i]     = s[t,i] if i in sel[t] else 0     (not renormalised)
+ *   h_t        = u_t + sum_{j shared} FFN_j(u_t) + sum_{i in sel[t]} g[t,i] FFN_i(u_t)
+ *   FFN(x)     = W_down (SiLU(W_gate x) * (W_up x)),  SiLU(z) = z / (1 + exp(-z))
+ *   count_i    = #{t : i in sel[t]},  P_i = (1/T) sum_t s[t,i],
+ *   aux_loss   = alpha1 * sum_i (count_i / T) * P_i
+ * Sources: "DeepSeekMoE: Towards Ultimate Expert Specialization in Mixture-of-Experts
+ * Language Models" (deepforge.srivtx.xyz article): section "Routing in a classic MoE
+ * layer" (routing equation with residual), "Top-k routing, from affinities to gates"
+ * (softmax before the top-k cut, no renormalisation, stable ranking), "Where this sits"
+ * (fine-grained segmentation mN/mK and K_s shared experts that every token uses),
+ * "Expert-level balance loss" (L_ExpBal = alpha_1 sum_i f_i P_i).  The SwiGLU form of the
+ * expert FFN follows the GLU-variants paper cited by the observer.broadside.tech card.
+ *
+ * Conventions for every entry point:
+ *   - Status codes are returned; nothing throws across the ABI.  On failure
+ *     moe_last_error() returns a thread-local, NUL-terminated description.
+ *   - "device" pointers are CUDA global-memory pointers of the current device; "host"
+ *     pointers are ordinary (pageable or pinned) host memory.
+ *   - All row-major, no padding between rows.  bf16 is IEEE-like bfloat16 (16-bit).
+ *   - stream: a cudaStream_t (NULL = the legacy default stream).
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_ABI_VERSION 1
+
+typedef struct CUstream_st* moe_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, inconsistent sizes            */
+  MOE_ERR_UNSUPPORTED = 2,  /* a valid layer this build does not handle (see create)  */
+  MOE_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed                      */
+  MOE_ERR_OOM = 4,          /* device allocation failed                               */
+  MOE_ERR_DEVICE_CHECK = 5  /* a kernel recorded an error (bounded wait ran out, ...) */
+} moe_status;
+
+typedef enum { MOE_FP32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+/* Layer description.  All weight pointers are DEVICE pointers in `dtype`, read only
+ * during moe_create (the library keeps its own re-laid-out copy; the caller may free
+ * them when moe_create returns).
+ *   T          tokens per forward call (fixed per handle; decode and prefill use
+ *              separate handles), 1 <= T <= 2^24
+ *   d          hidden width;  inter = I, intermediate width of every expert
+ *   n_routed   N_r = mN routed experts (1..256);  n_shared = K_s always-on experts
+ *   top_k      K' = mK - K_s routed experts per token (1..min(16, N_r))
+ *   alpha1     balance-loss factor alpha_1
+ *   centroids  [n_routed, d]
+ *   logit_bias [n_routed] fp32 added to the logits before the softmax, or NULL
+ *   w_gate     [n_shared + n_routed, inter, d]   shared experts first
+ *   w_up       [n_shared + n_routed, inter, d]
+ *   w_down     [n_shared + n_routed, d, inter]
+ * bf16 layers need d % 64 == 0 and inter % 64 == 0 (MOE_ERR_UNSUPPORTED otherwise);
+ * fp32 layers need d % 4 == 0. */
+typedef struct {
+  int32_t T;
+  int32_t d;
+  int32_t n_routed;
+  int32_t n_shared;
+  int32_t top_k;
+  int32_t inter;
+  int32_t dtype; /* moe_dtype */
+  float alpha1;
+  const void* centroids;
+  const float* logit_bias;
+  const void* w_gate;
+  const void* w_up;
+  const void* w_down;
+} moe_cfg;
+
+typedef struct moe_handle moe_handle;
+
+/* Validate cfg, allocate the handle's device workspace (sized for cfg->T), copy and
+ * re-lay-out the weights.  Synchronous (returns after the copies finished) on the
+ * current device.  *out is set to NULL on failure. */
+moe_status moe_create(const moe_cfg* cfg, moe_handle** out);
+
+/* One forward pass of the layer over cfg->T tokens, enqueued on `stream`; no host
+ * synchronisation and no allocation.  All pointers are DEVICE pointers owned by the
+ * caller:
+ *   u             [T, d] in dtype, 16-byte aligned (input)
+ *   h             [T, d] in dtype, 16-byte aligned (output)
+ *   topk_idx      [T, top_k] int32 routed expert ids in [0, n_routed), descending logit
+ *   topk_w        [T, top_k] fp32 gates g = s at those experts
+ *   expert_counts [n_routed] int32
+ *   aux_loss      [1] fp32
+ * Deterministic: identical inputs give bit-identical outputs.  Calls on one handle must
+ * not overlap in time (they share the handle's workspace).  A device-side failure is
+ * reported by moe_device_status(). */
+moe_status moe_forward(moe_handle* handle, const void* u, void* h, int32_t* topk_idx,
+                       float* topk_w, int32_t* expert_counts, float* aux_loss,
+                       moe_stream_t stream);
+
+/* moe_forward on HOST buffers: copies u host->device, runs the forward, copies every
+ * output device->host and synchronises `stream` before returning.  Sizes as in
+ * moe_forward; any output pointer except h_host may be NULL (not copied back). */
+moe_status moe_forward_host(moe_handle* handle, const void* u_host, void* h_host,
+                            int32_t* topk_idx_host, float* topk_w_host,
+                            int32_t* expert_counts_host, float* aux_loss_host,
+                            moe_stream_t stream);
+
+/* Synchronise `stream`, then read and clear the handle's device error word.
+ * Returns MOE_DEVICE_CHECK (with the kernel's code in moe_last_error()) if any kernel
+ * of an earlier forward recorded an error, else MOE_OK. */
+moe_status moe_device_status(moe_handle* handle, moe_stream_t stream);
+
+/* Per-expert affinity sums sum_t s[t,i] (fp32, [n_routed], DEVICE) of the most recent
+ * forward on this handle, copied on `stream`.  Data-parallel callers all-reduce these
+ * together with expert_counts and then call moe_balance_loss with the global T. */
+moe_status moe_expert_psum(moe_handle* handle, float* psum, moe_stream_t stream);
+
+/* aux_loss = alpha1 * sum_i (counts[i] / n_tokens) * (psum[i] / n_tokens), one kernel on
+ * `stream`, fixed summation order.  counts, psum, aux_loss are DEVICE pointers. */
+moe_status moe_balance_loss(const int32_t* counts, const float* psum, int32_t n_routed,
+                            int64_t n_tokens, float alpha1, float* aux_loss,
+                            moe_stream_t stream);
+
+/* Number of kernels one moe_forward launches on this handle. */
+int32_t moe_kernels_per_forward(const moe_handle* handle);
+
+/* Bytes of device memory the handle owns (weights copy + workspace). */
+size_t moe_device_bytes(const moe_handle* handle);
+
+/* Free everything the handle owns.  NULL-safe.  Synchronises the device first. */
+void moe_destroy(moe_handle* handle);
+
+/* Thread-local description of the last failure on this thread ("" if none). */
+const char* moe_last_error(void);
+
+int32_t moe_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

@@ -1,0 +1,57 @@
+"""Build the in-tree CUDA library ``libmoe.so`` for sm_100a with nvcc.
+
+Usage: ``python -m mixture_experts_layer_65_b200.build`` (or ``__graft_entry__.build()``).
+"""
+from __future__ import annotations
+
+import os
+import shutil
+import subprocess
+import sys
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(PKG)
+CSRC = os.path.join(PKG, "csrc")
+INCLUDE = os.path.join(ROOT, "include")
+LIB = os.path.join(PKG, "libmoe.so")
+SOURCES = [os.path.join(CSRC, "moe_api.cu")]
+GENCODE = "arch=compute_100a,code=sm_100a"
+
+
+def nvcc_path() -> str:
+    for cand in (shutil.which("nvcc"), "/usr/local/cuda/bin/nvcc"):
+        if cand and os.path.exists(cand):
+            return cand
+    raise RuntimeError("nvcc not found: the CUDA toolkit is required to build libmoe.so")
+
+
+def nvcc_cmd(out: str = LIB, extra: list[str] | None = None) -> list[str]:
+    return [nvcc_path(), "-gencode", GENCODE, "-O3", "-lineinfo", "-std=c++17",
+            "--expt-relaxed-constexpr", "-Xcompiler", "-fPIC,-O2", "-shared",
+            "-I", INCLUDE, "-I", CSRC, *(extra or []), "-o", out, *SOURCES]
+
+
+def _stale() -> bool:
+    if not os.path.exists(LIB):
+        return True
+    t = os.path.getmtime(LIB)
+    deps = [os.path.join(CSRC, f) for f in os.listdir(CSRC)] + [os.path.join(INCLUDE, "moe.h")]
+    return any(os.path.getmtime(p) > t for p in deps)
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    if not force and not _stale():
+        return LIB
+    tmp = LIB + ".tmp"
+    cmd = nvcc_cmd(tmp, ["-Xptxas", "-v"] if verbose else None)
+    proc = subprocess.run(cmd, capture_output=True, text=True)
+    if proc.returncode != 0:
+        raise RuntimeError("nvcc failed:\n" + " ".join(cmd) + "\n" + proc.stdout + proc.stderr)
+    if verbose:
+        sys.stderr.write(proc.stdout + proc.stderr)
+    os.replace(tmp, LIB)
+    return LIB
+
+
+if __name__ == "__main__":
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))

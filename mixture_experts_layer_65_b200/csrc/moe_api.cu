@@ -1,0 +1,581 @@
+// moe_api.cu -- the C-ABI (include/moe.h): validation, weight re-layout, workspace,
+// TMA descriptors and the launch sequence of one DeepSeekMoE layer forward pass.
+//
+// Launch sequence of moe_forward (one stream, no host synchronisation):
+//   1. router      logits -> softmax -> top-k, gates, per-tile histograms / ranks / sums
+//   2. scan        per-expert counts, padded offsets, tile tables, balance loss
+//   3. permute     token rows -> expert-contiguous rows (top_k copies per token)
+//   4. gate/up     grouped GEMM + SwiGLU (shared group reads the token rows directly)
+//   5. down        grouped GEMM
+//   6. combine     h = u + shared + sum_k g_k * routed_k (fp32, fixed order)
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "moe.h"
+#include "combine.cuh"
+#include "gemm_simt.cuh"
+#include "gemm_tc.cuh"
+#include "router.cuh"
+#include "scan_permute.cuh"
+
+using namespace moe;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+moe_status fail(moe_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+#define MOE_CUDA(expr)                                                                     \
+  do {                                                                                     \
+    cudaError_t e_ = (expr);                                                               \
+    if (e_ != cudaSuccess)                                                                 \
+      return fail(MOE_ERR_CUDA, "%s: %s (%s:%d)", #expr, cudaGetErrorString(e_), __FILE__, \
+                  __LINE__);                                                               \
+  } while (0)
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// bf16 row-major [outer, inner] matrix, box = box_outer rows x 64 columns, 128 B swizzle.
+bool encode_2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer,
+               uint32_t box_outer) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {64, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// bf16 [depth, outer, inner], box = box_outer rows x 64 columns of one matrix.
+bool encode_3d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t depth,
+               uint32_t box_outer) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {inner, outer, depth};
+  cuuint64_t strides[2] = {inner * 2, inner * outer * 2};
+  cuuint32_t box[3] = {64, box_outer, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+__global__ void balance_loss_kernel(const int32_t* counts, const float* psum, int n, double inv_t,
+                                    float alpha1, float* out) {
+  if (threadIdx.x == 0 && blockIdx.x == 0) {
+    double acc = 0.0;
+    for (int i = 0; i < n; ++i) acc += ((double)counts[i] * inv_t) * ((double)psum[i] * inv_t);
+    *out = (float)((double)alpha1 * acc);
+  }
+}
+
+constexpr int kKernelsPerForward = 6;
+
+}  // namespace
+
+struct moe_handle {
+  moe_cfg cfg;
+  int device = 0, n_sms = 0;
+  bool bf16 = true;
+  int es = 2;              // element size
+  int G = 0, has_shared = 0, inter_shared = 0;
+  int n_tiles = 0;         // router tiles of 128 tokens
+  int64_t T_pad = 0, rows_cap = 0;
+  int n_pad = 0, maxk = 16;
+  int router_stages = 0;
+  uint32_t router_tmem_cols = 0;
+  size_t router_smem = 0, simt_router_smem = 0;
+  // weights (library-owned, re-laid-out)
+  void* centroids = nullptr;
+  float* bias = nullptr;
+  void* w_gu_s = nullptr;  // bf16 [2*inter_shared, d], gate/up interleaved by 64 rows
+  void* w_gu_r = nullptr;  // bf16 [n_routed, 2*inter, d]
+  void* w_g = nullptr;     // fp32 [G, inter, d]
+  void* w_u = nullptr;     // fp32 [G, inter, d]
+  void* w_d_s = nullptr;   // [d, inter_shared]
+  void* w_d_r = nullptr;   // [n_routed, d, inter]
+  // workspace
+  int32_t *topk_rank = nullptr, *slot_row = nullptr, *tile_hist = nullptr, *tile_base = nullptr;
+  int32_t *grp_row = nullptr, *ts1 = nullptr, *ts2 = nullptr;
+  float *tile_psum = nullptr, *psum_total = nullptr;
+  void *xp = nullptr, *hs = nullptr, *hr = nullptr, *ys = nullptr, *yr = nullptr;
+  int* err = nullptr;
+  // staging for moe_forward_host
+  void *u_dev = nullptr, *h_dev = nullptr;
+  int32_t *idx_dev = nullptr, *cnt_dev = nullptr;
+  float *w_dev = nullptr, *aux_dev = nullptr;
+  CUtensorMap tmE, tmXp, tmWguS, tmWguR, tmHs, tmHr, tmWdS, tmWdR;
+  std::vector<void*> allocs;
+  size_t bytes = 0;
+};
+
+namespace {
+
+moe_status dalloc(moe_handle* H, void** p, size_t bytes) {
+  *p = nullptr;
+  if (bytes == 0) return MOE_OK;
+  cudaError_t e = cudaMalloc(p, bytes);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    *p = nullptr;
+    return fail(MOE_ERR_OOM, "cudaMalloc(%zu) failed: %s", bytes, cudaGetErrorString(e));
+  }
+  H->allocs.push_back(*p);
+  H->bytes += bytes;
+  return MOE_OK;
+}
+
+#define MOE_TRY(expr)              \
+  do {                             \
+    moe_status s_ = (expr);        \
+    if (s_ != MOE_OK) return s_;   \
+  } while (0)
+
+void free_handle(moe_handle* H) {
+  if (!H) return;
+  for (void* p : H->allocs) cudaFree(p);
+  delete H;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int pick_maxk(int k) { return k <= 4 ? 4 : (k <= 8 ? 8 : 16); }
+
+moe_status validate(const moe_cfg* c) {
+  if (!c) return fail(MOE_ERR_INVALID_ARG, "cfg is NULL");
+  if (c->T < 1 || c->T > (1 << 24)) return fail(MOE_ERR_INVALID_ARG, "T=%d outside [1, 2^24]", c->T);
+  if (c->d < 1 || c->inter < 1) return fail(MOE_ERR_INVALID_ARG, "d and inter must be positive");
+  if (c->n_routed < 1 || c->n_routed > kMaxRouted)
+    return fail(MOE_ERR_UNSUPPORTED, "n_routed=%d outside [1, %d]", c->n_routed, kMaxRouted);
+  if (c->n_shared < 0 || c->n_shared > 64)
+    return fail(MOE_ERR_INVALID_ARG, "n_shared=%d outside [0, 64]", c->n_shared);
+  if (c->top_k < 1 || c->top_k > c->n_routed)
+    return fail(MOE_ERR_INVALID_ARG, "top_k=%d outside [1, n_routed=%d]", c->top_k, c->n_routed);
+  if (c->top_k > kMaxTopK)
+    return fail(MOE_ERR_UNSUPPORTED, "top_k=%d above %d", c->top_k, kMaxTopK);
+  if (c->dtype != MOE_FP32 && c->dtype != MOE_BF16)
+    return fail(MOE_ERR_INVALID_ARG, "dtype=%d is not MOE_FP32 or MOE_BF16", c->dtype);
+  if (!c->centroids || !c->w_gate || !c->w_up || !c->w_down)
+    return fail(MOE_ERR_INVALID_ARG, "a weight pointer is NULL");
+  if (c->dtype == MOE_BF16) {
+    if (c->d % 64 || c->inter % 64)
+      return fail(MOE_ERR_UNSUPPORTED, "bf16 layers need d %% 64 == 0 and inter %% 64 == 0 (d=%d inter=%d)",
+                  c->d, c->inter);
+  } else {
+    if (c->d % 4 || c->inter % 4)
+      return fail(MOE_ERR_UNSUPPORTED, "fp32 layers need d %% 4 == 0 and inter %% 4 == 0 (d=%d inter=%d)",
+                  c->d, c->inter);
+  }
+  const int64_t rows_cap = (int64_t)c->T * c->top_k + (int64_t)c->n_routed * (kGemmBM - 1);
+  if (rows_cap >= (int64_t(1) << 30)) return fail(MOE_ERR_UNSUPPORTED, "T * top_k too large");
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t moe_abi_version(void) { return MOE_ABI_VERSION; }
+
+const char* moe_last_error(void) { return g_last_error.c_str(); }
+
+int32_t moe_kernels_per_forward(const moe_handle* handle) {
+  return handle ? kKernelsPerForward : 0;
+}
+
+size_t moe_device_bytes(const moe_handle* handle) { return handle ? handle->bytes : 0; }
+
+static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
+  const moe_cfg& c = *cfg;
+  MOE_CUDA(cudaGetDevice(&H->device));
+  int major = 0, minor = 0;
+  MOE_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, H->device));
+  MOE_CUDA(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, H->device));
+  if (major != 10 || minor != 0)
+    return fail(MOE_ERR_UNSUPPORTED, "this library is built for sm_100a (B200); device is sm_%d%d",
+                major, minor);
+  MOE_CUDA(cudaDeviceGetAttribute(&H->n_sms, cudaDevAttrMultiProcessorCount, H->device));
+
+  H->cfg = c;
+  H->cfg.centroids = H->cfg.w_gate = H->cfg.w_up = H->cfg.w_down = nullptr;
+  H->cfg.logit_bias = nullptr;
+  H->bf16 = c.dtype == MOE_BF16;
+  H->es = H->bf16 ? 2 : 4;
+  H->has_shared = c.n_shared > 0 ? 1 : 0;
+  H->inter_shared = c.n_shared * c.inter;
+  H->G = H->has_shared + c.n_routed;
+  H->n_tiles = (c.T + kRouterBM - 1) / kRouterBM;
+  H->T_pad = (int64_t)H->n_tiles * kRouterBM;
+  H->rows_cap = ((int64_t)c.T * c.top_k + (int64_t)c.n_routed * (kGemmBM - 1) + kGemmBM - 1) /
+                kGemmBM * kGemmBM;
+  H->n_pad = (c.n_routed + 15) / 16 * 16;
+  H->maxk = pick_maxk(c.top_k);
+  const size_t es = H->es;
+  const size_t d = c.d, I = c.inter, Is = H->inter_shared, nr = c.n_routed, ks = c.n_shared;
+
+  // ---- weights
+  cudaStream_t st;
+  MOE_CUDA(cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking));
+  struct StreamGuard {
+    cudaStream_t s;
+    ~StreamGuard() { cudaStreamDestroy(s); }
+  } guard{st};
+
+  MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->bias), (size_t)H->n_pad * 4));
+  MOE_CUDA(cudaMemsetAsync(H->bias, 0, (size_t)H->n_pad * 4, st));
+  if (c.logit_bias)
+    MOE_CUDA(cudaMemcpyAsync(H->bias, c.logit_bias, nr * 4, cudaMemcpyDeviceToDevice, st));
+  const size_t cen_rows = H->bf16 ? (size_t)H->n_pad : nr;
+  MOE_TRY(dalloc(H, &H->centroids, cen_rows * d * es));
+  MOE_CUDA(cudaMemsetAsync(H->centroids, 0, cen_rows * d * es, st));
+  MOE_CUDA(cudaMemcpyAsync(H->centroids, c.centroids, nr * d * es, cudaMemcpyDeviceToDevice, st));
+
+  const char* wg = static_cast<const char*>(c.w_gate);
+  const char* wu = static_cast<const char*>(c.w_up);
+  const char* wd = static_cast<const char*>(c.w_down);
+  if (H->bf16) {
+    // gate/up interleaved in blocks of 64 rows: [g0..63, u0..63, g64..127, u64..127, ...]
+    const size_t blk = 64 * d * es;
+    if (ks) {
+      MOE_TRY(dalloc(H, &H->w_gu_s, 2 * Is * d * es));
+      MOE_CUDA(cudaMemcpy2DAsync(H->w_gu_s, 2 * blk, wg, blk, blk, Is / 64, cudaMemcpyDeviceToDevice, st));
+      MOE_CUDA(cudaMemcpy2DAsync(static_cast<char*>(H->w_gu_s) + blk, 2 * blk, wu, blk, blk, Is / 64,
+                                 cudaMemcpyDeviceToDevice, st));
+    }
+    MOE_TRY(dalloc(H, &H->w_gu_r, 2 * nr * I * d * es));
+    MOE_CUDA(cudaMemcpy2DAsync(H->w_gu_r, 2 * blk, wg + ks * I * d * es, blk, blk, nr * I / 64,
+                               cudaMemcpyDeviceToDevice, st));
+    MOE_CUDA(cudaMemcpy2DAsync(static_cast<char*>(H->w_gu_r) + blk, 2 * blk, wu + ks * I * d * es, blk,
+                               blk, nr * I / 64, cudaMemcpyDeviceToDevice, st));
+  } else {
+    MOE_TRY(dalloc(H, &H->w_g, (ks + nr) * I * d * es));
+    MOE_TRY(dalloc(H, &H->w_u, (ks + nr) * I * d * es));
+    MOE_CUDA(cudaMemcpyAsync(H->w_g, wg, (ks + nr) * I * d * es, cudaMemcpyDeviceToDevice, st));
+    MOE_CUDA(cudaMemcpyAsync(H->w_u, wu, (ks + nr) * I * d * es, cudaMemcpyDeviceToDevice, st));
+  }
+  // down projection: shared experts side by side along the intermediate axis [d, ks*I]
+  if (ks) {
+    MOE_TRY(dalloc(H, &H->w_d_s, d * Is * es));
+    for (size_t j = 0; j < ks; ++j)
+      MOE_CUDA(cudaMemcpy2DAsync(static_cast<char*>(H->w_d_s) + j * I * es, Is * es, wd + j * d * I * es,
+                                 I * es, I * es, d, cudaMemcpyDeviceToDevice, st));
+  }
+  MOE_TRY(dalloc(H, &H->w_d_r, nr * d * I * es));
+  MOE_CUDA(cudaMemcpyAsync(H->w_d_r, wd + ks * d * I * es, nr * d * I * es, cudaMemcpyDeviceToDevice, st));
+
+  // ---- workspace
+  const size_t T = c.T, K = c.top_k, nt = H->n_tiles;
+  MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->topk_rank), T * K * 4));
+  MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->slot_row), T * K * 4));
+  MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->tile_hist), nt * nr * 4));
+  MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->tile_base), nt * nr * 4));
+  MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->tile_psum), nt * nr * 4));
+  MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->psum_total), nr * 4));
+  MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->grp_row), (size_t)H->G * 4));
+  MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->ts1), (size_t)(H->G + 1) * 4));
+  MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->ts2), (size_t)(H->G + 1) * 4));
+  MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->err), 256));
+  MOE_CUDA(cudaMemsetAsync(H->err, 0, 256, st));
+  const size_t rc = (size_t)H->rows_cap, tp = (size_t)H->T_pad;
+  MOE_TRY(dalloc(H, &H->xp, rc * d * es));
+  MOE_TRY(dalloc(H, &H->hr, rc * I * es));
+  MOE_TRY(dalloc(H, &H->yr, rc * d * es));
+  if (ks) {
+    MOE_TRY(dalloc(H, &H->hs, tp * Is * es));
+    MOE_TRY(dalloc(H, &H->ys, tp * d * es));
+  }
+  MOE_TRY(dalloc(H, &H->u_dev, T * d * es));
+  MOE_TRY(dalloc(H, &H->h_dev, T * d * es));
+  MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->idx_dev), T * K * 4));
+  MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->w_dev), T * K * 4));
+  MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->cnt_dev), nr * 4));
+  MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->aux_dev), 4));
+  MOE_CUDA(cudaStreamSynchronize(st));
+
+  // ---- kernels' launch attributes and TMA descriptors
+  if (H->bf16) {
+    const uint32_t b_bytes = ((uint32_t)H->n_pad * 128u + 1023u) & ~1023u;
+    const uint32_t stage_bytes = kRouterBM * 64 * 2 + b_bytes;
+    int stages = (int)((200u * 1024u) / stage_bytes);
+    if (stages > kRouterMaxStages) stages = kRouterMaxStages;
+    if (stages < 2) stages = 2;
+    H->router_stages = stages;
+    H->router_smem = 1024 + (size_t)stages * stage_bytes + 256;
+    if ((size_t)stages * stage_bytes < sizeof(RouterEpiSmem))
+      return fail(MOE_ERR_UNSUPPORTED, "router epilogue scratch does not fit");
+    uint32_t cols = 32;
+    while (cols < (uint32_t)H->n_pad) cols <<= 1;
+    H->router_tmem_cols = cols;
+    const void* rk = H->maxk == 4 ? (const void*)router_tc_kernel<4>
+                   : H->maxk == 8 ? (const void*)router_tc_kernel<8>
+                                  : (const void*)router_tc_kernel<16>;
+    MOE_CUDA(cudaFuncSetAttribute(rk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)H->router_smem));
+    MOE_CUDA(cudaFuncSetAttribute((const void*)grouped_gemm_tc_kernel<kGateUpSwiGLU>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmemBytes));
+    MOE_CUDA(cudaFuncSetAttribute((const void*)grouped_gemm_tc_kernel<kDown>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmemBytes));
+    bool ok = encode_2d(&H->tmE, H->centroids, d, (uint64_t)H->n_pad, (uint32_t)H->n_pad) &&
+              encode_2d(&H->tmXp, H->xp, d, rc, kGemmBM) &&
+              encode_3d(&H->tmWguR, H->w_gu_r, d, 2 * I, nr, kGemmBN) &&
+              encode_2d(&H->tmHr, H->hr, I, rc, kGemmBM) &&
+              encode_3d(&H->tmWdR, H->w_d_r, I, d, nr, kGemmBN);
+    if (ks)
+      ok = ok && encode_2d(&H->tmWguS, H->w_gu_s, d, 2 * Is, kGemmBN) &&
+           encode_2d(&H->tmHs, H->hs, Is, tp, kGemmBM) &&
+           encode_2d(&H->tmWdS, H->w_d_s, Is, d, kGemmBN);
+    else {
+      H->tmWguS = H->tmWguR;
+      H->tmHs = H->tmHr;
+      H->tmWdS = H->tmWdR;
+    }
+    if (!ok) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for a weight/workspace tensor");
+  } else {
+    H->simt_router_smem = sizeof(RouterEpiSmem) + (size_t)kRouterBM * (nr + 1) * 4;
+    const void* rk = H->maxk == 4 ? (const void*)router_simt_kernel<4>
+                   : H->maxk == 8 ? (const void*)router_simt_kernel<8>
+                                  : (const void*)router_simt_kernel<16>;
+    MOE_CUDA(cudaFuncSetAttribute(rk, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)H->simt_router_smem));
+  }
+  return MOE_OK;
+}
+
+moe_status moe_create(const moe_cfg* cfg, moe_handle** out) {
+  if (!out) return fail(MOE_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  MOE_TRY(validate(cfg));
+  moe_handle* H = new (std::nothrow) moe_handle();
+  if (!H) return fail(MOE_ERR_OOM, "host allocation failed");
+  moe_status s = create_impl(cfg, H);
+  if (s != MOE_OK) {
+    cudaDeviceSynchronize();
+    free_handle(H);
+    return s;
+  }
+  *out = H;
+  return MOE_OK;
+}
+
+moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx, float* topk_w,
+                       int32_t* expert_counts, float* aux_loss, moe_stream_t stream_) {
+  if (!H) return fail(MOE_ERR_INVALID_ARG, "handle is NULL");
+  if (!u || !h || !topk_idx || !topk_w || !expert_counts || !aux_loss)
+    return fail(MOE_ERR_INVALID_ARG, "an input/output pointer is NULL");
+  if (!aligned16(u) || !aligned16(h)) return fail(MOE_ERR_INVALID_ARG, "u and h must be 16-byte aligned");
+  int dev = -1;
+  MOE_CUDA(cudaGetDevice(&dev));
+  if (dev != H->device)
+    return fail(MOE_ERR_INVALID_ARG, "current device %d is not the handle's device %d", dev, H->device);
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const moe_cfg& c = H->cfg;
+  const int T = c.T, d = c.d, K = c.top_k, nr = c.n_routed;
+
+  RouterOut ro{topk_idx, topk_w, H->topk_rank, H->tile_hist, H->tile_psum, H->err};
+  CUtensorMap tmU;
+  if (H->bf16) {
+    if (!encode_2d(&tmU, u, d, T, kRouterBM))
+      return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for u");
+    RouterTcArgs ra{T, d, nr, H->n_pad, K, H->router_stages, H->router_tmem_cols, H->bias, ro};
+    if (H->maxk == 4)
+      router_tc_kernel<4><<<H->n_tiles, kRouterThreads, H->router_smem, stream>>>(tmU, H->tmE, ra);
+    else if (H->maxk == 8)
+      router_tc_kernel<8><<<H->n_tiles, kRouterThreads, H->router_smem, stream>>>(tmU, H->tmE, ra);
+    else
+      router_tc_kernel<16><<<H->n_tiles, kRouterThreads, H->router_smem, stream>>>(tmU, H->tmE, ra);
+  } else {
+    RouterSimtArgs ra{static_cast<const float*>(u), static_cast<const float*>(H->centroids), H->bias,
+                      T, d, nr, K, ro};
+    if (H->maxk == 4)
+      router_simt_kernel<4><<<H->n_tiles, kRouterBM, H->simt_router_smem, stream>>>(ra);
+    else if (H->maxk == 8)
+      router_simt_kernel<8><<<H->n_tiles, kRouterBM, H->simt_router_smem, stream>>>(ra);
+    else
+      router_simt_kernel<16><<<H->n_tiles, kRouterBM, H->simt_router_smem, stream>>>(ra);
+  }
+  MOE_CUDA(cudaGetLastError());
+
+  const int bn1 = H->bf16 ? kGemmBN / 2 : kSimtBN;
+  const int bn2 = H->bf16 ? kGemmBN : kSimtBN;
+  ScanArgs sa{H->tile_hist, H->tile_psum, H->n_tiles, nr, T, H->has_shared, H->inter_shared,
+              c.inter, d, bn1, bn2, c.alpha1, expert_counts, aux_loss, H->psum_total,
+              H->tile_base, H->grp_row, H->ts1, H->ts2};
+  scan_kernel<<<1, kScanThreads, 0, stream>>>(sa);
+  MOE_CUDA(cudaGetLastError());
+
+  PermuteArgs pa{static_cast<const uint8_t*>(u), topk_idx, H->topk_rank, H->tile_base, H->slot_row,
+                 static_cast<uint8_t*>(H->xp), T, K, nr, (int)H->rows_cap, d * H->es, H->err};
+  permute_kernel<<<(T + kPermuteWarps - 1) / kPermuteWarps, kPermuteWarps * 32, 0, stream>>>(pa);
+  MOE_CUDA(cudaGetLastError());
+
+  const int I = c.inter, Is = H->inter_shared;
+  if (H->bf16) {
+    GemmArgs g1{};
+    g1.grp_row = H->grp_row; g1.ts = H->ts1; g1.G = H->G; g1.has_shared = H->has_shared;
+    g1.kb_shared = d / kGemmBK; g1.kb_routed = d / kGemmBK;
+    g1.nt_shared = (Is + bn1 - 1) / bn1; g1.nt_routed = (I + bn1 - 1) / bn1;
+    g1.out_shared = static_cast<__nv_bfloat16*>(H->hs); g1.ld_shared = Is; g1.rows_shared = H->T_pad;
+    g1.cols_shared = Is;
+    g1.out_routed = static_cast<__nv_bfloat16*>(H->hr); g1.ld_routed = I; g1.rows_routed = H->rows_cap;
+    g1.cols_routed = I;
+    g1.err = H->err;
+    grouped_gemm_tc_kernel<kGateUpSwiGLU><<<H->n_sms, kGemmThreads, kGemmSmemBytes, stream>>>(
+        tmU, H->tmXp, H->tmWguS, H->tmWguR, g1);
+    MOE_CUDA(cudaGetLastError());
+
+    GemmArgs g2{};
+    g2.grp_row = H->grp_row; g2.ts = H->ts2; g2.G = H->G; g2.has_shared = H->has_shared;
+    g2.kb_shared = Is / kGemmBK; g2.kb_routed = I / kGemmBK;
+    g2.nt_shared = (d + bn2 - 1) / bn2; g2.nt_routed = (d + bn2 - 1) / bn2;
+    g2.out_shared = static_cast<__nv_bfloat16*>(H->ys); g2.ld_shared = d; g2.rows_shared = H->T_pad;
+    g2.cols_shared = d;
+    g2.out_routed = static_cast<__nv_bfloat16*>(H->yr); g2.ld_routed = d; g2.rows_routed = H->rows_cap;
+    g2.cols_routed = d;
+    g2.err = H->err;
+    grouped_gemm_tc_kernel<kDown><<<H->n_sms, kGemmThreads, kGemmSmemBytes, stream>>>(
+        H->tmHs, H->tmHr, H->tmWdS, H->tmWdR, g2);
+    MOE_CUDA(cudaGetLastError());
+
+    CombineArgs<__nv_bfloat16> ca{static_cast<const __nv_bfloat16*>(u),
+                                  static_cast<const __nv_bfloat16*>(H->ys),
+                                  static_cast<const __nv_bfloat16*>(H->yr), H->slot_row, topk_w,
+                                  static_cast<__nv_bfloat16*>(h), T, d, K};
+    combine_bf16_kernel<<<(T + kCombineWarps - 1) / kCombineWarps, kCombineWarps * 32, 0, stream>>>(ca);
+    MOE_CUDA(cudaGetLastError());
+  } else {
+    const size_t ks = c.n_shared;
+    const float* wg = static_cast<const float*>(H->w_g);
+    const float* wu = static_cast<const float*>(H->w_u);
+    const int grid = H->n_sms * 4;
+    SimtGemmArgs s1{};
+    s1.grp_row = H->grp_row; s1.ts = H->ts1; s1.G = H->G; s1.has_shared = H->has_shared;
+    s1.a_shared = static_cast<const float*>(u); s1.a_rows_shared = T;
+    s1.a_routed = static_cast<const float*>(H->xp); s1.a_rows_routed = H->rows_cap;
+    s1.K_shared = d; s1.K_routed = d;
+    s1.b0_shared = wg; s1.b1_shared = wu;
+    s1.b0_routed = wg + ks * I * (size_t)d; s1.b1_routed = wu + ks * I * (size_t)d;
+    s1.b_expert_stride = (int64_t)I * d;
+    s1.N_shared = Is; s1.N_routed = I;
+    s1.nt_shared = (Is + bn1 - 1) / bn1; s1.nt_routed = (I + bn1 - 1) / bn1;
+    s1.out_shared = static_cast<float*>(H->hs); s1.out_rows_shared = H->T_pad;
+    s1.out_routed = static_cast<float*>(H->hr); s1.out_rows_routed = H->rows_cap;
+    s1.err = H->err;
+    grouped_gemm_simt_kernel<kGateUpSwiGLU><<<grid, kSimtThreads, 0, stream>>>(s1);
+    MOE_CUDA(cudaGetLastError());
+
+    SimtGemmArgs s2{};
+    s2.grp_row = H->grp_row; s2.ts = H->ts2; s2.G = H->G; s2.has_shared = H->has_shared;
+    s2.a_shared = static_cast<const float*>(H->hs); s2.a_rows_shared = H->T_pad;
+    s2.a_routed = static_cast<const float*>(H->hr); s2.a_rows_routed = H->rows_cap;
+    s2.K_shared = Is; s2.K_routed = I;
+    s2.b0_shared = static_cast<const float*>(H->w_d_s); s2.b1_shared = nullptr;
+    s2.b0_routed = static_cast<const float*>(H->w_d_r); s2.b1_routed = nullptr;
+    s2.b_expert_stride = (int64_t)d * I;
+    s2.N_shared = d; s2.N_routed = d;
+    s2.nt_shared = (d + bn2 - 1) / bn2; s2.nt_routed = (d + bn2 - 1) / bn2;
+    s2.out_shared = static_cast<float*>(H->ys); s2.out_rows_shared = H->T_pad;
+    s2.out_routed = static_cast<float*>(H->yr); s2.out_rows_routed = H->rows_cap;
+    s2.err = H->err;
+    grouped_gemm_simt_kernel<kDown><<<grid, kSimtThreads, 0, stream>>>(s2);
+    MOE_CUDA(cudaGetLastError());
+
+    CombineArgs<float> ca{static_cast<const float*>(u), static_cast<const float*>(H->ys),
+                          static_cast<const float*>(H->yr), H->slot_row, topk_w,
+                          static_cast<float*>(h), T, d, K};
+    combine_f32_kernel<<<(T + kCombineWarps - 1) / kCombineWarps, kCombineWarps * 32, 0, stream>>>(ca);
+    MOE_CUDA(cudaGetLastError());
+  }
+  return MOE_OK;
+}
+
+moe_status moe_forward_host(moe_handle* H, const void* u_host, void* h_host, int32_t* topk_idx_host,
+                            float* topk_w_host, int32_t* expert_counts_host, float* aux_loss_host,
+                            moe_stream_t stream_) {
+  if (!H) return fail(MOE_ERR_INVALID_ARG, "handle is NULL");
+  if (!u_host || !h_host) return fail(MOE_ERR_INVALID_ARG, "u_host and h_host must not be NULL");
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const moe_cfg& c = H->cfg;
+  const size_t row = (size_t)c.T * c.d * H->es, tk = (size_t)c.T * c.top_k;
+  MOE_CUDA(cudaMemcpyAsync(H->u_dev, u_host, row, cudaMemcpyHostToDevice, stream));
+  MOE_TRY(moe_forward(H, H->u_dev, H->h_dev, H->idx_dev, H->w_dev, H->cnt_dev, H->aux_dev, stream_));
+  MOE_CUDA(cudaMemcpyAsync(h_host, H->h_dev, row, cudaMemcpyDeviceToHost, stream));
+  if (topk_idx_host)
+    MOE_CUDA(cudaMemcpyAsync(topk_idx_host, H->idx_dev, tk * 4, cudaMemcpyDeviceToHost, stream));
+  if (topk_w_host)
+    MOE_CUDA(cudaMemcpyAsync(topk_w_host, H->w_dev, tk * 4, cudaMemcpyDeviceToHost, stream));
+  if (expert_counts_host)
+    MOE_CUDA(cudaMemcpyAsync(expert_counts_host, H->cnt_dev, (size_t)c.n_routed * 4,
+                             cudaMemcpyDeviceToHost, stream));
+  if (aux_loss_host)
+    MOE_CUDA(cudaMemcpyAsync(aux_loss_host, H->aux_dev, 4, cudaMemcpyDeviceToHost, stream));
+  MOE_CUDA(cudaStreamSynchronize(stream));
+  return MOE_OK;
+}
+
+moe_status moe_device_status(moe_handle* H, moe_stream_t stream_) {
+  if (!H) return fail(MOE_ERR_INVALID_ARG, "handle is NULL");
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  MOE_CUDA(cudaStreamSynchronize(stream));
+  int code = 0;
+  MOE_CUDA(cudaMemcpy(&code, H->err, sizeof(int), cudaMemcpyDeviceToHost));
+  if (code != 0) {
+    MOE_CUDA(cudaMemset(H->err, 0, sizeof(int)));
+    return fail(MOE_ERR_DEVICE_CHECK, "a kernel recorded device error 0x%x", code);
+  }
+  return MOE_OK;
+}
+
+moe_status moe_expert_psum(moe_handle* H, float* psum, moe_stream_t stream_) {
+  if (!H || !psum) return fail(MOE_ERR_INVALID_ARG, "handle or psum is NULL");
+  MOE_CUDA(cudaMemcpyAsync(psum, H->psum_total, (size_t)H->cfg.n_routed * 4, cudaMemcpyDeviceToDevice,
+                           reinterpret_cast<cudaStream_t>(stream_)));
+  return MOE_OK;
+}
+
+moe_status moe_balance_loss(const int32_t* counts, const float* psum, int32_t n_routed,
+                            int64_t n_tokens, float alpha1, float* aux_loss, moe_stream_t stream_) {
+  if (!counts || !psum || !aux_loss) return fail(MOE_ERR_INVALID_ARG, "a pointer is NULL");
+  if (n_routed < 1 || n_tokens < 1) return fail(MOE_ERR_INVALID_ARG, "n_routed and n_tokens must be positive");
+  balance_loss_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream_)>>>(
+      counts, psum, n_routed, 1.0 / (double)n_tokens, alpha1, aux_loss);
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+void moe_destroy(moe_handle* H) {
+  if (!H) return;
+  cudaDeviceSynchronize();
+  free_handle(H);
+}
+
+}  // extern "C"

@@ -1,0 +1,154 @@
+"""Python face of the C-ABI: a DeepSeekMoE layer whose forward pass runs in libmoe.so.
+
+PyTorch is used for device memory and streams only; every step of the forward pass
+(router, scan/permute, grouped expert GEMMs, combine, balance statistics) runs in the
+library's CUDA kernels.  There is no CPU or PyTorch fallback: a missing library or a
+non-B200 device raises.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import NamedTuple
+
+import numpy as np
+import torch
+
+from . import _lib
+from ._lib import MoeCfg, check, lib
+
+
+class MoEOutput(NamedTuple):
+    h: torch.Tensor              # [T, d] layer output (dtype of the layer)
+    topk_idx: torch.Tensor       # [T, top_k] int32, descending logit order
+    topk_w: torch.Tensor         # [T, top_k] fp32 gates
+    expert_counts: torch.Tensor  # [n_routed] int32
+    aux_loss: torch.Tensor       # [1] fp32
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def to_device_tensor(a: np.ndarray, device) -> torch.Tensor:
+    """Upload a workload array: uint16 arrays are bf16 bit patterns, float32 stays fp32."""
+    if a.dtype == np.uint16:
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device).view(torch.bfloat16)
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device)
+
+
+class MoELayer:
+    """One DeepSeekMoE layer (fixed token count T per instance)."""
+
+    def __init__(self, *, T: int, d: int, n_routed: int, n_shared: int, top_k: int, inter: int,
+                 dtype: str, alpha1: float, centroids: torch.Tensor, w_gate: torch.Tensor,
+                 w_up: torch.Tensor, w_down: torch.Tensor, logit_bias: torch.Tensor | None = None):
+        self.T, self.d, self.n_routed, self.n_shared = T, d, n_routed, n_shared
+        self.top_k, self.inter, self.alpha1 = top_k, inter, alpha1
+        self.dtype = dtype
+        self.torch_dtype = torch.bfloat16 if dtype == "bf16" else torch.float32
+        self.device = centroids.device
+        for t in (centroids, w_gate, w_up, w_down):
+            if not t.is_cuda or not t.is_contiguous() or t.dtype != self.torch_dtype:
+                raise ValueError("weights must be contiguous CUDA tensors of the layer dtype")
+        if logit_bias is not None and (logit_bias.dtype != torch.float32 or not logit_bias.is_cuda):
+            raise ValueError("logit_bias must be a float32 CUDA tensor")
+        cfg = MoeCfg(T=T, d=d, n_routed=n_routed, n_shared=n_shared, top_k=top_k, inter=inter,
+                     dtype=_lib.MOE_BF16 if dtype == "bf16" else _lib.MOE_FP32, alpha1=alpha1,
+                     centroids=_ptr(centroids), logit_bias=_ptr(logit_bias), w_gate=_ptr(w_gate),
+                     w_up=_ptr(w_up), w_down=_ptr(w_down))
+        handle = ctypes.c_void_p()
+        with torch.cuda.device(self.device):
+            check(lib().moe_create(ctypes.byref(cfg), ctypes.byref(handle)))
+        self._h = handle
+
+    @classmethod
+    def from_workload(cls, w, device="cuda") -> "MoELayer":
+        dev = torch.device(device)
+        bias = None if w.logit_bias is None else torch.from_numpy(w.logit_bias).to(dev)
+        return cls(T=w.T, d=w.d, n_routed=w.n_routed, n_shared=w.n_shared, top_k=w.top_k,
+                   inter=w.inter, dtype=w.dtype, alpha1=w.alpha1,
+                   centroids=to_device_tensor(w.centroids, dev),
+                   w_gate=to_device_tensor(w.w_gate, dev), w_up=to_device_tensor(w.w_up, dev),
+                   w_down=to_device_tensor(w.w_down, dev), logit_bias=bias)
+
+    # -------------------------------------------------------------------------- calls
+    def alloc_outputs(self) -> MoEOutput:
+        dev = self.device
+        return MoEOutput(
+            h=torch.empty(self.T, self.d, dtype=self.torch_dtype, device=dev),
+            topk_idx=torch.empty(self.T, self.top_k, dtype=torch.int32, device=dev),
+            topk_w=torch.empty(self.T, self.top_k, dtype=torch.float32, device=dev),
+            expert_counts=torch.empty(self.n_routed, dtype=torch.int32, device=dev),
+            aux_loss=torch.empty(1, dtype=torch.float32, device=dev))
+
+    def forward(self, u: torch.Tensor, out: MoEOutput | None = None,
+                stream: torch.cuda.Stream | None = None) -> MoEOutput:
+        """Enqueue one forward pass on `stream` (default: the current stream)."""
+        if u.shape != (self.T, self.d) or u.dtype != self.torch_dtype or not u.is_contiguous():
+            raise ValueError(f"u must be a contiguous [{self.T}, {self.d}] {self.torch_dtype} tensor")
+        out = out or self.alloc_outputs()
+        s = stream or torch.cuda.current_stream(self.device)
+        check(lib().moe_forward(self._h, _ptr(u), _ptr(out.h), _ptr(out.topk_idx),
+                                _ptr(out.topk_w), _ptr(out.expert_counts), _ptr(out.aux_loss),
+                                s.cuda_stream))
+        return out
+
+    __call__ = forward
+
+    def forward_host(self, u: torch.Tensor, out: MoEOutput | None = None,
+                     stream: torch.cuda.Stream | None = None) -> MoEOutput:
+        """Forward pass on HOST tensors (pinned for overlap); copies in and out, synchronises."""
+        if u.is_cuda or u.shape != (self.T, self.d) or u.dtype != self.torch_dtype:
+            raise ValueError("u must be a host tensor of the layer shape and dtype")
+        if out is None:
+            out = MoEOutput(
+                h=torch.empty(self.T, self.d, dtype=self.torch_dtype, pin_memory=True),
+                topk_idx=torch.empty(self.T, self.top_k, dtype=torch.int32, pin_memory=True),
+                topk_w=torch.empty(self.T, self.top_k, dtype=torch.float32, pin_memory=True),
+                expert_counts=torch.empty(self.n_routed, dtype=torch.int32, pin_memory=True),
+                aux_loss=torch.empty(1, dtype=torch.float32, pin_memory=True))
+        s = stream or torch.cuda.current_stream(self.device)
+        check(lib().moe_forward_host(self._h, _ptr(u), _ptr(out.h), _ptr(out.topk_idx),
+                                     _ptr(out.topk_w), _ptr(out.expert_counts),
+                                     _ptr(out.aux_loss), s.cuda_stream))
+        return out
+
+    def device_status(self, stream: torch.cuda.Stream | None = None) -> None:
+        """Synchronise and raise if a kernel recorded a device-side error."""
+        s = stream or torch.cuda.current_stream(self.device)
+        check(lib().moe_device_status(self._h, s.cuda_stream))
+
+    def expert_psum(self, out: torch.Tensor | None = None) -> torch.Tensor:
+        out = out if out is not None else torch.empty(self.n_routed, dtype=torch.float32,
+                                                      device=self.device)
+        check(lib().moe_expert_psum(self._h, _ptr(out), torch.cuda.current_stream(self.device).cuda_stream))
+        return out
+
+    @property
+    def kernels_per_forward(self) -> int:
+        return int(lib().moe_kernels_per_forward(self._h))
+
+    @property
+    def device_bytes(self) -> int:
+        return int(lib().moe_device_bytes(self._h))
+
+    def close(self) -> None:
+        if getattr(self, "_h", None):
+            lib().moe_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def balance_loss(counts: torch.Tensor, psum: torch.Tensor, n_tokens: int, alpha1: float,
+                 out: torch.Tensor | None = None) -> torch.Tensor:
+    """aux = alpha1 * sum_i (counts_i / n_tokens) * (psum_i / n_tokens), on the device."""
+    out = out if out is not None else torch.empty(1, dtype=torch.float32, device=counts.device)
+    check(lib().moe_balance_loss(_ptr(counts), _ptr(psum), counts.numel(), int(n_tokens),
+                                 float(alpha1), _ptr(out),
+                                 torch.cuda.current_stream(counts.device).cuda_stream))
+    return out

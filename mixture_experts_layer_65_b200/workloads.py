@@ -16,7 +16,7 @@ The token counts, hidden sizes, intermediate widths, distributions and the Zipf 
 skew of the 145B layer are the workload recipe chosen for this library (no trained
 weights or datasets exist here):
   u ~ N(0, 1);  centroids e_i ~ N(0, variance 1/d) so logits are ~N(0, 1);
-  expert weights ~ N(0, std 0.02);  seed 0;  one PCG64 stream per tensor.
+  expert weights ~ N(0, std 0.02);  seed 0;  PCG64 streams per tensor and expert.
 bf16 configurations round the fp32 draws to bf16 (round-to-nearest-even) and keep the
 raw 16-bit patterns; both sides widen those patterns exactly.
 """
@@ -24,6 +24,8 @@ from __future__ import annotations
 
 import dataclasses
 import math
+import os
+from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
 
@@ -113,37 +115,59 @@ class Workload:
                     inter=self.inter, top_k=self.top_k, dtype=self.dtype, alpha1=self.alpha1)
 
 
-def _draw(rng: np.random.Generator, shape, std: float, dtype: str) -> np.ndarray:
-    x = rng.standard_normal(shape, dtype=np.float32)
+def _draw(seed_seq, shape, std: float, dtype: str) -> np.ndarray:
+    x = np.random.Generator(np.random.PCG64(seed_seq)).standard_normal(shape, dtype=np.float32)
     if std != 1.0:
         x *= np.float32(std)
     return f32_to_bf16_bits(x) if dtype == "bf16" else x
 
 
-def make_workload(name: str = "tiny", seed: int = 0, **overrides) -> Workload:
+_ROWS_PER_STREAM = 1024
+
+
+def make_workload(name: str = "tiny", seed: int = 0, threads: int | None = None,
+                  **overrides) -> Workload:
     """Draw the seeded inputs of a named configuration (fields may be overridden).
 
-    Each tensor has its own PCG64 stream spawned from SeedSequence(seed), so changing T
-    keeps the weights identical and keeps u's first rows identical (row-major draws).
+    Streams: SeedSequence(seed) spawns one child per tensor (u, centroids, w_gate, w_up,
+    w_down); each weight tensor's child spawns one PCG64 stream per expert and u's child one
+    stream per block of 1024 token rows.  Child i of a SeedSequence does not depend on how
+    many children are spawned, so changing T keeps every weight and u's first rows
+    identical, and the per-expert streams let the draws run on several threads.
     """
     spec = dict(CONFIGS[name]) if name in CONFIGS else {}
     spec.update(overrides)
     T, d, ks, nr = int(spec["T"]), int(spec["d"]), int(spec["n_shared"]), int(spec["n_routed"])
     inter, top_k, dtype = int(spec["inter"]), int(spec["top_k"]), spec["dtype"]
     g = ks + nr
-    rngs = {k: np.random.Generator(np.random.PCG64(s))
-            for k, s in zip(_STREAMS, np.random.SeedSequence(seed).spawn(len(_STREAMS)))}
-    u = _draw(rngs["u"], (T, d), 1.0, dtype)
-    cen = _draw(rngs["centroids"], (nr, d), 1.0 / math.sqrt(d), dtype)
-    # per-expert draws keep the fp32 temporaries small for the large layers
+    ss = dict(zip(_STREAMS, np.random.SeedSequence(seed).spawn(len(_STREAMS))))
     edt = np.uint16 if dtype == "bf16" else np.float32
+    u = np.empty((T, d), dtype=edt)
     w_gate = np.empty((g, inter, d), dtype=edt)
     w_up = np.empty((g, inter, d), dtype=edt)
     w_down = np.empty((g, d, inter), dtype=edt)
-    for e in range(g):
-        w_gate[e] = _draw(rngs["w_gate"], (inter, d), 0.02, dtype)
-        w_up[e] = _draw(rngs["w_up"], (inter, d), 0.02, dtype)
-        w_down[e] = _draw(rngs["w_down"], (d, inter), 0.02, dtype)
+    jobs = []
+    n_chunks = (T + _ROWS_PER_STREAM - 1) // _ROWS_PER_STREAM
+    for c, child in enumerate(ss["u"].spawn(n_chunks)):
+        r0, r1 = c * _ROWS_PER_STREAM, min(T, (c + 1) * _ROWS_PER_STREAM)
+        jobs.append((u, c, slice(r0, r1), child, (r1 - r0, d), 1.0))
+    for name_, arr, shape in (("w_gate", w_gate, (inter, d)), ("w_up", w_up, (inter, d)),
+                              ("w_down", w_down, (d, inter))):
+        for e, child in enumerate(ss[name_].spawn(g)):
+            jobs.append((arr, e, None, child, shape, 0.02))
+
+    def run(job):
+        arr, i, sl, child, shape, std = job
+        x = _draw(child, shape, std, dtype)
+        if sl is None:
+            arr[i] = x
+        else:
+            arr[sl] = x
+
+    n_thr = threads or min(32, os.cpu_count() or 1)
+    with ThreadPoolExecutor(max_workers=n_thr) as ex:
+        list(ex.map(run, jobs))
+    cen = _draw(ss["centroids"], (nr, d), 1.0 / math.sqrt(d), dtype)
     zs = spec.get("zipf_s")
     bias = zipf_logit_bias(nr, zs) if zs else None
     return Workload(name=name, T=T, d=d, n_shared=ks, n_routed=nr, inter=inter, top_k=top_k,

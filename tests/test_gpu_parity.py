@@ -1,0 +1,197 @@
+"""GPU parity: the CUDA path (through the C-ABI) against the fp64 oracle, element by element.
+
+Small layers are compared on every row; the full-size layers (2B, GShard, 16B prefill and
+decode, 145B) on all routing outputs and on sampled output rows, in the same launch
+configuration the benchmark uses.
+"""
+import numpy as np
+import pytest
+import torch
+
+from mixture_experts_layer_65_b200 import build
+from mixture_experts_layer_65_b200 import workloads as W
+from mixture_experts_layer_65_b200.layer import MoELayer, balance_loss, to_device_tensor
+from oracle import moe_oracle as O
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib_ready():
+    build.build()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+
+
+def run(w, layer=None):
+    layer = layer or MoELayer.from_workload(w)
+    u = to_device_tensor(w.u, "cuda")
+    out = layer.forward(u)
+    torch.cuda.synchronize()
+    layer.device_status()
+    return P.fetch(out), layer, u, out
+
+
+# ------------------------------------------------------------------------ small, every row
+def test_tiny_fp32():
+    w = W.make_workload("tiny")
+    g, *_ = run(w)
+    rep = P.compare(w, g)
+    print("tiny", rep)
+
+
+SMALL = [
+    # ragged T, shared group of 2, intermediate width with a half column tile
+    dict(T=333, d=256, n_shared=2, n_routed=16, inter=192, top_k=4, dtype="bf16"),
+    # N_r not a multiple of 16; hidden width with a tail tile in the down GEMM
+    dict(T=128, d=320, n_shared=1, n_routed=63, inter=128, top_k=7, dtype="bf16"),
+    # no shared expert (GShard-like)
+    dict(T=1000, d=512, n_shared=0, n_routed=16, inter=256, top_k=2, dtype="bf16"),
+    # a single token
+    dict(T=1, d=256, n_shared=1, n_routed=8, inter=128, top_k=2, dtype="bf16"),
+    # many experts and the largest top-k
+    dict(T=260, d=256, n_shared=1, n_routed=200, inter=64, top_k=16, dtype="bf16"),
+    # fp32 path, ragged sizes
+    dict(T=300, d=64, n_shared=2, n_routed=9, inter=48, top_k=3, dtype="fp32"),
+    dict(T=1, d=32, n_shared=0, n_routed=4, inter=16, top_k=4, dtype="fp32"),
+]
+
+
+@pytest.mark.parametrize("spec", SMALL, ids=lambda s: "T{T}_d{d}_s{n_shared}_r{n_routed}_i{inter}_k{top_k}_{dtype}".format(**s))
+def test_small_layers(spec):
+    w = W.make_workload("16b_prefill", alpha1=0.001, **spec)
+    g, *_ = run(w)
+    rep = P.compare(w, g)
+    print(spec, rep)
+
+
+# ------------------------------------------------------------------------ full sizes
+@pytest.mark.parametrize("name", ["2b", "gshard", "16b_prefill", "16b_decode", "145b"])
+def test_full_size_layer(name):
+    w = W.make_workload(name)
+    g, layer, *_ = run(w)
+    rows = None if w.T <= 512 else P.sample_rows(w.T)
+    rep = P.compare(w, g, rows=rows)
+    print(name, rep)
+    assert layer.kernels_per_forward == 6
+
+
+# ------------------------------------------------------------------------ edge cases
+def _bias_layer(bias, **spec):
+    w = W.make_workload("16b_prefill", alpha1=0.001, **spec)
+    w.logit_bias = np.asarray(bias, dtype=np.float32)
+    return w
+
+
+def test_expert_with_no_tokens():
+    nr = 16
+    bias = np.zeros(nr, np.float32)
+    bias[3] = -30.0
+    w = _bias_layer(bias, T=700, d=256, n_shared=1, n_routed=nr, inter=128, top_k=3, dtype="bf16")
+    g, *_ = run(w)
+    assert g.counts[3] == 0
+    P.compare(w, g)
+
+
+def test_all_tokens_to_one_expert():
+    nr = 8
+    bias = np.zeros(nr, np.float32)
+    bias[0] = 30.0
+    w = _bias_layer(bias, T=1100, d=256, n_shared=1, n_routed=nr, inter=128, top_k=1, dtype="bf16")
+    g, *_ = run(w)
+    assert g.counts[0] == w.T and g.counts[1:].sum() == 0
+    P.compare(w, g)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_top_k_equal_to_n_routed(dtype):
+    w = W.make_workload("16b_prefill", T=200, d=128, n_shared=1, n_routed=8, inter=64, top_k=8,
+                        dtype=dtype, alpha1=0.01)
+    g, *_ = run(w)
+    np.testing.assert_allclose(g.topk_w.sum(axis=1), 1.0, rtol=0, atol=1e-5)
+    P.compare(w, g)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_single_expert_layer_is_dense_ffn(dtype):
+    w = W.make_workload("16b_prefill", T=150, d=128, n_shared=0, n_routed=1, inter=64, top_k=1,
+                        dtype=dtype, alpha1=0.01)
+    g, *_ = run(w)
+    np.testing.assert_array_equal(g.topk_idx, 0)
+    np.testing.assert_allclose(g.topk_w, 1.0, rtol=0, atol=1e-6)
+    assert abs(g.aux - 0.01) < 1e-6
+    P.compare(w, g)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_equal_logits_lower_index_wins(dtype):
+    w = W.make_workload("16b_prefill", T=1024, d=256, n_shared=1, n_routed=16, inter=64, top_k=4,
+                        dtype=dtype, alpha1=0.01)
+    w.centroids[9] = w.centroids[2]          # experts 2 and 9 always tie exactly
+    g, *_ = run(w)
+    idx = g.topk_idx
+    has2 = (idx == 2).any(axis=1)
+    has9 = (idx == 9).any(axis=1)
+    assert np.all(has2[has9]), "expert 9 chosen without its lower-index twin 2"
+    both = np.nonzero(has2 & has9)[0]
+    for t in both:
+        row = idx[t].tolist()
+        assert row.index(2) < row.index(9)
+    straddle = int((has2 & ~has9).sum())
+    print("tokens where the tie straddles the cut:", straddle)
+    P.compare(w, g)
+
+
+def test_nan_row_propagates_without_hang():
+    w = W.make_workload("16b_prefill", T=300, d=256, n_shared=1, n_routed=16, inter=128, top_k=4,
+                        dtype="bf16", alpha1=0.01)
+    w.u[7] = 0x7FC0                            # bf16 quiet NaN
+    g, layer, *_ = run(w)                      # device_status() raises on a device error
+    assert np.all(np.isnan(g.h[7]))
+    idx = g.topk_idx
+    assert idx.min() >= 0 and idx.max() < w.n_routed
+    assert np.all(np.diff(np.sort(idx, axis=1), axis=1) > 0)
+    others = np.array([r for r in range(w.T) if r != 7])
+    ref = O.moe_forward(w.u, w.centroids, w.w_gate, w.w_up, w.w_down, w.n_shared, w.top_k,
+                        w.alpha1, rows=others)
+    assert np.all(np.isfinite(g.h[others]))
+    err = np.abs(g.h[others] - ref.h).max() / np.abs(ref.h).max()
+    assert err <= P.TOL["bf16"]
+
+
+def test_bitwise_deterministic():
+    w = W.make_workload("16b_prefill", T=3000)
+    layer = MoELayer.from_workload(w)
+    u = to_device_tensor(w.u, "cuda")
+    a = layer.forward(u)
+    b = layer.forward(u)
+    torch.cuda.synchronize()
+    layer.device_status()
+    for x, y in zip(a, b):
+        assert torch.equal(x.view(torch.uint8) if x.dtype == torch.bfloat16 else x, y.view(torch.uint8) if y.dtype == torch.bfloat16 else y)
+
+
+def test_forward_host_matches_forward():
+    w = W.make_workload("16b_prefill", T=500)
+    layer = MoELayer.from_workload(w)
+    u = to_device_tensor(w.u, "cuda")
+    dev = layer.forward(u)
+    torch.cuda.synchronize()
+    host = layer.forward_host(u.cpu().pin_memory())
+    for x, y in zip(dev, host):
+        assert torch.equal(x.cpu(), y)
+    layer.device_status()
+
+
+def test_expert_psum_and_balance_loss_kernel():
+    w = W.make_workload("2b", T=1000)
+    g, layer, u, out = run(w)
+    ref = O.moe_forward(w.u, w.centroids, w.w_gate, w.w_up, w.w_down, w.n_shared, w.top_k,
+                        w.alpha1, rows=[0])
+    ps = layer.expert_psum().cpu().numpy().astype(np.float64)
+    np.testing.assert_allclose(ps, ref.P * w.T, rtol=1e-4, atol=1e-4)
+    aux = balance_loss(out.expert_counts, layer.expert_psum(), w.T, w.alpha1)
+    torch.cuda.synchronize()
+    expect = w.alpha1 * np.sum((g.counts / w.T) * (ps / w.T))
+    assert abs(float(aux.cpu()[0]) - expect) <= 1e-6 * abs(expect)
+    assert abs(float(aux.cpu()[0]) - g.aux) <= 1e-6 * abs(expect)
