@@ -1,0 +1,385 @@
+#!/usr/bin/env python
+"""Throughput of the DeepSeekMoE layer forward pass on B200.
+
+One step = one full forward pass of the layer (router, scan/permute, gate/up GEMM with
+SwiGLU, down GEMM, combine, balance statistics) over one batch of T tokens already
+resident in HBM.  Default workload: the DeepSeekMoE-16B-shaped layer at prefill
+(T=16384, d=2048, 2 shared + 64 routed experts of width 1408, top-6, bf16).
+
+  python bench.py [--gpus N --steps K --warmup W] [--config NAME] [--impl ours|reference]
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own T tokens (data
+parallel, weights replicated, weak scaling); the only exchange is the all-reduce of the
+per-expert counts and affinity sums for the global balance loss.
+Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s and expert-GEMM TFLOP/s (% BF16 peak), 16B-shaped, 1 B200"
+L2_BYTES = 126 * 2 ** 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNELS = ("router", "scan", "permute", "gate_up_gemm", "down_gemm", "combine")
+
+
+def parse_args():
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=400)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--config", default="16b_prefill")
+    p.add_argument("--e2e-steps", type=int, default=20)
+    p.add_argument("--cpu-seconds", type=float, default=15.0,
+                   help="target CPU time of the oracle baseline sample")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return {k: float(pk[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_desc(w, n_gpus: int) -> dict:
+    return {"workload": f"{w.name}: T={w.T} d={w.d} shared={w.n_shared} routed={w.n_routed} "
+                        f"inter={w.inter} top_k={w.top_k} {w.dtype}",
+            "T_per_gpu": w.T, "d": w.d, "n_shared": w.n_shared, "n_routed": w.n_routed,
+            "inter": w.inter, "top_k": w.top_k, "global_batch": w.T * n_gpus,
+            "parallelism": f"dp{n_gpus}"}
+
+
+# --------------------------------------------------------------------------- work model
+def algorithmic_work(w) -> dict:
+    """Per-launch algorithmic work of each kernel (selected experts only, no padding)."""
+    es = 2 if w.dtype == "bf16" else 4
+    T, d, I, K, ks, nr = w.T, w.d, w.inter, w.top_k, w.n_shared, w.n_routed
+    passes = ks + K
+    return {
+        "router": ("hbm", T * d * es + nr * d * es + T * K * 12),
+        "scan": ("latency", 0),
+        "permute": ("hbm", T * d * es + T * K * d * es + T * K * 12),
+        "gate_up_gemm": ("tensor", 4.0 * T * d * I * passes),
+        "down_gemm": ("tensor", 2.0 * T * d * I * passes),
+        "combine": ("hbm", T * d * es * (2 + (1 if ks else 0) + K) + T * K * 8),
+    }
+
+
+def csrc_digest() -> str:
+    h = hashlib.sha1()
+    d = os.path.join(ROOT, "mixture_experts_layer_65_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()
+
+
+def ncu_traffic(kernel: str, config: str):
+    """DRAM bytes per launch from the committed ncu summary, if the kernels are unchanged."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        tab = json.load(f)
+    if tab.get("csrc_sha1") != csrc_digest():
+        return None
+    ent = tab.get("kernels", {}).get(config, {}).get(kernel)
+    return None if ent is None else float(ent["dram_bytes_per_launch"])
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}",
+                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                      stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.p = None
+
+    def stop(self) -> dict:
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.p.terminate()
+        try:
+            out = self.p.communicate(timeout=10)[0]
+        except subprocess.TimeoutExpired:
+            self.p.kill()
+            out = self.p.communicate()[0]
+        sm, smax, power, reasons = [], [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+                power.append(float(f[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "samples": len(sm),
+                "power_w_max": max(power) if power else None, "reasons": sorted(reasons)}
+
+
+# --------------------------------------------------------------------------- CPU oracle
+def oracle_tokens_per_s(w, seconds: float) -> tuple[float, dict]:
+    """Time the fp64 oracle (as it stands) on a bounded token sample of the workload."""
+    import numpy as np
+    import threadpoolctl
+
+    from oracle import moe_oracle as O
+
+    def run(n):
+        t0 = time.perf_counter()
+        O.moe_forward(w.u[:n], w.centroids, w.w_gate, w.w_up, w.w_down, w.n_shared, w.top_k,
+                      w.alpha1, bias=w.logit_bias)
+        return time.perf_counter() - t0
+
+    # grow the sample until one call takes about `seconds` (the oracle has a per-call cost
+    # for widening the experts it touches, so the rate depends on the sample size)
+    n = min(w.T, 64)
+    while True:
+        dt = run(n)
+        if dt >= 0.5 * seconds or n >= w.T:
+            break
+        n = int(min(w.T, max(2 * n, n * 0.8 * seconds / max(dt, 1e-6))))
+    info = threadpoolctl.threadpool_info()
+    threads = max([i.get("num_threads", 1) for i in info] or [1])
+    desc = {"kind": "oracle", "cores": threads,
+            "sample": f"first {n} of {w.T} tokens of the same layer (routing + all experts, fp64 "
+                      f"NumPy/{info[0]['internal_api'] if info else 'BLAS'}); {dt:.1f} s",
+            "value": n / dt, "unit": "tokens/s"}
+    _ = np
+    return n / dt, desc
+
+
+# --------------------------------------------------------------------------- reference arm
+def run_reference(args, rank: int, world: int):
+    if rank != 0:
+        return
+    from mixture_experts_layer_65_b200 import workloads as W
+    w = W.make_workload(args.config)
+    from oracle import moe_oracle as O
+    budget = 120.0 / max(1, args.steps + args.warmup)
+
+    t0 = time.perf_counter()
+    O.moe_forward(w.u[:16], w.centroids, w.w_gate, w.w_up, w.w_down, w.n_shared, w.top_k,
+                  w.alpha1, bias=w.logit_bias)
+    per_tok = (time.perf_counter() - t0) / 16
+    n = int(max(1, min(w.T, budget / max(per_tok, 1e-9))))
+    times = []
+    for i in range(args.warmup + args.steps):
+        s = (i * n) % max(1, w.T - n + 1)
+        t0 = time.perf_counter()
+        O.moe_forward(w.u[s:s + n], w.centroids, w.w_gate, w.w_up, w.w_down, w.n_shared,
+                      w.top_k, w.alpha1, bias=w.logit_bias)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    tot = sum(times)
+    value = n * len(times) / tot
+    import threadpoolctl
+    info = threadpoolctl.threadpool_info()
+    threads = max([i.get("num_threads", 1) for i in info] or [1])
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * tot / len(times), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_desc(w, world),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                             "sample": f"{n} tokens per step of the {w.name} layer (fp64 oracle)"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- our arm
+def run_ours(args, rank: int, world: int, local_rank: int):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from mixture_experts_layer_65_b200 import workloads as W
+    from mixture_experts_layer_65_b200.layer import MoELayer, balance_loss, to_device_tensor
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = W.make_workload(args.config)
+    layer = MoELayer.from_workload(w, dev)
+    es = 2 if w.dtype == "bf16" else 4
+    u_bytes = w.T * w.d * es
+    n_buf = int(min(8, max(2, math.ceil(2 * L2_BYTES / u_bytes))))
+    base = to_device_tensor(w.u, dev)
+    # distinct token batches per rank and per buffer (row rotations of the seeded batch)
+    ubufs = [torch.roll(base, shifts=(rank * n_buf + i) * 997, dims=0).contiguous()
+             for i in range(n_buf)]
+    del base
+    out = layer.alloc_outputs()
+    if world > 1:
+        psum = torch.empty(w.n_routed, dtype=torch.float32, device=dev)
+        cnt_g = torch.empty(w.n_routed, dtype=torch.int32, device=dev)
+        aux_g = torch.empty(1, dtype=torch.float32, device=dev)
+
+    def step(i):
+        layer.forward(ubufs[i % n_buf], out)
+        if world > 1:
+            layer.expert_psum(psum)
+            cnt_g.copy_(out.expert_counts)
+            dist.all_reduce(cnt_g)
+            dist.all_reduce(psum)
+            balance_loss(cnt_g, psum, world * w.T, w.alpha1, aux_g)
+
+    for i in range(max(3, args.warmup)):
+        step(i)
+    torch.cuda.synchronize()
+    layer.device_status()
+    if world > 1:
+        dist.barrier()
+    clocks = ClockSampler() if rank == 0 else None
+    time.sleep(0.3 if clocks else 0.0)
+    stream = torch.cuda.current_stream(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    layer.timing_begin(args.steps)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    kernel_ms, n_rec = layer.timing_end()
+    clk = clocks.stop() if clocks else None
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    layer.device_status()
+
+    # end to end through the public host-buffer call (pinned host memory)
+    u_host = ubufs[0].cpu().pin_memory()
+    host_out = None
+    for _ in range(2):
+        host_out = layer.forward_host(u_host, host_out)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        host_out = layer.forward_host(u_host, host_out)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    layer.device_status()
+
+    if rank != 0:
+        return
+    peaks, peak_src = load_peaks()
+    work = algorithmic_work(w)
+    per_kernel = {}
+    for k in KERNELS:
+        kind, amount = work[k]
+        avg_ms = kernel_ms[k] / max(1, n_rec)
+        ent = {"avg_ms": avg_ms, "share": kernel_ms[k] / max(1e-12, sum(kernel_ms.values()))}
+        if kind == "tensor":
+            ach = amount / (avg_ms * 1e-3) / 1e12
+            ent.update(bound="tensor", achieved=ach, unit="TFLOP/s",
+                       frac=ach / peaks["bf16_tflops_sustained"],
+                       frac_of_burst=ach / peaks["bf16_tflops"])
+        elif kind == "hbm":
+            ach = amount / (avg_ms * 1e-3) / 1e9
+            ent.update(bound="hbm", achieved=ach, unit="GB/s", frac=ach / peaks["hbm_gbs"])
+        per_kernel[k] = ent
+    dominant = max(KERNELS, key=lambda k: kernel_ms[k])
+    dk = per_kernel[dominant]
+    bound = dk.get("bound", "latency")
+    roofline = {"kernel": dominant, "bound": bound, "achieved": dk.get("achieved"),
+                "peak": (peaks["bf16_tflops_sustained"] if bound == "tensor" else peaks["hbm_gbs"]),
+                "unit": dk.get("unit"), "frac": dk.get("frac"),
+                "peak_source": f"{peak_src} ({'bf16 sustained' if bound == 'tensor' else 'HBM copy'})",
+                "traffic": ncu_traffic(dominant, w.name), "algorithmic_per_launch": work[dominant][1]}
+    gemm_flops = work["gate_up_gemm"][1] + work["down_gemm"][1]
+    gemm_ms = (kernel_ms["gate_up_gemm"] + kernel_ms["down_gemm"]) / max(1, n_rec)
+    gemm_tflops = gemm_flops / (gemm_ms * 1e-3) / 1e12
+    value = world * w.T * args.steps / (ms * 1e-3)
+    tk = w.T * w.top_k
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic (seeded N(0,1) tokens, N(0,0.02) random-init experts, no trained weights)",
+        "config": dict(workload_desc(w, world),
+                       l2=f"inputs rotate over {n_buf} token buffers "
+                          f"({n_buf * u_bytes / 2**20:.0f} MiB > 126 MiB L2); expert weights "
+                          f"{layer.device_bytes / 2**30:.2f} GiB with workspace"),
+        "expert_gemm_tflops": gemm_tflops,
+        "expert_gemm_frac_of_peak": gemm_tflops / peaks["bf16_tflops_sustained"],
+        "expert_gemm_frac_of_burst_peak": gemm_tflops / peaks["bf16_tflops"],
+        "roofline": roofline,
+        "kernels": per_kernel,
+        "e2e": {"value": world * w.T * args.e2e_steps / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": u_bytes,
+                "d2h_bytes_per_step": u_bytes + tk * 8 + w.n_routed * 4 + 4},
+        "gpu_launches": args.steps * (layer.kernels_per_forward + (1 if world > 1 else 0)),
+        "clocks": clk,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        _, desc = oracle_tokens_per_s(w, args.cpu_seconds)
+        line["cpu_baseline"] = desc
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    import torch.distributed as dist
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=None)
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

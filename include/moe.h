@@ -130,6 +130,16 @@ moe_status moe_balance_loss(const int32_t* counts, const float* psum, int32_t n_
                             int64_t n_tokens, float alpha1, float* aux_loss,
                             moe_stream_t stream);
 
+/* Per-kernel timing.  After moe_timing_begin(handle, n), each of the next n calls of
+ * moe_forward on this handle records a CUDA event on its stream before each of its
+ * kernels and after the last one (host-side event creation happens here, not in
+ * moe_forward).  moe_timing_end synchronises those events, writes the summed elapsed
+ * milliseconds of kernel i over the recorded calls to kernel_ms[i] (i < 6: router, scan,
+ * permute, gate/up GEMM, down GEMM, combine), the number of recorded calls to
+ * *n_forwards, and switches recording off. */
+moe_status moe_timing_begin(moe_handle* handle, int32_t max_forwards);
+moe_status moe_timing_end(moe_handle* handle, double* kernel_ms, int32_t* n_forwards);
+
 /* Number of kernels one moe_forward launches on this handle. */
 int32_t moe_kernels_per_forward(const moe_handle* handle);
 

@@ -136,6 +136,9 @@ struct moe_handle {
   int32_t *idx_dev = nullptr, *cnt_dev = nullptr;
   float *w_dev = nullptr, *aux_dev = nullptr;
   CUtensorMap tmE, tmXp, tmWguS, tmWguR, tmHs, tmHr, tmWdS, tmWdR;
+  // per-kernel timing (moe_timing_begin / moe_timing_end)
+  std::vector<cudaEvent_t> events;   // kKernelsPerForward + 1 per recorded call
+  int timing_cap = 0, timing_used = 0;
   std::vector<void*> allocs;
   size_t bytes = 0;
 };
@@ -164,6 +167,7 @@ moe_status dalloc(moe_handle* H, void** p, size_t bytes) {
 
 void free_handle(moe_handle* H) {
   if (!H) return;
+  for (cudaEvent_t e : H->events) cudaEventDestroy(e);
   for (void* p : H->allocs) cudaFree(p);
   delete H;
 }
@@ -387,6 +391,12 @@ moe_status moe_create(const moe_cfg* cfg, moe_handle** out) {
   return MOE_OK;
 }
 
+// Record timing event `slot` of the current call (no-op unless timing is on).
+static inline void tick(moe_handle* H, cudaStream_t s, int slot) {
+  if (H->timing_used < H->timing_cap)
+    cudaEventRecord(H->events[(size_t)H->timing_used * (kKernelsPerForward + 1) + slot], s);
+}
+
 moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx, float* topk_w,
                        int32_t* expert_counts, float* aux_loss, moe_stream_t stream_) {
   if (!H) return fail(MOE_ERR_INVALID_ARG, "handle is NULL");
@@ -403,6 +413,7 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
 
   RouterOut ro{topk_idx, topk_w, H->topk_rank, H->tile_hist, H->tile_psum, H->err};
   CUtensorMap tmU;
+  tick(H, stream, 0);
   if (H->bf16) {
     if (!encode_2d(&tmU, u, d, T, kRouterBM))
       return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for u");
@@ -430,11 +441,13 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
   ScanArgs sa{H->tile_hist, H->tile_psum, H->n_tiles, nr, T, H->has_shared, H->inter_shared,
               c.inter, d, bn1, bn2, c.alpha1, expert_counts, aux_loss, H->psum_total,
               H->tile_base, H->grp_row, H->ts1, H->ts2};
+  tick(H, stream, 1);
   scan_kernel<<<1, kScanThreads, 0, stream>>>(sa);
   MOE_CUDA(cudaGetLastError());
 
   PermuteArgs pa{static_cast<const uint8_t*>(u), topk_idx, H->topk_rank, H->tile_base, H->slot_row,
                  static_cast<uint8_t*>(H->xp), T, K, nr, (int)H->rows_cap, d * H->es, H->err};
+  tick(H, stream, 2);
   permute_kernel<<<(T + kPermuteWarps - 1) / kPermuteWarps, kPermuteWarps * 32, 0, stream>>>(pa);
   MOE_CUDA(cudaGetLastError());
 
@@ -449,6 +462,7 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
     g1.out_routed = static_cast<__nv_bfloat16*>(H->hr); g1.ld_routed = I; g1.rows_routed = H->rows_cap;
     g1.cols_routed = I;
     g1.err = H->err;
+    tick(H, stream, 3);
     grouped_gemm_tc_kernel<kGateUpSwiGLU><<<H->n_sms, kGemmThreads, kGemmSmemBytes, stream>>>(
         tmU, H->tmXp, H->tmWguS, H->tmWguR, g1);
     MOE_CUDA(cudaGetLastError());
@@ -462,6 +476,7 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
     g2.out_routed = static_cast<__nv_bfloat16*>(H->yr); g2.ld_routed = d; g2.rows_routed = H->rows_cap;
     g2.cols_routed = d;
     g2.err = H->err;
+    tick(H, stream, 4);
     grouped_gemm_tc_kernel<kDown><<<H->n_sms, kGemmThreads, kGemmSmemBytes, stream>>>(
         H->tmHs, H->tmHr, H->tmWdS, H->tmWdR, g2);
     MOE_CUDA(cudaGetLastError());
@@ -470,6 +485,7 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
                                   static_cast<const __nv_bfloat16*>(H->ys),
                                   static_cast<const __nv_bfloat16*>(H->yr), H->slot_row, topk_w,
                                   static_cast<__nv_bfloat16*>(h), T, d, K};
+    tick(H, stream, 5);
     combine_bf16_kernel<<<(T + kCombineWarps - 1) / kCombineWarps, kCombineWarps * 32, 0, stream>>>(ca);
     MOE_CUDA(cudaGetLastError());
   } else {
@@ -490,6 +506,7 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
     s1.out_shared = static_cast<float*>(H->hs); s1.out_rows_shared = H->T_pad;
     s1.out_routed = static_cast<float*>(H->hr); s1.out_rows_routed = H->rows_cap;
     s1.err = H->err;
+    tick(H, stream, 3);
     grouped_gemm_simt_kernel<kGateUpSwiGLU><<<grid, kSimtThreads, 0, stream>>>(s1);
     MOE_CUDA(cudaGetLastError());
 
@@ -506,15 +523,53 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
     s2.out_shared = static_cast<float*>(H->ys); s2.out_rows_shared = H->T_pad;
     s2.out_routed = static_cast<float*>(H->yr); s2.out_rows_routed = H->rows_cap;
     s2.err = H->err;
+    tick(H, stream, 4);
     grouped_gemm_simt_kernel<kDown><<<grid, kSimtThreads, 0, stream>>>(s2);
     MOE_CUDA(cudaGetLastError());
 
     CombineArgs<float> ca{static_cast<const float*>(u), static_cast<const float*>(H->ys),
                           static_cast<const float*>(H->yr), H->slot_row, topk_w,
                           static_cast<float*>(h), T, d, K};
+    tick(H, stream, 5);
     combine_f32_kernel<<<(T + kCombineWarps - 1) / kCombineWarps, kCombineWarps * 32, 0, stream>>>(ca);
     MOE_CUDA(cudaGetLastError());
   }
+  if (H->timing_used < H->timing_cap) {
+    tick(H, stream, kKernelsPerForward);
+    ++H->timing_used;
+  }
+  return MOE_OK;
+}
+
+moe_status moe_timing_begin(moe_handle* H, int32_t max_forwards) {
+  if (!H || max_forwards < 1) return fail(MOE_ERR_INVALID_ARG, "handle is NULL or max_forwards < 1");
+  const size_t need = (size_t)max_forwards * (kKernelsPerForward + 1);
+  while (H->events.size() < need) {
+    cudaEvent_t e;
+    MOE_CUDA(cudaEventCreate(&e));
+    H->events.push_back(e);
+  }
+  H->timing_cap = max_forwards;
+  H->timing_used = 0;
+  return MOE_OK;
+}
+
+moe_status moe_timing_end(moe_handle* H, double* kernel_ms, int32_t* n_forwards) {
+  if (!H || !kernel_ms || !n_forwards) return fail(MOE_ERR_INVALID_ARG, "a pointer is NULL");
+  for (int k = 0; k < kKernelsPerForward; ++k) kernel_ms[k] = 0.0;
+  const int n = H->timing_used;
+  H->timing_cap = 0;
+  H->timing_used = 0;
+  for (int f = 0; f < n; ++f) {
+    const cudaEvent_t* ev = &H->events[(size_t)f * (kKernelsPerForward + 1)];
+    MOE_CUDA(cudaEventSynchronize(ev[kKernelsPerForward]));
+    for (int k = 0; k < kKernelsPerForward; ++k) {
+      float ms = 0.f;
+      MOE_CUDA(cudaEventElapsedTime(&ms, ev[k], ev[k + 1]));
+      kernel_ms[k] += ms;
+    }
+  }
+  *n_forwards = n;
   return MOE_OK;
 }
 

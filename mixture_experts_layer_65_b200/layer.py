@@ -124,6 +124,19 @@ class MoELayer:
         check(lib().moe_expert_psum(self._h, _ptr(out), torch.cuda.current_stream(self.device).cuda_stream))
         return out
 
+    KERNEL_NAMES = ("router", "scan", "permute", "gate_up_gemm", "down_gemm", "combine")
+
+    def timing_begin(self, max_forwards: int) -> None:
+        """Record per-kernel CUDA events in the next `max_forwards` forward calls."""
+        check(lib().moe_timing_begin(self._h, int(max_forwards)))
+
+    def timing_end(self) -> tuple[dict, int]:
+        """Synchronise; return ({kernel: summed ms}, number of recorded forward calls)."""
+        ms = (ctypes.c_double * 6)()
+        n = ctypes.c_int32()
+        check(lib().moe_timing_end(self._h, ms, ctypes.byref(n)))
+        return dict(zip(self.KERNEL_NAMES, list(ms))), int(n.value)
+
     @property
     def kernels_per_forward(self) -> int:
         return int(lib().moe_kernels_per_forward(self._h))

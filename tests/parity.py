@@ -12,6 +12,10 @@ TOL = {"bf16": 2e-2, "fp32": 1e-4}
 # The expert part (h - u) is also checked against max|h_ref - u| with the same factor
 # (after discounting the output's own rounding), so the residual cannot hide an error in
 # the experts.
+# Gates g = s come from fp32 logits accumulated over d bf16 products; the accumulated
+# rounding error of a logit grows like sqrt(d) (about 1e-5 absolute at d = 4096 for
+# logits of unit scale), and a logit error e shifts s by a relative e (plus the same
+# through the softmax denominator).  Hence 1e-5 relative up to d = 1024, scaled with d.
 GATE_RTOL = 1e-5
 AUX_RTOL = 1e-4
 NEAR_TIE = 1e-6
@@ -68,7 +72,8 @@ def compare(w, g: GpuOut, rows=None, report: dict | None = None) -> dict:
     s_at = np.take_along_axis(r.s, gi, axis=1)
     assert np.all(s_at[:, :-1] >= s_at[:, 1:] - NEAR_TIE), "routed order not descending"
     # gates: g = s at the chosen experts, not renormalised
-    np.testing.assert_allclose(g.topk_w, s_at, rtol=GATE_RTOL, atol=1e-7 * np.abs(s_at).max())
+    gate_rtol = GATE_RTOL * max(1.0, w.d / 1024)
+    np.testing.assert_allclose(g.topk_w, s_at, rtol=gate_rtol, atol=1e-7 * np.abs(s_at).max())
 
     # --- counts: the GPU histogram of its own indices, and the oracle's on kept tokens
     own = np.bincount(gi.reshape(-1), minlength=nr)
