@@ -42,6 +42,8 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--config", default="16b_prefill")
+    p.add_argument("--tokens", type=int, default=None,
+                   help="override the token count T of the workload (profiling captures)")
     p.add_argument("--e2e-steps", type=int, default=20)
     p.add_argument("--cpu-seconds", type=float, default=15.0,
                    help="target CPU time of the oracle baseline sample")
@@ -185,7 +187,7 @@ def run_reference(args, rank: int, world: int):
     if rank != 0:
         return
     from mixture_experts_layer_65_b200 import workloads as W
-    w = W.make_workload(args.config)
+    w = W.make_workload(args.config, **({"T": args.tokens} if args.tokens else {}))
     from oracle import moe_oracle as O
     budget = 120.0 / max(1, args.steps + args.warmup)
 
@@ -230,7 +232,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    w = W.make_workload(args.config)
+    w = W.make_workload(args.config, **({"T": args.tokens} if args.tokens else {}))
     layer = MoELayer.from_workload(w, dev)
     es = 2 if w.dtype == "bf16" else 4
     u_bytes = w.T * w.d * es
@@ -286,24 +288,26 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     layer.device_status()
 
     # end to end through the public host-buffer call (pinned host memory)
-    u_host = ubufs[0].cpu().pin_memory()
-    host_out = None
-    for _ in range(2):
-        host_out = layer.forward_host(u_host, host_out)
-    if world > 1:
-        dist.barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.e2e_steps):
-        host_out = layer.forward_host(u_host, host_out)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    layer.device_status()
+    e2e_ms = None
+    if args.e2e_steps > 0:
+        u_host = ubufs[0].cpu().pin_memory()
+        host_out = None
+        for _ in range(2):
+            host_out = layer.forward_host(u_host, host_out)
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            host_out = layer.forward_host(u_host, host_out)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        layer.device_status()
 
     if rank != 0:
         return
@@ -350,9 +354,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "expert_gemm_frac_of_burst_peak": gemm_tflops / peaks["bf16_tflops"],
         "roofline": roofline,
         "kernels": per_kernel,
-        "e2e": {"value": world * w.T * args.e2e_steps / (e2e_ms * 1e-3), "unit": "tokens/s",
-                "h2d_bytes_per_step": u_bytes,
-                "d2h_bytes_per_step": u_bytes + tk * 8 + w.n_routed * 4 + 4},
+        "e2e": None if e2e_ms is None else {
+            "value": world * w.T * args.e2e_steps / (e2e_ms * 1e-3), "unit": "tokens/s",
+            "h2d_bytes_per_step": u_bytes, "d2h_bytes_per_step": u_bytes + tk * 8 + w.n_routed * 4 + 4},
         "gpu_launches": args.steps * (layer.kernels_per_forward + (1 if world > 1 else 0)),
         "clocks": clk,
     }
