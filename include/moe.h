@@ -140,6 +140,45 @@ moe_status moe_balance_loss(const int32_t* counts, const float* psum, int32_t n_
 moe_status moe_timing_begin(moe_handle* handle, int32_t max_forwards);
 moe_status moe_timing_end(moe_handle* handle, double* kernel_ms, int32_t* n_forwards);
 
+/* ---------------------------------------------------------------------------------
+ * Allocation-free router step.  (The DeepSeekMoE pages have no counterpart: this is a
+ * deployment convenience of this library.)
+ *
+ * Some callers cannot call cudaMalloc: code whose GPU memory is owned by another
+ * allocator (a framework's caching allocator or a serving engine's arena that has
+ * reserved the device's memory and forbids allocations behind its back), and code on a
+ * latency-critical path where cudaMalloc/cudaFree would implicitly synchronise the
+ * device.  For them moe_route_noalloc runs the routing part of the layer -- the same
+ * bf16 tcgen05 router and scan kernels moe_forward uses -- without a handle and without
+ * allocating: the kernels' scratch (per-tile expert histograms, within-tile ranks,
+ * per-tile affinity sums, tile tables, an error word) lives in one file-scope device
+ * array of MOE_NOALLOC_SCRATCH_BYTES, which every GPU that loads this library holds
+ * until the process exits.
+ *
+ * Inputs (DEVICE, 16-byte aligned): u [T, d] bf16; centroids [n_routed, d] bf16;
+ * logit_bias [n_routed] fp32 or NULL.  Outputs (DEVICE): topk_idx [T, top_k] int32,
+ * topk_w [T, top_k] fp32, expert_counts [n_routed] int32, aux_loss [1] fp32 -- the same
+ * values moe_forward returns for that layer -- and, if not NULL, device_error [1] int32
+ * (0, or the code a kernel recorded, e.g. a bounded wait that ran out).
+ * Limits: 1 <= T <= MOE_NOALLOC_MAX_TOKENS, 1 <= n_routed <= MOE_NOALLOC_MAX_ROUTED,
+ * 1 <= top_k <= min(MOE_NOALLOC_MAX_TOP_K, n_routed), d a multiple of 64; anything
+ * larger returns MOE_ERR_UNSUPPORTED before touching the GPU.
+ * The first call on a device does a one-time set-up with that device current (it looks
+ * up the array's device address with cudaGetSymbolAddress and reads the compute
+ * capability); make that first call before any stream capture.  No call allocates:
+ * no cudaMalloc/cudaFree and no allocating library routine.
+ * All calls share the one array and each call overwrites it (the error word is cleared
+ * at the start of every call), so calls that overlap on the GPU -- on different streams,
+ * or from several host threads -- race and give wrong results: serialise them. */
+#define MOE_NOALLOC_MAX_TOKENS 16384
+#define MOE_NOALLOC_MAX_ROUTED 256
+#define MOE_NOALLOC_MAX_TOP_K 16
+#define MOE_NOALLOC_SCRATCH_BYTES (1536u * 1024u)
+moe_status moe_route_noalloc(const void* u, const void* centroids, const float* logit_bias,
+                             int32_t T, int32_t d, int32_t n_routed, int32_t top_k, float alpha1,
+                             int32_t* topk_idx, float* topk_w, int32_t* expert_counts,
+                             float* aux_loss, int32_t* device_error, moe_stream_t stream);
+
 /* Number of kernels one moe_forward launches on this handle. */
 int32_t moe_kernels_per_forward(const moe_handle* handle);
 

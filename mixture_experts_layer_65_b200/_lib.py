@@ -45,6 +45,9 @@ _SIGS = {
     "moe_timing_begin": (ctypes.c_int, [_P, ctypes.c_int32]),
     "moe_timing_end": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_double),
                                       ctypes.POINTER(ctypes.c_int32)]),
+    "moe_route_noalloc": (ctypes.c_int, [_P, _P, _P, ctypes.c_int32, ctypes.c_int32,
+                                         ctypes.c_int32, ctypes.c_int32, ctypes.c_float,
+                                         _P, _P, _P, _P, _P, _P]),
     "moe_kernels_per_forward": (ctypes.c_int32, [_P]),
     "moe_device_bytes": (ctypes.c_size_t, [_P]),
     "moe_destroy": (None, [_P]),

@@ -35,7 +35,7 @@ __device__ __forceinline__ void add8(float (&acc)[8], const uint4& v, float w) {
 }
 
 // bf16 rows: 8 elements per 16-byte vector; each lane handles vectors lane, lane+32, ...
-__global__ void __launch_bounds__(kCombineWarps * 32)
+static __global__ void __launch_bounds__(kCombineWarps * 32)
 combine_bf16_kernel(CombineArgs<__nv_bfloat16> a) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * kCombineWarps + warp;
@@ -72,7 +72,7 @@ combine_bf16_kernel(CombineArgs<__nv_bfloat16> a) {
 }
 
 // fp32 rows: 4 elements per 16-byte vector
-__global__ void __launch_bounds__(kCombineWarps * 32) combine_f32_kernel(CombineArgs<float> a) {
+static __global__ void __launch_bounds__(kCombineWarps * 32) combine_f32_kernel(CombineArgs<float> a) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * kCombineWarps + warp;
   if (t >= a.T_) return;

@@ -104,6 +104,10 @@ constexpr int kKernelsPerForward = 6;
 
 }  // namespace
 
+namespace moe {
+void set_last_error(const char* msg) { g_last_error = msg; }
+}  // namespace moe
+
 struct moe_handle {
   moe_cfg cfg;
   int device = 0, n_sms = 0;

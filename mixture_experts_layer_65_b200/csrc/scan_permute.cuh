@@ -35,7 +35,7 @@ struct ScanArgs {
   int32_t* ts2;               // [G + 1] tile prefix of the down GEMM
 };
 
-__global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a) {
+static __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a) {
   __shared__ int32_t s_cnt[kScanThreads];
   __shared__ float s_ps[kScanThreads];
   __shared__ int32_t s_base[kScanThreads];
@@ -141,7 +141,7 @@ struct PermuteArgs {
 constexpr int kPermuteWarps = 8;
 constexpr int kPermuteVec = 8;   // 16-byte vectors held per lane per pass
 
-__global__ void __launch_bounds__(kPermuteWarps * 32) permute_kernel(PermuteArgs a) {
+static __global__ void __launch_bounds__(kPermuteWarps * 32) permute_kernel(PermuteArgs a) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * kPermuteWarps + warp;
   if (t >= a.T) return;
