@@ -1,4 +1,4 @@
-// gemm_tc.cuh -- grouped expert GEMMs on the 5th-generation tensor cores (tcgen05).
+// gemm_tc.cuh -- grouped expert GEMMs on the 5th-generation tensor cores (tcgen05, 2-SM).
 //
 // The expert FFN is SwiGLU, FFN(x) = W_down (SiLU(W_gate x) * (W_up x)) (the GLU-variant
 // FFN cited by the observer.broadside.tech card; the DeepSeekMoE pages only say "FFN").
@@ -12,30 +12,37 @@
 //   mode kGateUpSwiGLU:  Hmid[r, :] = SiLU(X W_gate^T) * (X W_up^T)      (K = d)
 //   mode kDown:          Y[r, :]    = Hmid W_down^T                        (K = I_g)
 //
-// Design (one persistent CTA per SM, 192 threads):
-//   warp 0      one thread issues TMA tile loads (A 128x64, B 256x64 bf16, 128-byte
-//               swizzle) into a 4-stage shared-memory ring;
-//   warp 1      allocates 512 TMEM columns (two 128x256 fp32 accumulators) and one
-//               thread issues tcgen05.mma (M=128, N=256, K=16) per 16-wide K step;
-//   warps 2..5  epilogue: tcgen05.ld the accumulator rows (one TMEM lane = one output
-//               row per thread), apply SiLU(gate)*up in fp32 or convert, store bf16.
-// The accumulators are double-buffered so the epilogue of tile i overlaps the MMAs of
-// tile i+1.  For the gate/up GEMM the weight rows are interleaved in blocks of 64
-// (64 gate rows, then the 64 matching up rows) so one 256-row B tile yields 128 Hmid
-// columns.  Tiles are enumerated group by group (row block major, column block minor)
-// and handed out round-robin over the CTAs.
+// Design: persistent clusters of two CTAs (one per SM); each cluster computes 256 x 256
+// output tiles with the paired-SM MMA (tcgen05.mma.cta_group::2, M = 256, N = 256,
+// K = 16): CTA r of the pair stages rows [128 r, 128 r + 128) of the A tile and rows
+// [128 r, 128 r + 128) of the B tile, so each SM holds half of B and the MMA reads both
+// SMs' shared memory.  192 threads per CTA:
+//   warp 0      one thread issues the TMA loads of this CTA's halves (128 x 64 bf16 each,
+//               128-byte swizzle) into a 6-stage ring; completion is counted on the
+//               leader CTA's "full" barrier (the leader expects both CTAs' bytes);
+//   warp 1      allocates 512 TMEM columns in both CTAs (two 256-column fp32
+//               accumulators); in the leader one thread issues the MMAs and commits with a
+//               multicast arrive to both CTAs' "empty" / "accumulator full" barriers;
+//   warps 2..5  epilogue in both CTAs: tcgen05.ld of the CTA's 128 accumulator rows (one
+//               TMEM lane per output row), SiLU(gate)*up in fp32 or a plain convert, bf16
+//               stores; one arrive per warp on the leader's "accumulator empty" barrier.
+// Gate/up weight rows are interleaved in blocks of 64 (64 gate rows, then the 64 matching
+// up rows), so a 256-row B tile yields 128 Hmid columns.  Tiles are enumerated group by
+// group (row block major, column block minor) and handed out round-robin over clusters.
+// No load uses multicast.
 #pragma once
 
 #include "scan_permute.cuh"
 
 namespace moe {
 
-constexpr int kGemmBN = 256;
+constexpr int kPairBM = 256;                 // output rows per cluster tile (128 per CTA)
+constexpr int kGemmBN = 256;                 // output columns (B rows) per tile
 constexpr int kGemmBK = 64;
-constexpr int kGemmStages = 4;
+constexpr int kGemmStages = 6;
 constexpr int kGemmThreads = 192;
-constexpr uint32_t kGemmABytes = kGemmBM * kGemmBK * 2;
-constexpr uint32_t kGemmBBytes = kGemmBN * kGemmBK * 2;
+constexpr uint32_t kGemmABytes = 128 * kGemmBK * 2;           // this CTA's half of A
+constexpr uint32_t kGemmBBytes = (kGemmBN / 2) * kGemmBK * 2; // this CTA's half of B
 constexpr uint32_t kGemmStageBytes = kGemmABytes + kGemmBBytes;
 constexpr uint32_t kGemmTmemCols = 512;
 constexpr size_t kGemmSmemBytes = 1024 + (size_t)kGemmStages * kGemmStageBytes + 256;
@@ -44,7 +51,7 @@ enum GemmMode : int { kGateUpSwiGLU = 0, kDown = 1 };
 
 struct GemmArgs {
   const int32_t* grp_row;   // [G] first row of the group in A (and in the output)
-  const int32_t* ts;        // [G + 1] tile prefix
+  const int32_t* ts;        // [G + 1] tile prefix (256-row tiles)
   int G, has_shared;
   int kb_shared, kb_routed; // K / 64 of the shared group and of a routed group
   int nt_shared, nt_routed; // column tiles per group
@@ -74,7 +81,7 @@ __device__ __forceinline__ void gemm_decode(int tile, int& g, const GemmArgs& a,
 }
 
 template <int MODE>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
                        const __grid_constant__ CUtensorMap tmA_r,
                        const __grid_constant__ CUtensorMap tmB_s,
@@ -83,15 +90,18 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* ctl = base + (size_t)kGemmStages * kGemmStageBytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(ctl);
-  uint64_t* empty = full + kGemmStages;
-  uint64_t* acc_full = empty + kGemmStages;
-  uint64_t* acc_empty = acc_full + 2;
-  uint64_t* drain = acc_empty + 2;
+  uint64_t* full = reinterpret_cast<uint64_t*>(ctl);   // used in the leader
+  uint64_t* empty = full + kGemmStages;                 // both CTAs
+  uint64_t* acc_full = empty + kGemmStages;             // both CTAs
+  uint64_t* acc_empty = acc_full + 2;                   // used in the leader
+  uint64_t* drain = acc_empty + 2;                      // both CTAs
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();            // 0 = leader, 1 = peer
+  const bool leader = rank == 0;
+  const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
   const int total = __ldg(&a.ts[a.G]);
 
   if (threadIdx.x == 0) {
@@ -101,7 +111,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&acc_full[s]), 1);
-      mbar_init(smem_u32(&acc_empty[s]), 128);
+      mbar_init(smem_u32(&acc_empty[s]), 8);   // 4 epilogue warps x 2 CTAs
     }
     mbar_init(smem_u32(drain), 1);
     *abort_flag = 0;
@@ -112,11 +122,11 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
     tma_prefetch_desc(&tmB_r);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), kGemmTmemCols);
-    tmem_relinquish();
+    tmem_alloc_pair(smem_u32(tmem_slot), kGemmTmemCols);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();   // barriers of both CTAs initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -124,41 +134,44 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int stage = 0, g = 0;
-      uint32_t phase = 0, issued = 0, last_par = 0;
+      uint32_t phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      for (int tile = cid; tile < total && ok; tile += ncl) {
         TileCoord c;
         gemm_decode(tile, g, a, c);
         const CUtensorMap* ta = c.shared ? &tmA_s : &tmA_r;
-        const int arow = __ldg(&a.grp_row[c.g]) + c.m * kGemmBM;
-        const int brow = c.n * kGemmBN;
+        const int arow = __ldg(&a.grp_row[c.g]) + c.m * kPairBM + (int)rank * 128;
+        const int brow = c.n * kGemmBN + (int)rank * (kGemmBN / 2);
         const int kbn = c.shared ? a.kb_shared : a.kb_routed;
         for (int kb = 0; kb < kbn; ++kb) {
           ok = mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, a.err, kErrWaitProducer);
           if (!ok) break;
           const uint32_t sa = smem_u32(base + (size_t)stage * kGemmStageBytes);
-          const uint32_t fb = smem_u32(&full[stage]);
-          mbar_arrive_expect_tx(fb, kGemmStageBytes);
-          tma_load_2d(sa, ta, fb, kb * kGemmBK, arow);
-          if (c.shared) tma_load_2d(sa + kGemmABytes, &tmB_s, fb, kb * kGemmBK, brow);
-          else tma_load_3d(sa + kGemmABytes, &tmB_r, fb, kb * kGemmBK, brow, c.e);
-          issued |= 1u << stage;
-          last_par = (last_par & ~(1u << stage)) | (phase << stage);
+          const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
+          if (leader) mbar_arrive_expect_tx(smem_u32(&full[stage]), 2 * kGemmStageBytes);
+          tma_load_2d_pair(sa, ta, fb, kb * kGemmBK, arow);
+          if (c.shared) tma_load_2d_pair(sa + kGemmABytes, &tmB_s, fb, kb * kGemmBK, brow);
+          else tma_load_3d_pair(sa + kGemmABytes, &tmB_r, fb, kb * kGemmBK, brow, c.e);
           if (++stage == kGemmStages) { stage = 0; phase ^= 1u; }
         }
       }
-      for (int s = 0; s < kGemmStages; ++s)
-        if (issued & (1u << s))
-          mbar_wait(smem_u32(&full[s]), (last_par >> s) & 1u, abort_flag, a.err, kErrWaitDrain);
+      // every copy this CTA started has landed once its stage came back empty: wait for
+      // the MMAs to release all stages (bounded), so no copy is in flight at exit
+      if (ok) {
+        for (int s = 0; s < kGemmStages; ++s) {
+          if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, a.err, kErrWaitDrain)) break;
+          if (++stage == kGemmStages) { stage = 0; phase ^= 1u; }
+        }
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(kGemmBM, kGemmBN);
+    if (lane == 0 && leader) {
+      const uint32_t idesc = idesc_bf16_f32(kPairBM, kGemmBN);
       int stage = 0, g = 0, it = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++it) {
+      for (int tile = cid; tile < total && ok; tile += ncl, ++it) {
         TileCoord c;
         gemm_decode(tile, g, a, c);
         const int kbn = c.shared ? a.kb_shared : a.kb_routed;
@@ -177,14 +190,13 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
           const uint64_t bdesc = sdesc_k_sw128(sa + kGemmABytes);
 #pragma unroll
           for (int k = 0; k < kGemmBK / 16; ++k)
-            tc_mma_f16(dt, adesc + 2u * k, bdesc + 2u * k, idesc, (kb | k) != 0);
-          tc_commit(smem_u32(&empty[stage]));
+            tc_mma_f16_pair(dt, adesc + 2u * k, bdesc + 2u * k, idesc, (kb | k) != 0);
+          tc_commit_pair_mc(smem_u32(&empty[stage]), 0x3);
           if (++stage == kGemmStages) { stage = 0; phase ^= 1u; }
         }
-        if (ok) tc_commit(smem_u32(&acc_full[acc]));
+        if (ok) tc_commit_pair_mc(smem_u32(&acc_full[acc]), 0x3);
       }
-      tc_commit(smem_u32(drain));
-      mbar_wait(smem_u32(drain), 0, abort_flag, a.err, kErrWaitDrain);
+      tc_commit_pair_mc(smem_u32(drain), 0x3);
     }
     __syncwarp();
   } else {
@@ -192,7 +204,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
     const int q = warp & 3;
     const int rr = q * 32 + lane;
     int g = 0, it = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+    for (int tile = cid; tile < total; tile += ncl, ++it) {
       TileCoord c;
       gemm_decode(tile, g, a, c);
       const int acc = it & 1;
@@ -203,7 +215,8 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
       tc_fence_after();
       const uint32_t trow =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * kGemmBN);
-      const int64_t orow = (int64_t)__ldg(&a.grp_row[c.g]) + (int64_t)c.m * kGemmBM + rr;
+      const int64_t orow = (int64_t)__ldg(&a.grp_row[c.g]) + (int64_t)c.m * kPairBM +
+                           (int64_t)rank * 128 + rr;
       __nv_bfloat16* out = c.shared ? a.out_shared : a.out_routed;
       const int64_t ld = c.shared ? a.ld_shared : a.ld_routed;
       const int64_t rows = c.shared ? a.rows_shared : a.rows_routed;
@@ -261,15 +274,20 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
         }
       }
       tc_fence_before();
-      mbar_arrive(smem_u32(&acc_empty[acc]));
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty[acc]), 0));
     }
   }
 
+  // teardown: all MMAs of the pair have completed before TMEM is released in either CTA
+  if (warp == 1 && lane == 0)
+    mbar_wait(smem_u32(drain), 0, abort_flag, a.err, kErrWaitDrain);
+  __syncwarp();
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, kGemmTmemCols);
+    tmem_dealloc_pair(tmem_base, kGemmTmemCols);
   }
 }
 

@@ -115,7 +115,9 @@ struct moe_handle {
   int es = 2;              // element size
   int G = 0, has_shared = 0, inter_shared = 0;
   int n_tiles = 0;         // router tiles of 128 tokens
-  int64_t T_pad = 0, rows_cap = 0;
+  int64_t T_pad = 0, rows_cap = 0;   // padded to bm, the GEMM row tile
+  int bm = 0;
+  int gemm_grid = 0;                  // CTAs of the paired-SM GEMMs (2 per cluster)
   int n_pad = 0, maxk = 16;
   int router_stages = 0;
   uint32_t router_tmem_cols = 0;
@@ -205,7 +207,7 @@ moe_status validate(const moe_cfg* c) {
       return fail(MOE_ERR_UNSUPPORTED, "fp32 layers need d %% 4 == 0 and inter %% 4 == 0 (d=%d inter=%d)",
                   c->d, c->inter);
   }
-  const int64_t rows_cap = (int64_t)c->T * c->top_k + (int64_t)c->n_routed * (kGemmBM - 1);
+  const int64_t rows_cap = (int64_t)c->T * c->top_k + (int64_t)c->n_routed * (kPairBM - 1);
   if (rows_cap >= (int64_t(1) << 30)) return fail(MOE_ERR_UNSUPPORTED, "T * top_k too large");
   return MOE_OK;
 }
@@ -244,9 +246,10 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
   H->inter_shared = c.n_shared * c.inter;
   H->G = H->has_shared + c.n_routed;
   H->n_tiles = (c.T + kRouterBM - 1) / kRouterBM;
-  H->T_pad = (int64_t)H->n_tiles * kRouterBM;
-  H->rows_cap = ((int64_t)c.T * c.top_k + (int64_t)c.n_routed * (kGemmBM - 1) + kGemmBM - 1) /
-                kGemmBM * kGemmBM;
+  H->bm = H->bf16 ? kPairBM : kSimtBM;
+  H->T_pad = ((int64_t)c.T + H->bm - 1) / H->bm * H->bm;
+  H->rows_cap = ((int64_t)c.T * c.top_k + (int64_t)c.n_routed * (H->bm - 1) + H->bm - 1) /
+                H->bm * H->bm;
   H->n_pad = (c.n_routed + 15) / 16 * 16;
   H->maxk = pick_maxk(c.top_k);
   const size_t es = H->es;
@@ -340,7 +343,7 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
     if (stages < 2) stages = 2;
     H->router_stages = stages;
     H->router_smem = 1024 + (size_t)stages * stage_bytes + 256;
-    if ((size_t)stages * stage_bytes < sizeof(RouterEpiSmem))
+    if ((size_t)stages * stage_bytes < router_epi_bytes(c.n_routed))
       return fail(MOE_ERR_UNSUPPORTED, "router epilogue scratch does not fit");
     uint32_t cols = 32;
     while (cols < (uint32_t)H->n_pad) cols <<= 1;
@@ -353,15 +356,34 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmemBytes));
     MOE_CUDA(cudaFuncSetAttribute((const void*)grouped_gemm_tc_kernel<kDown>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmemBytes));
+    // persistent grid: as many CTA pairs as can be resident at once
+    {
+      cudaLaunchConfig_t lc = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      lc.gridDim = dim3(2 * (H->n_sms / 2), 1, 1);
+      lc.blockDim = dim3(kGemmThreads, 1, 1);
+      lc.dynamicSmemBytes = kGemmSmemBytes;
+      lc.attrs = attr;
+      lc.numAttrs = 1;
+      int clusters = 0;
+      MOE_CUDA(cudaOccupancyMaxActiveClusters(
+          &clusters, (const void*)grouped_gemm_tc_kernel<kGateUpSwiGLU>, &lc));
+      if (clusters < 1) return fail(MOE_ERR_UNSUPPORTED, "no CTA pair of the GEMM kernel fits on this device");
+      H->gemm_grid = 2 * clusters;
+    }
     bool ok = encode_2d(&H->tmE, H->centroids, d, (uint64_t)H->n_pad, (uint32_t)H->n_pad) &&
-              encode_2d(&H->tmXp, H->xp, d, rc, kGemmBM) &&
-              encode_3d(&H->tmWguR, H->w_gu_r, d, 2 * I, nr, kGemmBN) &&
-              encode_2d(&H->tmHr, H->hr, I, rc, kGemmBM) &&
-              encode_3d(&H->tmWdR, H->w_d_r, I, d, nr, kGemmBN);
+              encode_2d(&H->tmXp, H->xp, d, rc, 128) &&
+              encode_3d(&H->tmWguR, H->w_gu_r, d, 2 * I, nr, kGemmBN / 2) &&
+              encode_2d(&H->tmHr, H->hr, I, rc, 128) &&
+              encode_3d(&H->tmWdR, H->w_d_r, I, d, nr, kGemmBN / 2);
     if (ks)
-      ok = ok && encode_2d(&H->tmWguS, H->w_gu_s, d, 2 * Is, kGemmBN) &&
-           encode_2d(&H->tmHs, H->hs, Is, tp, kGemmBM) &&
-           encode_2d(&H->tmWdS, H->w_d_s, Is, d, kGemmBN);
+      ok = ok && encode_2d(&H->tmWguS, H->w_gu_s, d, 2 * Is, kGemmBN / 2) &&
+           encode_2d(&H->tmHs, H->hs, Is, tp, 128) &&
+           encode_2d(&H->tmWdS, H->w_d_s, Is, d, kGemmBN / 2);
     else {
       H->tmWguS = H->tmWguR;
       H->tmHs = H->tmHr;
@@ -369,7 +391,7 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
     }
     if (!ok) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for a weight/workspace tensor");
   } else {
-    H->simt_router_smem = sizeof(RouterEpiSmem) + (size_t)kRouterBM * (nr + 1) * 4;
+    H->simt_router_smem = router_epi_bytes(c.n_routed);
     const void* rk = H->maxk == 4 ? (const void*)router_simt_kernel<4>
                    : H->maxk == 8 ? (const void*)router_simt_kernel<8>
                                   : (const void*)router_simt_kernel<16>;
@@ -443,7 +465,7 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
   const int bn1 = H->bf16 ? kGemmBN / 2 : kSimtBN;
   const int bn2 = H->bf16 ? kGemmBN : kSimtBN;
   ScanArgs sa{H->tile_hist, H->tile_psum, H->n_tiles, nr, T, H->has_shared, H->inter_shared,
-              c.inter, d, bn1, bn2, c.alpha1, expert_counts, aux_loss, H->psum_total,
+              c.inter, d, H->bm, bn1, bn2, c.alpha1, expert_counts, aux_loss, H->psum_total,
               H->tile_base, H->grp_row, H->ts1, H->ts2};
   tick(H, stream, 1);
   scan_kernel<<<1, kScanThreads, 0, stream>>>(sa);
@@ -467,7 +489,7 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
     g1.cols_routed = I;
     g1.err = H->err;
     tick(H, stream, 3);
-    grouped_gemm_tc_kernel<kGateUpSwiGLU><<<H->n_sms, kGemmThreads, kGemmSmemBytes, stream>>>(
+    grouped_gemm_tc_kernel<kGateUpSwiGLU><<<H->gemm_grid, kGemmThreads, kGemmSmemBytes, stream>>>(
         tmU, H->tmXp, H->tmWguS, H->tmWguR, g1);
     MOE_CUDA(cudaGetLastError());
 
@@ -481,7 +503,7 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
     g2.cols_routed = d;
     g2.err = H->err;
     tick(H, stream, 4);
-    grouped_gemm_tc_kernel<kDown><<<H->n_sms, kGemmThreads, kGemmSmemBytes, stream>>>(
+    grouped_gemm_tc_kernel<kDown><<<H->gemm_grid, kGemmThreads, kGemmSmemBytes, stream>>>(
         H->tmHs, H->tmHr, H->tmWdS, H->tmWdR, g2);
     MOE_CUDA(cudaGetLastError());
 

@@ -36,34 +36,51 @@ struct RouterOut {
 };
 
 struct RouterEpiSmem {
-  float sbuf[kRouterBM][33];
-  float part[4][32];
   uint32_t mask[kMaxRouted][4];   // bit r of mask[e][r/32]: token r of the tile chose e
+  float bias[kMaxRouted];
+  float inv_sum[kRouterBM];       // 1 / softmax denominator per row (0 for rows past T)
 };
 
+// Epilogue scratch: RouterEpiSmem followed by a [128][ld] fp32 row buffer.
+__host__ __device__ constexpr int router_row_ld(int n_routed) { return ((n_routed + 31) & ~31) + 1; }
+__host__ __device__ constexpr size_t router_epi_bytes(int n_routed) {
+  return sizeof(RouterEpiSmem) + (size_t)kRouterBM * router_row_ld(n_routed) * 4;
+}
+
+// Total order on (logit, expert): larger logit first; on equal logits the lower index.
+// NaN ranks as -inf and -0 as +0, so every slot gets a real index and equal values tie.
+__device__ __forceinline__ uint64_t route_key(float l, int i) {
+  uint32_t b = (l != l) ? 0xFF800000u : __float_as_uint(l);
+  if (b == 0x80000000u) b = 0u;
+  const uint32_t ord = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+  return (static_cast<uint64_t>(ord) << 32) | static_cast<uint64_t>(0xFFFFFFFFu - (uint32_t)i);
+}
+
 // One epilogue thread = one token row r (0..127) of tile `tile`.  `load(c, v)` yields the
-// 32 raw fp32 logits (bit patterns) of columns c..c+31 of this row; it is called
-// uniformly by all 128 threads.  `sync()` synchronises the 128 epilogue threads.
+// 32 raw fp32 logits (bit patterns) of columns c..c+31 of this row and is called uniformly
+// by all 128 threads; `sync()` synchronises the 128 epilogue threads.  `rows` is a
+// [128][ld] fp32 buffer (it may hold the logits on entry; load() reads a chunk before
+// this function overwrites it).
 template <int MAXK, class Load, class Sync>
 __device__ __forceinline__ void router_epilogue(int r, int tile, int T, int n_routed, int n_cols,
                                                 int top_k, const float* __restrict__ bias,
-                                                RouterEpiSmem& S, const RouterOut& o, Load load,
-                                                Sync sync) {
+                                                RouterEpiSmem& S, float* rows, const RouterOut& o,
+                                                Load load, Sync sync) {
   const int t = tile * kRouterBM + r;
   const bool valid = t < T;
-
+  const int ld = router_row_ld(n_routed);
+  float* my = rows + (size_t)r * ld;
   for (int e = r; e < kMaxRouted; e += kRouterBM) {
     S.mask[e][0] = 0u; S.mask[e][1] = 0u; S.mask[e][2] = 0u; S.mask[e][3] = 0u;
+    S.bias[e] = e < n_routed ? bias[e] : 0.f;
   }
+  sync();
 
-  // pass 1: running max and top-k (sorted descending; equal keys keep the earlier,
-  // lower index ahead).  NaN logits rank as -inf so every slot gets a real index.
-  float topv[MAXK];
-  int topi[MAXK];
+  // pass 1: row max and the MAXK largest (logit, index) keys, kept sorted descending by a
+  // compare-exchange chain in registers
+  uint64_t top[MAXK];
 #pragma unroll
-  for (int p = 0; p < MAXK; ++p) { topv[p] = -INFINITY; topi[p] = INT_MAX; }
-  float kth = -INFINITY;
-  bool kth_empty = true;
+  for (int p = 0; p < MAXK; ++p) top[p] = 0ull;
   float lmax = -INFINITY;
   uint32_t v[32];
   for (int c = 0; c < n_cols; c += 32) {
@@ -72,103 +89,85 @@ __device__ __forceinline__ void router_epilogue(int r, int tile, int T, int n_ro
     for (int j = 0; j < 32; ++j) {
       const int i = c + j;
       if (i < n_routed) {
-        const float l = __uint_as_float(v[j]) + bias[i];
+        const float l = __uint_as_float(v[j]) + S.bias[i];
         lmax = fmaxf(lmax, l);
-        const float key = (l != l) ? -INFINITY : l;
-        if (kth_empty || key > kth) {
-          float cv = key;
-          int ci = i;
-          bool moved = false;
+        uint64_t key = route_key(l, i);
+        if (key > top[MAXK - 1]) {
 #pragma unroll
           for (int p = 0; p < MAXK; ++p) {
-            if (p < top_k) {
-              const bool take = moved || topi[p] == INT_MAX || cv > topv[p];
-              if (take) {
-                const float tv = topv[p];
-                const int ti = topi[p];
-                topv[p] = cv; topi[p] = ci;
-                cv = tv; ci = ti;
-                moved = true;
-              }
-              if (p == top_k - 1) { kth = topv[p]; kth_empty = topi[p] == INT_MAX; }
-            }
+            const uint64_t hi = top[p] > key ? top[p] : key;
+            key = top[p] > key ? key : top[p];
+            top[p] = hi;
           }
         }
       }
     }
   }
 
-  // pass 2: softmax denominator, ascending expert order
+  // pass 2: exp(l - max) per expert into the row buffer, denominator in ascending order
   float sum = 0.f;
   for (int c = 0; c < n_cols; c += 32) {
     load(c, v);
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
       const int i = c + j;
-      if (i < n_routed) sum += expf(__uint_as_float(v[j]) + bias[i] - lmax);
+      if (i < n_routed) {
+        const float e = __expf(__uint_as_float(v[j]) + S.bias[i] - lmax);
+        sum += e;
+        my[i] = e;
+      }
     }
   }
   const float inv_sum = 1.0f / sum;
+  S.inv_sum[r] = valid ? inv_sum : 0.f;
 
-  // pass 3: affinities s and the tile's per-expert sums (fixed reduction order)
-  for (int c = 0; c < n_cols; c += 32) {
-    load(c, v);
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const int i = c + j;
-      S.sbuf[r][j] = (valid && i < n_routed)
-                         ? expf(__uint_as_float(v[j]) + bias[i] - lmax) * inv_sum : 0.f;
-    }
-    sync();
-    {
-      const int j = r & 31, q = r >> 5;
-      float a = 0.f;
-#pragma unroll 8
-      for (int rr = 0; rr < 32; ++rr) a += S.sbuf[q * 32 + rr][j];
-      S.part[q][j] = a;
-    }
-    sync();
-    if (r < 32 && c + r < n_routed)
-      o.tile_psum[(size_t)tile * n_routed + c + r] =
-          ((S.part[0][r] + S.part[1][r]) + S.part[2][r]) + S.part[3][r];
-  }
-
-  // counts and within-tile ranks from per-expert token bitmasks
+  // gates g = s at the selected experts, and the expert bitmasks of this tile
   if (valid) {
 #pragma unroll
     for (int p = 0; p < MAXK; ++p) {
       if (p < top_k) {
-        const int e = topi[p];
+        const int e = (int)(0xFFFFFFFFu - (uint32_t)top[p]);
         if (e >= 0 && e < n_routed) atomicOr(&S.mask[e][r >> 5], 1u << (r & 31));
       }
     }
   }
   sync();
+
+  // the tile's per-expert affinity sums: one column per thread, rows in order
+  for (int c = r; c < n_routed; c += kRouterBM) {
+    float a = 0.f;
+#pragma unroll 8
+    for (int rr = 0; rr < kRouterBM; ++rr) a += rows[(size_t)rr * ld + c] * S.inv_sum[rr];
+    o.tile_psum[(size_t)tile * n_routed + c] = a;
+    o.tile_hist[(size_t)tile * n_routed + c] =
+        __popc(S.mask[c][0]) + __popc(S.mask[c][1]) + __popc(S.mask[c][2]) + __popc(S.mask[c][3]);
+  }
+
+  // outputs and within-tile ranks (tokens of the tile that chose e before this one)
   if (valid) {
     const int q = r >> 5;
     const uint32_t below = (1u << (r & 31)) - 1u;
 #pragma unroll
     for (int p = 0; p < MAXK; ++p) {
       if (p < top_k) {
-        int e = topi[p];
+        int e = (int)(0xFFFFFFFFu - (uint32_t)top[p]);
         int rank = 0;
+        float g = 0.f;
         if (e >= 0 && e < n_routed) {
           for (int qq = 0; qq < q; ++qq) rank += __popc(S.mask[e][qq]);
           rank += __popc(S.mask[e][q] & below);
+          g = my[e] * inv_sum;
         } else {
           record_error(o.err, kErrRouteIndex);
           e = 0;
         }
         const size_t at = (size_t)t * top_k + p;
         o.topk_idx[at] = e;
-        o.topk_w[at] = expf(topv[p] - lmax) * inv_sum;
+        o.topk_w[at] = g;
         o.topk_rank[at] = rank;
       }
     }
   }
-  for (int e = r; e < n_routed; e += kRouterBM)
-    o.tile_hist[(size_t)tile * n_routed + e] =
-        __popc(S.mask[e][0]) + __popc(S.mask[e][1]) + __popc(S.mask[e][2]) + __popc(S.mask[e][3]);
 }
 
 // ------------------------------------------------------------------------ bf16, tcgen05
@@ -271,6 +270,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant_
     if (!named_bar_any(1, 128, !ok)) {
       tc_fence_after();
       RouterEpiSmem& E = *reinterpret_cast<RouterEpiSmem*>(base);
+      float* rows = reinterpret_cast<float*>(base + sizeof(RouterEpiSmem));
       const uint32_t trow = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
       auto load = [&](int c, uint32_t (&v)[32]) {
         __syncwarp();
@@ -278,7 +278,8 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant_
         tmem_ld_wait(v);
       };
       auto sync = [] { named_bar_sync(1, 128); };
-      router_epilogue<MAXK>(r, tile, a.T, a.n_routed, a.n_pad, a.top_k, a.bias, E, a.out, load, sync);
+      router_epilogue<MAXK>(r, tile, a.T, a.n_routed, a.n_pad, a.top_k, a.bias, E, rows, a.out,
+                            load, sync);
     }
   }
 
@@ -299,38 +300,37 @@ struct RouterSimtArgs {
   RouterOut out;
 };
 
-// dynamic smem: RouterEpiSmem + logits [128][n_routed + 1]
+// dynamic smem: router_epi_bytes(n_routed) (the row buffer first holds the logits)
 template <int MAXK>
 __global__ void __launch_bounds__(kRouterBM) router_simt_kernel(RouterSimtArgs a) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   RouterEpiSmem& E = *reinterpret_cast<RouterEpiSmem*>(smem_raw);
-  float* slog = reinterpret_cast<float*>(smem_raw + sizeof(RouterEpiSmem));
-  const int ld = a.n_routed + 1;
+  float* rows = reinterpret_cast<float*>(smem_raw + sizeof(RouterEpiSmem));
+  const int ld = router_row_ld(a.n_routed);
   const int r = threadIdx.x;
   const int tile = blockIdx.x;
   const int t = tile * kRouterBM + r;
-  if (t < a.T) {
-    const float4* ur = reinterpret_cast<const float4*>(a.u + (size_t)t * a.d);
-    for (int i = 0; i < a.n_routed; ++i) {
+  for (int i = 0; i < a.n_routed; ++i) {
+    float acc = 0.f;
+    if (t < a.T) {
+      const float4* ur = reinterpret_cast<const float4*>(a.u + (size_t)t * a.d);
       const float4* er = reinterpret_cast<const float4*>(a.cen + (size_t)i * a.d);
-      float acc = 0.f;
       for (int k = 0; k < a.d / 4; ++k) {
         const float4 x = ur[k], y = __ldg(&er[k]);
         acc = fmaf(x.x, y.x, acc); acc = fmaf(x.y, y.y, acc);
         acc = fmaf(x.z, y.z, acc); acc = fmaf(x.w, y.w, acc);
       }
-      slog[r * ld + i] = acc;
     }
+    rows[(size_t)r * ld + i] = acc;
   }
-  __syncthreads();
   const int n_cols = (a.n_routed + 31) & ~31;
   auto load = [&](int c, uint32_t (&v)[32]) {
 #pragma unroll
     for (int j = 0; j < 32; ++j)
-      v[j] = (c + j < a.n_routed) ? __float_as_uint(slog[r * ld + c + j]) : 0u;
+      v[j] = (c + j < a.n_routed) ? __float_as_uint(rows[(size_t)r * ld + c + j]) : 0u;
   };
   auto sync = [] { __syncthreads(); };
-  router_epilogue<MAXK>(r, tile, a.T, a.n_routed, n_cols, a.top_k, a.bias, E, a.out, load, sync);
+  router_epilogue<MAXK>(r, tile, a.T, a.n_routed, n_cols, a.top_k, a.bias, E, rows, a.out, load, sync);
 }
 
 }  // namespace moe

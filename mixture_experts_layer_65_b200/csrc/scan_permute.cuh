@@ -14,7 +14,6 @@
 
 namespace moe {
 
-constexpr int kGemmBM = 128;   // grouped-GEMM M tile: expert row blocks are padded to it
 constexpr int kScanThreads = 1024;
 
 struct ScanArgs {
@@ -23,6 +22,7 @@ struct ScanArgs {
   int n_tiles, n_routed, T;
   int has_shared;             // group 0 = all shared experts as one group
   int inter_shared, inter, d; // widths of the shared group and of a routed expert
+  int bm;                     // GEMM row tile: each group's rows are padded to it
   int bn1, bn2;               // output columns per tile of the gate/up and down GEMMs
   float alpha1;
   // outputs
@@ -88,7 +88,7 @@ static __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a
     a.ts2[0] = 0;
     int g = 0;
     if (a.has_shared) {
-      const int mt = (a.T + kGemmBM - 1) / kGemmBM;
+      const int mt = (a.T + a.bm - 1) / a.bm;
       const int nt1 = (a.inter_shared + a.bn1 - 1) / a.bn1;
       a.grp_row[0] = 0;
       acc1 += mt * nt1;
@@ -100,10 +100,10 @@ static __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a
     const int nt1 = (a.inter + a.bn1 - 1) / a.bn1;
     for (int i = 0; i < nr; ++i, ++g) {
       const int cnt = s_off[i];
-      const int mt = (cnt + kGemmBM - 1) / kGemmBM;
+      const int mt = (cnt + a.bm - 1) / a.bm;
       s_off[i] = off;
       a.grp_row[g] = off;
-      off += mt * kGemmBM;
+      off += mt * a.bm;
       acc1 += mt * nt1;
       acc2 += mt * nt2;
       a.ts1[g + 1] = acc1;
