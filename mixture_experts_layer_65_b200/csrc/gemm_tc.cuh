@@ -16,16 +16,17 @@
 // output tiles with the paired-SM MMA (tcgen05.mma.cta_group::2, M = 256, N = 256,
 // K = 16): CTA r of the pair stages rows [128 r, 128 r + 128) of the A tile and rows
 // [128 r, 128 r + 128) of the B tile, so each SM holds half of B and the MMA reads both
-// SMs' shared memory.  192 threads per CTA:
+// SMs' shared memory.  320 threads per CTA:
 //   warp 0      one thread issues the TMA loads of this CTA's halves (128 x 64 bf16 each,
 //               128-byte swizzle) into a 6-stage ring; completion is counted on the
 //               leader CTA's "full" barrier (the leader expects both CTAs' bytes);
 //   warp 1      allocates 512 TMEM columns in both CTAs (two 256-column fp32
 //               accumulators); in the leader one thread issues the MMAs and commits with a
 //               multicast arrive to both CTAs' "empty" / "accumulator full" barriers;
-//   warps 2..5  epilogue in both CTAs: tcgen05.ld of the CTA's 128 accumulator rows (one
-//               TMEM lane per output row), SiLU(gate)*up in fp32 or a plain convert, bf16
-//               stores; one arrive per warp on the leader's "accumulator empty" barrier.
+//   warps 2..9  epilogue in both CTAs: tcgen05.ld of the CTA's 128 accumulator rows (one
+//               TMEM lane per output row; two warps per lane quadrant, each taking half of
+//               the columns), SiLU(gate)*up in fp32 or a plain convert, bf16 stores; one
+//               arrive per warp on the leader's "accumulator empty" barrier.
 // Gate/up weight rows are interleaved in blocks of 64 (64 gate rows, then the 64 matching
 // up rows), so a 256-row B tile yields 128 Hmid columns.  Tiles are enumerated group by
 // group (row block major, column block minor) and handed out round-robin over clusters.
@@ -40,7 +41,8 @@ constexpr int kPairBM = 256;                 // output rows per cluster tile (12
 constexpr int kGemmBN = 256;                 // output columns (B rows) per tile
 constexpr int kGemmBK = 64;
 constexpr int kGemmStages = 6;
-constexpr int kGemmThreads = 192;
+constexpr int kGemmEpiWarps = 8;             // two warps per TMEM lane quadrant
+constexpr int kGemmThreads = 64 + 32 * kGemmEpiWarps;
 constexpr uint32_t kGemmABytes = 128 * kGemmBK * 2;           // this CTA's half of A
 constexpr uint32_t kGemmBBytes = (kGemmBN / 2) * kGemmBK * 2; // this CTA's half of B
 constexpr uint32_t kGemmStageBytes = kGemmABytes + kGemmBBytes;
@@ -111,7 +113,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&acc_full[s]), 1);
-      mbar_init(smem_u32(&acc_empty[s]), 8);   // 4 epilogue warps x 2 CTAs
+      mbar_init(smem_u32(&acc_empty[s]), 2 * kGemmEpiWarps);   // epilogue warps of both CTAs
     }
     mbar_init(smem_u32(drain), 1);
     *abort_flag = 0;
@@ -201,7 +203,8 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
     __syncwarp();
   } else {
     // ------------------------------------------------------------------ epilogue
-    const int q = warp & 3;
+    const int q = warp & 3;                 // TMEM lane quadrant this warp may access
+    const int half = (warp - 2) >> 2;       // which half of the tile's columns
     const int rr = q * 32 + lane;
     int g = 0, it = 0;
     for (int tile = cid; tile < total; tile += ncl, ++it) {
@@ -224,12 +227,11 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
       const bool row_ok = orow < rows;
       if (!row_ok) record_error(a.err, kErrOutRow);
       if (MODE == kGateUpSwiGLU) {
-#pragma unroll 1
-        for (int hb = 0; hb < 2; ++hb) {
+        {
+          const int hb = half;
           const int col0 = c.n * (kGemmBN / 2) + hb * 64;
-          if (col0 >= cols) break;
 #pragma unroll 1
-          for (int j = 0; j < 64; j += 32) {
+          for (int j = 0; j < 64 && col0 < cols; j += 32) {
             uint32_t gv[32], uv[32];
             __syncwarp();
             tmem_ld32(trow + static_cast<uint32_t>(hb * 128 + j), gv);
@@ -239,9 +241,9 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
             uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              const float h0 = silu_f32(__uint_as_float(gv[2 * i])) * __uint_as_float(uv[2 * i]);
+              const float h0 = silu_fast(__uint_as_float(gv[2 * i])) * __uint_as_float(uv[2 * i]);
               const float h1 =
-                  silu_f32(__uint_as_float(gv[2 * i + 1])) * __uint_as_float(uv[2 * i + 1]);
+                  silu_fast(__uint_as_float(gv[2 * i + 1])) * __uint_as_float(uv[2 * i + 1]);
               pk[i] = pack_bf16x2(h0, h1);
             }
             if (row_ok) {
@@ -254,7 +256,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
         }
       } else {
 #pragma unroll 1
-        for (int cc = 0; cc < kGemmBN; cc += 32) {
+        for (int cc = half * (kGemmBN / 2); cc < (half + 1) * (kGemmBN / 2); cc += 32) {
           const int col = c.n * kGemmBN + cc;
           if (col >= cols) break;
           uint32_t v[32];

@@ -114,7 +114,8 @@ struct moe_handle {
   bool bf16 = true;
   int es = 2;              // element size
   int G = 0, has_shared = 0, inter_shared = 0;
-  int n_tiles = 0;         // router tiles of 128 tokens
+  int n_tiles = 0;         // router tiles
+  int router_rows = 0;     // tokens per router tile
   int64_t T_pad = 0, rows_cap = 0;   // padded to bm, the GEMM row tile
   int bm = 0;
   int gemm_grid = 0;                  // CTAs of the paired-SM GEMMs (2 per cluster)
@@ -180,8 +181,6 @@ void free_handle(moe_handle* H) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int pick_maxk(int k) { return k <= 4 ? 4 : (k <= 8 ? 8 : 16); }
-
 moe_status validate(const moe_cfg* c) {
   if (!c) return fail(MOE_ERR_INVALID_ARG, "cfg is NULL");
   if (c->T < 1 || c->T > (1 << 24)) return fail(MOE_ERR_INVALID_ARG, "T=%d outside [1, 2^24]", c->T);
@@ -203,6 +202,8 @@ moe_status validate(const moe_cfg* c) {
       return fail(MOE_ERR_UNSUPPORTED, "bf16 layers need d %% 64 == 0 and inter %% 64 == 0 (d=%d inter=%d)",
                   c->d, c->inter);
   } else {
+    if (c->n_routed > 128)
+      return fail(MOE_ERR_UNSUPPORTED, "fp32 layers support n_routed <= 128 (got %d)", c->n_routed);
     if (c->d % 4 || c->inter % 4)
       return fail(MOE_ERR_UNSUPPORTED, "fp32 layers need d %% 4 == 0 and inter %% 4 == 0 (d=%d inter=%d)",
                   c->d, c->inter);
@@ -245,13 +246,20 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
   H->has_shared = c.n_shared > 0 ? 1 : 0;
   H->inter_shared = c.n_shared * c.inter;
   H->G = H->has_shared + c.n_routed;
-  H->n_tiles = (c.T + kRouterBM - 1) / kRouterBM;
+  if (H->bf16) {
+    // tiles of R <= 128 tokens (a multiple of 8) so that the router covers every SM
+    const int per_sm = (c.T + H->n_sms - 1) / H->n_sms;
+    H->router_rows = per_sm >= kRouterBM ? kRouterBM : ((per_sm + 7) / 8) * 8;
+  } else {
+    H->router_rows = kRouterBM;
+  }
+  H->n_tiles = (c.T + H->router_rows - 1) / H->router_rows;
   H->bm = H->bf16 ? kPairBM : kSimtBM;
   H->T_pad = ((int64_t)c.T + H->bm - 1) / H->bm * H->bm;
   H->rows_cap = ((int64_t)c.T * c.top_k + (int64_t)c.n_routed * (H->bm - 1) + H->bm - 1) /
                 H->bm * H->bm;
   H->n_pad = (c.n_routed + 15) / 16 * 16;
-  H->maxk = pick_maxk(c.top_k);
+  H->maxk = router_maxk(c.top_k);
   const size_t es = H->es;
   const size_t d = c.d, I = c.inter, Is = H->inter_shared, nr = c.n_routed, ks = c.n_shared;
 
@@ -336,14 +344,13 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
 
   // ---- kernels' launch attributes and TMA descriptors
   if (H->bf16) {
-    const uint32_t b_bytes = ((uint32_t)H->n_pad * 128u + 1023u) & ~1023u;
-    const uint32_t stage_bytes = kRouterBM * 64 * 2 + b_bytes;
+    const uint32_t stage_bytes = router_stage_bytes(H->n_pad);
     int stages = (int)((200u * 1024u) / stage_bytes);
     if (stages > kRouterMaxStages) stages = kRouterMaxStages;
     if (stages < 2) stages = 2;
     H->router_stages = stages;
     H->router_smem = 1024 + (size_t)stages * stage_bytes + 256;
-    if ((size_t)stages * stage_bytes < router_epi_bytes(c.n_routed))
+    if ((size_t)stages * stage_bytes < router_epi_bytes(c.n_routed, H->maxk))
       return fail(MOE_ERR_UNSUPPORTED, "router epilogue scratch does not fit");
     uint32_t cols = 32;
     while (cols < (uint32_t)H->n_pad) cols <<= 1;
@@ -391,7 +398,8 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
     }
     if (!ok) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for a weight/workspace tensor");
   } else {
-    H->simt_router_smem = router_epi_bytes(c.n_routed);
+    H->simt_router_smem = router_epi_bytes(c.n_routed, H->maxk) +
+                          (size_t)kRouterBM * router_row_ld(c.n_routed) * 4;
     const void* rk = H->maxk == 4 ? (const void*)router_simt_kernel<4>
                    : H->maxk == 8 ? (const void*)router_simt_kernel<8>
                                   : (const void*)router_simt_kernel<16>;
@@ -438,27 +446,28 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
   const int T = c.T, d = c.d, K = c.top_k, nr = c.n_routed;
 
   RouterOut ro{topk_idx, topk_w, H->topk_rank, H->tile_hist, H->tile_psum, H->err};
-  CUtensorMap tmU;
+  CUtensorMap tmU, tmUr;
   tick(H, stream, 0);
   if (H->bf16) {
-    if (!encode_2d(&tmU, u, d, T, kRouterBM))
+    if (!encode_2d(&tmU, u, d, T, 128) || !encode_2d(&tmUr, u, d, T, (uint32_t)H->router_rows))
       return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for u");
-    RouterTcArgs ra{T, d, nr, H->n_pad, K, H->router_stages, H->router_tmem_cols, H->bias, ro};
+    RouterTcArgs ra{T, d, nr, H->n_pad, K, H->router_stages, H->router_rows,
+                    H->router_tmem_cols, H->bias, ro};
     if (H->maxk == 4)
-      router_tc_kernel<4><<<H->n_tiles, kRouterThreads, H->router_smem, stream>>>(tmU, H->tmE, ra);
+      router_tc_kernel<4><<<H->n_tiles, kRouterThreads, H->router_smem, stream>>>(tmUr, H->tmE, ra);
     else if (H->maxk == 8)
-      router_tc_kernel<8><<<H->n_tiles, kRouterThreads, H->router_smem, stream>>>(tmU, H->tmE, ra);
+      router_tc_kernel<8><<<H->n_tiles, kRouterThreads, H->router_smem, stream>>>(tmUr, H->tmE, ra);
     else
-      router_tc_kernel<16><<<H->n_tiles, kRouterThreads, H->router_smem, stream>>>(tmU, H->tmE, ra);
+      router_tc_kernel<16><<<H->n_tiles, kRouterThreads, H->router_smem, stream>>>(tmUr, H->tmE, ra);
   } else {
     RouterSimtArgs ra{static_cast<const float*>(u), static_cast<const float*>(H->centroids), H->bias,
                       T, d, nr, K, ro};
     if (H->maxk == 4)
-      router_simt_kernel<4><<<H->n_tiles, kRouterBM, H->simt_router_smem, stream>>>(ra);
+      router_simt_kernel<4><<<H->n_tiles, kRouterEpiThreads, H->simt_router_smem, stream>>>(ra);
     else if (H->maxk == 8)
-      router_simt_kernel<8><<<H->n_tiles, kRouterBM, H->simt_router_smem, stream>>>(ra);
+      router_simt_kernel<8><<<H->n_tiles, kRouterEpiThreads, H->simt_router_smem, stream>>>(ra);
     else
-      router_simt_kernel<16><<<H->n_tiles, kRouterBM, H->simt_router_smem, stream>>>(ra);
+      router_simt_kernel<16><<<H->n_tiles, kRouterEpiThreads, H->simt_router_smem, stream>>>(ra);
   }
   MOE_CUDA(cudaGetLastError());
 
@@ -472,7 +481,8 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
   MOE_CUDA(cudaGetLastError());
 
   PermuteArgs pa{static_cast<const uint8_t*>(u), topk_idx, H->topk_rank, H->tile_base, H->slot_row,
-                 static_cast<uint8_t*>(H->xp), T, K, nr, (int)H->rows_cap, d * H->es, H->err};
+                 static_cast<uint8_t*>(H->xp), T, K, nr, (int)H->rows_cap, H->router_rows,
+                 d * H->es, H->err};
   tick(H, stream, 2);
   permute_kernel<<<(T + kPermuteWarps - 1) / kPermuteWarps, kPermuteWarps * 32, 0, stream>>>(pa);
   MOE_CUDA(cudaGetLastError());

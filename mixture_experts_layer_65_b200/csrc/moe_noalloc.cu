@@ -141,8 +141,7 @@ extern "C" moe_status moe_route_noalloc(const void* u, const void* centroids, co
   CUtensorMap tmU, tmE;
   if (!encode_rows(&tmU, u, d, T, kRouterBM) || !encode_rows(&tmE, centroids, d, n_routed, n_pad))
     return nfail(MOE_ERR_CUDA, "moe_route_noalloc: cuTensorMapEncodeTiled failed");
-  const uint32_t b_bytes = ((uint32_t)n_pad * 128u + 1023u) & ~1023u;
-  const uint32_t stage_bytes = kRouterBM * 64 * 2 + b_bytes;
+  const uint32_t stage_bytes = router_stage_bytes(n_pad);
   int stages = (int)((200u * 1024u) / stage_bytes);
   stages = stages > kRouterMaxStages ? kRouterMaxStages : (stages < 2 ? 2 : stages);
   const size_t smem = 1024 + (size_t)stages * stage_bytes + 256;
@@ -151,7 +150,10 @@ extern "C" moe_status moe_route_noalloc(const void* u, const void* centroids, co
 
   RouterOut ro{topk_idx, topk_w, reinterpret_cast<int32_t*>(sc + kOffRank),
                reinterpret_cast<int32_t*>(sc + kOffHist), reinterpret_cast<float*>(sc + kOffPsum), err};
-  RouterTcArgs ra{T, d, n_routed, n_pad, top_k, stages, cols, logit_bias ? logit_bias : zero_bias, ro};
+  if ((size_t)stages * stage_bytes < router_epi_bytes(n_routed, router_maxk(top_k)))
+    return nfail(MOE_ERR_UNSUPPORTED, "moe_route_noalloc: router scratch does not fit");
+  RouterTcArgs ra{T, d, n_routed, n_pad, top_k, stages, kRouterBM, cols,
+                  logit_bias ? logit_bias : zero_bias, ro};
   cudaError_t e = top_k <= 4 ? launch_router<4>(tmU, tmE, ra, n_tiles, smem, st)
                  : top_k <= 8 ? launch_router<8>(tmU, tmE, ra, n_tiles, smem, st)
                               : launch_router<16>(tmU, tmE, ra, n_tiles, smem, st);

@@ -312,4 +312,10 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 __device__ __forceinline__ float silu_f32(float z) { return z / (1.0f + expf(-z)); }
 
+// SiLU for a result that is rounded to bf16 next: fast exp and divide (a few ulp of fp32,
+// far below bf16 resolution).  The exponent is clamped so 1 + e^-z stays finite.
+__device__ __forceinline__ float silu_fast(float z) {
+  return __fdividef(z, 1.0f + __expf(fminf(-z, 80.0f)));
+}
+
 }  // namespace moe

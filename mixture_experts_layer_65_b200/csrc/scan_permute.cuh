@@ -134,6 +134,7 @@ struct PermuteArgs {
   int32_t* slot_row;           // [T, top_k] destination row (output)
   uint8_t* xp;                 // [rows_cap, row_bytes]
   int T, top_k, n_routed, rows_cap;
+  int tile_rows;               // tokens per router tile
   int row_bytes;               // multiple of 16
   int* err;
 };
@@ -149,7 +150,7 @@ static __global__ void __launch_bounds__(kPermuteWarps * 32) permute_kernel(Perm
   if (lane < a.top_k) {
     const int e = a.topk_idx[(size_t)t * a.top_k + lane];
     if (e >= 0 && e < a.n_routed) {
-      const int dst = a.tile_base[(size_t)(t / kRouterBM) * a.n_routed + e] +
+      const int dst = a.tile_base[(size_t)(t / a.tile_rows) * a.n_routed + e] +
                       a.topk_rank[(size_t)t * a.top_k + lane];
       if (dst >= 0 && dst < a.rows_cap) my_dest = dst;
       else record_error(a.err, kErrPermuteRow);
