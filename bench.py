@@ -228,7 +228,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     import torch.distributed as dist
 
     from mixture_experts_layer_65_b200 import workloads as W
-    from mixture_experts_layer_65_b200.layer import MoELayer, balance_loss, to_device_tensor
+    from mixture_experts_layer_65_b200.layer import MoELayer, to_device_tensor
+    from mixture_experts_layer_65_b200.parallel import global_balance_loss
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
@@ -250,12 +251,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
     def step(i):
         layer.forward(ubufs[i % n_buf], out)
-        if world > 1:
-            layer.expert_psum(psum)
-            cnt_g.copy_(out.expert_counts)
-            dist.all_reduce(cnt_g)
-            dist.all_reduce(psum)
-            balance_loss(cnt_g, psum, world * w.T, w.alpha1, aux_g)
+        if world > 1:   # balance loss of the global batch: all-reduce counts and sums
+            global_balance_loss(layer, out, psum, cnt_g, aux_g)
 
     for i in range(max(3, args.warmup)):
         step(i)

@@ -35,7 +35,9 @@ __device__ __forceinline__ void add8(float (&acc)[8], const uint4& v, float w) {
 }
 
 // bf16 rows: 8 elements per 16-byte vector; each lane handles vectors lane, lane+32, ...
-static __global__ void __launch_bounds__(kCombineWarps * 32)
+// All 2 + top_k loads of a vector are issued before the fixed-order accumulation.
+template <int MAXK>
+__global__ void __launch_bounds__(kCombineWarps * 32)
 combine_bf16_kernel(CombineArgs<__nv_bfloat16> a) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * kCombineWarps + warp;
@@ -47,21 +49,33 @@ combine_bf16_kernel(CombineArgs<__nv_bfloat16> a) {
     s_w[warp][lane] = a.topk_w[(size_t)t * a.top_k + lane];
   }
   __syncwarp();
+  const uint4* yk[MAXK];
+  float wk[MAXK];
+#pragma unroll
+  for (int k = 0; k < MAXK; ++k) {
+    const bool on = k < a.top_k;
+    yk[k] = reinterpret_cast<const uint4*>(a.yr + (size_t)(on ? s_row[warp][k] : 0) * a.d);
+    wk[k] = on ? s_w[warp][k] : 0.f;
+  }
   const int nvec = a.d >> 3;
   const uint4* ur = reinterpret_cast<const uint4*>(a.u + (size_t)t * a.d);
   const uint4* sr = a.ys ? reinterpret_cast<const uint4*>(a.ys + (size_t)t * a.d) : nullptr;
   uint4* hr = reinterpret_cast<uint4*>(a.h + (size_t)t * a.d);
   for (int v = lane; v < nvec; v += 32) {
+    uint4 x[MAXK];
+    const uint4 xu = __ldg(ur + v);
+    const uint4 xs = sr ? __ldg(sr + v) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int k = 0; k < MAXK; ++k)
+      if (k < a.top_k) x[k] = __ldg(yk[k] + v);
     float acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-    add8(acc, __ldg(ur + v), 1.0f);
-    if (sr) add8(acc, __ldg(sr + v), 1.0f);
-    for (int k = 0; k < a.top_k; ++k) {
-      const int rk = s_row[warp][k];
-      const float wk = s_w[warp][k];
-      add8(acc, __ldg(reinterpret_cast<const uint4*>(a.yr + (size_t)rk * a.d) + v), wk);
-    }
+    add8(acc, xu, 1.0f);
+    if (sr) add8(acc, xs, 1.0f);
+#pragma unroll
+    for (int k = 0; k < MAXK; ++k)
+      if (k < a.top_k) add8(acc, x[k], wk[k]);
     uint4 o;
     o.x = pack_bf16x2(acc[0], acc[1]);
     o.y = pack_bf16x2(acc[2], acc[3]);

@@ -212,9 +212,11 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
       gemm_decode(tile, g, a, c);
       const int acc = it & 1;
       const uint32_t acc_par = (it >> 1) & 1;
-      const bool ok =
-          mbar_wait(smem_u32(&acc_full[acc]), acc_par, abort_flag, a.err, kErrWaitEpilogue);
-      if (!__all_sync(0xffffffffu, ok)) break;   // warp-uniform decision
+      // lane 0 polls the accumulator barrier, the other lanes wait in __syncwarp
+      int ok = 1;
+      if (lane == 0)
+        ok = mbar_wait(smem_u32(&acc_full[acc]), acc_par, abort_flag, a.err, kErrWaitEpilogue);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;   // warp-uniform decision
       tc_fence_after();
       const uint32_t trow =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * kGemmBN);

@@ -522,7 +522,13 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
                                   static_cast<const __nv_bfloat16*>(H->yr), H->slot_row, topk_w,
                                   static_cast<__nv_bfloat16*>(h), T, d, K};
     tick(H, stream, 5);
-    combine_bf16_kernel<<<(T + kCombineWarps - 1) / kCombineWarps, kCombineWarps * 32, 0, stream>>>(ca);
+    const int cgrid = (T + kCombineWarps - 1) / kCombineWarps;
+    if (H->maxk == 4)
+      combine_bf16_kernel<4><<<cgrid, kCombineWarps * 32, 0, stream>>>(ca);
+    else if (H->maxk == 8)
+      combine_bf16_kernel<8><<<cgrid, kCombineWarps * 32, 0, stream>>>(ca);
+    else
+      combine_bf16_kernel<16><<<cgrid, kCombineWarps * 32, 0, stream>>>(ca);
     MOE_CUDA(cudaGetLastError());
   } else {
     const size_t ks = c.n_shared;

@@ -45,12 +45,12 @@ struct RouterEpiSmem {
   float ppart[4][kMaxRouted];     // per-expert sums over 32-row quarters of the tile
   float inv_sum[kRouterBM];       // 1 / softmax denominator per row (0 for rows past T)
   float rowmax[kRouterBM];
-  float maxpart[kRouterBM * 4];
-  float sumpart[kRouterBM * 4];
+  float maxpart[4][kRouterBM];    // [sub][row]: lanes of a warp hit consecutive banks
+  float sumpart[4][kRouterBM];
 };
 
 // Epilogue scratch: RouterEpiSmem, then one region that first holds the per-thread top-k
-// lists [128][4][MAXK] (u64) and then the exp(l - max) rows [128][ld] (fp32).
+// lists [4][MAXK][128] (u64, row fastest) and then the exp(l - max) rows [128][ld] (fp32).
 __host__ __device__ constexpr int router_row_ld(int n_routed) { return ((n_routed + 31) & ~31) + 1; }
 __host__ __device__ constexpr size_t router_region_bytes(int n_routed, int maxk) {
   return (size_t)kRouterBM * router_row_ld(n_routed) * 4 > (size_t)kRouterBM * 4 * maxk * 8
@@ -128,27 +128,27 @@ __device__ __forceinline__ void router_epilogue(int r, int sub, int tile, int ti
     }
   }
 #pragma unroll
-  for (int p = 0; p < MAXK; ++p) tops[(size_t)(r * 4 + sub) * MAXK + p] = top[p];
-  S.maxpart[r * 4 + sub] = lmax;
+  for (int p = 0; p < MAXK; ++p) tops[(size_t)(sub * MAXK + p) * kRouterBM + r] = top[p];
+  S.maxpart[sub][r] = lmax;
   sync();
 
   // row owner (sub 0): merge the four sorted lists, row max in a fixed order
   if (sub == 0) {
-    const uint64_t* L = tops + (size_t)r * 4 * MAXK;
+    const uint64_t* L = tops + r;    // element (s, p) at L[(s * MAXK + p) * 128]
     int h0 = 0, h1 = 0, h2 = 0, h3 = 0;
 #pragma unroll
     for (int p = 0; p < MAXK; ++p) {
-      const uint64_t a0 = h0 < MAXK ? L[h0] : 0ull;
-      const uint64_t a1 = h1 < MAXK ? L[MAXK + h1] : 0ull;
-      const uint64_t a2 = h2 < MAXK ? L[2 * MAXK + h2] : 0ull;
-      const uint64_t a3 = h3 < MAXK ? L[3 * MAXK + h3] : 0ull;
+      const uint64_t a0 = h0 < MAXK ? L[(size_t)h0 * kRouterBM] : 0ull;
+      const uint64_t a1 = h1 < MAXK ? L[(size_t)(MAXK + h1) * kRouterBM] : 0ull;
+      const uint64_t a2 = h2 < MAXK ? L[(size_t)(2 * MAXK + h2) * kRouterBM] : 0ull;
+      const uint64_t a3 = h3 < MAXK ? L[(size_t)(3 * MAXK + h3) * kRouterBM] : 0ull;
       const uint64_t m01 = a0 > a1 ? a0 : a1, m23 = a2 > a3 ? a2 : a3;
       const uint64_t m = m01 > m23 ? m01 : m23;
       top[p] = m;
       if (m == a0) ++h0; else if (m == a1) ++h1; else if (m == a2) ++h2; else ++h3;
     }
-    S.rowmax[r] = fmaxf(fmaxf(S.maxpart[r * 4], S.maxpart[r * 4 + 1]),
-                        fmaxf(S.maxpart[r * 4 + 2], S.maxpart[r * 4 + 3]));
+    S.rowmax[r] = fmaxf(fmaxf(S.maxpart[0][r], S.maxpart[1][r]),
+                        fmaxf(S.maxpart[2][r], S.maxpart[3][r]));
   }
   sync();   // the list region is reused for the exp rows below
 
@@ -170,13 +170,12 @@ __device__ __forceinline__ void router_epilogue(int r, int sub, int tile, int ti
         }
       }
     }
-    S.sumpart[r * 4 + sub] = part;
+    S.sumpart[sub][r] = part;
   }
   sync();
   float inv_sum = 0.f;
   if (sub == 0) {
-    const float sum = ((S.sumpart[r * 4] + S.sumpart[r * 4 + 1]) + S.sumpart[r * 4 + 2]) +
-                      S.sumpart[r * 4 + 3];
+    const float sum = ((S.sumpart[0][r] + S.sumpart[1][r]) + S.sumpart[2][r]) + S.sumpart[3][r];
     inv_sum = 1.0f / sum;
     S.inv_sum[r] = valid ? inv_sum : 0.f;
     if (valid) {
@@ -363,8 +362,11 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant_
     const int q = warp & 3;              // TMEM lane quadrant this warp may access
     const int sub = w >> 2;              // which slices of the row
     const int r = q * 32 + lane;
-    const bool ok = mbar_wait(smem_u32(acc_full), 0, abort_flag, a.out.err, kErrWaitEpilogue);
-    // all sixteen epilogue warps take the same branch (they synchronise inside it)
+    // one thread polls the accumulator barrier; the others sleep in the named barrier,
+    // and all sixteen warps take the same branch (they synchronise inside it)
+    bool ok = true;
+    if (w == 0 && lane == 0)
+      ok = mbar_wait(smem_u32(acc_full), 0, abort_flag, a.out.err, kErrWaitEpilogue);
     if (!named_bar_any(1, kRouterEpiThreads, !ok)) {
       tc_fence_after();
       const uint32_t trow = tmem_base + (static_cast<uint32_t>(q * 32) << 16);

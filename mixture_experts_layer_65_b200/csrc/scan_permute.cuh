@@ -77,41 +77,65 @@ static __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a
     s_off[tid] = run;   // count for now, offset after step 3
   }
   __syncthreads();
-  // 3. expert offsets (padded to the GEMM M tile), tile tables, balance loss
-  if (tid == 0) {
-    const int G = a.has_shared + nr;
-    const int nt2 = (a.d + a.bn2 - 1) / a.bn2;
-    int off = 0, acc1 = 0, acc2 = 0;
-    double aux = 0.0;
-    const double invT = 1.0 / (double)a.T;
-    a.ts1[0] = 0;
-    a.ts2[0] = 0;
-    int g = 0;
-    if (a.has_shared) {
-      const int mt = (a.T + a.bm - 1) / a.bm;
-      const int nt1 = (a.inter_shared + a.bn1 - 1) / a.bn1;
-      a.grp_row[0] = 0;
-      acc1 += mt * nt1;
-      acc2 += mt * nt2;
-      a.ts1[1] = acc1;
-      a.ts2[1] = acc2;
-      g = 1;
-    }
+  // 3. expert offsets (padded to the GEMM row tile), tile tables, balance loss: inclusive
+  //    scans over the experts (shuffles within a warp, then over warp totals) and a
+  //    fixed-shape tree sum for the loss, so the result does not depend on scheduling
+  {
+    __shared__ int w_off[kScanThreads / 32], w_t1[kScanThreads / 32], w_t2[kScanThreads / 32];
+    __shared__ double s_aux[kMaxRouted];
+    const int lane = tid & 31, wid = tid >> 5;
     const int nt1 = (a.inter + a.bn1 - 1) / a.bn1;
-    for (int i = 0; i < nr; ++i, ++g) {
-      const int cnt = s_off[i];
+    const int nt2 = (a.d + a.bn2 - 1) / a.bn2;
+    const int sh_mt = a.has_shared ? (a.T + a.bm - 1) / a.bm : 0;
+    const int sh_t1 = sh_mt * ((a.inter_shared + a.bn1 - 1) / a.bn1);
+    const int sh_t2 = sh_mt * nt2;
+    int cnt = 0, pad = 0, t1 = 0, t2 = 0;
+    if (tid < nr) {
+      cnt = s_off[tid];
       const int mt = (cnt + a.bm - 1) / a.bm;
-      s_off[i] = off;
-      a.grp_row[g] = off;
-      off += mt * a.bm;
-      acc1 += mt * nt1;
-      acc2 += mt * nt2;
-      a.ts1[g + 1] = acc1;
-      a.ts2[g + 1] = acc2;
-      aux += ((double)cnt * invT) * ((double)a.psum_total[i] * invT);
+      pad = mt * a.bm;
+      t1 = mt * nt1;
+      t2 = mt * nt2;
+      const double invT = 1.0 / (double)a.T;
+      s_aux[tid] = ((double)cnt * invT) * ((double)a.psum_total[tid] * invT);
+    } else if (tid < kMaxRouted) {
+      s_aux[tid] = 0.0;
     }
-    (void)G;
-    *a.aux_loss = (float)((double)a.alpha1 * aux);
+    int ip = pad, i1 = t1, i2 = t2;   // inclusive scans within the warp
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int xp = __shfl_up_sync(0xffffffffu, ip, o);
+      const int x1 = __shfl_up_sync(0xffffffffu, i1, o);
+      const int x2 = __shfl_up_sync(0xffffffffu, i2, o);
+      if (lane >= o) { ip += xp; i1 += x1; i2 += x2; }
+    }
+    if (lane == 31) { w_off[wid] = ip; w_t1[wid] = i1; w_t2[wid] = i2; }
+    __syncthreads();
+    int bp = 0, b1 = 0, b2 = 0;
+    for (int w2 = 0; w2 < wid; ++w2) { bp += w_off[w2]; b1 += w_t1[w2]; b2 += w_t2[w2]; }
+    if (tid < nr) {
+      const int g = a.has_shared + tid;
+      const int off = bp + ip - pad;            // exclusive prefix of the padded sizes
+      s_off[tid] = off;                         // read in step 4 after the barrier below
+      a.grp_row[g] = off;
+      a.ts1[g + 1] = sh_t1 + b1 + i1;
+      a.ts2[g + 1] = sh_t2 + b2 + i2;
+    }
+    if (tid == 0) {
+      a.ts1[0] = 0;
+      a.ts2[0] = 0;
+      if (a.has_shared) {
+        a.grp_row[0] = 0;
+        a.ts1[1] = sh_t1;
+        a.ts2[1] = sh_t2;
+      }
+    }
+    // loss: pairwise tree over 256 slots, always the same shape
+    for (int stride = kMaxRouted / 2; stride > 0; stride >>= 1) {
+      __syncthreads();
+      if (tid < stride) s_aux[tid] += s_aux[tid + stride];
+    }
+    if (tid == 0) *a.aux_loss = (float)((double)a.alpha1 * s_aux[0]);
   }
   __syncthreads();
   // 4. destination base of every (tile, expert)
