@@ -48,6 +48,8 @@ def parse_args():
     p.add_argument("--cpu-seconds", type=float, default=15.0,
                    help="target CPU time of the oracle baseline sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-graph", action="store_true",
+                   help="launch the forward eagerly instead of replaying captured CUDA graphs")
     return p.parse_args()
 
 
@@ -249,8 +251,31 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         cnt_g = torch.empty(w.n_routed, dtype=torch.int32, device=dev)
         aux_g = torch.empty(1, dtype=torch.float32, device=dev)
 
-    def step(i):
-        layer.forward(ubufs[i % n_buf], out)
+    stream = torch.cuda.current_stream(dev)
+    # one captured CUDA graph per input buffer: the six kernel launches of a forward are
+    # replayed without host launch overhead (the layer's inputs/outputs stay fixed)
+    graphs = None
+    if not args.no_graph:
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            for ub in ubufs:
+                layer.forward(ub, out)
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        graphs = []
+        for ub in ubufs:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                layer.forward(ub, out)
+            graphs.append(g)
+        torch.cuda.synchronize()
+
+    def step(i, eager=False):
+        if graphs is not None and not eager:
+            graphs[i % n_buf].replay()
+        else:
+            layer.forward(ubufs[i % n_buf], out)
         if world > 1:   # balance loss of the global batch: all-reduce counts and sums
             global_balance_loss(layer, out, psum, cnt_g, aux_g)
 
@@ -262,9 +287,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         dist.barrier()
     clocks = ClockSampler() if rank == 0 else None
     time.sleep(0.3 if clocks else 0.0)
-    stream = torch.cuda.current_stream(dev)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    layer.timing_begin(args.steps)
+    if graphs is None:
+        layer.timing_begin(args.steps)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -275,9 +300,16 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    kernel_ms, n_rec = layer.timing_end()
     clk = clocks.stop() if clocks else None
     ms = ev0.elapsed_time(ev1)
+    if graphs is not None:
+        # per-kernel durations: CUDA events between the kernels of eager forwards
+        n_prof = min(args.steps, 100)
+        layer.timing_begin(n_prof)
+        for i in range(n_prof):
+            step(i, eager=True)
+        torch.cuda.synchronize()
+    kernel_ms, n_rec = layer.timing_end()
     if world > 1:
         t = torch.tensor([ms], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -308,6 +340,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
     if rank != 0:
         return
+    del graphs
     peaks, peak_src = load_peaks()
     work = algorithmic_work(w)
     per_kernel = {}
@@ -355,6 +388,11 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             "value": world * w.T * args.e2e_steps / (e2e_ms * 1e-3), "unit": "tokens/s",
             "h2d_bytes_per_step": u_bytes, "d2h_bytes_per_step": u_bytes + tk * 8 + w.n_routed * 4 + 4},
         "gpu_launches": args.steps * (layer.kernels_per_forward + (1 if world > 1 else 0)),
+        "launch": "eager" if args.no_graph else "CUDA graph replay (one graph per input buffer)",
+        "kernel_timing": ("CUDA events between the library's kernels over the timed steps"
+                          if args.no_graph else
+                          f"CUDA events between the library's kernels over {n_rec} eager forwards "
+                          "after the timed region"),
         "clocks": clk,
     }
     if world == 1 and not args.no_cpu_baseline:

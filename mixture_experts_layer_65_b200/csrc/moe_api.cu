@@ -12,6 +12,7 @@
 #include <cstdio>
 #include <cstring>
 #include <string>
+#include <type_traits>
 #include <vector>
 
 #include "moe.h"
@@ -101,6 +102,18 @@ __global__ void balance_loss_kernel(const int32_t* counts, const float* psum, in
 }
 
 constexpr int kKernelsPerForward = 6;
+
+// Call f(std::integral_constant<int, MAXK>{}) for the compile-time list length of top_k.
+template <class F>
+auto with_maxk(int maxk, F&& f) {
+  switch (maxk) {
+    case 4: return f(std::integral_constant<int, 4>{});
+    case 6: return f(std::integral_constant<int, 6>{});
+    case 8: return f(std::integral_constant<int, 8>{});
+    case 12: return f(std::integral_constant<int, 12>{});
+    default: return f(std::integral_constant<int, 16>{});
+  }
+}
 
 }  // namespace
 
@@ -355,9 +368,7 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
     uint32_t cols = 32;
     while (cols < (uint32_t)H->n_pad) cols <<= 1;
     H->router_tmem_cols = cols;
-    const void* rk = H->maxk == 4 ? (const void*)router_tc_kernel<4>
-                   : H->maxk == 8 ? (const void*)router_tc_kernel<8>
-                                  : (const void*)router_tc_kernel<16>;
+    const void* rk = with_maxk(H->maxk, [](auto m) { return (const void*)router_tc_kernel<m()>; });
     MOE_CUDA(cudaFuncSetAttribute(rk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)H->router_smem));
     MOE_CUDA(cudaFuncSetAttribute((const void*)grouped_gemm_tc_kernel<kGateUpSwiGLU>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmemBytes));
@@ -400,9 +411,7 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
   } else {
     H->simt_router_smem = router_epi_bytes(c.n_routed, H->maxk) +
                           (size_t)kRouterBM * router_row_ld(c.n_routed) * 4;
-    const void* rk = H->maxk == 4 ? (const void*)router_simt_kernel<4>
-                   : H->maxk == 8 ? (const void*)router_simt_kernel<8>
-                                  : (const void*)router_simt_kernel<16>;
+    const void* rk = with_maxk(H->maxk, [](auto m) { return (const void*)router_simt_kernel<m()>; });
     MOE_CUDA(cudaFuncSetAttribute(rk, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)H->simt_router_smem));
   }
@@ -453,21 +462,17 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
       return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for u");
     RouterTcArgs ra{T, d, nr, H->n_pad, K, H->router_stages, H->router_rows,
                     H->router_tmem_cols, H->bias, ro};
-    if (H->maxk == 4)
-      router_tc_kernel<4><<<H->n_tiles, kRouterThreads, H->router_smem, stream>>>(tmUr, H->tmE, ra);
-    else if (H->maxk == 8)
-      router_tc_kernel<8><<<H->n_tiles, kRouterThreads, H->router_smem, stream>>>(tmUr, H->tmE, ra);
-    else
-      router_tc_kernel<16><<<H->n_tiles, kRouterThreads, H->router_smem, stream>>>(tmUr, H->tmE, ra);
+    with_maxk(H->maxk, [&](auto m) {
+      router_tc_kernel<m()><<<H->n_tiles, kRouterThreads, H->router_smem, stream>>>(tmUr, H->tmE, ra);
+      return 0;
+    });
   } else {
     RouterSimtArgs ra{static_cast<const float*>(u), static_cast<const float*>(H->centroids), H->bias,
                       T, d, nr, K, ro};
-    if (H->maxk == 4)
-      router_simt_kernel<4><<<H->n_tiles, kRouterEpiThreads, H->simt_router_smem, stream>>>(ra);
-    else if (H->maxk == 8)
-      router_simt_kernel<8><<<H->n_tiles, kRouterEpiThreads, H->simt_router_smem, stream>>>(ra);
-    else
-      router_simt_kernel<16><<<H->n_tiles, kRouterEpiThreads, H->simt_router_smem, stream>>>(ra);
+    with_maxk(H->maxk, [&](auto m) {
+      router_simt_kernel<m()><<<H->n_tiles, kRouterEpiThreads, H->simt_router_smem, stream>>>(ra);
+      return 0;
+    });
   }
   MOE_CUDA(cudaGetLastError());
 
@@ -523,12 +528,10 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
                                   static_cast<__nv_bfloat16*>(h), T, d, K};
     tick(H, stream, 5);
     const int cgrid = (T + kCombineWarps - 1) / kCombineWarps;
-    if (H->maxk == 4)
-      combine_bf16_kernel<4><<<cgrid, kCombineWarps * 32, 0, stream>>>(ca);
-    else if (H->maxk == 8)
-      combine_bf16_kernel<8><<<cgrid, kCombineWarps * 32, 0, stream>>>(ca);
-    else
-      combine_bf16_kernel<16><<<cgrid, kCombineWarps * 32, 0, stream>>>(ca);
+    with_maxk(H->maxk, [&](auto m) {
+      combine_bf16_kernel<m()><<<cgrid, kCombineWarps * 32, 0, stream>>>(ca);
+      return 0;
+    });
     MOE_CUDA(cudaGetLastError());
   } else {
     const size_t ks = c.n_shared;

@@ -154,9 +154,12 @@ extern "C" moe_status moe_route_noalloc(const void* u, const void* centroids, co
     return nfail(MOE_ERR_UNSUPPORTED, "moe_route_noalloc: router scratch does not fit");
   RouterTcArgs ra{T, d, n_routed, n_pad, top_k, stages, kRouterBM, cols,
                   logit_bias ? logit_bias : zero_bias, ro};
-  cudaError_t e = top_k <= 4 ? launch_router<4>(tmU, tmE, ra, n_tiles, smem, st)
-                 : top_k <= 8 ? launch_router<8>(tmU, tmE, ra, n_tiles, smem, st)
-                              : launch_router<16>(tmU, tmE, ra, n_tiles, smem, st);
+  const int mk = router_maxk(top_k);
+  cudaError_t e = mk == 4 ? launch_router<4>(tmU, tmE, ra, n_tiles, smem, st)
+                 : mk == 6 ? launch_router<6>(tmU, tmE, ra, n_tiles, smem, st)
+                 : mk == 8 ? launch_router<8>(tmU, tmE, ra, n_tiles, smem, st)
+                 : mk == 12 ? launch_router<12>(tmU, tmE, ra, n_tiles, smem, st)
+                            : launch_router<16>(tmU, tmE, ra, n_tiles, smem, st);
   if (e != cudaSuccess) return nfail(MOE_ERR_CUDA, "moe_route_noalloc: router launch failed");
 
   ScanArgs sa{ro.tile_hist, ro.tile_psum, n_tiles, n_routed, T, /*has_shared=*/0,

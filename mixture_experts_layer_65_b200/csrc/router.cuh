@@ -60,7 +60,11 @@ __host__ __device__ constexpr size_t router_region_bytes(int n_routed, int maxk)
 __host__ __device__ constexpr size_t router_epi_bytes(int n_routed, int maxk) {
   return sizeof(RouterEpiSmem) + router_region_bytes(n_routed, maxk);
 }
-__host__ __device__ constexpr int router_maxk(int top_k) { return top_k <= 4 ? 4 : (top_k <= 8 ? 8 : 16); }
+// Length of the per-thread top-k list (compile-time, so it stays in registers): the
+// insertion chain costs one 64-bit compare-exchange per slot, so it is sized tightly.
+__host__ __device__ constexpr int router_maxk(int top_k) {
+  return top_k <= 4 ? 4 : top_k <= 6 ? 6 : top_k <= 8 ? 8 : top_k <= 12 ? 12 : 16;
+}
 
 // Total order on (logit, expert): larger logit first; on equal logits the lower index.
 // NaN ranks as -inf and -0 as +0, so every slot gets a real index and equal values tie.
