@@ -71,12 +71,20 @@ def workload_desc(w, n_gpus: int) -> dict:
 
 
 # --------------------------------------------------------------------------- work model
-def algorithmic_work(w) -> dict:
-    """Per-launch algorithmic work of each kernel (selected experts only, no padding)."""
+SMALL_BATCH_MAX_T = 128   # the library streams weights (weights-on-M GEMMs) up to this T
+
+
+def algorithmic_work(w, active_experts: int | None = None) -> dict:
+    """Per-launch algorithmic work of each kernel (selected experts only, no padding).
+
+    Prefill-sized layers: the expert GEMMs are tensor-bound (FLOPs).  Decode-sized layers
+    (T <= 128, weights-on-M GEMMs): they are bound by streaming the weights of the experts
+    that received tokens (bytes), plus the shared experts.
+    """
     es = 2 if w.dtype == "bf16" else 4
     T, d, I, K, ks, nr = w.T, w.d, w.inter, w.top_k, w.n_shared, w.n_routed
     passes = ks + K
-    return {
+    work = {
         "router": ("hbm", T * d * es + nr * d * es + T * K * 12),
         "scan": ("latency", 0),
         "permute": ("hbm", T * d * es + T * K * d * es + T * K * 12),
@@ -84,6 +92,11 @@ def algorithmic_work(w) -> dict:
         "down_gemm": ("tensor", 2.0 * T * d * I * passes),
         "combine": ("hbm", T * d * es * (2 + (1 if ks else 0) + K) + T * K * 8),
     }
+    if w.dtype == "bf16" and T <= SMALL_BATCH_MAX_T and d % 128 == 0:
+        n = (nr if active_experts is None else active_experts) + ks
+        work["gate_up_gemm"] = ("hbm", n * 2 * I * d * es + T * passes * (d + I) * es)
+        work["down_gemm"] = ("hbm", n * I * d * es + T * passes * (I + d) * es)
+    return work
 
 
 def csrc_digest() -> str:
@@ -342,7 +355,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         return
     del graphs
     peaks, peak_src = load_peaks()
-    work = algorithmic_work(w)
+    work = algorithmic_work(w, int((out.expert_counts > 0).sum().item()))
     per_kernel = {}
     for k in KERNELS:
         kind, amount = work[k]
@@ -365,7 +378,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                 "unit": dk.get("unit"), "frac": dk.get("frac"),
                 "peak_source": f"{peak_src} ({'bf16 sustained' if bound == 'tensor' else 'HBM copy'})",
                 "traffic": ncu_traffic(dominant, w.name), "algorithmic_per_launch": work[dominant][1]}
-    gemm_flops = work["gate_up_gemm"][1] + work["down_gemm"][1]
+    gemm_flops = 6.0 * w.T * w.d * w.inter * (w.n_shared + w.top_k)
     gemm_ms = (kernel_ms["gate_up_gemm"] + kernel_ms["down_gemm"]) / max(1, n_rec)
     gemm_tflops = gemm_flops / (gemm_ms * 1e-3) / 1e12
     value = world * w.T * args.steps / (ms * 1e-3)

@@ -1,0 +1,274 @@
+// gemm_small.cuh -- grouped expert GEMMs for small token counts (decode), weights on M.
+//
+// Same FFN as gemm_tc.cuh (SwiGLU experts, K_s shared experts as one always-on group), for
+// layers whose groups hold few tokens (every group's token count <= n_tok <= 128).  The
+// products are computed transposed, D^T = W X^T, so the MMA's M dimension (128) runs over
+// weight rows and its N dimension over the group's tokens: each weight tile is streamed
+// from HBM once and the tensor cores do almost no padding work, which makes the kernel a
+// weight-streaming one, as a decode step is.  Groups without tokens get no tiles.
+//
+//   mode kGateUpSwiGLU: a 128-row tile of the interleaved gate/up weights is one block of
+//                       64 gate rows followed by the 64 matching up rows; TMEM lane L < 64
+//                       holds gate values, lane L + 64 the up values of the same column.
+//   mode kDown:         a 128-row tile of W_down gives 128 output features.
+//
+// One CTA per SM (persistent), 192 threads: warp 0 issues TMA loads (weights 128 x 64 and
+// tokens n_tok x 64, 128-byte swizzle) into a multi-stage ring; warp 1 allocates TMEM (two
+// n_tok-column fp32 accumulators) and one thread issues tcgen05.mma (M = 128, N = n_tok);
+// warps 2..5 drain the accumulator, transpose through shared memory and store whole token
+// rows (coalesced).
+#pragma once
+
+#include "gemm_tc.cuh"
+
+namespace moe {
+
+constexpr int kSmallBM = 128;
+constexpr int kSmallThreads = 192;
+constexpr int kSmallMaxTok = 128;
+constexpr int kSmallMaxStages = 8;
+
+struct SmallGemmArgs {
+  const int32_t* grp_row;   // [G] first token row of each group in the token operand / output
+  const int32_t* ts;        // [G + 1] tile prefix (a group has tiles only if it has tokens)
+  const int32_t* counts;    // [n_routed] tokens of each routed group (shared group: T)
+  int G, has_shared, T;
+  int n_tok;                // N of the MMA: multiple of 16, >= every group's token count
+  int stages;
+  int kb_shared, kb_routed; // K / 64
+  int mt_shared, mt_routed; // weight-row tiles per group
+  __nv_bfloat16* out_shared;
+  int64_t ld_shared;
+  __nv_bfloat16* out_routed;
+  int64_t ld_routed;
+  int* err;
+};
+
+// smem: stages x (weights 16 KB + tokens n_tok x 128 B) | epilogue buffers | barriers
+__host__ __device__ constexpr uint32_t small_stage_bytes(int n_tok) {
+  return kSmallBM * 128u + (((uint32_t)n_tok * 128u + 1023u) & ~1023u);
+}
+__host__ __device__ constexpr size_t small_epi_bytes(int n_tok) {
+  // up values [64][n_tok + 1] fp32 and the transposed output tile [n_tok][128] bf16
+  return (size_t)64 * (n_tok + 1) * 4 + (size_t)n_tok * kSmallBM * 2;
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kSmallThreads, 1)
+grouped_gemm_small_kernel(const __grid_constant__ CUtensorMap tmW_s,
+                          const __grid_constant__ CUtensorMap tmW_r,
+                          const __grid_constant__ CUtensorMap tmX_s,
+                          const __grid_constant__ CUtensorMap tmX_r, SmallGemmArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const int S = a.stages;
+  const int nt = a.n_tok;
+  const uint32_t stage_bytes = small_stage_bytes(nt);
+  const uint32_t x_bytes = (uint32_t)nt * 128u;
+  float* upbuf = reinterpret_cast<float*>(base + (size_t)S * stage_bytes);
+  __nv_bfloat16* obuf = reinterpret_cast<__nv_bfloat16*>(upbuf + 64 * (nt + 1));
+  uint8_t* ctl = base + (size_t)S * stage_bytes + ((small_epi_bytes(nt) + 15) & ~size_t(15));
+  uint64_t* full = reinterpret_cast<uint64_t*>(ctl);
+  uint64_t* empty = full + kSmallMaxStages;
+  uint64_t* acc_full = empty + kSmallMaxStages;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int total = __ldg(&a.ts[a.G]);
+  uint32_t tmem_cols = 32;
+  while (tmem_cols < 2u * (uint32_t)nt) tmem_cols <<= 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(smem_u32(&acc_full[s]), 1);
+      mbar_init(smem_u32(&acc_empty[s]), 4);   // one arrive per epilogue warp
+    }
+    mbar_init(smem_u32(drain), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmW_s);
+    tma_prefetch_desc(&tmW_r);
+    tma_prefetch_desc(&tmX_s);
+    tma_prefetch_desc(&tmX_r);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  // tile -> (group g, weight tile m); GemmArgs-style decode with one token tile per group
+  auto decode = [&](int tile, int& g, int& m, int& e, bool& sh) {
+    while (tile >= __ldg(&a.ts[g + 1])) ++g;
+    m = tile - __ldg(&a.ts[g]);
+    sh = a.has_shared && g == 0;
+    e = g - a.has_shared;
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0, g = 0;
+      uint32_t phase = 0, issued = 0, last_par = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        int m, e;
+        bool sh;
+        decode(tile, g, m, e, sh);
+        const int xrow = __ldg(&a.grp_row[g]);
+        const int kbn = sh ? a.kb_shared : a.kb_routed;
+        for (int kb = 0; kb < kbn; ++kb) {
+          ok = mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, a.err, kErrWaitProducer);
+          if (!ok) break;
+          const uint32_t sa = smem_u32(base + (size_t)stage * stage_bytes);
+          const uint32_t fb = smem_u32(&full[stage]);
+          mbar_arrive_expect_tx(fb, kSmallBM * 128u + x_bytes);
+          if (sh) {
+            tma_load_2d(sa, &tmW_s, fb, kb * 64, m * kSmallBM);
+            tma_load_2d(sa + kSmallBM * 128u, &tmX_s, fb, kb * 64, 0);
+          } else {
+            tma_load_3d(sa, &tmW_r, fb, kb * 64, m * kSmallBM, e);
+            tma_load_2d(sa + kSmallBM * 128u, &tmX_r, fb, kb * 64, xrow);
+          }
+          issued |= 1u << stage;
+          last_par = (last_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == S) { stage = 0; phase ^= 1u; }
+        }
+      }
+      for (int s = 0; s < S; ++s)
+        if (issued & (1u << s))
+          mbar_wait(smem_u32(&full[s]), (last_par >> s) & 1u, abort_flag, a.err, kErrWaitDrain);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(kSmallBM, nt);
+      int stage = 0, g = 0, it = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++it) {
+        int m, e;
+        bool sh;
+        decode(tile, g, m, e, sh);
+        const int kbn = sh ? a.kb_shared : a.kb_routed;
+        const int acc = it & 1;
+        const uint32_t acc_par = (it >> 1) & 1;
+        ok = mbar_wait(smem_u32(&acc_empty[acc]), acc_par ^ 1u, abort_flag, a.err, kErrWaitMma);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t dt = tmem_base + (uint32_t)(acc * nt);
+        for (int kb = 0; kb < kbn; ++kb) {
+          ok = mbar_wait(smem_u32(&full[stage]), phase, abort_flag, a.err, kErrWaitMma);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t sa = smem_u32(base + (size_t)stage * stage_bytes);
+          const uint64_t adesc = sdesc_k_sw128(sa), bdesc = sdesc_k_sw128(sa + kSmallBM * 128u);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            tc_mma_f16(dt, adesc + 2u * k, bdesc + 2u * k, idesc, (kb | k) != 0);
+          tc_commit(smem_u32(&empty[stage]));
+          if (++stage == S) { stage = 0; phase ^= 1u; }
+        }
+        if (ok) tc_commit(smem_u32(&acc_full[acc]));
+      }
+      tc_commit(smem_u32(drain));
+      mbar_wait(smem_u32(drain), 0, abort_flag, a.err, kErrWaitDrain);
+    }
+    __syncwarp();
+  } else {
+    const int q = warp & 3;              // TMEM lane quadrant
+    const int L = q * 32 + lane;         // TMEM lane = weight row of the tile
+    const int et = threadIdx.x - 64;     // 0..127
+    int g = 0, it = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+      int m, e;
+      bool sh;
+      decode(tile, g, m, e, sh);
+      const int acc = it & 1;
+      const uint32_t acc_par = (it >> 1) & 1;
+      bool ok = true;
+      if (et == 0) ok = mbar_wait(smem_u32(&acc_full[acc]), acc_par, abort_flag, a.err, kErrWaitEpilogue);
+      if (named_bar_any(2, 128, !ok)) break;
+      tc_fence_after();
+      const uint32_t trow = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + (uint32_t)(acc * nt);
+      const int rows = sh ? a.T : __ldg(&a.counts[e]);
+      const int64_t row0 = __ldg(&a.grp_row[g]);
+      __nv_bfloat16* out = sh ? a.out_shared : a.out_routed;
+      const int64_t ld = sh ? a.ld_shared : a.ld_routed;
+      if (MODE == kGateUpSwiGLU) {
+        if (L >= 64) {   // up rows: park them in shared memory for their gate partners
+          for (int c = 0; c < nt; c += 16) {
+            uint32_t v[16];
+            __syncwarp();
+            tmem_ld16(trow + (uint32_t)c, v);
+            tmem_ld_wait16(v);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) upbuf[(L - 64) * (nt + 1) + c + j] = __uint_as_float(v[j]);
+          }
+        }
+        named_bar_sync(2, 128);
+        if (L < 64) {    // gate rows: SiLU(gate) * up, token-major into the output tile
+          for (int c = 0; c < nt; c += 16) {
+            uint32_t v[16];
+            __syncwarp();
+            tmem_ld16(trow + (uint32_t)c, v);
+            tmem_ld_wait16(v);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const float h = silu_fast(__uint_as_float(v[j])) * upbuf[L * (nt + 1) + c + j];
+              obuf[(size_t)(c + j) * 64 + L] = __float2bfloat16_rn(h);
+            }
+          }
+        }
+        tc_fence_before();
+        named_bar_sync(2, 128);
+        // rows of 64 outputs (128 B = 8 vectors) per token
+        const int col0 = m * 64;
+        for (int idx = et; idx < rows * 8; idx += 128) {
+          const int n = idx >> 3, v8 = idx & 7;
+          *reinterpret_cast<uint4*>(out + (row0 + n) * ld + col0 + v8 * 8) =
+              *reinterpret_cast<const uint4*>(obuf + (size_t)n * 64 + v8 * 8);
+        }
+      } else {
+        for (int c = 0; c < nt; c += 16) {
+          uint32_t v[16];
+          __syncwarp();
+          tmem_ld16(trow + (uint32_t)c, v);
+          tmem_ld_wait16(v);
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            obuf[(size_t)(c + j) * kSmallBM + L] = __float2bfloat16_rn(__uint_as_float(v[j]));
+        }
+        tc_fence_before();
+        named_bar_sync(2, 128);
+        // rows of 128 outputs (256 B = 16 vectors) per token
+        const int col0 = m * kSmallBM;
+        for (int idx = et; idx < rows * 16; idx += 128) {
+          const int n = idx >> 4, v16 = idx & 15;
+          *reinterpret_cast<uint4*>(out + (row0 + n) * ld + col0 + v16 * 8) =
+              *reinterpret_cast<const uint4*>(obuf + (size_t)n * kSmallBM + v16 * 8);
+        }
+      }
+      named_bar_sync(2, 128);   // output tile and up buffer are reused by the next tile
+      if (lane == 0) mbar_arrive(smem_u32(&acc_empty[acc]));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, tmem_cols);
+  }
+}
+
+}  // namespace moe

@@ -18,6 +18,7 @@
 #include "moe.h"
 #include "combine.cuh"
 #include "gemm_simt.cuh"
+#include "gemm_small.cuh"
 #include "gemm_tc.cuh"
 #include "router.cuh"
 #include "scan_permute.cuh"
@@ -130,8 +131,12 @@ struct moe_handle {
   int n_tiles = 0;         // router tiles
   int router_rows = 0;     // tokens per router tile
   int64_t T_pad = 0, rows_cap = 0;   // padded to bm, the GEMM row tile
-  int bm = 0;
+  int bm = 0, tile_rows = 0;
   int gemm_grid = 0;                  // CTAs of the paired-SM GEMMs (2 per cluster)
+  // small-batch (decode) path: token counts <= n_tok, weights on the MMA's M dimension
+  bool small = false;
+  int n_tok = 0, small_stages = 0;
+  size_t small_smem = 0;
   int n_pad = 0, maxk = 16;
   int router_stages = 0;
   uint32_t router_tmem_cols = 0;
@@ -156,6 +161,7 @@ struct moe_handle {
   int32_t *idx_dev = nullptr, *cnt_dev = nullptr;
   float *w_dev = nullptr, *aux_dev = nullptr;
   CUtensorMap tmE, tmXp, tmWguS, tmWguR, tmHs, tmHr, tmWdS, tmWdR;
+  CUtensorMap tmXpN, tmHsN, tmHrN;   // token operands of the small-batch GEMMs (n_tok rows)
   // per-kernel timing (moe_timing_begin / moe_timing_end)
   std::vector<cudaEvent_t> events;   // kKernelsPerForward + 1 per recorded call
   int timing_cap = 0, timing_used = 0;
@@ -267,10 +273,14 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
     H->router_rows = kRouterBM;
   }
   H->n_tiles = (c.T + H->router_rows - 1) / H->router_rows;
-  H->bm = H->bf16 ? kPairBM : kSimtBM;
-  H->T_pad = ((int64_t)c.T + H->bm - 1) / H->bm * H->bm;
+  H->small = H->bf16 && c.T <= kSmallMaxTok && c.d % kSmallBM == 0;
+  H->n_tok = (c.T + 15) / 16 * 16;
+  H->bm = H->small ? 1 : (H->bf16 ? kPairBM : kSimtBM);
+  H->tile_rows = H->small ? 0 : H->bm;
+  H->T_pad = H->small ? H->n_tok : ((int64_t)c.T + H->bm - 1) / H->bm * H->bm;
   H->rows_cap = ((int64_t)c.T * c.top_k + (int64_t)c.n_routed * (H->bm - 1) + H->bm - 1) /
                 H->bm * H->bm;
+  if (H->small) H->rows_cap = ((int64_t)c.T * c.top_k + 15) / 16 * 16;
   H->n_pad = (c.n_routed + 15) / 16 * 16;
   H->maxk = router_maxk(c.top_k);
   const size_t es = H->es;
@@ -393,6 +403,7 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
       if (clusters < 1) return fail(MOE_ERR_UNSUPPORTED, "no CTA pair of the GEMM kernel fits on this device");
       H->gemm_grid = 2 * clusters;
     }
+
     bool ok = encode_2d(&H->tmE, H->centroids, d, (uint64_t)H->n_pad, (uint32_t)H->n_pad) &&
               encode_2d(&H->tmXp, H->xp, d, rc, 128) &&
               encode_3d(&H->tmWguR, H->w_gu_r, d, 2 * I, nr, kGemmBN / 2) &&
@@ -408,6 +419,23 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
       H->tmWdS = H->tmWdR;
     }
     if (!ok) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for a weight/workspace tensor");
+    if (H->small) {
+      const size_t epi = (small_epi_bytes(H->n_tok) + 15) & ~size_t(15);
+      const uint32_t sb = small_stage_bytes(H->n_tok);
+      int stages = (int)((200u * 1024u - epi) / sb);
+      stages = stages > kSmallMaxStages ? kSmallMaxStages : (stages < 2 ? 2 : stages);
+      H->small_stages = stages;
+      H->small_smem = 1024 + (size_t)stages * sb + epi + 256;
+      MOE_CUDA(cudaFuncSetAttribute((const void*)grouped_gemm_small_kernel<kGateUpSwiGLU>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)H->small_smem));
+      MOE_CUDA(cudaFuncSetAttribute((const void*)grouped_gemm_small_kernel<kDown>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)H->small_smem));
+      bool okn = encode_2d(&H->tmXpN, H->xp, d, rc, (uint32_t)H->n_tok) &&
+           encode_2d(&H->tmHrN, H->hr, I, rc, (uint32_t)H->n_tok);
+      if (ks) okn = okn && encode_2d(&H->tmHsN, H->hs, Is, tp, (uint32_t)H->n_tok);
+      else H->tmHsN = H->tmHrN;
+      if (!okn) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for a small-batch operand");
+    }
   } else {
     H->simt_router_smem = router_epi_bytes(c.n_routed, H->maxk) +
                           (size_t)kRouterBM * router_row_ld(c.n_routed) * 4;
@@ -476,10 +504,11 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
   }
   MOE_CUDA(cudaGetLastError());
 
-  const int bn1 = H->bf16 ? kGemmBN / 2 : kSimtBN;
-  const int bn2 = H->bf16 ? kGemmBN : kSimtBN;
+  const int bn1 = H->small ? 64 : (H->bf16 ? kGemmBN / 2 : kSimtBN);
+  const int bn2 = H->small ? kSmallBM : (H->bf16 ? kGemmBN : kSimtBN);
   ScanArgs sa{H->tile_hist, H->tile_psum, H->n_tiles, nr, T, H->has_shared, H->inter_shared,
-              c.inter, d, H->bm, bn1, bn2, c.alpha1, expert_counts, aux_loss, H->psum_total,
+              c.inter, d, H->bm, H->tile_rows, bn1, bn2, c.alpha1, expert_counts, aux_loss,
+              H->psum_total,
               H->tile_base, H->grp_row, H->ts1, H->ts2};
   tick(H, stream, 1);
   scan_kernel<<<1, kScanThreads, 0, stream>>>(sa);
@@ -493,7 +522,33 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
   MOE_CUDA(cudaGetLastError());
 
   const int I = c.inter, Is = H->inter_shared;
-  if (H->bf16) {
+  if (H->small) {
+    CUtensorMap tmUN;   // token rows of the shared group, n_tok per tile
+    if (!encode_2d(&tmUN, u, d, T, (uint32_t)H->n_tok))
+      return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for u");
+    SmallGemmArgs s1{};
+    s1.grp_row = H->grp_row; s1.ts = H->ts1; s1.counts = expert_counts; s1.G = H->G;
+    s1.has_shared = H->has_shared; s1.T = T; s1.n_tok = H->n_tok; s1.stages = H->small_stages;
+    s1.kb_shared = d / 64; s1.kb_routed = d / 64;
+    s1.mt_shared = Is / 64; s1.mt_routed = I / 64;
+    s1.out_shared = static_cast<__nv_bfloat16*>(H->hs); s1.ld_shared = Is;
+    s1.out_routed = static_cast<__nv_bfloat16*>(H->hr); s1.ld_routed = I;
+    s1.err = H->err;
+    tick(H, stream, 3);
+    grouped_gemm_small_kernel<kGateUpSwiGLU><<<H->n_sms, kSmallThreads, H->small_smem, stream>>>(
+        H->tmWguS, H->tmWguR, tmUN, H->tmXpN, s1);
+    MOE_CUDA(cudaGetLastError());
+    SmallGemmArgs s2 = s1;
+    s2.ts = H->ts2;
+    s2.kb_shared = Is / 64; s2.kb_routed = I / 64;
+    s2.mt_shared = d / kSmallBM; s2.mt_routed = d / kSmallBM;
+    s2.out_shared = static_cast<__nv_bfloat16*>(H->ys); s2.ld_shared = d;
+    s2.out_routed = static_cast<__nv_bfloat16*>(H->yr); s2.ld_routed = d;
+    tick(H, stream, 4);
+    grouped_gemm_small_kernel<kDown><<<H->n_sms, kSmallThreads, H->small_smem, stream>>>(
+        H->tmWdS, H->tmWdR, H->tmHsN, H->tmHrN, s2);
+    MOE_CUDA(cudaGetLastError());
+  } else if (H->bf16) {
     GemmArgs g1{};
     g1.grp_row = H->grp_row; g1.ts = H->ts1; g1.G = H->G; g1.has_shared = H->has_shared;
     g1.kb_shared = d / kGemmBK; g1.kb_routed = d / kGemmBK;
@@ -520,18 +575,6 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
     tick(H, stream, 4);
     grouped_gemm_tc_kernel<kDown><<<H->gemm_grid, kGemmThreads, kGemmSmemBytes, stream>>>(
         H->tmHs, H->tmHr, H->tmWdS, H->tmWdR, g2);
-    MOE_CUDA(cudaGetLastError());
-
-    CombineArgs<__nv_bfloat16> ca{static_cast<const __nv_bfloat16*>(u),
-                                  static_cast<const __nv_bfloat16*>(H->ys),
-                                  static_cast<const __nv_bfloat16*>(H->yr), H->slot_row, topk_w,
-                                  static_cast<__nv_bfloat16*>(h), T, d, K};
-    tick(H, stream, 5);
-    const int cgrid = (T + kCombineWarps - 1) / kCombineWarps;
-    with_maxk(H->maxk, [&](auto m) {
-      combine_bf16_kernel<m()><<<cgrid, kCombineWarps * 32, 0, stream>>>(ca);
-      return 0;
-    });
     MOE_CUDA(cudaGetLastError());
   } else {
     const size_t ks = c.n_shared;
@@ -577,6 +620,19 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
                           static_cast<float*>(h), T, d, K};
     tick(H, stream, 5);
     combine_f32_kernel<<<(T + kCombineWarps - 1) / kCombineWarps, kCombineWarps * 32, 0, stream>>>(ca);
+    MOE_CUDA(cudaGetLastError());
+  }
+  if (H->bf16) {
+    CombineArgs<__nv_bfloat16> ca{static_cast<const __nv_bfloat16*>(u),
+                                  static_cast<const __nv_bfloat16*>(H->ys),
+                                  static_cast<const __nv_bfloat16*>(H->yr), H->slot_row, topk_w,
+                                  static_cast<__nv_bfloat16*>(h), T, d, K};
+    tick(H, stream, 5);
+    const int cgrid = (T + kCombineWarps - 1) / kCombineWarps;
+    with_maxk(H->maxk, [&](auto m) {
+      combine_bf16_kernel<m()><<<cgrid, kCombineWarps * 32, 0, stream>>>(ca);
+      return 0;
+    });
     MOE_CUDA(cudaGetLastError());
   }
   if (H->timing_used < H->timing_cap) {

@@ -163,7 +163,8 @@ extern "C" moe_status moe_route_noalloc(const void* u, const void* centroids, co
   if (e != cudaSuccess) return nfail(MOE_ERR_CUDA, "moe_route_noalloc: router launch failed");
 
   ScanArgs sa{ro.tile_hist, ro.tile_psum, n_tiles, n_routed, T, /*has_shared=*/0,
-              /*inter_shared=*/0, /*inter=*/64, d, /*bm=*/128, /*bn1=*/128, /*bn2=*/256, alpha1,
+              /*inter_shared=*/0, /*inter=*/64, d, /*bm=*/128, /*tile_rows=*/128, /*bn1=*/128,
+              /*bn2=*/256, alpha1,
               expert_counts,
               aux_loss, reinterpret_cast<float*>(sc + kOffPsumTot),
               reinterpret_cast<int32_t*>(sc + kOffBase), reinterpret_cast<int32_t*>(sc + kOffGrp),

@@ -22,7 +22,8 @@ struct ScanArgs {
   int n_tiles, n_routed, T;
   int has_shared;             // group 0 = all shared experts as one group
   int inter_shared, inter, d; // widths of the shared group and of a routed expert
-  int bm;                     // GEMM row tile: each group's rows are padded to it
+  int bm;                     // each group's rows are padded to a multiple of bm
+  int tile_rows;              // rows per GEMM row tile; 0 = one tile per non-empty group
   int bn1, bn2;               // output columns per tile of the gate/up and down GEMMs
   float alpha1;
   // outputs
@@ -86,14 +87,14 @@ static __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a
     const int lane = tid & 31, wid = tid >> 5;
     const int nt1 = (a.inter + a.bn1 - 1) / a.bn1;
     const int nt2 = (a.d + a.bn2 - 1) / a.bn2;
-    const int sh_mt = a.has_shared ? (a.T + a.bm - 1) / a.bm : 0;
+    const int sh_mt = !a.has_shared ? 0 : a.tile_rows > 0 ? (a.T + a.tile_rows - 1) / a.tile_rows : 1;
     const int sh_t1 = sh_mt * ((a.inter_shared + a.bn1 - 1) / a.bn1);
     const int sh_t2 = sh_mt * nt2;
     int cnt = 0, pad = 0, t1 = 0, t2 = 0;
     if (tid < nr) {
       cnt = s_off[tid];
-      const int mt = (cnt + a.bm - 1) / a.bm;
-      pad = mt * a.bm;
+      const int mt = a.tile_rows > 0 ? (cnt + a.tile_rows - 1) / a.tile_rows : (cnt > 0 ? 1 : 0);
+      pad = (cnt + a.bm - 1) / a.bm * a.bm;
       t1 = mt * nt1;
       t2 = mt * nt2;
       const double invT = 1.0 / (double)a.T;

@@ -51,6 +51,10 @@ SMALL = [
     dict(T=1, d=256, n_shared=1, n_routed=8, inter=128, top_k=2, dtype="bf16"),
     # many experts and the largest top-k
     dict(T=260, d=256, n_shared=1, n_routed=200, inter=64, top_k=16, dtype="bf16"),
+    # small-batch (weights-on-M) GEMM path: ragged token count, two shared experts
+    dict(T=100, d=256, n_shared=2, n_routed=16, inter=192, top_k=4, dtype="bf16"),
+    # small-batch path at its largest token count, many experts without tokens
+    dict(T=128, d=384, n_shared=1, n_routed=64, inter=128, top_k=6, dtype="bf16"),
     # fp32 path, ragged sizes
     dict(T=300, d=64, n_shared=2, n_routed=9, inter=48, top_k=3, dtype="fp32"),
     dict(T=1, d=32, n_shared=0, n_routed=4, inter=16, top_k=4, dtype="fp32"),
