@@ -173,7 +173,7 @@ moe_status moe_timing_end(moe_handle* handle, double* kernel_ms, int32_t* n_forw
 #define MOE_NOALLOC_MAX_TOKENS 16384
 #define MOE_NOALLOC_MAX_ROUTED 256
 #define MOE_NOALLOC_MAX_TOP_K 16
-#define MOE_NOALLOC_SCRATCH_BYTES (1536u * 1024u)
+#define MOE_NOALLOC_SCRATCH_BYTES (2048u * 1024u)
 moe_status moe_route_noalloc(const void* u, const void* centroids, const float* logit_bias,
                              int32_t T, int32_t d, int32_t n_routed, int32_t top_k, float alpha1,
                              int32_t* topk_idx, float* topk_w, int32_t* expert_counts,

@@ -13,6 +13,11 @@ namespace moe {
 
 constexpr int kCombineWarps = 8;
 
+// Compile-time bound on top_k for the per-vector load batch.
+__host__ __device__ constexpr int combine_maxk(int top_k) {
+  return top_k <= 4 ? 4 : top_k <= 6 ? 6 : top_k <= 8 ? 8 : top_k <= 12 ? 12 : 16;
+}
+
 template <typename T>
 struct CombineArgs {
   const T* u;              // [T, d]

@@ -104,7 +104,19 @@ __global__ void balance_loss_kernel(const int32_t* counts, const float* psum, in
 
 constexpr int kKernelsPerForward = 6;
 
-// Call f(std::integral_constant<int, MAXK>{}) for the compile-time list length of top_k.
+// Call f(std::integral_constant<int, MAXC>{}) for the router's columns per thread bound.
+template <class F>
+auto with_maxc(int maxc, F&& f) {
+  switch (maxc) {
+    case 2: return f(std::integral_constant<int, 2>{});
+    case 4: return f(std::integral_constant<int, 4>{});
+    case 8: return f(std::integral_constant<int, 8>{});
+    case 16: return f(std::integral_constant<int, 16>{});
+    default: return f(std::integral_constant<int, 32>{});
+  }
+}
+
+// Call f(std::integral_constant<int, MAXK>{}) for the combine's bound on top_k.
 template <class F>
 auto with_maxk(int maxk, F&& f) {
   switch (maxk) {
@@ -137,8 +149,8 @@ struct moe_handle {
   bool small = false;
   int n_tok = 0, small_stages = 0;
   size_t small_smem = 0;
-  int n_pad = 0, maxk = 16;
-  int router_stages = 0;
+  int n_pad = 0, maxk = 16, maxc = 32;
+  int router_stages = 0, router_kps = 1;
   uint32_t router_tmem_cols = 0;
   size_t router_smem = 0, simt_router_smem = 0;
   // weights (library-owned, re-laid-out)
@@ -221,8 +233,6 @@ moe_status validate(const moe_cfg* c) {
       return fail(MOE_ERR_UNSUPPORTED, "bf16 layers need d %% 64 == 0 and inter %% 64 == 0 (d=%d inter=%d)",
                   c->d, c->inter);
   } else {
-    if (c->n_routed > 128)
-      return fail(MOE_ERR_UNSUPPORTED, "fp32 layers support n_routed <= 128 (got %d)", c->n_routed);
     if (c->d % 4 || c->inter % 4)
       return fail(MOE_ERR_UNSUPPORTED, "fp32 layers need d %% 4 == 0 and inter %% 4 == 0 (d=%d inter=%d)",
                   c->d, c->inter);
@@ -265,13 +275,7 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
   H->has_shared = c.n_shared > 0 ? 1 : 0;
   H->inter_shared = c.n_shared * c.inter;
   H->G = H->has_shared + c.n_routed;
-  if (H->bf16) {
-    // tiles of R <= 128 tokens (a multiple of 8) so that the router covers every SM
-    const int per_sm = (c.T + H->n_sms - 1) / H->n_sms;
-    H->router_rows = per_sm >= kRouterBM ? kRouterBM : ((per_sm + 7) / 8) * 8;
-  } else {
-    H->router_rows = kRouterBM;
-  }
+  H->router_rows = H->bf16 ? router_tile_rows(c.T, H->n_sms) : kRouterPass;
   H->n_tiles = (c.T + H->router_rows - 1) / H->router_rows;
   H->small = H->bf16 && c.T <= kSmallMaxTok && c.d % kSmallBM == 0;
   H->n_tok = (c.T + 15) / 16 * 16;
@@ -282,7 +286,8 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
                 H->bm * H->bm;
   if (H->small) H->rows_cap = ((int64_t)c.T * c.top_k + 15) / 16 * 16;
   H->n_pad = (c.n_routed + 15) / 16 * 16;
-  H->maxk = router_maxk(c.top_k);
+  H->maxk = combine_maxk(c.top_k);
+  H->maxc = router_maxc(H->n_pad);
   const size_t es = H->es;
   const size_t d = c.d, I = c.inter, Is = H->inter_shared, nr = c.n_routed, ks = c.n_shared;
 
@@ -367,18 +372,15 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
 
   // ---- kernels' launch attributes and TMA descriptors
   if (H->bf16) {
-    const uint32_t stage_bytes = router_stage_bytes(H->n_pad);
-    int stages = (int)((200u * 1024u) / stage_bytes);
-    if (stages > kRouterMaxStages) stages = kRouterMaxStages;
-    if (stages < 2) stages = 2;
-    H->router_stages = stages;
-    H->router_smem = 1024 + (size_t)stages * stage_bytes + 256;
-    if ((size_t)stages * stage_bytes < router_epi_bytes(c.n_routed, H->maxk))
-      return fail(MOE_ERR_UNSUPPORTED, "router epilogue scratch does not fit");
+    const RouterStages rs = router_stages(H->n_pad, H->router_rows);
+    if (rs.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "router stages do not fit in shared memory");
+    H->router_kps = rs.kps;
+    H->router_stages = rs.stages;
+    H->router_smem = router_smem_bytes(H->n_pad, rs.kps, H->router_rows, rs.stages);
     uint32_t cols = 32;
-    while (cols < (uint32_t)H->n_pad) cols <<= 1;
+    while (cols < 2u * (uint32_t)H->n_pad) cols <<= 1;
     H->router_tmem_cols = cols;
-    const void* rk = with_maxk(H->maxk, [](auto m) { return (const void*)router_tc_kernel<m()>; });
+    const void* rk = with_maxc(H->maxc, [](auto m) { return (const void*)router_tc_kernel<m()>; });
     MOE_CUDA(cudaFuncSetAttribute(rk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)H->router_smem));
     MOE_CUDA(cudaFuncSetAttribute((const void*)grouped_gemm_tc_kernel<kGateUpSwiGLU>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmemBytes));
@@ -437,9 +439,8 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
       if (!okn) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for a small-batch operand");
     }
   } else {
-    H->simt_router_smem = router_epi_bytes(c.n_routed, H->maxk) +
-                          (size_t)kRouterBM * router_row_ld(c.n_routed) * 4;
-    const void* rk = with_maxk(H->maxk, [](auto m) { return (const void*)router_simt_kernel<m()>; });
+    H->simt_router_smem = router_epi_bytes(H->n_pad);
+    const void* rk = with_maxc(H->maxc, [](auto m) { return (const void*)router_simt_kernel<m()>; });
     MOE_CUDA(cudaFuncSetAttribute(rk, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)H->simt_router_smem));
   }
@@ -488,16 +489,17 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
   if (H->bf16) {
     if (!encode_2d(&tmU, u, d, T, 128) || !encode_2d(&tmUr, u, d, T, (uint32_t)H->router_rows))
       return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for u");
-    RouterTcArgs ra{T, d, nr, H->n_pad, K, H->router_stages, H->router_rows,
+    RouterTcArgs ra{T, d, nr, H->n_pad, K, H->router_kps, H->router_stages, H->router_rows, H->n_tiles,
                     H->router_tmem_cols, H->bias, ro};
-    with_maxk(H->maxk, [&](auto m) {
-      router_tc_kernel<m()><<<H->n_tiles, kRouterThreads, H->router_smem, stream>>>(tmUr, H->tmE, ra);
+    const int rgrid = H->n_tiles < H->n_sms ? H->n_tiles : H->n_sms;
+    with_maxc(H->maxc, [&](auto m) {
+      router_tc_kernel<m()><<<rgrid, kRouterThreads, H->router_smem, stream>>>(tmUr, H->tmE, ra);
       return 0;
     });
   } else {
     RouterSimtArgs ra{static_cast<const float*>(u), static_cast<const float*>(H->centroids), H->bias,
                       T, d, nr, K, ro};
-    with_maxk(H->maxk, [&](auto m) {
+    with_maxc(H->maxc, [&](auto m) {
       router_simt_kernel<m()><<<H->n_tiles, kRouterEpiThreads, H->simt_router_smem, stream>>>(ra);
       return 0;
     });

@@ -15,7 +15,9 @@ using namespace moe;
 
 namespace {
 
-constexpr int kNoAllocTiles = MOE_NOALLOC_MAX_TOKENS / kRouterBM;
+// router tiles: the tiling moe_forward uses, or tiles of 128 tokens where that would need more
+constexpr int kNoAllocTiles = 320;
+static_assert(kNoAllocTiles * kRouterBM >= MOE_NOALLOC_MAX_TOKENS, "tiles of 128 must fit");
 // byte offsets inside the scratch array
 constexpr size_t kOffRank = 0;                                                      // [T, top_k] i32
 constexpr size_t kOffHist = kOffRank + (size_t)MOE_NOALLOC_MAX_TOKENS * kMaxTopK * 4;  // [tiles, N_r] i32
@@ -51,7 +53,7 @@ struct DeviceSetup {
   std::once_flag once;
   unsigned char* scratch = nullptr;   // device address of g_noalloc_scratch on this device
   cudaError_t status = cudaSuccess;
-  int sm_major = 0, sm_minor = 0;
+  int sm_major = 0, sm_minor = 0, n_sms = 0;
 };
 DeviceSetup g_setup[64];
 
@@ -79,13 +81,13 @@ bool encode_rows(CUtensorMap* m, const void* ptr, uint64_t d, uint64_t rows, uin
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int MAXK>
+template <int MAXC>
 cudaError_t launch_router(const CUtensorMap& tmU, const CUtensorMap& tmE, const RouterTcArgs& ra,
-                          int n_tiles, size_t smem, cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute((const void*)router_tc_kernel<MAXK>,
+                          int grid, size_t smem, cudaStream_t st) {
+  cudaError_t e = cudaFuncSetAttribute((const void*)router_tc_kernel<MAXC>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  router_tc_kernel<MAXK><<<n_tiles, kRouterThreads, smem, st>>>(tmU, tmE, ra);
+  router_tc_kernel<MAXC><<<grid, kRouterThreads, smem, st>>>(tmU, tmE, ra);
   return cudaGetLastError();
 }
 
@@ -120,6 +122,8 @@ extern "C" moe_status moe_route_noalloc(const void* u, const void* centroids, co
     if (S.status == cudaSuccess)
       S.status = cudaDeviceGetAttribute(&S.sm_minor, cudaDevAttrComputeCapabilityMinor, dev);
     if (S.status == cudaSuccess)
+      S.status = cudaDeviceGetAttribute(&S.n_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (S.status == cudaSuccess)
       S.status = cudaGetSymbolAddress(reinterpret_cast<void**>(&S.scratch), g_noalloc_scratch);
   });
   if (S.status != cudaSuccess || !S.scratch)
@@ -137,29 +141,29 @@ extern "C" moe_status moe_route_noalloc(const void* u, const void* centroids, co
     return nfail(MOE_ERR_CUDA, "moe_route_noalloc: cudaMemsetAsync on the scratch failed");
 
   const int n_pad = (n_routed + 15) / 16 * 16;
-  const int n_tiles = (T + kRouterBM - 1) / kRouterBM;
+  int rows = router_tile_rows(T, S.n_sms);
+  if ((T + rows - 1) / rows > kNoAllocTiles) rows = kRouterBM;
+  const int n_tiles = (T + rows - 1) / rows;
   CUtensorMap tmU, tmE;
-  if (!encode_rows(&tmU, u, d, T, kRouterBM) || !encode_rows(&tmE, centroids, d, n_routed, n_pad))
+  if (!encode_rows(&tmU, u, d, T, (uint32_t)rows) || !encode_rows(&tmE, centroids, d, n_routed, n_pad))
     return nfail(MOE_ERR_CUDA, "moe_route_noalloc: cuTensorMapEncodeTiled failed");
-  const uint32_t stage_bytes = router_stage_bytes(n_pad);
-  int stages = (int)((200u * 1024u) / stage_bytes);
-  stages = stages > kRouterMaxStages ? kRouterMaxStages : (stages < 2 ? 2 : stages);
-  const size_t smem = 1024 + (size_t)stages * stage_bytes + 256;
+  const RouterStages rs = router_stages(n_pad, rows);
+  if (rs.stages < 2) return nfail(MOE_ERR_UNSUPPORTED, "moe_route_noalloc: router stages do not fit");
+  const size_t smem = router_smem_bytes(n_pad, rs.kps, rows, rs.stages);
   uint32_t cols = 32;
-  while (cols < (uint32_t)n_pad) cols <<= 1;
+  while (cols < 2u * (uint32_t)n_pad) cols <<= 1;
 
   RouterOut ro{topk_idx, topk_w, reinterpret_cast<int32_t*>(sc + kOffRank),
                reinterpret_cast<int32_t*>(sc + kOffHist), reinterpret_cast<float*>(sc + kOffPsum), err};
-  if ((size_t)stages * stage_bytes < router_epi_bytes(n_routed, router_maxk(top_k)))
-    return nfail(MOE_ERR_UNSUPPORTED, "moe_route_noalloc: router scratch does not fit");
-  RouterTcArgs ra{T, d, n_routed, n_pad, top_k, stages, kRouterBM, cols,
+  RouterTcArgs ra{T, d, n_routed, n_pad, top_k, rs.kps, rs.stages, rows, n_tiles, cols,
                   logit_bias ? logit_bias : zero_bias, ro};
-  const int mk = router_maxk(top_k);
-  cudaError_t e = mk == 4 ? launch_router<4>(tmU, tmE, ra, n_tiles, smem, st)
-                 : mk == 6 ? launch_router<6>(tmU, tmE, ra, n_tiles, smem, st)
-                 : mk == 8 ? launch_router<8>(tmU, tmE, ra, n_tiles, smem, st)
-                 : mk == 12 ? launch_router<12>(tmU, tmE, ra, n_tiles, smem, st)
-                            : launch_router<16>(tmU, tmE, ra, n_tiles, smem, st);
+  const int grid = n_tiles < S.n_sms ? n_tiles : S.n_sms;
+  const int mc = router_maxc(n_pad);
+  cudaError_t e = mc == 2 ? launch_router<2>(tmU, tmE, ra, grid, smem, st)
+                 : mc == 4 ? launch_router<4>(tmU, tmE, ra, grid, smem, st)
+                 : mc == 8 ? launch_router<8>(tmU, tmE, ra, grid, smem, st)
+                 : mc == 16 ? launch_router<16>(tmU, tmE, ra, grid, smem, st)
+                            : launch_router<32>(tmU, tmE, ra, grid, smem, st);
   if (e != cudaSuccess) return nfail(MOE_ERR_CUDA, "moe_route_noalloc: router launch failed");
 
   ScanArgs sa{ro.tile_hist, ro.tile_psum, n_tiles, n_routed, T, /*has_shared=*/0,

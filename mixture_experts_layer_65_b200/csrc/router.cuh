@@ -8,13 +8,19 @@
 // renormalised, stable ranking (equal logits -> lower index first); "Expert-level balance
 // loss": counts and mean affinities per routed expert.
 //
-// One CTA handles a tile of R <= 128 tokens (R is chosen so the tiles cover all SMs).
-// The bf16 kernel computes the 128 x N_pad logit tile with tcgen05.mma into tensor memory
-// (A = the tile's token rows streamed by TMA, B = the padded centroid matrix; rows past R
-// are never read back).  Sixteen epilogue warps then share the rows: four threads per
-// token row (one per 16-column slice modulo 4), which reduce their partial maxima, sums
-// and top-k lists through shared memory.  The fp32 kernel computes the same logits with
-// FMA and shares the epilogue.
+// Tiles of R <= 128 tokens, as many as there are SMs, so that each SM streams the centroid
+// matrix once per tile and issues the fewest MMAs: at the layer sizes of interest the
+// tile loads run close to HBM bandwidth and the per-instruction MMA cost does not shrink
+// below N = 256, so smaller tiles only add centroid traffic and MMA instructions.  The bf16
+// kernel computes the 128 x N_pad logit tile with tcgen05.mma into one of two
+// tensor-memory accumulators (A = the tile's token rows streamed by TMA, B = the padded
+// centroid matrix; accumulator rows past R are never read back); a CTA with several tiles
+// (large T) overlaps the next tile's loads with the epilogue.  Sixteen epilogue warps copy
+// the logits (+ bias) to shared memory in passes of 64 rows and work on each pass with
+// eight threads per token row: row max and softmax denominator by shuffles, the top-k by
+// a bitonic sort of each thread's keys and three bitonic merges across the row's threads
+// (or, for top_k > 8 or wide rows, top_k rounds of a group-wide maximum).  The fp32 kernel
+// computes the same logits with FMA into the same shared-memory layout and shares the rest.
 #pragma once
 
 #include <climits>
@@ -25,10 +31,14 @@ namespace moe {
 
 constexpr int kMaxTopK = 16;
 constexpr int kMaxRouted = 256;
-constexpr int kRouterBM = 128;          // MMA rows (and the largest token tile)
-constexpr int kRouterEpiThreads = 512;  // 4 threads per row
+constexpr int kRouterBM = 128;          // MMA rows = largest token tile
+constexpr int kRouterPass = 64;         // token rows per epilogue pass
+constexpr int kRouterGroup = 8;         // threads per token row in the epilogue
+constexpr int kRouterEpiThreads = 512;  // kRouterPass * kRouterGroup
 constexpr int kRouterThreads = 64 + kRouterEpiThreads;   // warp 0 TMA, warp 1 MMA
 constexpr int kRouterMaxStages = 8;
+constexpr size_t kRouterSmemBudget = 232448;   // opt-in dynamic shared memory per block
+constexpr size_t kRouterCtlBytes = 512;        // mbarriers, TMEM slot, abort flag
 
 struct RouterOut {
   int32_t* topk_idx;    // [T, top_k]
@@ -40,30 +50,35 @@ struct RouterOut {
 };
 
 struct RouterEpiSmem {
-  uint32_t mask[kMaxRouted][4];   // bit r of mask[e][r/32]: token r of the tile chose e
   float bias[kMaxRouted];
-  float ppart[4][kMaxRouted];     // per-expert sums over 32-row quarters of the tile
-  float inv_sum[kRouterBM];       // 1 / softmax denominator per row (0 for rows past T)
-  float rowmax[kRouterBM];
-  float maxpart[4][kRouterBM];    // [sub][row]: lanes of a warp hit consecutive banks
-  float sumpart[4][kRouterBM];
+  uint32_t mask[kMaxRouted][4];            // bit r of mask[e][r/32]: token r of the tile chose e
+  int32_t sel[kRouterBM][kMaxTopK];        // chosen experts of each row, in rank order
+  float gsel[kRouterBM][kMaxTopK];         // their gates s[t, e]
+  float inv_sum[kRouterPass];              // 1 / softmax denominator (0 for rows past T)
+  float ppart[8][kMaxRouted];              // per-expert sums over row parts of the tile
 };
 
-// Epilogue scratch: RouterEpiSmem, then one region that first holds the per-thread top-k
-// lists [4][MAXK][128] (u64, row fastest) and then the exp(l - max) rows [128][ld] (fp32).
-__host__ __device__ constexpr int router_row_ld(int n_routed) { return ((n_routed + 31) & ~31) + 1; }
-__host__ __device__ constexpr size_t router_region_bytes(int n_routed, int maxk) {
-  return (size_t)kRouterBM * router_row_ld(n_routed) * 4 > (size_t)kRouterBM * 4 * maxk * 8
-             ? (size_t)kRouterBM * router_row_ld(n_routed) * 4
-             : (size_t)kRouterBM * 4 * maxk * 8;
+// Epilogue scratch: RouterEpiSmem, then the logit rows of one pass lg[64][ld] (fp32, bias
+// added), overwritten in place by exp(l - max).  ld = N_pad + 4 keeps the float4 row
+// stores of a warp and the eight-thread row reads free of bank conflicts.
+__host__ __device__ constexpr int router_ld(int n_pad) { return n_pad + 4; }
+__host__ __device__ constexpr size_t router_epi_bytes(int n_pad) {
+  return sizeof(RouterEpiSmem) + (size_t)kRouterPass * router_ld(n_pad) * 4;
 }
-__host__ __device__ constexpr size_t router_epi_bytes(int n_routed, int maxk) {
-  return sizeof(RouterEpiSmem) + router_region_bytes(n_routed, maxk);
+// Columns per epilogue thread, N_pad / 8, rounded up to the compile-time bound.
+__host__ __device__ constexpr int router_maxc(int n_pad) {
+  return n_pad <= 16 ? 2 : n_pad <= 32 ? 4 : n_pad <= 64 ? 8 : n_pad <= 128 ? 16 : 32;
 }
-// Length of the per-thread top-k list (compile-time, so it stays in registers): the
-// insertion chain costs one 64-bit compare-exchange per slot, so it is sized tightly.
-__host__ __device__ constexpr int router_maxk(int top_k) {
-  return top_k <= 4 ? 4 : top_k <= 6 ? 6 : top_k <= 8 ? 8 : top_k <= 12 ? 12 : 16;
+// Tokens per bf16 router tile for T tokens on n_sms SMs: the fewest tiles of <= 128
+// tokens (a multiple of 8) with one tile per SM per round.
+inline int router_tile_rows(int T, int n_sms) {
+  const int per_sm = (T + n_sms - 1) / n_sms;
+  const int k = (per_sm + kRouterBM - 1) / kRouterBM;
+  return (((per_sm + k - 1) / k) + 7) / 8 * 8;
+}
+// Parts the rows of a pass are split into for the per-expert sums.
+__host__ __device__ constexpr int router_psum_parts(int n_pad) {
+  return kRouterEpiThreads / n_pad > 8 ? 8 : kRouterEpiThreads / n_pad;
 }
 
 // Total order on (logit, expert): larger logit first; on equal logits the lower index.
@@ -79,165 +94,191 @@ __device__ __forceinline__ int key_index(uint64_t key) {
   return (int)(0xFFFFFFFFu - (uint32_t)key);
 }
 
-// Epilogue of one token tile.  Thread (r, sub), r < 128, sub < 4, owns the 16-column
-// slices j == sub (mod 4) of row r.  `load16(col, v)` yields the 16 raw fp32 logits of
-// columns col..col+15 of row r (called uniformly by all 512 threads); `sync()`
-// synchronises the 512 epilogue threads.
-template <int MAXK, class Load16, class Sync>
-__device__ __forceinline__ void router_epilogue(int r, int sub, int tile, int tile_rows, int T,
-                                                int n_routed, int n_pad, int top_k,
-                                                const float* __restrict__ bias, uint8_t* epi,
-                                                const RouterOut& o, Load16 load16, Sync sync) {
-  RouterEpiSmem& S = *reinterpret_cast<RouterEpiSmem*>(epi);
-  uint8_t* region = epi + sizeof(RouterEpiSmem);
-  uint64_t* tops = reinterpret_cast<uint64_t*>(region);
-  float* rows = reinterpret_cast<float*>(region);
-  const int ld = router_row_ld(n_routed);
-  const int tid = sub * kRouterBM + r;
-  const int t = tile * tile_rows + r;
-  const bool valid = r < tile_rows && t < T;
-  const int nch = n_pad >> 4;
-
-  for (int e = tid; e < kMaxRouted; e += kRouterEpiThreads) {
-    S.mask[e][0] = 0u; S.mask[e][1] = 0u; S.mask[e][2] = 0u; S.mask[e][3] = 0u;
-    S.bias[e] = e < n_routed ? bias[e] : 0.f;
+// Descending bitonic sort of N keys held in registers.
+template <int N>
+__device__ __forceinline__ void bitonic_sort_desc(uint64_t (&k)[N]) {
+#pragma unroll
+  for (int size = 2; size <= N; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+#pragma unroll
+      for (int i = 0; i < N; ++i) {
+        const int l = i ^ stride;
+        if (l > i) {
+          const bool desc = (i & size) == 0;
+          const uint64_t x = k[i], y = k[l];
+          const bool sw = desc ? (x < y) : (x > y);
+          k[i] = sw ? y : x;
+          k[l] = sw ? x : y;
+        }
+      }
+    }
   }
-  sync();
+}
 
-  // pass 1: partial max and partial top-MAXK (64-bit keys, sorted by a compare-exchange
-  // chain in registers) over this thread's slices
-  uint64_t top[MAXK];
-#pragma unroll
-  for (int p = 0; p < MAXK; ++p) top[p] = 0ull;
+// One epilogue pass: the pass's logit rows (bias added) are in lg[r][i] for r < rows,
+// i < N_pad, and the masks are zero (first pass) or hold the earlier passes' choices.
+// Thread tid (of 512) works on row r = tid / 8 of the pass (tile row 64 * pass + r) with
+// the eight threads of its row owning consecutive column blocks of C = N_pad / 8.  Writes
+// sel/gsel/mask for its rows and adds the pass's per-expert affinity sums into ppart.
+// `sync()` synchronises the 512 threads; returns with the scratch still in use.
+template <int MAXC, class Sync>
+__device__ __forceinline__ void router_pass(int tid, int pass, int tile, int R, int T,
+                                            int n_routed, int n_pad, int top_k, uint8_t* epi,
+                                            const RouterOut& o, Sync sync) {
+  RouterEpiSmem& S = *reinterpret_cast<RouterEpiSmem*>(epi);
+  float* lg = reinterpret_cast<float*>(epi + sizeof(RouterEpiSmem));
+  const int ld = router_ld(n_pad);
+  const int r = tid >> 3, j = tid & 7;
+  const int tr = pass * kRouterPass + r;                  // row in the tile
+  const int rows = min(kRouterPass, R - pass * kRouterPass);
+  const int C = n_pad >> 3;              // even: N_pad is a multiple of 16
+  const int c0 = j * C;
+  const int t = tile * R + tr;
+  const bool valid = r < rows && t < T;
+  float* row = lg + (size_t)r * ld;
+
+  // keys and the row max; rows past the tile or past T are treated as zeros
+  uint64_t key[MAXC];
   float lmax = -INFINITY;
-  uint32_t v[16];
-  for (int j = sub; j < nch; j += 4) {
-    load16(j * 16, v);
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      const int i = j * 16 + k;
-      if (i < n_routed) {
-        const float l = __uint_as_float(v[k]) + S.bias[i];
-        lmax = fmaxf(lmax, l);
-        uint64_t key = route_key(l, i);
-        if (key > top[MAXK - 1]) {
+  for (int k = 0; k < MAXC; k += 2) {
+    float2 x = make_float2(0.f, 0.f);
+    if (k < C && valid) x = *reinterpret_cast<const float2*>(row + c0 + k);
+    const bool in0 = k < C && c0 + k < n_routed, in1 = k < C && c0 + k + 1 < n_routed;
+    key[k] = in0 ? route_key(x.x, c0 + k) : 0ull;
+    key[k + 1] = in1 ? route_key(x.y, c0 + k + 1) : 0ull;
+    if (in0) lmax = fmaxf(lmax, x.x);
+    if (in1) lmax = fmaxf(lmax, x.y);
+  }
 #pragma unroll
-          for (int p = 0; p < MAXK; ++p) {
-            const uint64_t hi = top[p] > key ? top[p] : key;
-            key = top[p] > key ? key : top[p];
-            top[p] = hi;
+  for (int m = 1; m < kRouterGroup; m <<= 1)
+    lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, m));
+
+  // exp(l - max) in place, denominator: column order within a thread, then a fixed tree
+  float part = 0.f;
+#pragma unroll
+  for (int k = 0; k < MAXC; k += 2) {
+    if (k < C) {
+      const float2 x = *reinterpret_cast<const float2*>(row + c0 + k);
+      const float e0 = (valid && c0 + k < n_routed) ? __expf(x.x - lmax) : 0.f;
+      const float e1 = (valid && c0 + k + 1 < n_routed) ? __expf(x.y - lmax) : 0.f;
+      part += e0;
+      part += e1;
+      *reinterpret_cast<float2*>(row + c0 + k) = make_float2(e0, e1);
+    }
+  }
+#pragma unroll
+  for (int m = 1; m < kRouterGroup; m <<= 1) part += __shfl_xor_sync(0xffffffffu, part, m);
+  const float inv_sum = 1.0f / part;
+  if (j == 0) S.inv_sum[r] = valid ? inv_sum : 0.f;
+  __syncwarp();   // the row's exp values (written by the eight threads of a warp) are read below
+
+  auto record = [&](int p, uint64_t g) {
+    int e = key_index(g);
+    if (e < 0 || e >= n_routed) {
+      record_error(o.err, kErrRouteIndex);
+      e = 0;
+    }
+    if (valid) {
+      S.sel[tr][p] = e;
+      S.gsel[tr][p] = row[e] * inv_sum;
+      atomicOr(&S.mask[e][tr >> 5], 1u << (tr & 31));
+    }
+  };
+
+  if (MAXC <= 8 && top_k <= 8) {
+    // sort the thread's keys (padded to 8 with zeros), then three bitonic merges with the
+    // partner threads: every thread of the row ends up with the row's 8 largest keys
+    uint64_t kk[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) kk[i] = i < MAXC ? key[i < MAXC ? i : 0] : 0ull;
+    bitonic_sort_desc<8>(kk);
+#pragma unroll
+    for (int m = 1; m < kRouterGroup; m <<= 1) {
+      uint64_t pk[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) pk[i] = __shfl_xor_sync(0xffffffffu, kk[i], m);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) kk[i] = kk[i] > pk[7 - i] ? kk[i] : pk[7 - i];   // bitonic
+#pragma unroll
+      for (int stride = 4; stride > 0; stride >>= 1) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int l = i ^ stride;
+          if (l > i) {
+            const uint64_t x = kk[i], y = kk[l];
+            kk[i] = x > y ? x : y;
+            kk[l] = x > y ? y : x;
           }
         }
       }
     }
-  }
+    // thread j of the row records rank j
+    uint64_t mine = 0ull;
 #pragma unroll
-  for (int p = 0; p < MAXK; ++p) tops[(size_t)(sub * MAXK + p) * kRouterBM + r] = top[p];
-  S.maxpart[sub][r] = lmax;
-  sync();
-
-  // row owner (sub 0): merge the four sorted lists, row max in a fixed order
-  if (sub == 0) {
-    const uint64_t* L = tops + r;    // element (s, p) at L[(s * MAXK + p) * 128]
-    int h0 = 0, h1 = 0, h2 = 0, h3 = 0;
+    for (int i = 0; i < 8; ++i) mine = i == j ? kk[i] : mine;
+    if (j < top_k) record(j, mine);
+  } else {
+    // top_k rounds: the group's largest remaining key; its owner records it and drops it
+#pragma unroll 1
+    for (int p = 0; p < top_k; ++p) {
+      uint64_t best = key[0];
 #pragma unroll
-    for (int p = 0; p < MAXK; ++p) {
-      const uint64_t a0 = h0 < MAXK ? L[(size_t)h0 * kRouterBM] : 0ull;
-      const uint64_t a1 = h1 < MAXK ? L[(size_t)(MAXK + h1) * kRouterBM] : 0ull;
-      const uint64_t a2 = h2 < MAXK ? L[(size_t)(2 * MAXK + h2) * kRouterBM] : 0ull;
-      const uint64_t a3 = h3 < MAXK ? L[(size_t)(3 * MAXK + h3) * kRouterBM] : 0ull;
-      const uint64_t m01 = a0 > a1 ? a0 : a1, m23 = a2 > a3 ? a2 : a3;
-      const uint64_t m = m01 > m23 ? m01 : m23;
-      top[p] = m;
-      if (m == a0) ++h0; else if (m == a1) ++h1; else if (m == a2) ++h2; else ++h3;
-    }
-    S.rowmax[r] = fmaxf(fmaxf(S.maxpart[0][r], S.maxpart[1][r]),
-                        fmaxf(S.maxpart[2][r], S.maxpart[3][r]));
-  }
-  sync();   // the list region is reused for the exp rows below
-
-  // pass 2: exp(l - max) into the row buffer, partial denominators in slice order
-  {
-    const float rmax = S.rowmax[r];
-    float part = 0.f;
-    float* my = rows + (size_t)r * ld;
-    for (int j = sub; j < nch; j += 4) {
-      load16(j * 16, v);
+      for (int k = 1; k < MAXC; ++k) best = key[k] > best ? key[k] : best;
+      uint64_t g = best;
 #pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        const int i = j * 16 + k;
-        if (i < n_routed) {
-          // rows past the tile hold values computed from stale shared memory: store 0
-          const float e = valid ? __expf(__uint_as_float(v[k]) + S.bias[i] - rmax) : 0.f;
-          part += e;
-          my[i] = e;
-        }
+      for (int m = 1; m < kRouterGroup; m <<= 1) {
+        const uint64_t y = __shfl_xor_sync(0xffffffffu, g, m);
+        g = y > g ? y : g;
       }
-    }
-    S.sumpart[sub][r] = part;
-  }
-  sync();
-  float inv_sum = 0.f;
-  if (sub == 0) {
-    const float sum = ((S.sumpart[0][r] + S.sumpart[1][r]) + S.sumpart[2][r]) + S.sumpart[3][r];
-    inv_sum = 1.0f / sum;
-    S.inv_sum[r] = valid ? inv_sum : 0.f;
-    if (valid) {
+      if (best == g) {   // keys are distinct (distinct indices): exactly one owner
+        record(p, g);
 #pragma unroll
-      for (int p = 0; p < MAXK; ++p) {
-        if (p < top_k) {
-          const int e = key_index(top[p]);
-          if (e >= 0 && e < n_routed) atomicOr(&S.mask[e][r >> 5], 1u << (r & 31));
-        }
+        for (int k = 0; k < MAXC; ++k) key[k] = key[k] == g ? 0ull : key[k];
       }
     }
   }
   sync();
 
-  // the tile's per-expert affinity sums: four 32-row quarters, then a fixed-order total
-  {
-    const int quarter = tid >> 7;
-    for (int c = tid & (kRouterBM - 1); c < n_routed; c += kRouterBM) {
-      float a = 0.f;
-#pragma unroll 8
-      for (int rr = quarter * 32; rr < quarter * 32 + 32; ++rr)
-        a += rows[(size_t)rr * ld + c] * S.inv_sum[rr];
-      S.ppart[quarter][c] = a;
-    }
+  // the pass's per-expert affinity sums: row parts, added to the earlier passes' parts
+  const int P = router_psum_parts(n_pad);
+  const int RP = (rows + P - 1) / P;
+  for (int idx = tid; idx < P * n_pad; idx += kRouterEpiThreads) {
+    const int pp = idx / n_pad, c = idx - pp * n_pad;
+    const int r0 = pp * RP, r1 = min(rows, r0 + RP);
+    float a = 0.f;
+    for (int rr = r0; rr < r1; ++rr) a += lg[(size_t)rr * ld + c] * S.inv_sum[rr];
+    S.ppart[pp][c] = pass == 0 ? a : S.ppart[pp][c] + a;
   }
-  sync();
+}
+
+// After every pass of the tile (and a sync): the tile's histogram and affinity sums, and
+// the routing outputs with within-tile ranks (tokens of the tile that chose e before this
+// one), written in [T, top_k] order.
+__device__ __forceinline__ void router_tile_outputs(int tid, int tile, int R, int T, int n_routed,
+                                                    int n_pad, int top_k, uint8_t* epi,
+                                                    const RouterOut& o) {
+  RouterEpiSmem& S = *reinterpret_cast<RouterEpiSmem*>(epi);
+  const int P = router_psum_parts(n_pad);
   for (int c = tid; c < n_routed; c += kRouterEpiThreads) {
-    o.tile_psum[(size_t)tile * n_routed + c] =
-        ((S.ppart[0][c] + S.ppart[1][c]) + S.ppart[2][c]) + S.ppart[3][c];
-    o.tile_hist[(size_t)tile * n_routed + c] =
-        __popc(S.mask[c][0]) + __popc(S.mask[c][1]) + __popc(S.mask[c][2]) + __popc(S.mask[c][3]);
+    float a = 0.f;
+    for (int pp = 0; pp < P; ++pp) a += S.ppart[pp][c];
+    o.tile_psum[(size_t)tile * n_routed + c] = a;
+    o.tile_hist[(size_t)tile * n_routed + c] = __popc(S.mask[c][0]) + __popc(S.mask[c][1]) +
+                                               __popc(S.mask[c][2]) + __popc(S.mask[c][3]);
   }
-
-  // outputs and within-tile ranks (tokens of the tile that chose e before this one)
-  if (sub == 0 && valid) {
-    const int q = r >> 5;
-    const uint32_t below = (1u << (r & 31)) - 1u;
-    const float* my = rows + (size_t)r * ld;
-#pragma unroll
-    for (int p = 0; p < MAXK; ++p) {
-      if (p < top_k) {
-        int e = key_index(top[p]);
-        int rank = 0;
-        float g = 0.f;
-        if (e >= 0 && e < n_routed) {
-          for (int qq = 0; qq < q; ++qq) rank += __popc(S.mask[e][qq]);
-          rank += __popc(S.mask[e][q] & below);
-          g = my[e] * inv_sum;
-        } else {
-          record_error(o.err, kErrRouteIndex);
-          e = 0;
-        }
-        const size_t at = (size_t)t * top_k + p;
-        o.topk_idx[at] = e;
-        o.topk_w[at] = g;
-        o.topk_rank[at] = rank;
-      }
-    }
+  const int rows = min(R, T - tile * R);
+  for (int idx = tid; idx < rows * top_k; idx += kRouterEpiThreads) {
+    const int tr = idx / top_k, p = idx - tr * top_k;
+    const int e = S.sel[tr][p];
+    const int q = tr >> 5;
+    int rank = __popc(S.mask[e][q] & ((1u << (tr & 31)) - 1u));
+    for (int qq = 0; qq < q; ++qq) rank += __popc(S.mask[e][qq]);
+    const size_t at = (size_t)tile * R * top_k + idx;
+    o.topk_idx[at] = e;
+    o.topk_w[at] = S.gsel[tr][p];
+    o.topk_rank[at] = rank;
   }
 }
 
@@ -264,45 +305,82 @@ __device__ __forceinline__ void tmem_ld_wait16(uint32_t (&r)[16]) {
 
 // ------------------------------------------------------------------------ bf16, tcgen05
 struct RouterTcArgs {
-  int T, d, n_routed, n_pad, top_k, stages;
-  int tile_rows;       // R: tokens per CTA (<= 128, multiple of 8); the U map's box height
-  uint32_t tmem_cols;
+  int T, d, n_routed, n_pad, top_k;
+  int kps, stages;     // k-blocks per stage (1 or 2), stages in the ring
+  int tile_rows;       // R: tokens per tile (<= 128, multiple of 8); the U map's box height
+  int n_tiles;         // tiles, handed out round-robin over the CTAs
+  uint32_t tmem_cols;  // power of two >= 2 * n_pad: two accumulators
   const float* bias;   // [>= n_routed] (zeros where no bias)
   RouterOut out;
 };
 
-// stage = A (room for 128 rows of 128 B; R are written) + B (n_pad rows of 128 B)
-__host__ __device__ constexpr uint32_t router_stage_bytes(int n_pad) {
-  return kRouterBM * 128u + (((uint32_t)n_pad * 128u + 1023u) & ~1023u);
+// A stage holds kps (1 or 2) 64-wide k-blocks: A_0 .. A_{kps-1} (the tile's R token rows of
+// 128 B, rounded up to 1 KB) then B_0 .. B_{kps-1} (n_pad centroid rows of 128 B each, also
+// rounded up).  A barrier round trip (the producer's wait on `empty`, the MMA issuer's
+// wait on `full`) costs a few hundred cycles, about as long as the four N <= 64 MMAs of
+// one k-block, so a stage carries two where three stages of that size fit.  The M = 128
+// MMA reads 128 A rows; rows R..127 fall on the next block of the same stage (or the tail
+// padding), which the same TMA batch has filled: they only produce accumulator rows that
+// are never read.
+__host__ __device__ constexpr uint32_t router_a_bytes(int R) { return ((uint32_t)R * 128u + 1023u) & ~1023u; }
+__host__ __device__ constexpr uint32_t router_b_bytes(int n_pad) { return ((uint32_t)n_pad * 128u + 1023u) & ~1023u; }
+__host__ __device__ constexpr uint32_t router_stage_bytes(int n_pad, int kps, int R) {
+  return (uint32_t)kps * (router_a_bytes(R) + router_b_bytes(n_pad)) >
+                 (uint32_t)(kps - 1) * router_a_bytes(R) + kRouterBM * 128u
+             ? (uint32_t)kps * (router_a_bytes(R) + router_b_bytes(n_pad))
+             : (uint32_t)(kps - 1) * router_a_bytes(R) + kRouterBM * 128u;
+}
+// dynamic shared memory: alignment slack, stage ring, epilogue scratch, control block
+__host__ __device__ constexpr size_t router_smem_bytes(int n_pad, int kps, int R, int stages) {
+  return 1024 + (size_t)stages * router_stage_bytes(n_pad, kps, R) + router_epi_bytes(n_pad) +
+         kRouterCtlBytes;
+}
+// Stage shape: {k-blocks per stage, stages} that fit kRouterSmemBudget; stages < 2 when
+// nothing does.
+struct RouterStages { int kps, stages; };
+inline RouterStages router_stages(int n_pad, int R) {
+  for (int kps = 2; kps >= 1; --kps) {
+    long st = ((long)kRouterSmemBudget - (long)router_smem_bytes(n_pad, kps, R, 0)) /
+              (long)router_stage_bytes(n_pad, kps, R);
+    if (st > kRouterMaxStages) st = kRouterMaxStages;
+    if (st >= 3 || kps == 1) return RouterStages{kps, (int)st};
+  }
+  return RouterStages{1, 0};
 }
 
-template <int MAXK>
+// Persistent: CTA b handles tiles b, b + gridDim.x, ...  With several tiles per CTA the
+// producer and the MMA issuer run ahead into the next tile while the epilogue warps work.
+template <int MAXC>
 __global__ void __launch_bounds__(kRouterThreads, 1)
 router_tc_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmE,
                  RouterTcArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  const uint32_t a_off = kRouterBM * 128u;                         // B's offset in a stage
-  const uint32_t a_bytes = (uint32_t)a.tile_rows * 128u;           // bytes TMA writes for A
-  const uint32_t b_bytes = static_cast<uint32_t>(a.n_pad) * 128u;
-  const uint32_t stage_bytes = router_stage_bytes(a.n_pad);
+  const uint32_t a_bytes = (uint32_t)a.tile_rows * 128u;           // bytes TMA writes per A block
+  const uint32_t b_bytes = static_cast<uint32_t>(a.n_pad) * 128u;   // per B block
+  const uint32_t a_slot = router_a_bytes(a.tile_rows);
+  const uint32_t b_slot = router_b_bytes(a.n_pad);
+  const uint32_t b_off = (uint32_t)a.kps * a_slot;                 // B_0's offset in a stage
+  const uint32_t stage_bytes = router_stage_bytes(a.n_pad, a.kps, a.tile_rows);
   const int S = a.stages;
-  uint8_t* ctl = base + (size_t)S * stage_bytes;
+  uint8_t* epi = base + (size_t)S * stage_bytes;
+  uint8_t* ctl = epi + router_epi_bytes(a.n_pad);
   uint64_t* full = reinterpret_cast<uint64_t*>(ctl);
   uint64_t* empty = full + kRouterMaxStages;
   uint64_t* acc_full = empty + kRouterMaxStages;
-  uint64_t* drain = acc_full + 1;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* drain = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tile = blockIdx.x;
   const int kblocks = a.d / 64;
+  const int ksteps = (kblocks + a.kps - 1) / a.kps;   // stages per tile
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) { mbar_init(smem_u32(&full[s]), 1); mbar_init(smem_u32(&empty[s]), 1); }
-    mbar_init(smem_u32(acc_full), 1);
+    for (int s = 0; s < 2; ++s) { mbar_init(smem_u32(&acc_full[s]), 1); mbar_init(smem_u32(&acc_empty[s]), 1); }
     mbar_init(smem_u32(drain), 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -323,15 +401,24 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant_
       int stage = 0;
       uint32_t phase = 0;
       uint32_t issued = 0, last_par = 0;
-      for (int kb = 0; kb < kblocks; ++kb) {
-        if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, a.out.err, kErrWaitProducer)) break;
-        const uint32_t sa = smem_u32(base + (size_t)stage * stage_bytes);
-        mbar_arrive_expect_tx(smem_u32(&full[stage]), a_bytes + b_bytes);
-        tma_load_2d(sa, &tmU, smem_u32(&full[stage]), kb * 64, tile * a.tile_rows);
-        tma_load_2d(sa + a_off, &tmE, smem_u32(&full[stage]), kb * 64, 0);
-        issued |= 1u << stage;
-        last_par = (last_par & ~(1u << stage)) | (phase << stage);
-        if (++stage == S) { stage = 0; phase ^= 1u; }
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < a.n_tiles && ok; tile += gridDim.x) {
+        for (int ks = 0; ks < ksteps; ++ks) {
+          ok = mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, a.out.err, kErrWaitProducer);
+          if (!ok) break;
+          const uint32_t sa = smem_u32(base + (size_t)stage * stage_bytes);
+          const int kb0 = ks * a.kps;
+          const int nk = kblocks - kb0 < a.kps ? kblocks - kb0 : a.kps;
+          mbar_arrive_expect_tx(smem_u32(&full[stage]), (uint32_t)nk * (a_bytes + b_bytes));
+          for (int j = 0; j < nk; ++j) {
+            tma_load_2d(sa + j * a_slot, &tmU, smem_u32(&full[stage]), (kb0 + j) * 64,
+                        tile * a.tile_rows);
+            tma_load_2d(sa + b_off + j * b_slot, &tmE, smem_u32(&full[stage]), (kb0 + j) * 64, 0);
+          }
+          issued |= 1u << stage;
+          last_par = (last_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == S) { stage = 0; phase ^= 1u; }
+        }
       }
       // every copy this thread started must have landed before the CTA exits
       for (int s = 0; s < S; ++s)
@@ -340,48 +427,98 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant_
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(128, a.n_pad);
-      int stage = 0;
+      const uint32_t idesc = idesc_bf16_f32(kRouterBM, a.n_pad);
+      int stage = 0, it = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int kb = 0; kb < kblocks && ok; ++kb) {
-        ok = mbar_wait(smem_u32(&full[stage]), phase, abort_flag, a.out.err, kErrWaitMma);
+      for (int tile = blockIdx.x; tile < a.n_tiles && ok; tile += gridDim.x, ++it) {
+        const int acc = it & 1;
+        ok = mbar_wait(smem_u32(&acc_empty[acc]), ((it >> 1) & 1) ^ 1u, abort_flag, a.out.err,
+                       kErrWaitMma);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t sa = smem_u32(base + (size_t)stage * stage_bytes);
-        const uint64_t adesc = sdesc_k_sw128(sa), bdesc = sdesc_k_sw128(sa + a_off);
+        const uint32_t dt = tmem_base + (uint32_t)(acc * a.n_pad);
+        for (int ks = 0; ks < ksteps; ++ks) {
+          ok = mbar_wait(smem_u32(&full[stage]), phase, abort_flag, a.out.err, kErrWaitMma);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t sa = smem_u32(base + (size_t)stage * stage_bytes);
+          const int kb0 = ks * a.kps;
+          const int nk = kblocks - kb0 < a.kps ? kblocks - kb0 : a.kps;
+          for (int j = 0; j < nk; ++j) {
+            const uint64_t adesc = sdesc_k_sw128(sa + j * a_slot);
+            const uint64_t bdesc = sdesc_k_sw128(sa + b_off + j * b_slot);
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          tc_mma_f16(tmem_base, adesc + 2u * k, bdesc + 2u * k, idesc, (kb | k) != 0);
-        tc_commit(smem_u32(&empty[stage]));
-        if (++stage == S) { stage = 0; phase ^= 1u; }
+            for (int k = 0; k < 4; ++k)
+              tc_mma_f16(dt, adesc + 2u * k, bdesc + 2u * k, idesc, (ks | j | k) != 0);
+          }
+          tc_commit(smem_u32(&empty[stage]));
+          if (++stage == S) { stage = 0; phase ^= 1u; }
+        }
+        if (ok) tc_commit(smem_u32(&acc_full[acc]));
       }
-      if (ok) tc_commit(smem_u32(acc_full));
       tc_commit(smem_u32(drain));
       mbar_wait(smem_u32(drain), 0, abort_flag, a.out.err, kErrWaitDrain);
     }
     __syncwarp();
   } else {
-    const int w = warp - 2;              // 0..15
-    const int q = warp & 3;              // TMEM lane quadrant this warp may access
-    const int sub = w >> 2;              // which slices of the row
-    const int r = q * 32 + lane;
-    // one thread polls the accumulator barrier; the others sleep in the named barrier,
-    // and all sixteen warps take the same branch (they synchronise inside it)
-    bool ok = true;
-    if (w == 0 && lane == 0)
-      ok = mbar_wait(smem_u32(acc_full), 0, abort_flag, a.out.err, kErrWaitEpilogue);
-    if (!named_bar_any(1, kRouterEpiThreads, !ok)) {
+    const int tid = threadIdx.x - 64;     // 0..511
+    const int w = warp - 2;               // 0..15
+    const int q = warp & 3;               // TMEM lane quadrant this warp may access
+    const int sub = w >> 2;               // which 16-column slices it copies
+    RouterEpiSmem& SM = *reinterpret_cast<RouterEpiSmem*>(epi);
+    float* lg = reinterpret_cast<float*>(epi + sizeof(RouterEpiSmem));
+    const int ld = router_ld(a.n_pad);
+    const int nch = a.n_pad >> 4;
+    const int npass = (a.tile_rows + kRouterPass - 1) / kRouterPass;
+    auto sync = [] { named_bar_sync(1, kRouterEpiThreads); };
+    for (int e = tid; e < kMaxRouted; e += kRouterEpiThreads)
+      SM.bias[e] = e < a.n_routed ? a.bias[e] : 0.f;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < a.n_tiles; tile += gridDim.x, ++it) {
+      const int acc = it & 1;
+      // one thread polls the accumulator barrier; the others sleep in the named barrier,
+      // and all sixteen warps take the same branch (they synchronise inside it)
+      bool ok = true;
+      if (tid == 0)
+        ok = mbar_wait(smem_u32(&acc_full[acc]), (it >> 1) & 1, abort_flag, a.out.err,
+                       kErrWaitEpilogue);
+      if (named_bar_any(1, kRouterEpiThreads, !ok)) break;
       tc_fence_after();
-      const uint32_t trow = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-      auto load16 = [&](int c, uint32_t (&v)[16]) {
-        __syncwarp();
-        tmem_ld16(trow + static_cast<uint32_t>(c), v);
-        tmem_ld_wait16(v);
-      };
-      auto sync = [] { named_bar_sync(1, kRouterEpiThreads); };
-      router_epilogue<MAXK>(r, sub, tile, a.tile_rows, a.T, a.n_routed, a.n_pad, a.top_k, a.bias,
-                            base, a.out, load16, sync);
+      for (int e = tid; e < 4 * kMaxRouted; e += kRouterEpiThreads) (&SM.mask[0][0])[e] = 0u;
+      for (int pass = 0; pass < npass; ++pass) {
+        // accumulator rows 64 pass .. 64 pass + 63 -> shared memory (bias added): the
+        // quadrants 2 pass and 2 pass + 1, four warps each, one 16-column slice per turn
+        if ((q >> 1) == pass) {
+          const int tr = q * 32 + lane;
+          const uint32_t trow =
+              tmem_base + (static_cast<uint32_t>(q * 32) << 16) + (uint32_t)(acc * a.n_pad);
+          for (int jj = sub; jj < nch; jj += 4) {
+            uint32_t v[16];
+            __syncwarp();
+            tmem_ld16(trow + static_cast<uint32_t>(jj * 16), v);
+            tmem_ld_wait16(v);
+            if (tr < a.tile_rows) {
+              float4* dst = reinterpret_cast<float4*>(lg + (size_t)(tr - pass * kRouterPass) * ld + jj * 16);
+              const float* bb = SM.bias + jj * 16;
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                dst[k] = make_float4(__uint_as_float(v[4 * k]) + bb[4 * k],
+                                     __uint_as_float(v[4 * k + 1]) + bb[4 * k + 1],
+                                     __uint_as_float(v[4 * k + 2]) + bb[4 * k + 2],
+                                     __uint_as_float(v[4 * k + 3]) + bb[4 * k + 3]);
+            }
+          }
+        }
+        if (pass == npass - 1) tc_fence_before();
+        sync();
+        if (pass == npass - 1 && tid == 0) mbar_arrive(smem_u32(&acc_empty[acc]));   // accumulator free
+        router_pass<MAXC>(tid, pass, tile, a.tile_rows, a.T, a.n_routed, a.n_pad, a.top_k, epi,
+                          a.out, sync);
+        sync();
+      }
+      router_tile_outputs(tid, tile, a.tile_rows, a.T, a.n_routed, a.n_pad, a.top_k, epi, a.out);
+      sync();   // scratch free for the next tile
     }
   }
 
@@ -402,42 +539,39 @@ struct RouterSimtArgs {
   RouterOut out;
 };
 
-// 512 threads, tiles of 128 tokens.  dynamic smem: router_epi_bytes(n_routed, MAXK) plus a
-// [128][ld] logit buffer.  n_routed <= 128.
-template <int MAXK>
+// 512 threads, one tile of 64 tokens (one epilogue pass) per CTA.  dynamic smem:
+// router_epi_bytes(n_pad).
+template <int MAXC>
 __global__ void __launch_bounds__(kRouterEpiThreads) router_simt_kernel(RouterSimtArgs a) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  const int ld = router_row_ld(a.n_routed);
-  float* logits = reinterpret_cast<float*>(smem_raw + router_epi_bytes(a.n_routed, MAXK));
+  RouterEpiSmem& SM = *reinterpret_cast<RouterEpiSmem*>(smem_raw);
+  float* lg = reinterpret_cast<float*>(smem_raw + sizeof(RouterEpiSmem));
   const int tid = threadIdx.x;
-  const int r = tid & (kRouterBM - 1), sub = tid >> 7;
   const int tile = blockIdx.x;
-  const int t = tile * kRouterBM + r;
   const int n_pad = (a.n_routed + 15) & ~15;
-  // thread (r, sub) computes the logits of the slices it owns in the epilogue
-  for (int j = sub; j < (n_pad >> 4); j += 4) {
-    for (int i = j * 16; i < j * 16 + 16 && i < a.n_routed; ++i) {
-      float acc = 0.f;
-      if (t < a.T) {
-        const float4* ur = reinterpret_cast<const float4*>(a.u + (size_t)t * a.d);
-        const float4* er = reinterpret_cast<const float4*>(a.cen + (size_t)i * a.d);
-        for (int k = 0; k < a.d / 4; ++k) {
-          const float4 x = ur[k], y = __ldg(&er[k]);
-          acc = fmaf(x.x, y.x, acc); acc = fmaf(x.y, y.y, acc);
-          acc = fmaf(x.z, y.z, acc); acc = fmaf(x.w, y.w, acc);
-        }
+  const int ld = router_ld(n_pad);
+  for (int e = tid; e < 4 * kMaxRouted; e += kRouterEpiThreads) (&SM.mask[0][0])[e] = 0u;
+  for (int idx = tid; idx < kRouterPass * a.n_routed; idx += kRouterEpiThreads) {
+    const int r = idx / a.n_routed, i = idx - r * a.n_routed;
+    const int t = tile * kRouterPass + r;
+    float acc = 0.f;
+    if (t < a.T) {
+      const float4* ur = reinterpret_cast<const float4*>(a.u + (size_t)t * a.d);
+      const float4* er = reinterpret_cast<const float4*>(a.cen + (size_t)i * a.d);
+      for (int k = 0; k < a.d / 4; ++k) {
+        const float4 x = ur[k], y = __ldg(&er[k]);
+        acc = fmaf(x.x, y.x, acc); acc = fmaf(x.y, y.y, acc);
+        acc = fmaf(x.z, y.z, acc); acc = fmaf(x.w, y.w, acc);
       }
-      logits[(size_t)r * ld + i] = acc;
     }
+    lg[(size_t)r * ld + i] = acc + a.bias[i];
   }
-  auto load16 = [&](int c, uint32_t (&v)[16]) {
-#pragma unroll
-    for (int k = 0; k < 16; ++k)
-      v[k] = (c + k < a.n_routed) ? __float_as_uint(logits[(size_t)r * ld + c + k]) : 0u;
-  };
+  __syncthreads();
   auto sync = [] { __syncthreads(); };
-  router_epilogue<MAXK>(r, sub, tile, kRouterBM, a.T, a.n_routed, n_pad, a.top_k, a.bias,
-                        smem_raw, a.out, load16, sync);
+  router_pass<MAXC>(tid, 0, tile, kRouterPass, a.T, a.n_routed, n_pad, a.top_k, smem_raw, a.out,
+                    sync);
+  __syncthreads();
+  router_tile_outputs(tid, tile, kRouterPass, a.T, a.n_routed, n_pad, a.top_k, smem_raw, a.out);
 }
 
 }  // namespace moe
