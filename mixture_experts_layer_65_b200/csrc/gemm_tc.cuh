@@ -39,13 +39,18 @@ namespace moe {
 
 constexpr int kPairBM = 256;                 // output rows per cluster tile (128 per CTA)
 constexpr int kGemmBN = 256;                 // output columns (B rows) per tile
-constexpr int kGemmBK = 64;
-constexpr int kGemmStages = 6;
+constexpr int kGemmBK = 64;                  // k-block (one 128-byte swizzle row of bf16)
+// A stage carries two k-blocks: the MMA issuer's wait on a stage (and the producer's)
+// costs a few hundred cycles of issue latency, which two k-blocks of MMAs hide better
+// than one.  Three such stages keep the same bytes in flight as six single ones.
+constexpr int kGemmKPS = 2;
+constexpr int kGemmStages = 3;
 constexpr int kGemmEpiWarps = 8;             // two warps per TMEM lane quadrant
 constexpr int kGemmThreads = 64 + 32 * kGemmEpiWarps;
-constexpr uint32_t kGemmABytes = 128 * kGemmBK * 2;           // this CTA's half of A
-constexpr uint32_t kGemmBBytes = (kGemmBN / 2) * kGemmBK * 2; // this CTA's half of B
-constexpr uint32_t kGemmStageBytes = kGemmABytes + kGemmBBytes;
+constexpr uint32_t kGemmABytes = 128 * kGemmBK * 2;           // this CTA's half of A, per k-block
+constexpr uint32_t kGemmBBytes = (kGemmBN / 2) * kGemmBK * 2; // this CTA's half of B, per k-block
+constexpr uint32_t kGemmBOff = kGemmKPS * kGemmABytes;        // B blocks after the A blocks
+constexpr uint32_t kGemmStageBytes = kGemmKPS * (kGemmABytes + kGemmBBytes);
 constexpr uint32_t kGemmTmemCols = 512;
 constexpr size_t kGemmSmemBytes = 1024 + (size_t)kGemmStages * kGemmStageBytes + 256;
 
@@ -145,15 +150,20 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
         const int arow = __ldg(&a.grp_row[c.g]) + c.m * kPairBM + (int)rank * 128;
         const int brow = c.n * kGemmBN + (int)rank * (kGemmBN / 2);
         const int kbn = c.shared ? a.kb_shared : a.kb_routed;
-        for (int kb = 0; kb < kbn; ++kb) {
+        for (int kb0 = 0; kb0 < kbn; kb0 += kGemmKPS) {
           ok = mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, a.err, kErrWaitProducer);
           if (!ok) break;
           const uint32_t sa = smem_u32(base + (size_t)stage * kGemmStageBytes);
           const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
-          if (leader) mbar_arrive_expect_tx(smem_u32(&full[stage]), 2 * kGemmStageBytes);
-          tma_load_2d_pair(sa, ta, fb, kb * kGemmBK, arow);
-          if (c.shared) tma_load_2d_pair(sa + kGemmABytes, &tmB_s, fb, kb * kGemmBK, brow);
-          else tma_load_3d_pair(sa + kGemmABytes, &tmB_r, fb, kb * kGemmBK, brow, c.e);
+          const int nk = kbn - kb0 < kGemmKPS ? kbn - kb0 : kGemmKPS;
+          if (leader)
+            mbar_arrive_expect_tx(smem_u32(&full[stage]), 2u * (uint32_t)nk * (kGemmABytes + kGemmBBytes));
+          for (int j = 0; j < nk; ++j) {
+            const int kx = (kb0 + j) * kGemmBK;
+            tma_load_2d_pair(sa + j * kGemmABytes, ta, fb, kx, arow);
+            if (c.shared) tma_load_2d_pair(sa + kGemmBOff + j * kGemmBBytes, &tmB_s, fb, kx, brow);
+            else tma_load_3d_pair(sa + kGemmBOff + j * kGemmBBytes, &tmB_r, fb, kx, brow, c.e);
+          }
           if (++stage == kGemmStages) { stage = 0; phase ^= 1u; }
         }
       }
@@ -183,16 +193,19 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
         if (!ok) break;
         tc_fence_after();
         const uint32_t dt = tmem_base + static_cast<uint32_t>(acc * kGemmBN);
-        for (int kb = 0; kb < kbn; ++kb) {
+        for (int kb0 = 0; kb0 < kbn; kb0 += kGemmKPS) {
           ok = mbar_wait(smem_u32(&full[stage]), phase, abort_flag, a.err, kErrWaitMma);
           if (!ok) break;
           tc_fence_after();
           const uint32_t sa = smem_u32(base + (size_t)stage * kGemmStageBytes);
-          const uint64_t adesc = sdesc_k_sw128(sa);
-          const uint64_t bdesc = sdesc_k_sw128(sa + kGemmABytes);
+          const int nk = kbn - kb0 < kGemmKPS ? kbn - kb0 : kGemmKPS;
+          for (int j = 0; j < nk; ++j) {
+            const uint64_t adesc = sdesc_k_sw128(sa + j * kGemmABytes);
+            const uint64_t bdesc = sdesc_k_sw128(sa + kGemmBOff + j * kGemmBBytes);
 #pragma unroll
-          for (int k = 0; k < kGemmBK / 16; ++k)
-            tc_mma_f16_pair(dt, adesc + 2u * k, bdesc + 2u * k, idesc, (kb | k) != 0);
+            for (int k = 0; k < kGemmBK / 16; ++k)
+              tc_mma_f16_pair(dt, adesc + 2u * k, bdesc + 2u * k, idesc, (kb0 | j | k) != 0);
+          }
           tc_commit_pair_mc(smem_u32(&empty[stage]), 0x3);
           if (++stage == kGemmStages) { stage = 0; phase ^= 1u; }
         }
