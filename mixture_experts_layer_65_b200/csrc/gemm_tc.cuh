@@ -46,7 +46,8 @@ constexpr int kGemmBK = 64;                  // k-block (one 128-byte swizzle ro
 constexpr int kGemmKPS = 2;
 constexpr int kGemmStages = 3;
 constexpr int kGemmEpiWarps = 8;             // two warps per TMEM lane quadrant
-constexpr int kGemmThreads = 64 + 32 * kGemmEpiWarps;
+constexpr int kGemmCopyWarps = 4;            // row copies of the fused permute (gate/up GEMM)
+constexpr int kGemmThreads = 64 + 32 * (kGemmEpiWarps + kGemmCopyWarps);
 constexpr uint32_t kGemmABytes = 128 * kGemmBK * 2;           // this CTA's half of A, per k-block
 constexpr uint32_t kGemmBBytes = (kGemmBN / 2) * kGemmBK * 2; // this CTA's half of B, per k-block
 constexpr uint32_t kGemmBOff = kGemmKPS * kGemmABytes;        // B blocks after the A blocks
@@ -69,6 +70,15 @@ struct GemmArgs {
   int64_t ld_routed, rows_routed;
   int cols_routed;
   int* err;
+  // Fused permute (gate/up GEMM with a shared group): the copy warps of every CTA copy the
+  // token rows to their expert-contiguous A rows (`perm`) while the shared group's tiles,
+  // which read the token matrix itself, run first; each copy warp then adds 1 to
+  // *copy_done, and a CTA's producer waits for all gridDim.x * kGemmCopyWarps of them
+  // before loading its first routed tile.  copy_done == nullptr: no fused copy.  The
+  // wait relies on the whole grid being resident at once (it is sized from the occupancy
+  // of this kernel).
+  PermuteArgs perm;
+  int* copy_done;
 };
 
 struct TileCoord {
@@ -143,9 +153,17 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
       int stage = 0, g = 0;
       uint32_t phase = 0;
       bool ok = true;
+      bool rows_ready = a.copy_done == nullptr;
       for (int tile = cid; tile < total && ok; tile += ncl) {
         TileCoord c;
         gemm_decode(tile, g, a, c);
+        if (!c.shared && !rows_ready) {
+          ok = counter_wait(a.copy_done, (int)gridDim.x * kGemmCopyWarps, abort_flag, a.err,
+                            kErrWaitCopy);
+          if (!ok) break;
+          fence_proxy_async_global();   // the copied rows, seen by the TMA loads below
+          rows_ready = true;
+        }
         const CUtensorMap* ta = c.shared ? &tmA_s : &tmA_r;
         const int arow = __ldg(&a.grp_row[c.g]) + c.m * kPairBM + (int)rank * 128;
         const int brow = c.n * kGemmBN + (int)rank * (kGemmBN / 2);
@@ -214,6 +232,18 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
       tc_commit_pair_mc(smem_u32(drain), 0x3);
     }
     __syncwarp();
+  } else if (warp >= 2 + kGemmEpiWarps) {
+    // ------------------------------------------------------------------ row copies
+    if (a.copy_done != nullptr) {
+      const int nw = (int)gridDim.x * kGemmCopyWarps;
+      for (int t = (int)blockIdx.x * kGemmCopyWarps + (warp - 2 - kGemmEpiWarps); t < a.perm.T;
+           t += nw)
+        permute_token(a.perm, t, lane);
+      fence_proxy_async_global();
+      __threadfence();
+      __syncwarp();
+      if (lane == 0) atomicAdd(a.copy_done, 1);
+    }
   } else {
     // ------------------------------------------------------------------ epilogue
     const int q = warp & 3;                 // TMEM lane quadrant this warp may access

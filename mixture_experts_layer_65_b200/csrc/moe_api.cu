@@ -168,6 +168,8 @@ struct moe_handle {
   float *tile_psum = nullptr, *psum_total = nullptr;
   void *xp = nullptr, *hs = nullptr, *hr = nullptr, *ys = nullptr, *yr = nullptr;
   int* err = nullptr;
+  int* copy_done = nullptr;   // counter of the fused permute (paired bf16 path with a shared group)
+  bool fuse_permute = false;
   // staging for moe_forward_host
   void *u_dev = nullptr, *h_dev = nullptr;
   int32_t *idx_dev = nullptr, *cnt_dev = nullptr;
@@ -251,7 +253,7 @@ int32_t moe_abi_version(void) { return MOE_ABI_VERSION; }
 const char* moe_last_error(void) { return g_last_error.c_str(); }
 
 int32_t moe_kernels_per_forward(const moe_handle* handle) {
-  return handle ? kKernelsPerForward : 0;
+  return handle ? kKernelsPerForward - (handle->fuse_permute ? 1 : 0) : 0;
 }
 
 size_t moe_device_bytes(const moe_handle* handle) { return handle ? handle->bytes : 0; }
@@ -281,6 +283,8 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
   H->n_tok = (c.T + 15) / 16 * 16;
   H->bm = H->small ? 1 : (H->bf16 ? kPairBM : kSimtBM);
   H->tile_rows = H->small ? 0 : H->bm;
+  // the paired GEMM copies the routed rows itself while the shared group's tiles run
+  H->fuse_permute = H->bf16 && !H->small && H->has_shared;
   H->T_pad = H->small ? H->n_tok : ((int64_t)c.T + H->bm - 1) / H->bm * H->bm;
   H->rows_cap = ((int64_t)c.T * c.top_k + (int64_t)c.n_routed * (H->bm - 1) + H->bm - 1) /
                 H->bm * H->bm;
@@ -354,6 +358,8 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
   MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->ts2), (size_t)(H->G + 1) * 4));
   MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->err), 256));
   MOE_CUDA(cudaMemsetAsync(H->err, 0, 256, st));
+  MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->copy_done), 256));
+  MOE_CUDA(cudaMemsetAsync(H->copy_done, 0, 256, st));
   const size_t rc = (size_t)H->rows_cap, tp = (size_t)H->T_pad;
   MOE_TRY(dalloc(H, &H->xp, rc * d * es));
   MOE_TRY(dalloc(H, &H->hr, rc * I * es));
@@ -511,7 +517,8 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
   ScanArgs sa{H->tile_hist, H->tile_psum, H->n_tiles, nr, T, H->has_shared, H->inter_shared,
               c.inter, d, H->bm, H->tile_rows, bn1, bn2, c.alpha1, expert_counts, aux_loss,
               H->psum_total,
-              H->tile_base, H->grp_row, H->ts1, H->ts2};
+              H->tile_base, H->grp_row, H->ts1, H->ts2,
+              H->fuse_permute ? H->copy_done : nullptr};
   tick(H, stream, 1);
   scan_kernel<<<1, kScanThreads, 0, stream>>>(sa);
   MOE_CUDA(cudaGetLastError());
@@ -520,8 +527,10 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
                  static_cast<uint8_t*>(H->xp), T, K, nr, (int)H->rows_cap, H->router_rows,
                  d * H->es, H->err};
   tick(H, stream, 2);
-  permute_kernel<<<(T + kPermuteWarps - 1) / kPermuteWarps, kPermuteWarps * 32, 0, stream>>>(pa);
-  MOE_CUDA(cudaGetLastError());
+  if (!H->fuse_permute) {
+    permute_kernel<<<(T + kPermuteWarps - 1) / kPermuteWarps, kPermuteWarps * 32, 0, stream>>>(pa);
+    MOE_CUDA(cudaGetLastError());
+  }
 
   const int I = c.inter, Is = H->inter_shared;
   if (H->small) {
@@ -560,6 +569,10 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
     g1.out_routed = static_cast<__nv_bfloat16*>(H->hr); g1.ld_routed = I; g1.rows_routed = H->rows_cap;
     g1.cols_routed = I;
     g1.err = H->err;
+    if (H->fuse_permute) {
+      g1.perm = pa;
+      g1.copy_done = H->copy_done;
+    }
     tick(H, stream, 3);
     grouped_gemm_tc_kernel<kGateUpSwiGLU><<<H->gemm_grid, kGemmThreads, kGemmSmemBytes, stream>>>(
         tmU, H->tmXp, H->tmWguS, H->tmWguR, g1);

@@ -18,6 +18,7 @@ enum DevErr : int {
   kErrWaitMma = 0x102,        // MMA issuer gave up waiting for data / accumulator
   kErrWaitEpilogue = 0x103,   // epilogue gave up waiting for an accumulator
   kErrWaitDrain = 0x104,      // teardown gave up waiting for in-flight copies / MMAs
+  kErrWaitCopy = 0x105,       // fused GEMM producer gave up waiting for the row copies
   kErrRouteIndex = 0x201,     // routed index outside [0, n_routed)
   kErrPermuteRow = 0x202,     // destination row outside the permuted buffer
   kErrOutRow = 0x203,         // GEMM output row outside its buffer
@@ -81,6 +82,38 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 255u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        record_error(err, code);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// Generic-proxy global writes (plain stores) ordered before later async-proxy (TMA)
+// accesses of this thread.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Wait until *counter >= target (written by other CTAs with release semantics).  Gives
+// up like mbar_wait: on `abort_flag`, or after kWaitLimitNs, recording `code`.
+__device__ __forceinline__ bool counter_wait(const int* counter, int target, volatile int* abort_flag,
+                                             int* err, int code) {
+  if (ld_acquire_gpu(counter) >= target) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(256);
+    if (ld_acquire_gpu(counter) >= target) return true;
+    if ((it & 63u) == 0) {
       if (*abort_flag) return false;
       if (globaltimer_ns() - t0 > kWaitLimitNs) {
         record_error(err, code);

@@ -34,6 +34,7 @@ struct ScanArgs {
   int32_t* grp_row;           // [G] first row of each group in its A matrix
   int32_t* ts1;               // [G + 1] tile prefix of the gate/up GEMM
   int32_t* ts2;               // [G + 1] tile prefix of the down GEMM
+  int32_t* copy_done;         // counter of the fused GEMM's copy warps, zeroed here; or nullptr
 };
 
 static __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a) {
@@ -51,6 +52,7 @@ static __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a
   const bool active = seg < nseg;
   const int t0 = seg * seg_len;
   const int t1 = min(a.n_tiles, t0 + seg_len);
+  if (tid == 0 && a.copy_done) *a.copy_done = 0;
 
   // 1. per-segment sums (tiles in ascending order)
   if (active) {
@@ -167,10 +169,9 @@ struct PermuteArgs {
 constexpr int kPermuteWarps = 8;
 constexpr int kPermuteVec = 8;   // 16-byte vectors held per lane per pass
 
-static __global__ void __launch_bounds__(kPermuteWarps * 32) permute_kernel(PermuteArgs a) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = blockIdx.x * kPermuteWarps + warp;
-  if (t >= a.T) return;
+// One warp copies token t's row to its top_k destinations (and records them for the
+// combine).  Used by permute_kernel and by the copy warps of the fused gate/up GEMM.
+__device__ __forceinline__ void permute_token(const PermuteArgs& a, int t, int lane) {
   int my_dest = -1;
   if (lane < a.top_k) {
     const int e = a.topk_idx[(size_t)t * a.top_k + lane];
@@ -204,6 +205,13 @@ static __global__ void __launch_bounds__(kPermuteWarps * 32) permute_kernel(Perm
       }
     }
   }
+}
+
+static __global__ void __launch_bounds__(kPermuteWarps * 32) permute_kernel(PermuteArgs a) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kPermuteWarps + warp;
+  if (t >= a.T) return;
+  permute_token(a, t, lane);
 }
 
 }  // namespace moe

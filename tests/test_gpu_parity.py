@@ -77,7 +77,10 @@ def test_full_size_layer(name):
     rows = None if w.T <= 512 else P.sample_rows(w.T)
     rep = P.compare(w, g, rows=rows)
     print(name, rep)
-    assert layer.kernels_per_forward == 6
+    # the paired bf16 GEMM path with a shared group fuses the row permute into the
+    # gate/up GEMM; decode-sized layers and layers without shared experts launch it
+    fused = w.dtype == "bf16" and w.T > 128 and w.n_shared > 0
+    assert layer.kernels_per_forward == (5 if fused else 6)
 
 
 # ------------------------------------------------------------------------ edge cases
