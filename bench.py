@@ -329,19 +329,24 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         ms = float(t.item())
     layer.device_status()
 
-    # end to end through the public host-buffer call (pinned host memory)
+    # end to end through the public host-buffer call (pinned host memory): a stream of
+    # batches through moe_forward_host_pipelined, which overlaps each step's host->device
+    # and device->host copies with the neighbouring steps' forwards
     e2e_ms = None
     if args.e2e_steps > 0:
-        u_host = ubufs[0].cpu().pin_memory()
-        host_out = None
-        for _ in range(2):
-            host_out = layer.forward_host(u_host, host_out)
+        u_hosts = [ubufs[i % len(ubufs)].cpu().pin_memory() for i in range(2)]
+        host_outs = [layer.host_outputs() for _ in range(2)]
+        for i in range(2):
+            layer.forward_host_pipelined(u_hosts[i], host_outs[i], stream)
+        layer.pipeline_wait(stream)
+        torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for _ in range(args.e2e_steps):
-            host_out = layer.forward_host(u_host, host_out)
+        for i in range(args.e2e_steps):
+            layer.forward_host_pipelined(u_hosts[i % 2], host_outs[i % 2], stream)
+        layer.pipeline_wait(stream)
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1)
@@ -404,7 +409,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "kernels": per_kernel,
         "e2e": None if e2e_ms is None else {
             "value": world * w.T * args.e2e_steps / (e2e_ms * 1e-3), "unit": "tokens/s",
-            "h2d_bytes_per_step": u_bytes, "d2h_bytes_per_step": u_bytes + tk * 8 + w.n_routed * 4 + 4},
+            "h2d_bytes_per_step": u_bytes, "d2h_bytes_per_step": u_bytes + tk * 8 + w.n_routed * 4 + 4,
+            "api": "moe_forward_host_pipelined (two steps in flight), then moe_pipeline_wait"},
         "gpu_launches": args.steps * (layer.kernels_per_forward + (1 if world > 1 else 0)),
         "launch": "eager" if args.no_graph else "CUDA graph replay (one graph per input buffer)",
         "kernel_timing": ("CUDA events between the library's kernels over the timed steps"

@@ -114,6 +114,29 @@ moe_status moe_forward_host(moe_handle* handle, const void* u_host, void* h_host
                             int32_t* expert_counts_host, float* aux_loss_host,
                             moe_stream_t stream);
 
+/* Pipelined moe_forward on HOST buffers, for a caller that streams batch after batch
+ * through one layer.  Enqueues the host->device copy of u, the forward and the
+ * device->host copies of the outputs on the handle's own copy-in, forward and copy-out
+ * streams and returns without waiting.  The handle double-buffers its device staging, so
+ * two calls can be in flight and the copies of one overlap the forward of its neighbours
+ * (the two copy directions use separate copy engines).  Ordering: a call's copy-in
+ * starts after the work enqueued on `stream` before the call, and after the forward two
+ * calls earlier (which read the same staging slot); its forward runs after the copy-out two
+ * calls earlier.  Host buffers must be pinned; u_host must stay unchanged and the output
+ * buffers unread until moe_pipeline_wait(handle, stream) has been called and `stream`
+ * synchronised.  The first call creates the streams and allocates the staging (twice the
+ * input and output sizes).  Sizes as in moe_forward; any output except h_host may be NULL.
+ * Calls must come from one host thread at a time and must not overlap moe_forward or
+ * moe_forward_host calls on the same handle (they share its workspace). */
+moe_status moe_forward_host_pipelined(moe_handle* handle, const void* u_host, void* h_host,
+                                      int32_t* topk_idx_host, float* topk_w_host,
+                                      int32_t* expert_counts_host, float* aux_loss_host,
+                                      moe_stream_t stream);
+
+/* Make `stream` wait for every moe_forward_host_pipelined call issued so far (their
+ * device->host copies included).  Does not block the host. */
+moe_status moe_pipeline_wait(moe_handle* handle, moe_stream_t stream);
+
 /* Synchronise `stream`, then read and clear the handle's device error word.
  * Returns MOE_DEVICE_CHECK (with the kernel's code in moe_last_error()) if any kernel
  * of an earlier forward recorded an error, else MOE_OK. */

@@ -38,6 +38,8 @@ _SIGS = {
     "moe_create": (ctypes.c_int, [ctypes.POINTER(MoeCfg), ctypes.POINTER(ctypes.c_void_p)]),
     "moe_forward": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_forward_host": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_forward_host_pipelined": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_pipeline_wait": (ctypes.c_int, [_P, _P]),
     "moe_device_status": (ctypes.c_int, [_P, _P]),
     "moe_expert_psum": (ctypes.c_int, [_P, _P, _P]),
     "moe_balance_loss": (ctypes.c_int, [_P, _P, ctypes.c_int32, ctypes.c_int64, ctypes.c_float,

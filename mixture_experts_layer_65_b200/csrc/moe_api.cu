@@ -176,6 +176,19 @@ struct moe_handle {
   float *w_dev = nullptr, *aux_dev = nullptr;
   CUtensorMap tmE, tmXp, tmWguS, tmWguR, tmHs, tmHr, tmWdS, tmWdR;
   CUtensorMap tmXpN, tmHsN, tmHrN;   // token operands of the small-batch GEMMs (n_tok rows)
+  // moe_forward_host_pipelined: copy-in / forward / copy-out streams, two staging slots
+  struct PipeSlot {
+    void *u = nullptr, *h = nullptr;
+    int32_t *idx = nullptr, *cnt = nullptr;
+    float *w = nullptr, *aux = nullptr;
+    cudaEvent_t in_done = nullptr, comp_done = nullptr, out_done = nullptr;
+    bool used = false;
+  };
+  cudaStream_t p_in = nullptr, p_c = nullptr, p_out = nullptr;
+  cudaEvent_t p_entry = nullptr;
+  PipeSlot pslot[2];
+  int64_t p_calls = 0;
+  bool p_ready = false;
   // per-kernel timing (moe_timing_begin / moe_timing_end)
   std::vector<cudaEvent_t> events;   // kKernelsPerForward + 1 per recorded call
   int timing_cap = 0, timing_used = 0;
@@ -208,6 +221,12 @@ moe_status dalloc(moe_handle* H, void** p, size_t bytes) {
 void free_handle(moe_handle* H) {
   if (!H) return;
   for (cudaEvent_t e : H->events) cudaEventDestroy(e);
+  for (auto& P : H->pslot)
+    for (cudaEvent_t e : {P.in_done, P.comp_done, P.out_done})
+      if (e) cudaEventDestroy(e);
+  if (H->p_entry) cudaEventDestroy(H->p_entry);
+  for (cudaStream_t st : {H->p_in, H->p_c, H->p_out})
+    if (st) cudaStreamDestroy(st);
   for (void* p : H->allocs) cudaFree(p);
   delete H;
 }
@@ -710,6 +729,82 @@ moe_status moe_forward_host(moe_handle* H, const void* u_host, void* h_host, int
   if (aux_loss_host)
     MOE_CUDA(cudaMemcpyAsync(aux_loss_host, H->aux_dev, 4, cudaMemcpyDeviceToHost, stream));
   MOE_CUDA(cudaStreamSynchronize(stream));
+  return MOE_OK;
+}
+
+namespace {
+moe_status pipe_init(moe_handle* H) {
+  const moe_cfg& c = H->cfg;
+  const size_t row = (size_t)c.T * c.d * H->es, tk = (size_t)c.T * c.top_k;
+  for (cudaStream_t* st : {&H->p_in, &H->p_c, &H->p_out})
+    MOE_CUDA(cudaStreamCreateWithFlags(st, cudaStreamNonBlocking));
+  MOE_CUDA(cudaEventCreateWithFlags(&H->p_entry, cudaEventDisableTiming));
+  for (auto& P : H->pslot) {
+    MOE_TRY(dalloc(H, &P.u, row));
+    MOE_TRY(dalloc(H, &P.h, row));
+    MOE_TRY(dalloc(H, reinterpret_cast<void**>(&P.idx), tk * 4));
+    MOE_TRY(dalloc(H, reinterpret_cast<void**>(&P.w), tk * 4));
+    MOE_TRY(dalloc(H, reinterpret_cast<void**>(&P.cnt), (size_t)c.n_routed * 4));
+    MOE_TRY(dalloc(H, reinterpret_cast<void**>(&P.aux), 4));
+    for (cudaEvent_t* e : {&P.in_done, &P.comp_done, &P.out_done})
+      MOE_CUDA(cudaEventCreateWithFlags(e, cudaEventDisableTiming));
+  }
+  H->p_ready = true;
+  return MOE_OK;
+}
+}  // namespace
+
+moe_status moe_forward_host_pipelined(moe_handle* H, const void* u_host, void* h_host,
+                                      int32_t* topk_idx_host, float* topk_w_host,
+                                      int32_t* expert_counts_host, float* aux_loss_host,
+                                      moe_stream_t stream_) {
+  if (!H) return fail(MOE_ERR_INVALID_ARG, "handle is NULL");
+  if (!u_host || !h_host) return fail(MOE_ERR_INVALID_ARG, "u_host and h_host must not be NULL");
+  int dev = -1;
+  MOE_CUDA(cudaGetDevice(&dev));
+  if (dev != H->device)
+    return fail(MOE_ERR_INVALID_ARG, "current device %d is not the handle's device %d", dev, H->device);
+  if (!H->p_ready) MOE_TRY(pipe_init(H));
+  cudaStream_t us = reinterpret_cast<cudaStream_t>(stream_);
+  const moe_cfg& c = H->cfg;
+  const size_t row = (size_t)c.T * c.d * H->es, tk = (size_t)c.T * c.top_k;
+  moe_handle::PipeSlot& P = H->pslot[H->p_calls & 1];
+  // copy-in: after the caller's earlier work and after the forward that last read the slot
+  MOE_CUDA(cudaEventRecord(H->p_entry, us));
+  MOE_CUDA(cudaStreamWaitEvent(H->p_in, H->p_entry, 0));
+  if (P.used) MOE_CUDA(cudaStreamWaitEvent(H->p_in, P.comp_done, 0));
+  MOE_CUDA(cudaMemcpyAsync(P.u, u_host, row, cudaMemcpyHostToDevice, H->p_in));
+  MOE_CUDA(cudaEventRecord(P.in_done, H->p_in));
+  // forward: after its input and after the copy-out that last read the slot's outputs
+  MOE_CUDA(cudaStreamWaitEvent(H->p_c, P.in_done, 0));
+  if (P.used) MOE_CUDA(cudaStreamWaitEvent(H->p_c, P.out_done, 0));
+  MOE_TRY(moe_forward(H, P.u, P.h, P.idx, P.w, P.cnt, P.aux,
+                      reinterpret_cast<moe_stream_t>(H->p_c)));
+  MOE_CUDA(cudaEventRecord(P.comp_done, H->p_c));
+  // copy-out
+  MOE_CUDA(cudaStreamWaitEvent(H->p_out, P.comp_done, 0));
+  MOE_CUDA(cudaMemcpyAsync(h_host, P.h, row, cudaMemcpyDeviceToHost, H->p_out));
+  if (topk_idx_host)
+    MOE_CUDA(cudaMemcpyAsync(topk_idx_host, P.idx, tk * 4, cudaMemcpyDeviceToHost, H->p_out));
+  if (topk_w_host)
+    MOE_CUDA(cudaMemcpyAsync(topk_w_host, P.w, tk * 4, cudaMemcpyDeviceToHost, H->p_out));
+  if (expert_counts_host)
+    MOE_CUDA(cudaMemcpyAsync(expert_counts_host, P.cnt, (size_t)c.n_routed * 4,
+                             cudaMemcpyDeviceToHost, H->p_out));
+  if (aux_loss_host)
+    MOE_CUDA(cudaMemcpyAsync(aux_loss_host, P.aux, 4, cudaMemcpyDeviceToHost, H->p_out));
+  MOE_CUDA(cudaEventRecord(P.out_done, H->p_out));
+  P.used = true;
+  ++H->p_calls;
+  return MOE_OK;
+}
+
+moe_status moe_pipeline_wait(moe_handle* H, moe_stream_t stream_) {
+  if (!H) return fail(MOE_ERR_INVALID_ARG, "handle is NULL");
+  if (H->p_calls == 0) return MOE_OK;
+  // copy-outs run in issue order on one stream: the last one covers all earlier ones
+  const moe_handle::PipeSlot& P = H->pslot[(H->p_calls - 1) & 1];
+  MOE_CUDA(cudaStreamWaitEvent(reinterpret_cast<cudaStream_t>(stream_), P.out_done, 0));
   return MOE_OK;
 }
 

@@ -113,6 +113,35 @@ class MoELayer:
                                      _ptr(out.aux_loss), s.cuda_stream))
         return out
 
+    def host_outputs(self) -> MoEOutput:
+        """Pinned host tensors for the outputs of forward_host / forward_host_pipelined."""
+        return MoEOutput(
+            h=torch.empty(self.T, self.d, dtype=self.torch_dtype, pin_memory=True),
+            topk_idx=torch.empty(self.T, self.top_k, dtype=torch.int32, pin_memory=True),
+            topk_w=torch.empty(self.T, self.top_k, dtype=torch.float32, pin_memory=True),
+            expert_counts=torch.empty(self.n_routed, dtype=torch.int32, pin_memory=True),
+            aux_loss=torch.empty(1, dtype=torch.float32, pin_memory=True))
+
+    def forward_host_pipelined(self, u: torch.Tensor, out: MoEOutput,
+                               stream: torch.cuda.Stream | None = None) -> MoEOutput:
+        """Enqueue a forward on pinned HOST tensors without waiting (two calls in flight,
+        copies overlapped with the neighbouring forwards).  `u` must stay unchanged and
+        `out` unread until pipeline_wait() and a synchronisation of `stream`."""
+        if u.is_cuda or u.shape != (self.T, self.d) or u.dtype != self.torch_dtype:
+            raise ValueError("u must be a host tensor of the layer shape and dtype")
+        if not (u.is_pinned() and out.h.is_pinned()):
+            raise ValueError("forward_host_pipelined needs pinned host tensors")
+        s = stream or torch.cuda.current_stream(self.device)
+        check(lib().moe_forward_host_pipelined(self._h, _ptr(u), _ptr(out.h), _ptr(out.topk_idx),
+                                               _ptr(out.topk_w), _ptr(out.expert_counts),
+                                               _ptr(out.aux_loss), s.cuda_stream))
+        return out
+
+    def pipeline_wait(self, stream: torch.cuda.Stream | None = None) -> None:
+        """Make `stream` wait for every forward_host_pipelined call issued so far."""
+        s = stream or torch.cuda.current_stream(self.device)
+        check(lib().moe_pipeline_wait(self._h, s.cuda_stream))
+
     def device_status(self, stream: torch.cuda.Stream | None = None) -> None:
         """Synchronise and raise if a kernel recorded a device-side error."""
         s = stream or torch.cuda.current_stream(self.device)

@@ -190,6 +190,30 @@ def test_forward_host_matches_forward():
     layer.device_status()
 
 
+def test_forward_host_pipelined_matches_forward():
+    # four batches through the two-slot pipeline (slots reused), each checked bit for bit
+    # against the device-buffer forward of the same input
+    w = W.make_workload("16b_prefill", T=500)
+    layer = MoELayer.from_workload(w)
+    rng = np.random.default_rng(5)
+    us = [to_device_tensor(w.u, "cuda")]
+    for _ in range(3):
+        us.append(to_device_tensor(W.f32_to_bf16_bits(rng.standard_normal(w.u.shape, dtype=np.float32)), "cuda"))
+    hosts = [u.cpu().pin_memory() for u in us]
+    outs = [layer.host_outputs() for _ in us]
+    for u_h, o in zip(hosts, outs):
+        layer.forward_host_pipelined(u_h, o)
+    layer.pipeline_wait()
+    torch.cuda.synchronize()
+    layer.device_status()
+    for u, o in zip(us, outs):
+        dev = layer.forward(u)
+        torch.cuda.synchronize()
+        for x, y in zip(dev, o):
+            assert torch.equal(x.cpu(), y)
+    layer.device_status()
+
+
 def test_expert_psum_and_balance_loss_kernel():
     w = W.make_workload("2b", T=1000)
     g, layer, u, out = run(w)
