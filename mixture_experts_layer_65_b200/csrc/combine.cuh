@@ -44,6 +44,8 @@ __device__ __forceinline__ void add8(float (&acc)[8], const uint4& v, float w) {
 template <int MAXK>
 __global__ void __launch_bounds__(kCombineWarps * 32)
 combine_bf16_kernel(CombineArgs<__nv_bfloat16> a) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * kCombineWarps + warp;
   if (t >= a.T_) return;
@@ -92,6 +94,8 @@ combine_bf16_kernel(CombineArgs<__nv_bfloat16> a) {
 
 // fp32 rows: 4 elements per 16-byte vector
 static __global__ void __launch_bounds__(kCombineWarps * 32) combine_f32_kernel(CombineArgs<float> a) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * kCombineWarps + warp;
   if (t >= a.T_) return;

@@ -38,6 +38,8 @@ struct SimtGemmArgs {
 
 template <int MODE>
 __global__ void __launch_bounds__(kSimtThreads) grouped_gemm_simt_kernel(SimtGemmArgs a) {
+  pdl_launch_dependents();
+  pdl_wait();
   __shared__ float As[kSimtBK][kSimtBM + 4];
   __shared__ float Bs[2][kSimtBK][kSimtBN + 4];
   const int tid = threadIdx.x;

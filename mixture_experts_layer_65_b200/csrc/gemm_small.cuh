@@ -59,6 +59,7 @@ grouped_gemm_small_kernel(const __grid_constant__ CUtensorMap tmW_s,
                           const __grid_constant__ CUtensorMap tmW_r,
                           const __grid_constant__ CUtensorMap tmX_s,
                           const __grid_constant__ CUtensorMap tmX_r, SmallGemmArgs a) {
+  pdl_launch_dependents();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -78,7 +79,6 @@ grouped_gemm_small_kernel(const __grid_constant__ CUtensorMap tmW_s,
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int total = __ldg(&a.ts[a.G]);
   uint32_t tmem_cols = 32;
   while (tmem_cols < 2u * (uint32_t)nt) tmem_cols <<= 1;
 
@@ -107,6 +107,8 @@ grouped_gemm_small_kernel(const __grid_constant__ CUtensorMap tmW_s,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();   // the tile tables and operands come from the previous kernels
+  const int total = __ldg(&a.ts[a.G]);
 
   // tile -> (group g, weight tile m); GemmArgs-style decode with one token tile per group
   auto decode = [&](int tile, int& g, int& m, int& e, bool& sh) {

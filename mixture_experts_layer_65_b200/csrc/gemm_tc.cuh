@@ -103,6 +103,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
                        const __grid_constant__ CUtensorMap tmA_r,
                        const __grid_constant__ CUtensorMap tmB_s,
                        const __grid_constant__ CUtensorMap tmB_r, GemmArgs a) {
+  pdl_launch_dependents();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -119,7 +120,6 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
   const uint32_t rank = cluster_ctarank();            // 0 = leader, 1 = peer
   const bool leader = rank == 0;
   const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
-  const int total = __ldg(&a.ts[a.G]);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kGemmStages; ++s) {
@@ -146,6 +146,8 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
   cluster_sync_all();   // barriers of both CTAs initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();   // the tile tables and operands come from the previous kernels
+  const int total = __ldg(&a.ts[a.G]);
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer

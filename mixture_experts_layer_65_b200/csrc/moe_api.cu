@@ -95,6 +95,8 @@ bool encode_3d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, 
 
 __global__ void balance_loss_kernel(const int32_t* counts, const float* psum, int n, double inv_t,
                                     float alpha1, float* out) {
+  pdl_launch_dependents();
+  pdl_wait();
   if (threadIdx.x == 0 && blockIdx.x == 0) {
     double acc = 0.0;
     for (int i = 0; i < n; ++i) acc += ((double)counts[i] * inv_t) * ((double)psum[i] * inv_t);
@@ -518,14 +520,14 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
                     H->router_tmem_cols, H->bias, ro};
     const int rgrid = H->n_tiles < H->n_sms ? H->n_tiles : H->n_sms;
     with_maxc(H->maxc, [&](auto m) {
-      router_tc_kernel<m()><<<rgrid, kRouterThreads, H->router_smem, stream>>>(tmUr, H->tmE, ra);
+      launch_pdl(router_tc_kernel<m()>, dim3(rgrid), dim3(kRouterThreads), H->router_smem, stream, tmUr, H->tmE, ra);
       return 0;
     });
   } else {
     RouterSimtArgs ra{static_cast<const float*>(u), static_cast<const float*>(H->centroids), H->bias,
                       T, d, nr, K, ro};
     with_maxc(H->maxc, [&](auto m) {
-      router_simt_kernel<m()><<<H->n_tiles, kRouterEpiThreads, H->simt_router_smem, stream>>>(ra);
+      launch_pdl(router_simt_kernel<m()>, dim3(H->n_tiles), dim3(kRouterEpiThreads), H->simt_router_smem, stream, ra);
       return 0;
     });
   }
@@ -539,7 +541,7 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
               H->tile_base, H->grp_row, H->ts1, H->ts2,
               H->fuse_permute ? H->copy_done : nullptr};
   tick(H, stream, 1);
-  scan_kernel<<<1, kScanThreads, 0, stream>>>(sa);
+  launch_pdl(scan_kernel, dim3(1), dim3(kScanThreads), 0, stream, sa);
   MOE_CUDA(cudaGetLastError());
 
   PermuteArgs pa{static_cast<const uint8_t*>(u), topk_idx, H->topk_rank, H->tile_base, H->slot_row,
@@ -547,7 +549,7 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
                  d * H->es, H->err};
   tick(H, stream, 2);
   if (!H->fuse_permute) {
-    permute_kernel<<<(T + kPermuteWarps - 1) / kPermuteWarps, kPermuteWarps * 32, 0, stream>>>(pa);
+    launch_pdl(permute_kernel, dim3((T + kPermuteWarps - 1) / kPermuteWarps), dim3(kPermuteWarps * 32), 0, stream, pa);
     MOE_CUDA(cudaGetLastError());
   }
 
@@ -565,8 +567,7 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
     s1.out_routed = static_cast<__nv_bfloat16*>(H->hr); s1.ld_routed = I;
     s1.err = H->err;
     tick(H, stream, 3);
-    grouped_gemm_small_kernel<kGateUpSwiGLU><<<H->n_sms, kSmallThreads, H->small_smem, stream>>>(
-        H->tmWguS, H->tmWguR, tmUN, H->tmXpN, s1);
+    launch_pdl(grouped_gemm_small_kernel<kGateUpSwiGLU>, dim3(H->n_sms), dim3(kSmallThreads), H->small_smem, stream,  H->tmWguS, H->tmWguR, tmUN, H->tmXpN, s1);
     MOE_CUDA(cudaGetLastError());
     SmallGemmArgs s2 = s1;
     s2.ts = H->ts2;
@@ -575,8 +576,7 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
     s2.out_shared = static_cast<__nv_bfloat16*>(H->ys); s2.ld_shared = d;
     s2.out_routed = static_cast<__nv_bfloat16*>(H->yr); s2.ld_routed = d;
     tick(H, stream, 4);
-    grouped_gemm_small_kernel<kDown><<<H->n_sms, kSmallThreads, H->small_smem, stream>>>(
-        H->tmWdS, H->tmWdR, H->tmHsN, H->tmHrN, s2);
+    launch_pdl(grouped_gemm_small_kernel<kDown>, dim3(H->n_sms), dim3(kSmallThreads), H->small_smem, stream,  H->tmWdS, H->tmWdR, H->tmHsN, H->tmHrN, s2);
     MOE_CUDA(cudaGetLastError());
   } else if (H->bf16) {
     GemmArgs g1{};
@@ -593,8 +593,7 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
       g1.copy_done = H->copy_done;
     }
     tick(H, stream, 3);
-    grouped_gemm_tc_kernel<kGateUpSwiGLU><<<H->gemm_grid, kGemmThreads, kGemmSmemBytes, stream>>>(
-        tmU, H->tmXp, H->tmWguS, H->tmWguR, g1);
+    launch_pdl(grouped_gemm_tc_kernel<kGateUpSwiGLU>, dim3(H->gemm_grid), dim3(kGemmThreads), kGemmSmemBytes, stream,  tmU, H->tmXp, H->tmWguS, H->tmWguR, g1);
     MOE_CUDA(cudaGetLastError());
 
     GemmArgs g2{};
@@ -607,8 +606,7 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
     g2.cols_routed = d;
     g2.err = H->err;
     tick(H, stream, 4);
-    grouped_gemm_tc_kernel<kDown><<<H->gemm_grid, kGemmThreads, kGemmSmemBytes, stream>>>(
-        H->tmHs, H->tmHr, H->tmWdS, H->tmWdR, g2);
+    launch_pdl(grouped_gemm_tc_kernel<kDown>, dim3(H->gemm_grid), dim3(kGemmThreads), kGemmSmemBytes, stream,  H->tmHs, H->tmHr, H->tmWdS, H->tmWdR, g2);
     MOE_CUDA(cudaGetLastError());
   } else {
     const size_t ks = c.n_shared;
@@ -629,7 +627,7 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
     s1.out_routed = static_cast<float*>(H->hr); s1.out_rows_routed = H->rows_cap;
     s1.err = H->err;
     tick(H, stream, 3);
-    grouped_gemm_simt_kernel<kGateUpSwiGLU><<<grid, kSimtThreads, 0, stream>>>(s1);
+    launch_pdl(grouped_gemm_simt_kernel<kGateUpSwiGLU>, dim3(grid), dim3(kSimtThreads), 0, stream, s1);
     MOE_CUDA(cudaGetLastError());
 
     SimtGemmArgs s2{};
@@ -646,14 +644,14 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
     s2.out_routed = static_cast<float*>(H->yr); s2.out_rows_routed = H->rows_cap;
     s2.err = H->err;
     tick(H, stream, 4);
-    grouped_gemm_simt_kernel<kDown><<<grid, kSimtThreads, 0, stream>>>(s2);
+    launch_pdl(grouped_gemm_simt_kernel<kDown>, dim3(grid), dim3(kSimtThreads), 0, stream, s2);
     MOE_CUDA(cudaGetLastError());
 
     CombineArgs<float> ca{static_cast<const float*>(u), static_cast<const float*>(H->ys),
                           static_cast<const float*>(H->yr), H->slot_row, topk_w,
                           static_cast<float*>(h), T, d, K};
     tick(H, stream, 5);
-    combine_f32_kernel<<<(T + kCombineWarps - 1) / kCombineWarps, kCombineWarps * 32, 0, stream>>>(ca);
+    launch_pdl(combine_f32_kernel, dim3((T + kCombineWarps - 1) / kCombineWarps), dim3(kCombineWarps * 32), 0, stream, ca);
     MOE_CUDA(cudaGetLastError());
   }
   if (H->bf16) {
@@ -664,7 +662,7 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
     tick(H, stream, 5);
     const int cgrid = (T + kCombineWarps - 1) / kCombineWarps;
     with_maxk(H->maxk, [&](auto m) {
-      combine_bf16_kernel<m()><<<cgrid, kCombineWarps * 32, 0, stream>>>(ca);
+      launch_pdl(combine_bf16_kernel<m()>, dim3(cgrid), dim3(kCombineWarps * 32), 0, stream, ca);
       return 0;
     });
     MOE_CUDA(cudaGetLastError());
@@ -832,8 +830,7 @@ moe_status moe_balance_loss(const int32_t* counts, const float* psum, int32_t n_
                             int64_t n_tokens, float alpha1, float* aux_loss, moe_stream_t stream_) {
   if (!counts || !psum || !aux_loss) return fail(MOE_ERR_INVALID_ARG, "a pointer is NULL");
   if (n_routed < 1 || n_tokens < 1) return fail(MOE_ERR_INVALID_ARG, "n_routed and n_tokens must be positive");
-  balance_loss_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream_)>>>(
-      counts, psum, n_routed, 1.0 / (double)n_tokens, alpha1, aux_loss);
+  launch_pdl(balance_loss_kernel, dim3(1), dim3(32), 0, reinterpret_cast<cudaStream_t>(stream_),  counts, psum, n_routed, 1.0 / (double)n_tokens, alpha1, aux_loss);
   MOE_CUDA(cudaGetLastError());
   return MOE_OK;
 }

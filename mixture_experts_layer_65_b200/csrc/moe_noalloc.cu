@@ -87,7 +87,7 @@ cudaError_t launch_router(const CUtensorMap& tmU, const CUtensorMap& tmE, const 
   cudaError_t e = cudaFuncSetAttribute((const void*)router_tc_kernel<MAXC>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  router_tc_kernel<MAXC><<<grid, kRouterThreads, smem, st>>>(tmU, tmE, ra);
+  launch_pdl(router_tc_kernel<MAXC>, dim3(grid), dim3(kRouterThreads), smem, st, tmU, tmE, ra);
   return cudaGetLastError();
 }
 
@@ -173,7 +173,7 @@ extern "C" moe_status moe_route_noalloc(const void* u, const void* centroids, co
               aux_loss, reinterpret_cast<float*>(sc + kOffPsumTot),
               reinterpret_cast<int32_t*>(sc + kOffBase), reinterpret_cast<int32_t*>(sc + kOffGrp),
               reinterpret_cast<int32_t*>(sc + kOffTs1), reinterpret_cast<int32_t*>(sc + kOffTs2)};
-  scan_kernel<<<1, kScanThreads, 0, st>>>(sa);
+  launch_pdl(scan_kernel, dim3(1), dim3(kScanThreads), 0, st, sa);
   if (cudaGetLastError() != cudaSuccess) return nfail(MOE_ERR_CUDA, "moe_route_noalloc: scan launch failed");
   if (device_error &&
       cudaMemcpyAsync(device_error, err, sizeof(int32_t), cudaMemcpyDeviceToDevice, st) != cudaSuccess)

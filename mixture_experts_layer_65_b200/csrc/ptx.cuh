@@ -8,6 +8,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace moe {
 
 // ----------------------------------------------------------------------------- errors
@@ -122,6 +124,35 @@ __device__ __forceinline__ bool counter_wait(const int* counter, int target, vol
       }
     }
   }
+}
+
+// ------------------------------------------------------ programmatic dependent launch
+// Every kernel of the layer signals at entry that the next kernel in the stream may be
+// scheduled (its CTAs then run their prologue while this grid finishes: the signal of a
+// grid counts once all of its CTAs have given it or exited, i.e. once all of them are
+// resident, so a waiting dependent never keeps one of them off an SM), and waits for
+// the previous kernel's completion and memory before reading anything that kernel or an
+// earlier one wrote.  Both are no-ops in a launch without programmatic serialisation.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Host side: launch `kernel` on `stream` with programmatic stream serialisation.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 // ----------------------------------------------------------------------------- TMA

@@ -354,6 +354,7 @@ template <int MAXC>
 __global__ void __launch_bounds__(kRouterThreads, 1)
 router_tc_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmE,
                  RouterTcArgs a) {
+  pdl_launch_dependents();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -395,6 +396,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant_
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();   // u (and the bias) may come from the previous kernel
 
   if (warp == 0) {
     if (lane == 0) {
@@ -543,6 +545,8 @@ struct RouterSimtArgs {
 // router_epi_bytes(n_pad).
 template <int MAXC>
 __global__ void __launch_bounds__(kRouterEpiThreads) router_simt_kernel(RouterSimtArgs a) {
+  pdl_launch_dependents();
+  pdl_wait();
   extern __shared__ __align__(16) uint8_t smem_raw[];
   RouterEpiSmem& SM = *reinterpret_cast<RouterEpiSmem*>(smem_raw);
   float* lg = reinterpret_cast<float*>(smem_raw + sizeof(RouterEpiSmem));

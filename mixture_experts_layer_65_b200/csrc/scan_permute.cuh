@@ -38,6 +38,8 @@ struct ScanArgs {
 };
 
 static __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a) {
+  pdl_launch_dependents();
+  pdl_wait();
   __shared__ int32_t s_cnt[kScanThreads];
   __shared__ float s_ps[kScanThreads];
   __shared__ int32_t s_base[kScanThreads];
@@ -208,6 +210,8 @@ __device__ __forceinline__ void permute_token(const PermuteArgs& a, int t, int l
 }
 
 static __global__ void __launch_bounds__(kPermuteWarps * 32) permute_kernel(PermuteArgs a) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * kPermuteWarps + warp;
   if (t >= a.T) return;
