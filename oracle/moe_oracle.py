@@ -43,7 +43,8 @@ import numpy as np
 
 __all__ = ["widen", "router_logits", "affinity_softmax", "select_topk", "route",
            "swiglu_ffn", "balance_stats", "moe_forward", "near_tie_tokens",
-           "brute_force_layer", "Routing", "LayerOut"]
+           "brute_force_layer", "Routing", "LayerOut", "E4M3_MAX", "e4m3_round",
+           "quantize_rows_e4m3"]
 
 
 def widen(a) -> np.ndarray:
@@ -105,12 +106,63 @@ def _silu(z: np.ndarray) -> np.ndarray:
         return z / (1.0 + np.exp(-z))
 
 
-def swiglu_ffn(x, w_gate, w_up, w_down) -> np.ndarray:
-    """FFN(x) = W_down (SiLU(W_gate x) * (W_up x)); x [n, d], W_gate/W_up [I, d], W_down [d, I]."""
+def swiglu_ffn(x, w_gate, w_up, w_down, gate_up_e4m3: bool = False) -> np.ndarray:
+    """FFN(x) = W_down (SiLU(W_gate x) * (W_up x)); x [n, d], W_gate/W_up [I, d], W_down [d, I].
+
+    gate_up_e4m3: the e4m3 variant -- x's rows and W_gate's / W_up's rows are replaced by
+    their scaled e4m3 approximations (quantize_rows_e4m3) in the two gate/up products."""
+    if gate_up_e4m3:
+        x, w_gate, w_up = _dequantized(x), _dequantized(w_gate), _dequantized(w_up)
     x = widen(x)
     a = x @ widen(w_gate).T
     b = x @ widen(w_up).T
     return (_silu(a) * b) @ widen(w_down).T
+
+
+# ---------------------------------------------------------------- e4m3 gate/up variant
+# Not on the pages: a reduced-precision variant of the layer in which the gate/up
+# products take e4m3 operands.  Each token row and each gate/up weight row (one output
+# channel, d values) is quantised with its own fp32 scale; everything else (router,
+# down projection, residual, combine) is the plain layer.  Definition, per row x of
+# fp32-valued entries:  a = max_i |x_i|;  if a = 0 every q_i = 0 and the scale is 0;
+# otherwise inv = fp32(448 / a), q_i = e4m3(fp32(x_i * inv)) and scale = fp32(a / 448),
+# so that x_i ~ q_i * scale.  e4m3 is the 8-bit float with 1 sign, 4 exponent (bias 7)
+# and 3 mantissa bits, no infinities, largest finite value 448; e4m3(y) rounds to the
+# nearest value, ties to the even mantissa, and clamps |y| > 448 to 448.
+E4M3_MAX = 448.0
+
+
+def e4m3_round(y) -> np.ndarray:
+    """Nearest e4m3 value of each entry (ties to even), saturating at +-448."""
+    y = np.asarray(y, dtype=np.float64)
+    a = np.abs(y)
+    out = np.zeros_like(a)
+    big = a > E4M3_MAX
+    nz = (a > 0) & ~big
+    e = np.maximum(np.floor(np.log2(a[nz])), -6.0)   # binade; below 2^-6 the subnormal step
+    step = np.exp2(e - 3.0)                          # 3 mantissa bits
+    out[nz] = np.rint(a[nz] / step) * step
+    out[big] = E4M3_MAX
+    return np.copysign(out, y)
+
+
+def quantize_rows_e4m3(x):
+    """Per-row scaled e4m3 quantisation (definition above).  Returns (q [n, m] fp64 with
+    e4m3 values, scale [n] fp64 with fp32 values); x_i is approximated by q_i * scale."""
+    x32 = np.ascontiguousarray(widen(x), dtype=np.float32)   # bf16/fp32 values are exact
+    a = np.max(np.abs(x32), axis=1)
+    safe = np.where(a > 0, a, np.float32(1.0)).astype(np.float32)
+    inv = (np.float32(E4M3_MAX) / safe).astype(np.float32)
+    y = (x32 * inv[:, None]).astype(np.float32)
+    q = e4m3_round(y.astype(np.float64))
+    q[a == 0] = 0.0
+    scale = np.where(a > 0, (safe / np.float32(E4M3_MAX)).astype(np.float32), np.float32(0.0))
+    return q, scale.astype(np.float64)
+
+
+def _dequantized(x) -> np.ndarray:
+    q, scale = quantize_rows_e4m3(x)
+    return q * scale[:, None]
 
 
 # ---------------------------------------------------------------- balance statistics
@@ -141,7 +193,7 @@ class LayerOut:
 
 
 def moe_forward(u, centroids, w_gate, w_up, w_down, n_shared: int, top_k: int,
-                alpha1: float, bias=None, rows=None) -> LayerOut:
+                alpha1: float, bias=None, rows=None, gate_up_e4m3: bool = False) -> LayerOut:
     """h = u + sum_{j shared} FFN_j(u) + sum_{i routed, selected} g_i FFN_i(u).
 
     Weights: w_gate/w_up [n_shared + N_r, I, d], w_down [n_shared + N_r, d, I], shared
@@ -149,6 +201,8 @@ def moe_forward(u, centroids, w_gate, w_up, w_down, n_shared: int, top_k: int,
     all T tokens; `rows` (token ids) restricts only which output rows are computed.
     Per routed expert the selecting tokens are gathered and run as one fp64 GEMM chain
     (the grouping the deepforge article names for production implementations).
+    gate_up_e4m3 selects the e4m3 gate/up variant (quantize_rows_e4m3); routing, the
+    residual and the down projection use the unquantised values either way.
     """
     u64 = widen(u)
     T = u64.shape[0]
@@ -160,7 +214,7 @@ def moe_forward(u, centroids, w_gate, w_up, w_down, n_shared: int, top_k: int,
     x = u64[rows]
     h = x.copy()                                          # residual
     for j in range(n_shared):                             # shared experts, gate 1
-        h += swiglu_ffn(x, w_gate[j], w_up[j], w_down[j])
+        h += swiglu_ffn(x, w_gate[j], w_up[j], w_down[j], gate_up_e4m3)
     sel = r.topk_idx[rows]                                # [n, K']
     gate = r.topk_w[rows]
     for e in range(n_routed):
@@ -168,7 +222,7 @@ def moe_forward(u, centroids, w_gate, w_up, w_down, n_shared: int, top_k: int,
         if hit_r.size == 0:
             continue
         y = swiglu_ffn(x[hit_r], w_gate[n_shared + e], w_up[n_shared + e],
-                       w_down[n_shared + e])
+                       w_down[n_shared + e], gate_up_e4m3)
         h[hit_r] += gate[hit_r, hit_k][:, None] * y
     return LayerOut(h=h, rows=rows, routing=r, counts=counts, f=f, P=P, aux=aux)
 

@@ -294,3 +294,82 @@ def test_workload_is_seeded_and_prefix_stable():
     assert z.logit_bias is not None and z.logit_bias.shape == (16,)
     assert np.all(np.diff(z.logit_bias) < 0)
     np.testing.assert_allclose(np.exp(z.logit_bias.astype(np.float64)).sum(), 1.0, rtol=1e-6)
+
+
+# ------------------------------------------------------------------ e4m3 gate/up variant
+def _e4m3_values() -> np.ndarray:
+    """Every finite e4m3 value, decoded from its bit pattern by torch's float8 type."""
+    bits = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    v = bits.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    return np.unique(v[np.isfinite(v)])
+
+
+def test_e4m3_round_matches_torch_and_the_value_grid():
+    grid = _e4m3_values()
+    assert grid.size == 253 and grid.max() == O.E4M3_MAX      # 126 per sign, +0 and -0 merge
+    np.testing.assert_array_equal(O.e4m3_round(grid), grid)   # representable values stay
+    pos = grid[grid >= 0]
+    mids = (pos[:-1] + pos[1:]) / 2                           # exact ties: to the even mantissa
+    rng = np.random.default_rng(3)
+    y = np.concatenate([mids, -mids, rng.uniform(-448, 448, 20000), rng.uniform(-0.03, 0.03, 20000)])
+    y = y.astype(np.float32).astype(np.float64)
+    ref = torch.from_numpy(y).to(torch.float32).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    np.testing.assert_array_equal(O.e4m3_round(y), ref)
+    # saturation beyond the largest finite value
+    np.testing.assert_array_equal(O.e4m3_round(np.array([448.5, 463.9, 1e9, -500.0])),
+                                  [448.0, 448.0, 448.0, -448.0])
+
+
+def test_quantize_rows_e4m3_scales_and_error_bound():
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal((64, 300)).astype(np.float32)
+    x[5] = 0.0                                                # an all-zero row
+    q, s = O.quantize_rows_e4m3(x)
+    grid = set(_e4m3_values().tolist())
+    assert set(np.unique(q).tolist()) <= grid
+    a = np.abs(x).max(axis=1)
+    assert s[5] == 0.0 and np.all(q[5] == 0.0)
+    nz = a > 0
+    # the row maximum maps to +-448 and the scale is fp32(a / 448)
+    np.testing.assert_array_equal(np.abs(q[nz]).max(axis=1), O.E4M3_MAX)
+    np.testing.assert_array_equal(s[nz], (a[nz] / np.float32(448)).astype(np.float32))
+    # half an e4m3 step: 2^-4 relative in the normal range, 2^-10 * scale below it
+    err = np.abs(x.astype(np.float64) - q * s[:, None])
+    bound = 2.0 ** -4 * np.abs(x) * (1 + 1e-6) + 2.0 ** -10 * s[:, None] * (1 + 1e-6)
+    assert np.all(err <= bound)
+
+
+def test_e4m3_variant_is_exact_when_quantisation_is_lossless():
+    # rows whose entries are e4m3 values times 2^k with the row maximum at 448 * 2^k
+    # quantise without loss, so the variant must equal the plain layer
+    rng = np.random.default_rng(6)
+    grid = _e4m3_values()
+    grid = grid[np.abs(grid) > 0.5]
+
+    def lossless(shape, k):
+        v = rng.choice(grid, size=shape)
+        v[..., 0] = O.E4M3_MAX
+        return v * 2.0 ** k
+
+    T, d, ns, nr, I, K = 40, 64, 1, 6, 32, 2
+    u = lossless((T, d), -9)
+    cen = rng.standard_normal((nr, d)) / 8
+    wg = lossless((ns + nr, I, d), -12)
+    wu = lossless((ns + nr, I, d), -11)
+    wd = rng.standard_normal((ns + nr, d, I)) * 0.02
+    a = O.moe_forward(u, cen, wg, wu, wd, ns, K, 0.01)
+    b = O.moe_forward(u, cen, wg, wu, wd, ns, K, 0.01, gate_up_e4m3=True)
+    np.testing.assert_array_equal(a.routing.topk_idx, b.routing.topk_idx)
+    np.testing.assert_allclose(b.h, a.h, rtol=1e-13, atol=1e-13)
+
+
+def test_e4m3_variant_changes_only_the_expert_part_and_by_little():
+    w = W.make_workload("tiny")
+    a = O.moe_forward(w.u, w.centroids, w.w_gate, w.w_up, w.w_down, w.n_shared, w.top_k, w.alpha1)
+    b = O.moe_forward(w.u, w.centroids, w.w_gate, w.w_up, w.w_down, w.n_shared, w.top_k, w.alpha1,
+                      gate_up_e4m3=True)
+    np.testing.assert_array_equal(a.routing.topk_idx, b.routing.topk_idx)   # routing untouched
+    assert a.aux == b.aux
+    u = O.widen(w.u)
+    rel = np.abs((b.h - u) - (a.h - u)).max() / np.abs(a.h - u).max()
+    assert 1e-4 < rel < 0.1, rel                                           # quantised, not broken
