@@ -64,7 +64,8 @@ def load_peaks():
 
 def workload_desc(w, n_gpus: int) -> dict:
     return {"workload": f"{w.name}: T={w.T} d={w.d} shared={w.n_shared} routed={w.n_routed} "
-                        f"inter={w.inter} top_k={w.top_k} {w.dtype}",
+                        f"inter={w.inter} top_k={w.top_k} {w.dtype}"
+                        f"{' (gate/up e4m3)' if getattr(w, 'gate_up_e4m3', False) else ''}",
             "T_per_gpu": w.T, "d": w.d, "n_shared": w.n_shared, "n_routed": w.n_routed,
             "inter": w.inter, "top_k": w.top_k, "global_batch": w.T * n_gpus,
             "parallelism": f"dp{n_gpus}"}
@@ -176,7 +177,7 @@ def oracle_tokens_per_s(w, seconds: float) -> tuple[float, dict]:
     def run(n):
         t0 = time.perf_counter()
         O.moe_forward(w.u[:n], w.centroids, w.w_gate, w.w_up, w.w_down, w.n_shared, w.top_k,
-                      w.alpha1, bias=w.logit_bias)
+                      w.alpha1, bias=w.logit_bias, gate_up_e4m3=w.gate_up_e4m3)
         return time.perf_counter() - t0
 
     # grow the sample until one call takes about `seconds` (the oracle has a per-call cost
@@ -208,7 +209,7 @@ def run_reference(args, rank: int, world: int):
 
     t0 = time.perf_counter()
     O.moe_forward(w.u[:16], w.centroids, w.w_gate, w.w_up, w.w_down, w.n_shared, w.top_k,
-                  w.alpha1, bias=w.logit_bias)
+                  w.alpha1, bias=w.logit_bias, gate_up_e4m3=w.gate_up_e4m3)
     per_tok = (time.perf_counter() - t0) / 16
     n = int(max(1, min(w.T, budget / max(per_tok, 1e-9))))
     times = []
@@ -216,7 +217,7 @@ def run_reference(args, rank: int, world: int):
         s = (i * n) % max(1, w.T - n + 1)
         t0 = time.perf_counter()
         O.moe_forward(w.u[s:s + n], w.centroids, w.w_gate, w.w_up, w.w_down, w.n_shared,
-                      w.top_k, w.alpha1, bias=w.logit_bias)
+                      w.top_k, w.alpha1, bias=w.logit_bias, gate_up_e4m3=w.gate_up_e4m3)
         if i >= args.warmup:
             times.append(time.perf_counter() - t0)
     tot = sum(times)
@@ -362,20 +363,29 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     peaks, peak_src = load_peaks()
     work = algorithmic_work(w, int((out.expert_counts > 0).sum().item()))
     per_kernel = {}
+    # e4m3 gate/up variant: that GEMM's peak is the measured bf16 peak times the nominal
+    # dense e4m3 : bf16 ratio (4.5 : 2.25 PFLOP/s), and the token rows are quantised (one
+    # extra kernel, timed in the permute slot)
+    e4m3 = bool(getattr(w, "gate_up_e4m3", False))
+    tensor_ratio = {k: (2.0 if (e4m3 and k == "gate_up_gemm") else 1.0) for k in KERNELS}
+    if e4m3:
+        work["permute"] = ("hbm", w.T * w.d * 3 + w.T * 4)   # quantise: bf16 in, e4m3 + scale out
     # with a shared group the paired bf16 GEMM copies the routed rows itself (its copy
     # warps run beside the shared group's tiles): no permute kernel is launched
-    fused_permute = layer.kernels_per_forward == len(KERNELS) - 1
+    fused_permute = layer.kernels_per_forward - (1 if e4m3 else 0) == len(KERNELS) - 1
     for k in KERNELS:
         kind, amount = work[k]
         avg_ms = kernel_ms[k] / max(1, n_rec)
         ent = {"avg_ms": avg_ms, "share": kernel_ms[k] / max(1e-12, sum(kernel_ms.values()))}
-        if k == "permute" and fused_permute:
+        if k == "permute" and fused_permute and not e4m3:
             ent.update(fused_into="gate_up_gemm")
         elif kind == "tensor":
             ach = amount / (avg_ms * 1e-3) / 1e12
             ent.update(bound="tensor", achieved=ach, unit="TFLOP/s",
-                       frac=ach / peaks["bf16_tflops_sustained"],
-                       frac_of_burst=ach / peaks["bf16_tflops"])
+                       frac=ach / (tensor_ratio[k] * peaks["bf16_tflops_sustained"]),
+                       frac_of_burst=ach / (tensor_ratio[k] * peaks["bf16_tflops"]))
+            if tensor_ratio[k] != 1.0:
+                ent.update(operands="e4m3", peak_note="measured bf16 peak x 2 (nominal dense e4m3/bf16)")
         elif kind == "hbm":
             ach = amount / (avg_ms * 1e-3) / 1e9
             ent.update(bound="hbm", achieved=ach, unit="GB/s", frac=ach / peaks["hbm_gbs"])
@@ -384,27 +394,33 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     dk = per_kernel[dominant]
     bound = dk.get("bound", "latency")
     roofline = {"kernel": dominant, "bound": bound, "achieved": dk.get("achieved"),
-                "peak": (peaks["bf16_tflops_sustained"] if bound == "tensor" else peaks["hbm_gbs"]),
+                "peak": (tensor_ratio[dominant] * peaks["bf16_tflops_sustained"] if bound == "tensor"
+                         else peaks["hbm_gbs"]),
                 "unit": dk.get("unit"), "frac": dk.get("frac"),
-                "peak_source": f"{peak_src} ({'bf16 sustained' if bound == 'tensor' else 'HBM copy'})",
+                "peak_source": f"{peak_src} ({'HBM copy' if bound != 'tensor' else 'bf16 sustained' if tensor_ratio[dominant] == 1.0 else 'bf16 sustained x 2 for e4m3 operands'})",
                 "traffic": ncu_traffic(dominant, w.name), "algorithmic_per_launch": work[dominant][1]}
     gemm_flops = 6.0 * w.T * w.d * w.inter * (w.n_shared + w.top_k)
     gemm_ms = (kernel_ms["gate_up_gemm"] + kernel_ms["down_gemm"]) / max(1, n_rec)
     gemm_tflops = gemm_flops / (gemm_ms * 1e-3) / 1e12
+    # fraction of peak = time at peak / measured time (each GEMM at its operands' peak)
+    ideal = {key: sum(work[k][1] / (tensor_ratio[k] * peaks[key] * 1e12)
+                      for k in ("gate_up_gemm", "down_gemm"))
+             for key in ("bf16_tflops_sustained", "bf16_tflops")}
     value = world * w.T * args.steps / (ms * 1e-3)
     tk = w.T * w.top_k
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms / args.steps,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 (gate/up GEMM on e4m3 operands)" if e4m3 else w.dtype,
         "data": "synthetic (seeded N(0,1) tokens, N(0,0.02) random-init experts, no trained weights)",
         "config": dict(workload_desc(w, world),
                        l2=f"inputs rotate over {n_buf} token buffers "
                           f"({n_buf * u_bytes / 2**20:.0f} MiB > 126 MiB L2); expert weights "
                           f"{layer.device_bytes / 2**30:.2f} GiB with workspace"),
         "expert_gemm_tflops": gemm_tflops,
-        "expert_gemm_frac_of_peak": gemm_tflops / peaks["bf16_tflops_sustained"],
-        "expert_gemm_frac_of_burst_peak": gemm_tflops / peaks["bf16_tflops"],
+        "expert_gemm_frac_of_peak": ideal["bf16_tflops_sustained"] / (gemm_ms * 1e-3),
+        "expert_gemm_frac_of_burst_peak": ideal["bf16_tflops"] / (gemm_ms * 1e-3),
         "roofline": roofline,
         "kernels": per_kernel,
         "e2e": None if e2e_ms is None else {

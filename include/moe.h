@@ -49,7 +49,16 @@ typedef enum {
   MOE_ERR_DEVICE_CHECK = 5  /* a kernel recorded an error (bounded wait ran out, ...) */
 } moe_status;
 
-typedef enum { MOE_FP32 = 0, MOE_BF16 = 1 } moe_dtype;
+/* MOE_BF16_E4M3_GATEUP: a bf16 layer (bf16 inputs, weights and outputs) whose gate/up
+ * GEMM runs on e4m3 operands -- a reduced-precision variant this library adds (the
+ * DeepSeekMoE pages define the layer only in full precision).  Every token row and
+ * every gate/up weight row (one output channel, d values) is quantised with its own
+ * fp32 scale: a = max |x_i|; a = 0 gives q = 0 and scale 0; otherwise
+ * q_i = e4m3(fp32(x_i * fp32(448 / a))) (round to nearest even, saturating at 448) and
+ * scale = fp32(a / 448).  The gate/up products are computed on q with fp32 accumulation
+ * and multiplied by the two row scales; the router, the down projection, the residual and
+ * the combine are those of MOE_BF16.  Needs d % 128 == 0. */
+typedef enum { MOE_FP32 = 0, MOE_BF16 = 1, MOE_BF16_E4M3_GATEUP = 2 } moe_dtype;
 
 /* Layer description.  All weight pointers are DEVICE pointers in `dtype`, read only
  * during moe_create (the library keeps its own re-laid-out copy; the caller may free
@@ -66,7 +75,8 @@ typedef enum { MOE_FP32 = 0, MOE_BF16 = 1 } moe_dtype;
  *   w_up       [n_shared + n_routed, inter, d]
  *   w_down     [n_shared + n_routed, d, inter]
  * bf16 layers need d % 64 == 0 and inter % 64 == 0 (MOE_ERR_UNSUPPORTED otherwise);
- * fp32 layers need d % 4 == 0. */
+ * MOE_BF16_E4M3_GATEUP layers also d % 128 == 0; fp32 layers need d % 4 == 0.  The
+ * weights of MOE_BF16_E4M3_GATEUP layers are given in bf16 and quantised by moe_create. */
 typedef struct {
   int32_t T;
   int32_t d;

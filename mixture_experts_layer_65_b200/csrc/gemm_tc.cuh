@@ -79,6 +79,14 @@ struct GemmArgs {
   // of this kernel).
   PermuteArgs perm;
   int* copy_done;
+  // e4m3 operands (kernel template F8): per-row scales of A (token rows of the shared
+  // group, permuted rows of the routed groups) and of B (gate/up weight rows in their
+  // interleaved order; routed: sb_routed + e * sb_routed_stride)
+  const float* sa_shared;
+  const float* sa_routed;
+  const float* sb_shared;
+  const float* sb_routed;
+  int64_t sb_routed_stride;
 };
 
 struct TileCoord {
@@ -97,7 +105,9 @@ __device__ __forceinline__ void gemm_decode(int tile, int& g, const GemmArgs& a,
   c.g = g;
 }
 
-template <int MODE>
+// F8: A and B are e4m3 (k-blocks of 128 elements = the same 128-byte rows), MMAs of kind
+// f8f6f4, and the gate/up epilogue multiplies each accumulator by its two row scales.
+template <int MODE, bool F8 = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
                        const __grid_constant__ CUtensorMap tmA_r,
@@ -179,7 +189,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
           if (leader)
             mbar_arrive_expect_tx(smem_u32(&full[stage]), 2u * (uint32_t)nk * (kGemmABytes + kGemmBBytes));
           for (int j = 0; j < nk; ++j) {
-            const int kx = (kb0 + j) * kGemmBK;
+            const int kx = (kb0 + j) * (F8 ? 2 * kGemmBK : kGemmBK);   // elements
             tma_load_2d_pair(sa + j * kGemmABytes, ta, fb, kx, arow);
             if (c.shared) tma_load_2d_pair(sa + kGemmBOff + j * kGemmBBytes, &tmB_s, fb, kx, brow);
             else tma_load_3d_pair(sa + kGemmBOff + j * kGemmBBytes, &tmB_r, fb, kx, brow, c.e);
@@ -199,7 +209,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0 && leader) {
-      const uint32_t idesc = idesc_bf16_f32(kPairBM, kGemmBN);
+      const uint32_t idesc = F8 ? idesc_e4m3_f32(kPairBM, kGemmBN) : idesc_bf16_f32(kPairBM, kGemmBN);
       int stage = 0, g = 0, it = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -223,8 +233,10 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
             const uint64_t adesc = sdesc_k_sw128(sa + j * kGemmABytes);
             const uint64_t bdesc = sdesc_k_sw128(sa + kGemmBOff + j * kGemmBBytes);
 #pragma unroll
-            for (int k = 0; k < kGemmBK / 16; ++k)
-              tc_mma_f16_pair(dt, adesc + 2u * k, bdesc + 2u * k, idesc, (kb0 | j | k) != 0);
+            for (int k = 0; k < 4; ++k) {   // 32-byte K steps: 16 bf16 or 32 e4m3 values
+              if (F8) tc_mma_f8_pair(dt, adesc + 2u * k, bdesc + 2u * k, idesc, (kb0 | j | k) != 0);
+              else tc_mma_f16_pair(dt, adesc + 2u * k, bdesc + 2u * k, idesc, (kb0 | j | k) != 0);
+            }
           }
           tc_commit_pair_mc(smem_u32(&empty[stage]), 0x3);
           if (++stage == kGemmStages) { stage = 0; phase ^= 1u; }
@@ -274,6 +286,13 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
       const bool row_ok = orow < rows;
       if (!row_ok) record_error(a.err, kErrOutRow);
       if (MODE == kGateUpSwiGLU) {
+        float sa = 1.f;                 // e4m3: the A row's scale, and the B rows' scales
+        const float* sbv = nullptr;
+        if (F8) {
+          sa = row_ok ? __ldg((c.shared ? a.sa_shared : a.sa_routed) + orow) : 0.f;
+          sbv = (c.shared ? a.sb_shared : a.sb_routed + (int64_t)c.e * a.sb_routed_stride) +
+                (int64_t)c.n * kGemmBN;
+        }
         {
           const int hb = half;
           const int col0 = c.n * (kGemmBN / 2) + hb * 64;
@@ -285,6 +304,14 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
             tmem_ld32(trow + static_cast<uint32_t>(hb * 128 + 64 + j), uv);
             tmem_ld_wait(gv);
             tmem_ld_wait(uv);
+            if (F8) {
+              const float* sg = sbv + hb * 128 + j;        // gate rows of these 32 columns
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                gv[i] = __float_as_uint(__uint_as_float(gv[i]) * sa * __ldg(sg + i));
+                uv[i] = __float_as_uint(__uint_as_float(uv[i]) * sa * __ldg(sg + 64 + i));
+              }
+            }
             uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {

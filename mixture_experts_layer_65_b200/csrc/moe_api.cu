@@ -21,6 +21,7 @@
 #include "gemm_small.cuh"
 #include "gemm_tc.cuh"
 #include "router.cuh"
+#include "quant.cuh"
 #include "scan_permute.cuh"
 
 using namespace moe;
@@ -93,6 +94,43 @@ bool encode_3d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, 
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// e4m3 bytes: row-major [outer, inner] matrix, box = box_outer rows x 128 columns (128 B).
+bool encode_2d_e4m3(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer,
+                    uint32_t box_outer) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner};
+  cuuint32_t box[2] = {128, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// e4m3 bytes [depth, outer, inner], box = box_outer rows x 128 columns of one matrix.
+bool encode_3d_e4m3(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer,
+                    uint64_t depth, uint32_t box_outer) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {inner, outer, depth};
+  cuuint64_t strides[2] = {inner, inner * outer};
+  cuuint32_t box[3] = {128, box_outer, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Quantise `rows` bf16 rows of `cols` values to e4m3 with per-row scales, on `st`.
+cudaError_t launch_quant(const void* src, int64_t rows, int cols, void* dst, float* scale,
+                         int n_sms, cudaStream_t st) {
+  int64_t blocks = (rows + kQuantWarps - 1) / kQuantWarps;
+  if (blocks > (int64_t)n_sms * 16) blocks = (int64_t)n_sms * 16;
+  QuantArgs qa{static_cast<const __nv_bfloat16*>(src), rows, cols, static_cast<uint8_t*>(dst), scale};
+  return launch_pdl(quant_rows_e4m3_kernel, dim3((unsigned)blocks), dim3(kQuantWarps * 32), 0, st, qa);
+}
+
 __global__ void balance_loss_kernel(const int32_t* counts, const float* psum, int n, double inv_t,
                                     float alpha1, float* out) {
   pdl_launch_dependents();
@@ -139,7 +177,8 @@ void set_last_error(const char* msg) { g_last_error = msg; }
 struct moe_handle {
   moe_cfg cfg;
   int device = 0, n_sms = 0;
-  bool bf16 = true;
+  bool bf16 = true;        // bf16 storage (MOE_BF16 and MOE_BF16_E4M3_GATEUP)
+  bool e4m3 = false;       // gate/up GEMM on e4m3 operands (MOE_BF16_E4M3_GATEUP)
   int es = 2;              // element size
   int G = 0, has_shared = 0, inter_shared = 0;
   int n_tiles = 0;         // router tiles
@@ -147,6 +186,7 @@ struct moe_handle {
   int64_t T_pad = 0, rows_cap = 0;   // padded to bm, the GEMM row tile
   int bm = 0, tile_rows = 0;
   int gemm_grid = 0;                  // CTAs of the paired-SM GEMMs (2 per cluster)
+  int gemm_grid_f8 = 0;               // same, e4m3 gate/up GEMM
   // small-batch (decode) path: token counts <= n_tok, weights on the MMA's M dimension
   bool small = false;
   int n_tok = 0, small_stages = 0;
@@ -171,6 +211,10 @@ struct moe_handle {
   void *xp = nullptr, *hs = nullptr, *hr = nullptr, *ys = nullptr, *yr = nullptr;
   int* err = nullptr;
   int* copy_done = nullptr;   // counter of the fused permute (paired bf16 path with a shared group)
+  // e4m3 gate/up: quantised weights (interleaved rows), per-row scales, quantised tokens
+  void *w8_gu_s = nullptr, *w8_gu_r = nullptr, *u8 = nullptr;
+  float *sw_s = nullptr, *sw_r = nullptr, *su = nullptr, *su_p = nullptr;
+  CUtensorMap tmU8, tmXp8, tmW8guS, tmW8guR;
   bool fuse_permute = false;
   // staging for moe_forward_host
   void *u_dev = nullptr, *h_dev = nullptr;
@@ -247,11 +291,14 @@ moe_status validate(const moe_cfg* c) {
     return fail(MOE_ERR_INVALID_ARG, "top_k=%d outside [1, n_routed=%d]", c->top_k, c->n_routed);
   if (c->top_k > kMaxTopK)
     return fail(MOE_ERR_UNSUPPORTED, "top_k=%d above %d", c->top_k, kMaxTopK);
-  if (c->dtype != MOE_FP32 && c->dtype != MOE_BF16)
-    return fail(MOE_ERR_INVALID_ARG, "dtype=%d is not MOE_FP32 or MOE_BF16", c->dtype);
+  if (c->dtype != MOE_FP32 && c->dtype != MOE_BF16 && c->dtype != MOE_BF16_E4M3_GATEUP)
+    return fail(MOE_ERR_INVALID_ARG, "dtype=%d is not MOE_FP32, MOE_BF16 or MOE_BF16_E4M3_GATEUP",
+                c->dtype);
   if (!c->centroids || !c->w_gate || !c->w_up || !c->w_down)
     return fail(MOE_ERR_INVALID_ARG, "a weight pointer is NULL");
-  if (c->dtype == MOE_BF16) {
+  if (c->dtype == MOE_BF16_E4M3_GATEUP && c->d % 128)
+    return fail(MOE_ERR_UNSUPPORTED, "e4m3 gate/up layers need d %% 128 == 0 (d=%d)", c->d);
+  if (c->dtype != MOE_FP32) {
     if (c->d % 64 || c->inter % 64)
       return fail(MOE_ERR_UNSUPPORTED, "bf16 layers need d %% 64 == 0 and inter %% 64 == 0 (d=%d inter=%d)",
                   c->d, c->inter);
@@ -274,7 +321,7 @@ int32_t moe_abi_version(void) { return MOE_ABI_VERSION; }
 const char* moe_last_error(void) { return g_last_error.c_str(); }
 
 int32_t moe_kernels_per_forward(const moe_handle* handle) {
-  return handle ? kKernelsPerForward - (handle->fuse_permute ? 1 : 0) : 0;
+  return handle ? kKernelsPerForward - (handle->fuse_permute ? 1 : 0) + (handle->e4m3 ? 1 : 0) : 0;
 }
 
 size_t moe_device_bytes(const moe_handle* handle) { return handle ? handle->bytes : 0; }
@@ -293,14 +340,15 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
   H->cfg = c;
   H->cfg.centroids = H->cfg.w_gate = H->cfg.w_up = H->cfg.w_down = nullptr;
   H->cfg.logit_bias = nullptr;
-  H->bf16 = c.dtype == MOE_BF16;
+  H->bf16 = c.dtype != MOE_FP32;
+  H->e4m3 = c.dtype == MOE_BF16_E4M3_GATEUP;
   H->es = H->bf16 ? 2 : 4;
   H->has_shared = c.n_shared > 0 ? 1 : 0;
   H->inter_shared = c.n_shared * c.inter;
   H->G = H->has_shared + c.n_routed;
   H->router_rows = H->bf16 ? router_tile_rows(c.T, H->n_sms) : kRouterPass;
   H->n_tiles = (c.T + H->router_rows - 1) / H->router_rows;
-  H->small = H->bf16 && c.T <= kSmallMaxTok && c.d % kSmallBM == 0;
+  H->small = H->bf16 && !H->e4m3 && c.T <= kSmallMaxTok && c.d % kSmallBM == 0;
   H->n_tok = (c.T + 15) / 16 * 16;
   H->bm = H->small ? 1 : (H->bf16 ? kPairBM : kSimtBM);
   H->tile_rows = H->small ? 0 : H->bm;
@@ -365,6 +413,17 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
   }
   MOE_TRY(dalloc(H, &H->w_d_r, nr * d * I * es));
   MOE_CUDA(cudaMemcpyAsync(H->w_d_r, wd + ks * d * I * es, nr * d * I * es, cudaMemcpyDeviceToDevice, st));
+  if (H->e4m3) {
+    // e4m3 copies of the interleaved gate/up rows, one fp32 scale per row
+    if (ks) {
+      MOE_TRY(dalloc(H, &H->w8_gu_s, 2 * Is * d));
+      MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->sw_s), 2 * Is * 4));
+      MOE_CUDA(launch_quant(H->w_gu_s, (int64_t)(2 * Is), (int)d, H->w8_gu_s, H->sw_s, H->n_sms, st));
+    }
+    MOE_TRY(dalloc(H, &H->w8_gu_r, 2 * nr * I * d));
+    MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->sw_r), 2 * nr * I * 4));
+    MOE_CUDA(launch_quant(H->w_gu_r, (int64_t)(2 * nr * I), (int)d, H->w8_gu_r, H->sw_r, H->n_sms, st));
+  }
 
   // ---- workspace
   const size_t T = c.T, K = c.top_k, nt = H->n_tiles;
@@ -382,7 +441,15 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
   MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->copy_done), 256));
   MOE_CUDA(cudaMemsetAsync(H->copy_done, 0, 256, st));
   const size_t rc = (size_t)H->rows_cap, tp = (size_t)H->T_pad;
-  MOE_TRY(dalloc(H, &H->xp, rc * d * es));
+  MOE_TRY(dalloc(H, &H->xp, rc * d * (H->e4m3 ? 1 : es)));   // e4m3 rows on that path
+  if (H->e4m3) {
+    MOE_TRY(dalloc(H, &H->u8, tp * d));
+    MOE_CUDA(cudaMemsetAsync(H->u8, 0, tp * d, st));
+    MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->su), tp * 4));
+    MOE_CUDA(cudaMemsetAsync(H->su, 0, tp * 4, st));
+    MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->su_p), rc * 4));
+    MOE_CUDA(cudaMemsetAsync(H->su_p, 0, rc * 4, st));
+  }
   MOE_TRY(dalloc(H, &H->hr, rc * I * es));
   MOE_TRY(dalloc(H, &H->yr, rc * d * es));
   if (ks) {
@@ -431,10 +498,18 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
           &clusters, (const void*)grouped_gemm_tc_kernel<kGateUpSwiGLU>, &lc));
       if (clusters < 1) return fail(MOE_ERR_UNSUPPORTED, "no CTA pair of the GEMM kernel fits on this device");
       H->gemm_grid = 2 * clusters;
+      if (H->e4m3) {
+        MOE_CUDA(cudaFuncSetAttribute((const void*)grouped_gemm_tc_kernel<kGateUpSwiGLU, true>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmemBytes));
+        MOE_CUDA(cudaOccupancyMaxActiveClusters(
+            &clusters, (const void*)grouped_gemm_tc_kernel<kGateUpSwiGLU, true>, &lc));
+        if (clusters < 1) return fail(MOE_ERR_UNSUPPORTED, "no CTA pair of the e4m3 GEMM fits on this device");
+        H->gemm_grid_f8 = 2 * clusters;
+      }
     }
 
     bool ok = encode_2d(&H->tmE, H->centroids, d, (uint64_t)H->n_pad, (uint32_t)H->n_pad) &&
-              encode_2d(&H->tmXp, H->xp, d, rc, 128) &&
+              (H->e4m3 || encode_2d(&H->tmXp, H->xp, d, rc, 128)) &&
               encode_3d(&H->tmWguR, H->w_gu_r, d, 2 * I, nr, kGemmBN / 2) &&
               encode_2d(&H->tmHr, H->hr, I, rc, 128) &&
               encode_3d(&H->tmWdR, H->w_d_r, I, d, nr, kGemmBN / 2);
@@ -446,6 +521,13 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
       H->tmWguS = H->tmWguR;
       H->tmHs = H->tmHr;
       H->tmWdS = H->tmWdR;
+    }
+    if (H->e4m3) {
+      ok = ok && encode_2d_e4m3(&H->tmU8, H->u8, d, tp, 128) &&
+           encode_2d_e4m3(&H->tmXp8, H->xp, d, rc, 128) &&
+           encode_3d_e4m3(&H->tmW8guR, H->w8_gu_r, d, 2 * I, nr, kGemmBN / 2);
+      if (ks) ok = ok && encode_2d_e4m3(&H->tmW8guS, H->w8_gu_s, d, 2 * Is, kGemmBN / 2);
+      else H->tmW8guS = H->tmW8guR;
     }
     if (!ok) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for a weight/workspace tensor");
     if (H->small) {
@@ -548,6 +630,14 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
                  static_cast<uint8_t*>(H->xp), T, K, nr, (int)H->rows_cap, H->router_rows,
                  d * H->es, H->err};
   tick(H, stream, 2);
+  if (H->e4m3) {
+    // e4m3 token rows and scales; the row copy then moves those
+    MOE_CUDA(launch_quant(u, T, d, H->u8, H->su, H->n_sms, stream));
+    pa.u = static_cast<const uint8_t*>(H->u8);
+    pa.row_bytes = d;
+    pa.scale_src = H->su;
+    pa.scale_dst = H->su_p;
+  }
   if (!H->fuse_permute) {
     launch_pdl(permute_kernel, dim3((T + kPermuteWarps - 1) / kPermuteWarps), dim3(kPermuteWarps * 32), 0, stream, pa);
     MOE_CUDA(cudaGetLastError());
@@ -593,7 +683,19 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
       g1.copy_done = H->copy_done;
     }
     tick(H, stream, 3);
-    launch_pdl(grouped_gemm_tc_kernel<kGateUpSwiGLU>, dim3(H->gemm_grid), dim3(kGemmThreads), kGemmSmemBytes, stream,  tmU, H->tmXp, H->tmWguS, H->tmWguR, g1);
+    if (H->e4m3) {
+      g1.kb_shared = d / (2 * kGemmBK);   // k-blocks of 128 e4m3 values
+      g1.kb_routed = d / (2 * kGemmBK);
+      g1.sa_shared = H->su;
+      g1.sa_routed = H->su_p;
+      g1.sb_shared = H->sw_s;
+      g1.sb_routed = H->sw_r;
+      g1.sb_routed_stride = 2 * (int64_t)I;
+      launch_pdl(grouped_gemm_tc_kernel<kGateUpSwiGLU, true>, dim3(H->gemm_grid_f8), dim3(kGemmThreads),
+                 kGemmSmemBytes, stream, H->tmU8, H->tmXp8, H->tmW8guS, H->tmW8guR, g1);
+    } else {
+      launch_pdl(grouped_gemm_tc_kernel<kGateUpSwiGLU>, dim3(H->gemm_grid), dim3(kGemmThreads), kGemmSmemBytes, stream,  tmU, H->tmXp, H->tmWguS, H->tmWguR, g1);
+    }
     MOE_CUDA(cudaGetLastError());
 
     GemmArgs g2{};

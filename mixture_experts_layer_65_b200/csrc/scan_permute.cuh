@@ -166,6 +166,8 @@ struct PermuteArgs {
   int tile_rows;               // tokens per router tile
   int row_bytes;               // multiple of 16
   int* err;
+  const float* scale_src;      // [T] per-row scales copied along with the rows, or nullptr
+  float* scale_dst;            // [rows_cap]
 };
 
 constexpr int kPermuteWarps = 8;
@@ -186,6 +188,7 @@ __device__ __forceinline__ void permute_token(const PermuteArgs& a, int t, int l
       record_error(a.err, kErrRouteIndex);
     }
     a.slot_row[(size_t)t * a.top_k + lane] = my_dest < 0 ? 0 : my_dest;
+    if (my_dest >= 0 && a.scale_dst) a.scale_dst[my_dest] = a.scale_src[t];
   }
   const int nvec = a.row_bytes >> 4;
   const uint4* src = reinterpret_cast<const uint4*>(a.u + (size_t)t * a.row_bytes);

@@ -51,6 +51,10 @@ CONFIGS: dict[str, dict] = {
     # 145B-shaped layer with a Zipf(1.1) per-expert router bias (skewed load)
     "145b": dict(T=32768, d=4096, n_shared=4, n_routed=128, inter=1536, top_k=12,
                  dtype="bf16", alpha1=0.001, zipf_s=1.1),
+    # the 16B-shaped prefill layer with its gate/up GEMM on e4m3 operands (the library's
+    # reduced-precision variant; same draws as "16b_prefill")
+    "16b_prefill_e4m3": dict(T=16384, d=2048, n_shared=2, n_routed=64, inter=1408, top_k=6,
+                             dtype="bf16", alpha1=0.001, zipf_s=None, gate_up_e4m3=True),
 }
 
 _STREAMS = ("u", "centroids", "w_gate", "w_up", "w_down")
@@ -105,6 +109,7 @@ class Workload:
     w_up: np.ndarray
     w_down: np.ndarray
     logit_bias: np.ndarray | None
+    gate_up_e4m3: bool = False     # bf16 layer whose gate/up products take e4m3 operands
 
     @property
     def n_experts(self) -> int:
@@ -112,7 +117,8 @@ class Workload:
 
     def spec(self) -> dict:
         return dict(T=self.T, d=self.d, n_shared=self.n_shared, n_routed=self.n_routed,
-                    inter=self.inter, top_k=self.top_k, dtype=self.dtype, alpha1=self.alpha1)
+                    inter=self.inter, top_k=self.top_k, dtype=self.dtype, alpha1=self.alpha1,
+                    gate_up_e4m3=self.gate_up_e4m3)
 
 
 def _draw(seed_seq, shape, std: float, dtype: str) -> np.ndarray:
@@ -172,4 +178,5 @@ def make_workload(name: str = "tiny", seed: int = 0, threads: int | None = None,
     bias = zipf_logit_bias(nr, zs) if zs else None
     return Workload(name=name, T=T, d=d, n_shared=ks, n_routed=nr, inter=inter, top_k=top_k,
                     dtype=dtype, alpha1=float(spec["alpha1"]), u=u, centroids=cen,
-                    w_gate=w_gate, w_up=w_up, w_down=w_down, logit_bias=bias)
+                    w_gate=w_gate, w_up=w_up, w_down=w_down, logit_bias=bias,
+                    gate_up_e4m3=bool(spec.get("gate_up_e4m3", False)))

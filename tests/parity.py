@@ -50,7 +50,8 @@ def sample_rows(T: int, n: int = 256, seed: int = 1) -> np.ndarray:
 def compare(w, g: GpuOut, rows=None, report: dict | None = None) -> dict:
     """Assert parity of every output; returns a report dict (excluded tokens, errors)."""
     ref = O.moe_forward(w.u, w.centroids, w.w_gate, w.w_up, w.w_down, w.n_shared, w.top_k,
-                        w.alpha1, bias=w.logit_bias, rows=rows)
+                        w.alpha1, bias=w.logit_bias, rows=rows,
+                        gate_up_e4m3=getattr(w, "gate_up_e4m3", False))
     r = ref.routing
     T, K, nr = w.T, w.top_k, w.n_routed
     rep = report if report is not None else {}
