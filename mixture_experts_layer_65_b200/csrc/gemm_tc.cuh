@@ -48,6 +48,13 @@ constexpr int kGemmStages = 3;
 constexpr int kGemmEpiWarps = 8;             // two warps per TMEM lane quadrant
 constexpr int kGemmCopyWarps = 4;            // row copies of the fused permute (gate/up GEMM)
 constexpr int kGemmThreads = 64 + 32 * (kGemmEpiWarps + kGemmCopyWarps);
+// The e4m3 gate/up GEMM finishes a tile's MMAs in half the time, so its SwiGLU epilogue
+// (which also applies the row scales) gets twice the warps: four per TMEM lane quadrant,
+// working in steps of 16 outputs to stay within the smaller register budget.
+__host__ __device__ constexpr int gemm_epi_warps(bool f8) { return f8 ? 16 : kGemmEpiWarps; }
+__host__ __device__ constexpr int gemm_threads(bool f8) {
+  return 64 + 32 * (gemm_epi_warps(f8) + kGemmCopyWarps);
+}
 constexpr uint32_t kGemmABytes = 128 * kGemmBK * 2;           // this CTA's half of A, per k-block
 constexpr uint32_t kGemmBBytes = (kGemmBN / 2) * kGemmBK * 2; // this CTA's half of B, per k-block
 constexpr uint32_t kGemmBOff = kGemmKPS * kGemmABytes;        // B blocks after the A blocks
@@ -108,7 +115,7 @@ __device__ __forceinline__ void gemm_decode(int tile, int& g, const GemmArgs& a,
 // F8: A and B are e4m3 (k-blocks of 128 elements = the same 128-byte rows), MMAs of kind
 // f8f6f4, and the gate/up epilogue multiplies each accumulator by its two row scales.
 template <int MODE, bool F8 = false>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm_threads(F8), 1)
 grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
                        const __grid_constant__ CUtensorMap tmA_r,
                        const __grid_constant__ CUtensorMap tmB_s,
@@ -138,7 +145,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&acc_full[s]), 1);
-      mbar_init(smem_u32(&acc_empty[s]), 2 * kGemmEpiWarps);   // epilogue warps of both CTAs
+      mbar_init(smem_u32(&acc_empty[s]), 2 * gemm_epi_warps(F8));   // epilogue warps of both CTAs
     }
     mbar_init(smem_u32(drain), 1);
     *abort_flag = 0;
@@ -246,11 +253,11 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
       tc_commit_pair_mc(smem_u32(drain), 0x3);
     }
     __syncwarp();
-  } else if (warp >= 2 + kGemmEpiWarps) {
+  } else if (warp >= 2 + gemm_epi_warps(F8)) {
     // ------------------------------------------------------------------ row copies
     if (a.copy_done != nullptr) {
       const int nw = (int)gridDim.x * kGemmCopyWarps;
-      for (int t = (int)blockIdx.x * kGemmCopyWarps + (warp - 2 - kGemmEpiWarps); t < a.perm.T;
+      for (int t = (int)blockIdx.x * kGemmCopyWarps + (warp - 2 - gemm_epi_warps(F8)); t < a.perm.T;
            t += nw)
         permute_token(a.perm, t, lane);
       fence_proxy_async_global();
@@ -261,7 +268,9 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
   } else {
     // ------------------------------------------------------------------ epilogue
     const int q = warp & 3;                 // TMEM lane quadrant this warp may access
-    const int half = (warp - 2) >> 2;       // which half of the tile's columns
+    constexpr int WPQ = gemm_epi_warps(F8) / 4;   // epilogue warps per quadrant
+    const int part = (warp - 2) >> 2;       // which 1/WPQ of the tile's columns
+    const int half = part;                  // (WPQ == 2) which half of the tile's columns
     const int rr = q * 32 + lane;
     int g = 0, it = 0;
     for (int tile = cid; tile < total; tile += ncl, ++it) {
@@ -293,7 +302,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
           sbv = (c.shared ? a.sb_shared : a.sb_routed + (int64_t)c.e * a.sb_routed_stride) +
                 (int64_t)c.n * kGemmBN;
         }
-        {
+        if constexpr (!F8) {
           const int hb = half;
           const int col0 = c.n * (kGemmBN / 2) + hb * 64;
 #pragma unroll 1
@@ -304,14 +313,6 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
             tmem_ld32(trow + static_cast<uint32_t>(hb * 128 + 64 + j), uv);
             tmem_ld_wait(gv);
             tmem_ld_wait(uv);
-            if (F8) {
-              const float* sg = sbv + hb * 128 + j;        // gate rows of these 32 columns
-#pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                gv[i] = __float_as_uint(__uint_as_float(gv[i]) * sa * __ldg(sg + i));
-                uv[i] = __float_as_uint(__uint_as_float(uv[i]) * sa * __ldg(sg + 64 + i));
-              }
-            }
             uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
@@ -325,6 +326,43 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
 #pragma unroll
               for (int v = 0; v < 4; ++v)
                 dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            }
+          }
+        } else {
+          // four warps per quadrant: 32 of the tile's 128 outputs each, 16 per step
+          const int hb = part >> 1;
+          const int jb = (part & 1) * 32;
+          const int col0 = c.n * (kGemmBN / 2) + hb * 64;
+          const float* sg = sbv + hb * 128;      // weight-row scales of the gate columns
+#pragma unroll 1
+          for (int j = jb; j < jb + 32 && col0 < cols; j += 16) {
+            uint32_t gv[16], uv[16];
+            __syncwarp();
+            tmem_ld16(trow + static_cast<uint32_t>(hb * 128 + j), gv);
+            tmem_ld16(trow + static_cast<uint32_t>(hb * 128 + 64 + j), uv);
+            tmem_ld_wait16(gv);
+            tmem_ld_wait16(uv);
+            const float4* sg4 = reinterpret_cast<const float4*>(sg + j);
+            const float4* su4 = reinterpret_cast<const float4*>(sg + 64 + j);
+            uint32_t pk[8];
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const float4 a4 = __ldg(sg4 + v), b4 = __ldg(su4 + v);
+              const float ga[4] = {a4.x, a4.y, a4.z, a4.w}, ub[4] = {b4.x, b4.y, b4.z, b4.w};
+              float hv[4];
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float gg = __uint_as_float(gv[4 * v + i]) * sa * ga[i];
+                const float uu = __uint_as_float(uv[4 * v + i]) * sa * ub[i];
+                hv[i] = silu_fast(gg) * uu;
+              }
+              pk[2 * v] = pack_bf16x2(hv[0], hv[1]);
+              pk[2 * v + 1] = pack_bf16x2(hv[2], hv[3]);
+            }
+            if (row_ok) {
+              uint4* dst = reinterpret_cast<uint4*>(out + orow * ld + col0 + j);
+              dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
             }
           }
         }

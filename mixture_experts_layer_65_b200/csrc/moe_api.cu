@@ -501,6 +501,7 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
       if (H->e4m3) {
         MOE_CUDA(cudaFuncSetAttribute((const void*)grouped_gemm_tc_kernel<kGateUpSwiGLU, true>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmemBytes));
+        lc.blockDim = dim3(gemm_threads(true), 1, 1);
         MOE_CUDA(cudaOccupancyMaxActiveClusters(
             &clusters, (const void*)grouped_gemm_tc_kernel<kGateUpSwiGLU, true>, &lc));
         if (clusters < 1) return fail(MOE_ERR_UNSUPPORTED, "no CTA pair of the e4m3 GEMM fits on this device");
@@ -691,7 +692,7 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
       g1.sb_shared = H->sw_s;
       g1.sb_routed = H->sw_r;
       g1.sb_routed_stride = 2 * (int64_t)I;
-      launch_pdl(grouped_gemm_tc_kernel<kGateUpSwiGLU, true>, dim3(H->gemm_grid_f8), dim3(kGemmThreads),
+      launch_pdl(grouped_gemm_tc_kernel<kGateUpSwiGLU, true>, dim3(H->gemm_grid_f8), dim3(gemm_threads(true)),
                  kGemmSmemBytes, stream, H->tmU8, H->tmXp8, H->tmW8guS, H->tmW8guR, g1);
     } else {
       launch_pdl(grouped_gemm_tc_kernel<kGateUpSwiGLU>, dim3(H->gemm_grid), dim3(kGemmThreads), kGemmSmemBytes, stream,  tmU, H->tmXp, H->tmWguS, H->tmWguR, g1);
