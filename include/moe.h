@@ -212,6 +212,16 @@ moe_status moe_route_noalloc(const void* u, const void* centroids, const float* 
                              int32_t* topk_idx, float* topk_w, int32_t* expert_counts,
                              float* aux_loss, int32_t* device_error, moe_stream_t stream);
 
+/* Diagnostic (no counterpart on the DeepSeekMoE pages): checks, on the current device,
+ * that the library's bounded waits give up.  Runs one one-block kernel whose thread waits,
+ * for at most limit_ns nanoseconds (1e6 .. 2e9), on something nothing will complete --
+ * kind 0: an mbarrier phase (the wait of the GEMM/router pipelines), kind 1: a global
+ * counter (the wait of the fused row copy) -- then synchronises the current stream of the
+ * device and stores the error code the kernel recorded in *device_code (HOST pointer):
+ * 0x102 for kind 0, 0x105 for kind 1 when the wait ran out as designed.  The kernel
+ * returns normally, so the context stays usable.  Allocates a 4-byte word. */
+moe_status moe_selftest_wait_timeout(int32_t kind, int64_t limit_ns, int32_t* device_code);
+
 /* Number of kernels one moe_forward launches on this handle. */
 int32_t moe_kernels_per_forward(const moe_handle* handle);
 

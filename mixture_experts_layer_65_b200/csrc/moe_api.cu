@@ -131,6 +131,23 @@ cudaError_t launch_quant(const void* src, int64_t rows, int cols, void* dst, flo
   return launch_pdl(quant_rows_e4m3_kernel, dim3((unsigned)blocks), dim3(kQuantWarps * 32), 0, st, qa);
 }
 
+__device__ int g_never_set = 0;   // a counter no kernel writes (bounded-wait self-test)
+
+__global__ void wait_selftest_kernel(int kind, uint64_t limit_ns, int* err) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);   // expects one arrival, which never comes
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (kind == 0) mbar_wait(smem_u32(&bar), 0, &abort_flag, err, kErrWaitMma, limit_ns);
+    else counter_wait(&g_never_set, 1, &abort_flag, err, kErrWaitCopy, limit_ns);
+  }
+}
+
 __global__ void balance_loss_kernel(const int32_t* counts, const float* psum, int n, double inv_t,
                                     float alpha1, float* out) {
   pdl_launch_dependents();
@@ -935,6 +952,27 @@ moe_status moe_balance_loss(const int32_t* counts, const float* psum, int32_t n_
   if (n_routed < 1 || n_tokens < 1) return fail(MOE_ERR_INVALID_ARG, "n_routed and n_tokens must be positive");
   launch_pdl(balance_loss_kernel, dim3(1), dim3(32), 0, reinterpret_cast<cudaStream_t>(stream_),  counts, psum, n_routed, 1.0 / (double)n_tokens, alpha1, aux_loss);
   MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+moe_status moe_selftest_wait_timeout(int32_t kind, int64_t limit_ns, int32_t* device_code) {
+  if (!device_code) return fail(MOE_ERR_INVALID_ARG, "device_code is NULL");
+  if (kind != 0 && kind != 1) return fail(MOE_ERR_INVALID_ARG, "kind must be 0 or 1");
+  if (limit_ns < 1000000 || limit_ns > 2000000000)
+    return fail(MOE_ERR_INVALID_ARG, "limit_ns outside [1e6, 2e9]");
+  int* err = nullptr;
+  MOE_CUDA(cudaMalloc(&err, sizeof(int)));
+  cudaError_t e = cudaMemset(err, 0, sizeof(int));
+  if (e == cudaSuccess) {
+    wait_selftest_kernel<<<1, 32>>>(kind, (uint64_t)limit_ns, err);
+    e = cudaGetLastError();
+  }
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  int code = 0;
+  if (e == cudaSuccess) e = cudaMemcpy(&code, err, sizeof(int), cudaMemcpyDeviceToHost);
+  cudaFree(err);
+  if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "self-test kernel: %s", cudaGetErrorString(e));
+  *device_code = code;
   return MOE_OK;
 }
 

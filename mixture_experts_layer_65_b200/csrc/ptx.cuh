@@ -76,16 +76,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Wait for the phase of `bar` with the given parity to complete.  Gives up (returns
 // false) when `abort_flag` (shared memory, set by another role of this CTA) is raised,
-// or after kWaitLimitNs, in which case it records `code` and raises the abort flag.
+// or after `limit_ns` (kWaitLimitNs unless given), in which case it records `code` and
+// raises the abort flag.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          int* err, int code) {
+                                          int* err, int code, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 255u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         record_error(err, code);
         *abort_flag = 1;
         return false;
@@ -109,7 +110,7 @@ __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
 // Wait until *counter >= target (written by other CTAs with release semantics).  Gives
 // up like mbar_wait: on `abort_flag`, or after kWaitLimitNs, recording `code`.
 __device__ __forceinline__ bool counter_wait(const int* counter, int target, volatile int* abort_flag,
-                                             int* err, int code) {
+                                             int* err, int code, uint64_t limit_ns = kWaitLimitNs) {
   if (ld_acquire_gpu(counter) >= target) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
@@ -117,7 +118,7 @@ __device__ __forceinline__ bool counter_wait(const int* counter, int target, vol
     if (ld_acquire_gpu(counter) >= target) return true;
     if ((it & 63u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         record_error(err, code);
         *abort_flag = 1;
         return false;

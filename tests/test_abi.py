@@ -71,3 +71,11 @@ def test_product_path_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="missing"):
         _lib.lib()
+
+
+def test_wait_selftest_validates_arguments_before_touching_the_device():
+    L = _lib.lib()
+    code = ctypes.c_int32(0)
+    assert L.moe_selftest_wait_timeout(2, 50_000_000, ctypes.byref(code)) == _lib.MOE_ERR_INVALID_ARG
+    assert L.moe_selftest_wait_timeout(0, 10, ctypes.byref(code)) == _lib.MOE_ERR_INVALID_ARG
+    assert L.moe_selftest_wait_timeout(0, 50_000_000, None) == _lib.MOE_ERR_INVALID_ARG
