@@ -363,9 +363,14 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
   H->has_shared = c.n_shared > 0 ? 1 : 0;
   H->inter_shared = c.n_shared * c.inter;
   H->G = H->has_shared + c.n_routed;
+  // (the small-batch path, decided below, takes one token per router CTA)
   H->router_rows = H->bf16 ? router_tile_rows(c.T, H->n_sms) : kRouterPass;
   H->n_tiles = (c.T + H->router_rows - 1) / H->router_rows;
   H->small = H->bf16 && !H->e4m3 && c.T <= kSmallMaxTok && c.d % kSmallBM == 0;
+  if (H->small) {
+    H->router_rows = 1;
+    H->n_tiles = c.T;
+  }
   H->n_tok = (c.T + 15) / 16 * 16;
   H->bm = H->small ? 1 : (H->bf16 ? kPairBM : kSimtBM);
   H->tile_rows = H->small ? 0 : H->bm;
@@ -549,6 +554,10 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
     }
     if (!ok) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for a weight/workspace tensor");
     if (H->small) {
+      H->simt_router_smem = router_epi_bytes(H->n_pad);
+      const void* rk = with_maxc(H->maxc, [](auto m) { return (const void*)router_small_kernel<m()>; });
+      MOE_CUDA(cudaFuncSetAttribute(rk, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)H->simt_router_smem));
       const size_t epi = (small_epi_bytes(H->n_tok) + 15) & ~size_t(15);
       const uint32_t sb = small_stage_bytes(H->n_tok);
       int stages = (int)((200u * 1024u - epi) / sb);
@@ -613,7 +622,16 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
   RouterOut ro{topk_idx, topk_w, H->topk_rank, H->tile_hist, H->tile_psum, H->err};
   CUtensorMap tmU, tmUr;
   tick(H, stream, 0);
-  if (H->bf16) {
+  if (H->small) {
+    RouterSmallArgs ra{static_cast<const __nv_bfloat16*>(u),
+                       static_cast<const __nv_bfloat16*>(H->centroids), H->bias, T, d, nr, K,
+                       H->router_rows, ro};
+    with_maxc(H->maxc, [&](auto m) {
+      launch_pdl(router_small_kernel<m()>, dim3(H->n_tiles), dim3(kRouterEpiThreads),
+                 H->simt_router_smem, stream, ra);
+      return 0;
+    });
+  } else if (H->bf16) {
     if (!encode_2d(&tmU, u, d, T, 128) || !encode_2d(&tmUr, u, d, T, (uint32_t)H->router_rows))
       return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for u");
     RouterTcArgs ra{T, d, nr, H->n_pad, K, H->router_kps, H->router_stages, H->router_rows, H->n_tiles,

@@ -23,16 +23,6 @@ struct QuantArgs {
   float* scale;               // [rows]
 };
 
-__device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
-  const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 x = __bfloat1622float2(p[i]);
-    f[2 * i] = x.x;
-    f[2 * i + 1] = x.y;
-  }
-}
-
 // One warp per row: the row maximum by shuffles, then the row converted 8 values per lane
 // and step.
 static __global__ void __launch_bounds__(kQuantWarps * 32) quant_rows_e4m3_kernel(QuantArgs a) {

@@ -138,6 +138,9 @@ __device__ __forceinline__ void router_pass(int tid, int pass, int tile, int R, 
   const bool valid = r < rows && t < T;
   float* row = lg + (size_t)r * ld;
 
+  // warps whose four rows all lie past the pass skip the per-row work (they still take
+  // part in every barrier)
+  if ((tid >> 5) * 4 < rows) {
   // keys and the row max; rows past the tile or past T are treated as zeros
   uint64_t key[MAXC];
   float lmax = -INFINITY;
@@ -239,6 +242,7 @@ __device__ __forceinline__ void router_pass(int tid, int pass, int tile, int R, 
       }
     }
   }
+  }   // warps with rows
   sync();
 
   // the pass's per-expert affinity sums: row parts, added to the earlier passes' parts
@@ -576,6 +580,60 @@ __global__ void __launch_bounds__(kRouterEpiThreads) router_simt_kernel(RouterSi
                     sync);
   __syncthreads();
   router_tile_outputs(tid, tile, kRouterPass, a.T, a.n_routed, n_pad, a.top_k, smem_raw, a.out);
+}
+
+// ------------------------------------------------------------------------ bf16, few tokens
+struct RouterSmallArgs {
+  const __nv_bfloat16* u;     // [T, d]
+  const __nv_bfloat16* cen;   // [n_routed, d]
+  const float* bias;          // [>= n_routed]
+  int T, d, n_routed, top_k;
+  int tile_rows;              // tokens per CTA (1..64)
+  RouterOut out;
+};
+
+// For decode-sized batches (a handful of tokens), where the tensor-core router would
+// stream the whole centroid matrix through its TMA ring for a tile of a few rows: each
+// CTA takes tile_rows tokens, each warp one (token, expert) dot product at a time with
+// the lanes splitting d (16-byte vectors) and a fixed shuffle tree, then the shared
+// epilogue.  512 threads; dynamic smem router_epi_bytes(n_pad).
+template <int MAXC>
+__global__ void __launch_bounds__(kRouterEpiThreads) router_small_kernel(RouterSmallArgs a) {
+  pdl_launch_dependents();
+  pdl_wait();
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  RouterEpiSmem& SM = *reinterpret_cast<RouterEpiSmem*>(smem_raw);
+  float* lg = reinterpret_cast<float*>(smem_raw + sizeof(RouterEpiSmem));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tile = blockIdx.x, R = a.tile_rows;
+  const int n_pad = (a.n_routed + 15) & ~15;
+  const int ld = router_ld(n_pad);
+  const int nv = a.d >> 3;
+  for (int e = tid; e < 4 * kMaxRouted; e += kRouterEpiThreads) (&SM.mask[0][0])[e] = 0u;
+  for (int p = warp; p < R * a.n_routed; p += kRouterEpiThreads / 32) {
+    const int r = p / a.n_routed, i = p - r * a.n_routed;
+    const int t = tile * R + r;
+    float acc = 0.f;
+    if (t < a.T) {
+      const uint4* ur = reinterpret_cast<const uint4*>(a.u + (size_t)t * a.d);
+      const uint4* er = reinterpret_cast<const uint4*>(a.cen + (size_t)i * a.d);
+      for (int v = lane; v < nv; v += 32) {
+        float x[8], y[8];
+        bf16x8_to_f32(__ldg(ur + v), x);
+        bf16x8_to_f32(__ldg(er + v), y);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc = fmaf(x[k], y[k], acc);
+      }
+    }
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+    if (lane == 0) lg[(size_t)r * ld + i] = acc + a.bias[i];
+  }
+  __syncthreads();
+  auto sync = [] { __syncthreads(); };
+  router_pass<MAXC>(tid, 0, tile, R, a.T, a.n_routed, n_pad, a.top_k, smem_raw, a.out, sync);
+  __syncthreads();
+  router_tile_outputs(tid, tile, R, a.T, a.n_routed, n_pad, a.top_k, smem_raw, a.out);
 }
 
 }  // namespace moe
