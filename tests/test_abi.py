@@ -43,6 +43,8 @@ def _cfg(**kw):
     (dict(dtype=7), _lib.MOE_ERR_INVALID_ARG),
     (dict(w_down=None), _lib.MOE_ERR_INVALID_ARG),
     (dict(n_shared=-1), _lib.MOE_ERR_INVALID_ARG),
+    (dict(dtype=_lib.MOE_BF16_E4M3_GATEUP, d=192), _lib.MOE_ERR_UNSUPPORTED),   # d % 128
+    (dict(dtype=_lib.MOE_BF16_E4M3_GATEUP, inter=96), _lib.MOE_ERR_UNSUPPORTED),
 ])
 def test_create_rejects_invalid_config(L, kw, status):
     h = ctypes.c_void_p(123)
@@ -58,6 +60,8 @@ def test_null_arguments_are_rejected(L):
     assert L.moe_forward(None, 16, 16, 16, 16, 16, 16, None) == _lib.MOE_ERR_INVALID_ARG
     assert L.moe_forward_host(None, 16, 16, 16, 16, 16, 16, None) == _lib.MOE_ERR_INVALID_ARG
     assert L.moe_device_status(None, None) == _lib.MOE_ERR_INVALID_ARG
+    assert L.moe_forward_host_pipelined(None, 16, 16, 16, 16, 16, 16, None) == _lib.MOE_ERR_INVALID_ARG
+    assert L.moe_pipeline_wait(None, None) == _lib.MOE_ERR_INVALID_ARG
     assert L.moe_expert_psum(None, 16, None) == _lib.MOE_ERR_INVALID_ARG
     assert L.moe_balance_loss(None, 16, 4, 10, 0.01, 16, None) == _lib.MOE_ERR_INVALID_ARG
     assert L.moe_balance_loss(16, 16, 0, 10, 0.01, 16, None) == _lib.MOE_ERR_INVALID_ARG

@@ -166,8 +166,9 @@ def test_nan_row_propagates_without_hang():
     assert err <= P.TOL["bf16"]
 
 
-def test_bitwise_deterministic():
-    w = W.make_workload("16b_prefill", T=3000)
+@pytest.mark.parametrize("e4m3", [False, True], ids=["bf16", "e4m3_gate_up"])
+def test_bitwise_deterministic(e4m3):
+    w = W.make_workload("16b_prefill", T=3000, gate_up_e4m3=e4m3)
     layer = MoELayer.from_workload(w)
     u = to_device_tensor(w.u, "cuda")
     a = layer.forward(u)
@@ -190,10 +191,11 @@ def test_forward_host_matches_forward():
     layer.device_status()
 
 
-def test_forward_host_pipelined_matches_forward():
+@pytest.mark.parametrize("e4m3", [False, True], ids=["bf16", "e4m3_gate_up"])
+def test_forward_host_pipelined_matches_forward(e4m3):
     # four batches through the two-slot pipeline (slots reused), each checked bit for bit
     # against the device-buffer forward of the same input
-    w = W.make_workload("16b_prefill", T=500)
+    w = W.make_workload("16b_prefill", T=500, gate_up_e4m3=e4m3)
     layer = MoELayer.from_workload(w)
     rng = np.random.default_rng(5)
     us = [to_device_tensor(w.u, "cuda")]
