@@ -42,7 +42,7 @@ import math
 import numpy as np
 
 __all__ = ["widen", "router_logits", "affinity_softmax", "select_topk", "route",
-           "swiglu_ffn", "balance_stats", "moe_forward", "near_tie_tokens",
+           "swiglu_hidden", "swiglu_ffn", "balance_stats", "moe_forward", "near_tie_tokens",
            "brute_force_layer", "Routing", "LayerOut", "E4M3_MAX", "e4m3_round",
            "quantize_rows_e4m3"]
 
@@ -106,8 +106,8 @@ def _silu(z: np.ndarray) -> np.ndarray:
         return z / (1.0 + np.exp(-z))
 
 
-def swiglu_ffn(x, w_gate, w_up, w_down, gate_up_e4m3: bool = False) -> np.ndarray:
-    """FFN(x) = W_down (SiLU(W_gate x) * (W_up x)); x [n, d], W_gate/W_up [I, d], W_down [d, I].
+def swiglu_hidden(x, w_gate, w_up, gate_up_e4m3: bool = False) -> np.ndarray:
+    """The expert's hidden activation SiLU(W_gate x) * (W_up x); x [n, d], W_gate/W_up [I, d].
 
     gate_up_e4m3: the e4m3 variant -- x's rows and W_gate's / W_up's rows are replaced by
     their scaled e4m3 approximations (quantize_rows_e4m3) in the two gate/up products."""
@@ -116,7 +116,12 @@ def swiglu_ffn(x, w_gate, w_up, w_down, gate_up_e4m3: bool = False) -> np.ndarra
     x = widen(x)
     a = x @ widen(w_gate).T
     b = x @ widen(w_up).T
-    return (_silu(a) * b) @ widen(w_down).T
+    return _silu(a) * b
+
+
+def swiglu_ffn(x, w_gate, w_up, w_down, gate_up_e4m3: bool = False) -> np.ndarray:
+    """FFN(x) = W_down (SiLU(W_gate x) * (W_up x)); x [n, d], W_gate/W_up [I, d], W_down [d, I]."""
+    return swiglu_hidden(x, w_gate, w_up, gate_up_e4m3) @ widen(w_down).T
 
 
 # ---------------------------------------------------------------- e4m3 gate/up variant
