@@ -222,6 +222,21 @@ moe_status moe_route_noalloc(const void* u, const void* centroids, const float* 
  * returns normally, so the context stays usable.  Allocates a 4-byte word. */
 moe_status moe_selftest_wait_timeout(int32_t kind, int64_t limit_ns, int32_t* device_code);
 
+/* Diagnostic (for per-kernel tests): copy one of the handle's workspace buffers, as the
+ * most recent forward left it, to DEVICE memory `dst` on `stream` (bytes <= its size), or
+ * with dst == NULL only report its size in *size.  which:
+ *   0 slot_row [T, top_k] int32   destination row of each (token, slot) in the buffers below
+ *   1 xp  [rows_cap, d]    expert-contiguous token rows (layer dtype; e4m3 bytes for
+ *                          MOE_BF16_E4M3_GATEUP; unused padding rows are unspecified)
+ *   2 hr  [rows_cap, inter] routed experts' SwiGLU activations (bf16 / fp32)
+ *   3 yr  [rows_cap, d]    routed experts' outputs before the gates
+ *   4 hs  [T_pad, n_shared*inter]  shared experts' activations, experts side by side
+ *   5 ys  [T_pad, d]       sum of the shared experts' outputs
+ *   6 grp_row [G] int32    first row of each group (shared group first when n_shared > 0)
+ * Buffers 4 and 5 are empty (size 0) when n_shared == 0. */
+moe_status moe_debug_copy(const moe_handle* handle, int32_t which, void* dst, size_t bytes,
+                          size_t* size, moe_stream_t stream);
+
 /* Number of kernels one moe_forward launches on this handle. */
 int32_t moe_kernels_per_forward(const moe_handle* handle);
 

@@ -41,6 +41,7 @@ _SIGS = {
     "moe_forward_host_pipelined": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_pipeline_wait": (ctypes.c_int, [_P, _P]),
     "moe_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int64, _P]),
+    "moe_debug_copy": (ctypes.c_int, [_P, ctypes.c_int32, _P, ctypes.c_size_t, _P, _P]),
     "moe_device_status": (ctypes.c_int, [_P, _P]),
     "moe_expert_psum": (ctypes.c_int, [_P, _P, _P]),
     "moe_balance_loss": (ctypes.c_int, [_P, _P, ctypes.c_int32, ctypes.c_int64, ctypes.c_float,

@@ -973,6 +973,33 @@ moe_status moe_balance_loss(const int32_t* counts, const float* psum, int32_t n_
   return MOE_OK;
 }
 
+moe_status moe_debug_copy(const moe_handle* H, int32_t which, void* dst, size_t bytes,
+                          size_t* size, moe_stream_t stream_) {
+  if (!H || !size) return fail(MOE_ERR_INVALID_ARG, "handle and size must not be NULL");
+  const moe_cfg& c = H->cfg;
+  const size_t rc = (size_t)H->rows_cap, tp = (size_t)H->T_pad, d = c.d, I = c.inter;
+  const size_t es = H->es, xes = H->e4m3 ? 1 : es;
+  const void* src = nullptr;
+  size_t n = 0;
+  switch (which) {
+    case 0: src = H->slot_row; n = (size_t)c.T * c.top_k * 4; break;
+    case 1: src = H->xp; n = rc * d * xes; break;
+    case 2: src = H->hr; n = rc * I * es; break;
+    case 3: src = H->yr; n = rc * d * es; break;
+    case 4: src = H->hs; n = H->hs ? tp * (size_t)H->inter_shared * es : 0; break;
+    case 5: src = H->ys; n = H->ys ? tp * d * es : 0; break;
+    case 6: src = H->grp_row; n = (size_t)H->G * 4; break;
+    default: return fail(MOE_ERR_INVALID_ARG, "which=%d outside [0, 6]", which);
+  }
+  *size = n;
+  if (!dst) return MOE_OK;
+  if (bytes > n) return fail(MOE_ERR_INVALID_ARG, "bytes=%zu above the buffer's %zu", bytes, n);
+  if (bytes)
+    MOE_CUDA(cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice,
+                             reinterpret_cast<cudaStream_t>(stream_)));
+  return MOE_OK;
+}
+
 moe_status moe_selftest_wait_timeout(int32_t kind, int64_t limit_ns, int32_t* device_code) {
   if (!device_code) return fail(MOE_ERR_INVALID_ARG, "device_code is NULL");
   if (kind != 0 && kind != 1) return fail(MOE_ERR_INVALID_ARG, "kind must be 0 or 1");

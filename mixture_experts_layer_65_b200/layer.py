@@ -151,6 +151,28 @@ class MoELayer:
         s = stream or torch.cuda.current_stream(self.device)
         check(lib().moe_pipeline_wait(self._h, s.cuda_stream))
 
+    DEBUG_BUFFERS = {"slot_row": 0, "xp": 1, "hr": 2, "yr": 3, "hs": 4, "ys": 5, "grp_row": 6}
+
+    def debug_buffer(self, name: str) -> torch.Tensor:
+        """A copy (flat, device) of a workspace buffer as the last forward left it: for
+        per-kernel tests.  int32 for slot_row/grp_row, uint8 bytes for xp of e4m3 gate/up
+        layers, else the layer dtype."""
+        which = self.DEBUG_BUFFERS[name]
+        size = ctypes.c_size_t(0)
+        s = torch.cuda.current_stream(self.device)
+        check(lib().moe_debug_copy(self._h, which, None, 0, ctypes.byref(size), s.cuda_stream))
+        if name in ("slot_row", "grp_row"):
+            dt = torch.int32
+        elif name == "xp" and self.gate_up_e4m3:
+            dt = torch.uint8
+        else:
+            dt = self.torch_dtype
+        esz = torch.empty(0, dtype=dt).element_size()
+        out = torch.empty(size.value // esz, dtype=dt, device=self.device)
+        check(lib().moe_debug_copy(self._h, which, _ptr(out), size.value, ctypes.byref(size),
+                                   s.cuda_stream))
+        return out
+
     def device_status(self, stream: torch.cuda.Stream | None = None) -> None:
         """Synchronise and raise if a kernel recorded a device-side error."""
         s = stream or torch.cuda.current_stream(self.device)

@@ -1,0 +1,104 @@
+"""Per-kernel parity: the intermediates of one forward against the oracle.
+
+Besides the layer outputs (tests/test_gpu_parity.py), the workspace a forward leaves
+behind is checked step by step:
+  * the row copy (fused into the gate/up GEMM, or the permute kernel): every (token, slot)
+    has its own row, inside its expert's group, tokens of an expert in ascending order,
+    and the row holds the token's values byte for byte (for e4m3 gate/up layers: the
+    oracle's quantised token row, byte for byte);
+  * the gate/up GEMM: each routed row's SwiGLU activation, and the shared group's
+    activations (experts side by side), against the oracle's;
+  * the down GEMM: each routed row's expert output and the shared experts' summed output.
+"""
+import numpy as np
+import pytest
+import torch
+
+from mixture_experts_layer_65_b200 import build
+from mixture_experts_layer_65_b200 import workloads as W
+from mixture_experts_layer_65_b200.layer import MoELayer, to_device_tensor
+from oracle import moe_oracle as O
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+SPECS = [
+    dict(T=333, d=256, n_shared=2, n_routed=16, inter=192, top_k=4),   # row copy in the GEMM
+    dict(T=700, d=256, n_shared=0, n_routed=16, inter=128, top_k=2),   # permute kernel
+]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib_ready():
+    build.build()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+
+
+def _f64(t: torch.Tensor) -> np.ndarray:
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def _close(got: np.ndarray, ref: np.ndarray, what: str):
+    err = np.abs(got - ref).max() / max(np.abs(ref).max(), 1e-30)
+    assert err <= P.TOL["bf16"], (what, err)
+    return err
+
+
+@pytest.mark.parametrize("e4m3", [False, True], ids=["bf16", "e4m3_gate_up"])
+@pytest.mark.parametrize("spec", SPECS, ids=lambda s: "T{T}_s{n_shared}_r{n_routed}_k{top_k}".format(**s))
+def test_intermediates_match_the_oracle(spec, e4m3):
+    w = W.make_workload("16b_prefill", alpha1=0.001, gate_up_e4m3=e4m3, **spec)
+    layer = MoELayer.from_workload(w)
+    out = layer.forward(to_device_tensor(w.u, "cuda"))
+    torch.cuda.synchronize()
+    layer.device_status()
+    T, d, I, K, ks, nr = w.T, w.d, w.inter, w.top_k, w.n_shared, w.n_routed
+    idx = out.topk_idx.cpu().numpy()
+    slot = layer.debug_buffer("slot_row").cpu().numpy().reshape(T, K)
+    grp = layer.debug_buffer("grp_row").cpu().numpy()
+    hs_first = 1 if ks else 0
+
+    # row copy: a bijection onto each expert's rows, tokens in ascending order
+    assert np.unique(slot).size == slot.size
+    for e in range(nr):
+        ts, kk = np.nonzero(idx == e)
+        order = np.argsort(ts, kind="stable")
+        np.testing.assert_array_equal(slot[ts, kk][order], grp[hs_first + e] + np.arange(ts.size))
+    xp = layer.debug_buffer("xp").cpu()
+    rows = slot.reshape(-1)
+    toks = np.repeat(np.arange(T), K)
+    if e4m3:
+        xp8 = xp.view(-1, d)[torch.from_numpy(rows)]
+        got = xp8.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+        q, _ = O.quantize_rows_e4m3(w.u)
+        np.testing.assert_array_equal(got, q[toks])
+    else:
+        got = xp.view(-1, d)[torch.from_numpy(rows)].view(torch.int16).numpy().view(np.uint16)
+        np.testing.assert_array_equal(got, w.u[toks])
+
+    # gate/up and down GEMMs, routed experts
+    hr = _f64(layer.debug_buffer("hr")).reshape(-1, I)
+    yr = _f64(layer.debug_buffer("yr")).reshape(-1, d)
+    for e in range(nr):
+        ts, kk = np.nonzero(idx == e)
+        if ts.size == 0:
+            continue
+        x = w.u[ts]
+        hid = O.swiglu_hidden(x, w.w_gate[ks + e], w.w_up[ks + e], e4m3)
+        y = O.swiglu_ffn(x, w.w_gate[ks + e], w.w_up[ks + e], w.w_down[ks + e], e4m3)
+        r = slot[ts, kk]
+        _close(hr[r], hid, f"hidden of expert {e}")
+        _close(yr[r], y, f"output of expert {e}")
+
+    # shared group
+    if ks:
+        hs = _f64(layer.debug_buffer("hs")).reshape(-1, ks * I)[:T]
+        ys = _f64(layer.debug_buffer("ys")).reshape(-1, d)[:T]
+        y_ref = np.zeros((T, d))
+        for j in range(ks):
+            _close(hs[:, j * I:(j + 1) * I], O.swiglu_hidden(w.u, w.w_gate[j], w.w_up[j], e4m3),
+                   f"hidden of shared expert {j}")
+            y_ref += O.swiglu_ffn(w.u, w.w_gate[j], w.w_up[j], w.w_down[j], e4m3)
+        _close(ys, y_ref, "shared output")
+    else:
+        assert layer.debug_buffer("hs").numel() == 0
