@@ -266,7 +266,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         aux_g = torch.empty(1, dtype=torch.float32, device=dev)
 
     stream = torch.cuda.current_stream(dev)
-    # one captured CUDA graph per input buffer: the six kernel launches of a forward are
+    # one captured CUDA graph per input buffer: the kernel launches of a forward are
     # replayed without host launch overhead (the layer's inputs/outputs stay fixed)
     graphs = None
     if not args.no_graph:

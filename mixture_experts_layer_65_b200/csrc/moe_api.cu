@@ -1,13 +1,17 @@
 // moe_api.cu -- the C-ABI (include/moe.h): validation, weight re-layout, workspace,
 // TMA descriptors and the launch sequence of one DeepSeekMoE layer forward pass.
 //
-// Launch sequence of moe_forward (one stream, no host synchronisation):
+// Launch sequence of moe_forward (one stream, no host synchronisation, every launch with
+// programmatic dependent launch):
 //   1. router      logits -> softmax -> top-k, gates, per-tile histograms / ranks / sums
+//                  (tensor-core kernel; a SIMT kernel for decode-sized batches and fp32)
 //   2. scan        per-expert counts, padded offsets, tile tables, balance loss
-//   3. permute     token rows -> expert-contiguous rows (top_k copies per token)
-//   4. gate/up     grouped GEMM + SwiGLU (shared group reads the token rows directly)
-//   5. down        grouped GEMM
-//   6. combine     h = u + shared + sum_k g_k * routed_k (fp32, fixed order)
+//   3. quantise    (e4m3 gate/up layers only) e4m3 token rows + per-row scales
+//   4. permute     token rows -> expert-contiguous rows (top_k copies per token); on bf16
+//                  layers with shared experts this copy runs inside step 5 instead
+//   5. gate/up     grouped GEMM + SwiGLU (shared group reads the token rows directly)
+//   6. down        grouped GEMM
+//   7. combine     h = u + shared + sum_k g_k * routed_k (fp32, fixed order)
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
