@@ -21,6 +21,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -100,12 +101,19 @@ def algorithmic_work(w, active_experts: int | None = None) -> dict:
     return work
 
 
+def _code_only(src: str) -> str:
+    """C/C++ source without comments and whitespace (comment edits keep the digest)."""
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    return "".join(src.split())
+
+
 def csrc_digest() -> str:
     h = hashlib.sha1()
     d = os.path.join(ROOT, "mixture_experts_layer_65_b200", "csrc")
     for f in sorted(os.listdir(d)):
-        with open(os.path.join(d, f), "rb") as fh:
-            h.update(f.encode() + fh.read())
+        with open(os.path.join(d, f), encoding="utf-8") as fh:
+            h.update(f.encode() + _code_only(fh.read()).encode())
     return h.hexdigest()
 
 
