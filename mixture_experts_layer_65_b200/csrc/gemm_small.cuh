@@ -111,8 +111,18 @@ grouped_gemm_small_kernel(const __grid_constant__ CUtensorMap tmW_s,
   const int total = __ldg(&a.ts[a.G]);
 
   // tile -> (group g, weight tile m); GemmArgs-style decode with one token tile per group
-  auto decode = [&](int tile, int& g, int& m, int& e, bool& sh) {
-    while (tile >= __ldg(&a.ts[g + 1])) ++g;
+  // Tiles go round-robin to the CTAs, so the first total % gridDim.x CTAs get one tile
+  // more.  When the shared group's tiles are heavier (K = n_shared * inter), they are
+  // placed on CTAs that get one tile fewer: position p of the round-robin order visits
+  // tile remap(p).  Each CTA's tile indices stay increasing (the group search relies on it).
+  const int n_sh = a.has_shared ? __ldg(&a.ts[1]) : 0;
+  const int r0 = total % (int)gridDim.x;
+  // (the remap needs the positions r0 .. r0 + n_sh - 1 to exist: r0 + n_sh <= total)
+  const bool rebalance = n_sh > 0 && a.kb_shared > a.kb_routed && r0 > 0 &&
+                         n_sh <= (int)gridDim.x - r0 && r0 + n_sh <= total;
+  auto decode = [&](int pos, int& g, int& m, int& e, bool& sh) {
+    const int tile = !rebalance ? pos : pos < r0 ? n_sh + pos : pos < r0 + n_sh ? pos - r0 : pos;
+    while (g < a.G - 1 && tile >= __ldg(&a.ts[g + 1])) ++g;
     m = tile - __ldg(&a.ts[g]);
     sh = a.has_shared && g == 0;
     e = g - a.has_shared;
