@@ -253,7 +253,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
     from mixture_experts_layer_65_b200 import workloads as W
     from mixture_experts_layer_65_b200.layer import MoELayer, to_device_tensor
-    from mixture_experts_layer_65_b200.parallel import global_balance_loss
+    from mixture_experts_layer_65_b200.parallel import global_balance_loss, global_token_count
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
@@ -272,6 +272,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         psum = torch.empty(w.n_routed, dtype=torch.float32, device=dev)
         cnt_g = torch.empty(w.n_routed, dtype=torch.int32, device=dev)
         aux_g = torch.empty(1, dtype=torch.float32, device=dev)
+        n_global = global_token_count(w.T, dev)   # once: the per-rank token count is fixed
 
     stream = torch.cuda.current_stream(dev)
     # one captured CUDA graph per input buffer: the kernel launches of a forward are
@@ -299,7 +300,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         else:
             layer.forward(ubufs[i % n_buf], out)
         if world > 1:   # balance loss of the global batch: all-reduce counts and sums
-            global_balance_loss(layer, out, psum, cnt_g, aux_g)
+            global_balance_loss(layer, out, psum, cnt_g, aux_g, n_global=n_global)
 
     for i in range(max(3, args.warmup)):
         step(i)

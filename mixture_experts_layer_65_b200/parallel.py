@@ -15,25 +15,35 @@ import torch
 import torch.distributed as dist
 
 
-def all_reduce_balance_stats(counts: torch.Tensor, psum: torch.Tensor, n_tokens: int,
-                             group=None) -> int:
-    """Sum `counts` [N_r] and `psum` [N_r] over the ranks of `group`, in place.
-
-    Returns the global token count (the sum of every rank's `n_tokens`).  Every rank must
-    call this in the same order (it issues three all-reduces).
-    """
-    dist.all_reduce(counts, group=group)
-    dist.all_reduce(psum, group=group)
-    t = torch.tensor([int(n_tokens)], dtype=torch.int64, device=counts.device)
+def global_token_count(n_tokens: int, device, group=None) -> int:
+    """The sum of every rank's `n_tokens` (one all-reduce and a host read: call it once,
+    not per step, when the per-rank token counts do not change)."""
+    t = torch.tensor([int(n_tokens)], dtype=torch.int64, device=device)
     dist.all_reduce(t, group=group)
     return int(t.item())
 
 
+def all_reduce_balance_stats(counts: torch.Tensor, psum: torch.Tensor, n_tokens: int,
+                             group=None, n_global: int | None = None) -> int:
+    """Sum `counts` [N_r] and `psum` [N_r] over the ranks of `group`, in place.
+
+    Returns the global token count: `n_global` when the caller already knows it (then no
+    host synchronisation happens here), else the sum of every rank's `n_tokens`.  Every
+    rank must call this in the same order and with the same choice of `n_global`.
+    """
+    dist.all_reduce(counts, group=group)
+    dist.all_reduce(psum, group=group)
+    if n_global is not None:
+        return int(n_global)
+    return global_token_count(n_tokens, counts.device, group)
+
+
 def global_balance_loss(layer, out, psum_buf: torch.Tensor, counts_buf: torch.Tensor,
-                        aux_buf: torch.Tensor, group=None) -> torch.Tensor:
-    """After `layer.forward(u, out)`: the balance loss of the global batch into `aux_buf`."""
+                        aux_buf: torch.Tensor, group=None, n_global: int | None = None) -> torch.Tensor:
+    """After `layer.forward(u, out)`: the balance loss of the global batch into `aux_buf`
+    (`n_global`: the global token count, if known -- see global_token_count)."""
     from .layer import balance_loss
     layer.expert_psum(psum_buf)
     counts_buf.copy_(out.expert_counts)
-    n_global = all_reduce_balance_stats(counts_buf, psum_buf, layer.T, group)
+    n_global = all_reduce_balance_stats(counts_buf, psum_buf, layer.T, group, n_global)
     return balance_loss(counts_buf, psum_buf, n_global, layer.alpha1, aux_buf)

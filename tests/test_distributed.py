@@ -36,6 +36,12 @@ def _worker(rank, world, port, bounds, q):
         psum = torch.from_numpy(r.s.sum(axis=0))
         n = parallel.all_reduce_balance_stats(counts, psum, hi - lo)
         aux = w.alpha1 * float(torch.sum((counts / n) * (psum / n)))
+        # the same with the global token count computed once up front (no per-step read)
+        n_once = parallel.global_token_count(hi - lo, "cpu")
+        c2 = torch.from_numpy(np.bincount(r.topk_idx.reshape(-1), minlength=w.n_routed))
+        p2 = torch.from_numpy(r.s.sum(axis=0))
+        n2 = parallel.all_reduce_balance_stats(c2, p2, hi - lo, n_global=n_once)
+        assert n2 == n and torch.equal(c2, counts) and torch.equal(p2, psum)
         q.put((rank, n, counts.numpy(), psum.numpy(), aux, r.topk_idx))
     finally:
         dist.destroy_process_group()
