@@ -2,9 +2,10 @@
 //
 // DeepSeekMoE (deepforge.srivtx.xyz article), "Routing in a classic MoE layer":
 // h = sum_i g_i FFN_i(u) + u, with the K_s shared experts ("Where this sits", shared
-// expert isolation) added with gate 1.  One warp owns one token row and sums, in fp32 and
-// in a fixed order, u + (shared-group output) + g_0 Y_0 + ... + g_{K'-1} Y_{K'-1}, then
-// rounds once to the output type.
+// expert isolation) added with gate 1.  One warp owns one part of one token row (the
+// whole row, unless there are too few tokens to keep the SMs' load slots busy) and sums,
+// in fp32 and in a fixed order, u + (shared-group output) + g_0 Y_0 + ... + g_{K'-1}
+// Y_{K'-1}, then rounds once to the output type.
 #pragma once
 
 #include "router.cuh"
@@ -27,7 +28,23 @@ struct CombineArgs {
   const float* topk_w;     // [T, top_k]
   T* h;                    // [T, d]
   int T_, d, top_k;
+  int parts;               // warps per token row, each a contiguous range of its vectors
 };
+
+// Warps per token row: 1 for large batches; for small ones enough to give the SMs about
+// 16 warps each, with at least 32 vectors (one per lane) per part.
+inline int combine_parts(int T, int nvec, int n_sms) {
+  int p = (n_sms * 16) / (T > 0 ? T : 1);
+  const int pmax = nvec / 32 > 1 ? nvec / 32 : 1;
+  return p < 1 ? 1 : (p > pmax ? pmax : p);
+}
+
+// Vector range [v0, v1) of part `part` of a row of nvec vectors split into `parts`.
+__device__ __forceinline__ void combine_range(int nvec, int parts, int part, int& v0, int& v1) {
+  const int per = (nvec + parts - 1) / parts;
+  v0 = part * per;
+  v1 = v0 + per < nvec ? v0 + per : nvec;
+}
 
 __device__ __forceinline__ void add8(float (&acc)[8], const uint4& v, float w) {
   const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
@@ -47,7 +64,8 @@ combine_bf16_kernel(CombineArgs<__nv_bfloat16> a) {
   pdl_launch_dependents();
   pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = blockIdx.x * kCombineWarps + warp;
+  const int gw = blockIdx.x * kCombineWarps + warp;
+  const int t = gw / a.parts;
   if (t >= a.T_) return;
   __shared__ int s_row[kCombineWarps][kMaxTopK];
   __shared__ float s_w[kCombineWarps][kMaxTopK];
@@ -64,11 +82,12 @@ combine_bf16_kernel(CombineArgs<__nv_bfloat16> a) {
     yk[k] = reinterpret_cast<const uint4*>(a.yr + (size_t)(on ? s_row[warp][k] : 0) * a.d);
     wk[k] = on ? s_w[warp][k] : 0.f;
   }
-  const int nvec = a.d >> 3;
+  int v0, v1;
+  combine_range(a.d >> 3, a.parts, gw - t * a.parts, v0, v1);
   const uint4* ur = reinterpret_cast<const uint4*>(a.u + (size_t)t * a.d);
   const uint4* sr = a.ys ? reinterpret_cast<const uint4*>(a.ys + (size_t)t * a.d) : nullptr;
   uint4* hr = reinterpret_cast<uint4*>(a.h + (size_t)t * a.d);
-  for (int v = lane; v < nvec; v += 32) {
+  for (int v = v0 + lane; v < v1; v += 32) {
     uint4 x[MAXK];
     const uint4 xu = __ldg(ur + v);
     const uint4 xs = sr ? __ldg(sr + v) : make_uint4(0u, 0u, 0u, 0u);
@@ -97,7 +116,8 @@ static __global__ void __launch_bounds__(kCombineWarps * 32) combine_f32_kernel(
   pdl_launch_dependents();
   pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = blockIdx.x * kCombineWarps + warp;
+  const int gw = blockIdx.x * kCombineWarps + warp;
+  const int t = gw / a.parts;
   if (t >= a.T_) return;
   __shared__ int s_row[kCombineWarps][kMaxTopK];
   __shared__ float s_w[kCombineWarps][kMaxTopK];
@@ -106,11 +126,12 @@ static __global__ void __launch_bounds__(kCombineWarps * 32) combine_f32_kernel(
     s_w[warp][lane] = a.topk_w[(size_t)t * a.top_k + lane];
   }
   __syncwarp();
-  const int nvec = a.d >> 2;
+  int v0, v1;
+  combine_range(a.d >> 2, a.parts, gw - t * a.parts, v0, v1);
   const float4* ur = reinterpret_cast<const float4*>(a.u + (size_t)t * a.d);
   const float4* sr = a.ys ? reinterpret_cast<const float4*>(a.ys + (size_t)t * a.d) : nullptr;
   float4* hr = reinterpret_cast<float4*>(a.h + (size_t)t * a.d);
-  for (int v = lane; v < nvec; v += 32) {
+  for (int v = v0 + lane; v < v1; v += 32) {
     float4 acc = __ldg(ur + v);
     if (sr) {
       const float4 s = __ldg(sr + v);

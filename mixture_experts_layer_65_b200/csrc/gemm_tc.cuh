@@ -16,17 +16,21 @@
 // output tiles with the paired-SM MMA (tcgen05.mma.cta_group::2, M = 256, N = 256,
 // K = 16): CTA r of the pair stages rows [128 r, 128 r + 128) of the A tile and rows
 // [128 r, 128 r + 128) of the B tile, so each SM holds half of B and the MMA reads both
-// SMs' shared memory.  320 threads per CTA:
-//   warp 0      one thread issues the TMA loads of this CTA's halves (128 x 64 bf16 each,
-//               128-byte swizzle) into a 6-stage ring; completion is counted on the
-//               leader CTA's "full" barrier (the leader expects both CTAs' bytes);
+// SMs' shared memory.  448 threads per CTA (640 for the e4m3 gate/up GEMM):
+//   warp 0      one thread issues the TMA loads of this CTA's halves (128 rows x 128
+//               bytes each per k-block, 128-byte swizzle) into a ring of 3 stages of two
+//               k-blocks; completion is counted on the leader CTA's "full" barrier (the
+//               leader expects both CTAs' bytes);
 //   warp 1      allocates 512 TMEM columns in both CTAs (two 256-column fp32
 //               accumulators); in the leader one thread issues the MMAs and commits with a
 //               multicast arrive to both CTAs' "empty" / "accumulator full" barriers;
-//   warps 2..9  epilogue in both CTAs: tcgen05.ld of the CTA's 128 accumulator rows (one
-//               TMEM lane per output row; two warps per lane quadrant, each taking half of
-//               the columns), SiLU(gate)*up in fp32 or a plain convert, bf16 stores; one
-//               arrive per warp on the leader's "accumulator empty" barrier.
+//   warps 2..9  epilogue in both CTAs (warps 2..17 for e4m3): tcgen05.ld of the CTA's
+//               128 accumulator rows (one TMEM lane per output row; two warps per lane
+//               quadrant, each taking half of the columns, or four for e4m3), SiLU(gate)*up
+//               in fp32 or a plain convert, bf16 stores; one arrive per warp on the
+//               leader's "accumulator empty" barrier;
+//   4 warps     after the epilogue warps: the fused row copy of the gate/up GEMM (idle
+//               when there is none).
 // Gate/up weight rows are interleaved in blocks of 64 (64 gate rows, then the 64 matching
 // up rows), so a 256-row B tile yields 128 Hmid columns.  Tiles are enumerated group by
 // group (row block major, column block minor) and handed out round-robin over clusters.

@@ -789,20 +789,23 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
     launch_pdl(grouped_gemm_simt_kernel<kDown>, dim3(grid), dim3(kSimtThreads), 0, stream, s2);
     MOE_CUDA(cudaGetLastError());
 
+    const int parts = combine_parts(T, d / 4, H->n_sms);
     CombineArgs<float> ca{static_cast<const float*>(u), static_cast<const float*>(H->ys),
                           static_cast<const float*>(H->yr), H->slot_row, topk_w,
-                          static_cast<float*>(h), T, d, K};
+                          static_cast<float*>(h), T, d, K, parts};
     tick(H, stream, 5);
-    launch_pdl(combine_f32_kernel, dim3((T + kCombineWarps - 1) / kCombineWarps), dim3(kCombineWarps * 32), 0, stream, ca);
+    const int cgrid = (int)(((int64_t)T * parts + kCombineWarps - 1) / kCombineWarps);
+    launch_pdl(combine_f32_kernel, dim3(cgrid), dim3(kCombineWarps * 32), 0, stream, ca);
     MOE_CUDA(cudaGetLastError());
   }
   if (H->bf16) {
+    const int parts = combine_parts(T, d / 8, H->n_sms);
     CombineArgs<__nv_bfloat16> ca{static_cast<const __nv_bfloat16*>(u),
                                   static_cast<const __nv_bfloat16*>(H->ys),
                                   static_cast<const __nv_bfloat16*>(H->yr), H->slot_row, topk_w,
-                                  static_cast<__nv_bfloat16*>(h), T, d, K};
+                                  static_cast<__nv_bfloat16*>(h), T, d, K, parts};
     tick(H, stream, 5);
-    const int cgrid = (T + kCombineWarps - 1) / kCombineWarps;
+    const int cgrid = (int)(((int64_t)T * parts + kCombineWarps - 1) / kCombineWarps);
     with_maxk(H->maxk, [&](auto m) {
       launch_pdl(combine_bf16_kernel<m()>, dim3(cgrid), dim3(kCombineWarps * 32), 0, stream, ca);
       return 0;
