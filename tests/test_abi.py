@@ -34,6 +34,7 @@ def _cfg(**kw):
 
 @pytest.mark.parametrize("kw,status", [
     (dict(T=0), _lib.MOE_ERR_INVALID_ARG),
+    (dict(T=(1 << 24) + 1), _lib.MOE_ERR_INVALID_ARG),
     (dict(top_k=17, n_routed=32), _lib.MOE_ERR_UNSUPPORTED),
     (dict(top_k=5, n_routed=4), _lib.MOE_ERR_INVALID_ARG),
     (dict(n_routed=257), _lib.MOE_ERR_UNSUPPORTED),

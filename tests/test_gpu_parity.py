@@ -83,6 +83,21 @@ def test_full_size_layer(name):
     assert layer.kernels_per_forward == (5 if fused else 6)
 
 
+# ------------------------------------------------------------------------ the limits
+def test_largest_expert_count_and_top_k_every_row():
+    """N_r = 256 and top_k = 16, the library's limits, with more tokens than the SMs take
+    in one router tile each (128 tokens per tile): every router CTA walks two tiles, with
+    two 256-column TMEM accumulators (512 columns), the widest top-k path (rounds of a
+    group-wide maximum) and the combine's largest load batch.  Every row is compared."""
+    n_sms = torch.cuda.get_device_properties(0).multi_processor_count
+    spec = dict(T=20000, d=256, n_shared=1, n_routed=256, inter=64, top_k=16)
+    assert spec["T"] > n_sms * 128
+    w = W.make_workload("16b_prefill", alpha1=0.001, **spec)
+    g, *_ = run(w)
+    rep = P.compare(w, g)
+    print(spec, rep)
+
+
 # ------------------------------------------------------------------------ edge cases
 def _bias_layer(bias, **spec):
     w = W.make_workload("16b_prefill", alpha1=0.001, **spec)
