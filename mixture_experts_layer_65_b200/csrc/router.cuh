@@ -583,6 +583,8 @@ __global__ void __launch_bounds__(kRouterEpiThreads) router_simt_kernel(RouterSi
 }
 
 // ------------------------------------------------------------------------ bf16, few tokens
+constexpr int kSmallPairs = 4;   // (token, expert) dot products a warp computes together
+
 struct RouterSmallArgs {
   const __nv_bfloat16* u;     // [T, d]
   const __nv_bfloat16* cen;   // [n_routed, d]
@@ -610,24 +612,54 @@ __global__ void __launch_bounds__(kRouterEpiThreads) router_small_kernel(RouterS
   const int ld = router_ld(n_pad);
   const int nv = a.d >> 3;
   for (int e = tid; e < 4 * kMaxRouted; e += kRouterEpiThreads) (&SM.mask[0][0])[e] = 0u;
-  for (int p = warp; p < R * a.n_routed; p += kRouterEpiThreads / 32) {
-    const int r = p / a.n_routed, i = p - r * a.n_routed;
-    const int t = tile * R + r;
-    float acc = 0.f;
-    if (t < a.T) {
-      const uint4* ur = reinterpret_cast<const uint4*>(a.u + (size_t)t * a.d);
-      const uint4* er = reinterpret_cast<const uint4*>(a.cen + (size_t)i * a.d);
-      for (int v = lane; v < nv; v += 32) {
-        float x[8], y[8];
-        bf16x8_to_f32(__ldg(ur + v), x);
-        bf16x8_to_f32(__ldg(er + v), y);
+  // each warp takes kSmallPairs consecutive (token, expert) pairs at once, so that their
+  // loads are in flight together; every dot product keeps its own order of operations
+  const int npairs = R * a.n_routed;
+  for (int p0 = warp * kSmallPairs; p0 < npairs; p0 += (kRouterEpiThreads / 32) * kSmallPairs) {
+    const uint4* ur[kSmallPairs];
+    const uint4* er[kSmallPairs];
+    bool on[kSmallPairs];
+    float acc[kSmallPairs];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) acc = fmaf(x[k], y[k], acc);
+    for (int j = 0; j < kSmallPairs; ++j) {
+      const int p = p0 + j < npairs ? p0 + j : npairs - 1;
+      const int r = p / a.n_routed, i = p - r * a.n_routed;
+      const int t = tile * R + r;
+      on[j] = p0 + j < npairs && t < a.T;
+      ur[j] = reinterpret_cast<const uint4*>(a.u + (size_t)(t < a.T ? t : 0) * a.d);
+      er[j] = reinterpret_cast<const uint4*>(a.cen + (size_t)i * a.d);
+      acc[j] = 0.f;
+    }
+    for (int v = lane; v < nv; v += 32) {
+      uint4 xu[kSmallPairs], xe[kSmallPairs];
+#pragma unroll
+      for (int j = 0; j < kSmallPairs; ++j) {
+        if (on[j]) {
+          xu[j] = __ldg(ur[j] + v);
+          xe[j] = __ldg(er[j] + v);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < kSmallPairs; ++j) {
+        if (on[j]) {
+          float x[8], y[8];
+          bf16x8_to_f32(xu[j], x);
+          bf16x8_to_f32(xe[j], y);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) acc[j] = fmaf(x[k], y[k], acc[j]);
+        }
       }
     }
 #pragma unroll
-    for (int m = 16; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
-    if (lane == 0) lg[(size_t)r * ld + i] = acc + a.bias[i];
+    for (int j = 0; j < kSmallPairs; ++j) {
+#pragma unroll
+      for (int m = 16; m > 0; m >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], m);
+      const int p = p0 + j;
+      if (lane == 0 && p < npairs) {
+        const int r = p / a.n_routed, i = p - r * a.n_routed;
+        lg[(size_t)r * ld + i] = acc[j] + a.bias[i];
+      }
+    }
   }
   __syncthreads();
   auto sync = [] { __syncthreads(); };
