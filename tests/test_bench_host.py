@@ -1,0 +1,69 @@
+"""Host-side arithmetic of the benchmark (CPU only): the per-kernel algorithmic work that
+the roofline fractions divide by, pinned to figures computed independently from the layer
+shapes, and the source digest that decides whether the committed ncu traffic still applies."""
+import types
+
+import pytest
+
+import bench
+from mixture_experts_layer_65_b200 import workloads as W
+
+
+def _gb(x):
+    return x / 1e9
+
+
+def _shape(name: str):
+    """The layer's sizes without drawing its tensors."""
+    return types.SimpleNamespace(name=name, **W.CONFIGS[name])
+
+
+@pytest.mark.parametrize("name,gflop", [
+    ("2b", 451.0), ("gshard", 451.0), ("16b_prefill", 2268.0), ("145b", 19791.0)])
+def test_expert_gemm_flops_of_the_layers(name, gflop):
+    # 6 d I (K_s + K') FLOPs per token: three d x I products per selected expert, 2 FLOPs
+    # per multiply-add; 2B and GShard-like layers are iso-compute by construction
+    work = bench.algorithmic_work(_shape(name))
+    assert work["gate_up_gemm"][0] == "tensor" and work["down_gemm"][0] == "tensor"
+    total = work["gate_up_gemm"][1] + work["down_gemm"][1]
+    assert abs(total / 1e9 - gflop) / gflop < 1e-3
+    assert work["gate_up_gemm"][1] == pytest.approx(2 * work["down_gemm"][1])
+
+
+def test_memory_bound_bytes_of_the_16b_layer():
+    work = bench.algorithmic_work(_shape("16b_prefill"))
+    T, d = 16384, 2048
+    # router: token matrix + centroids read, (index, gate, rank) per selected slot written
+    assert work["router"] == ("hbm", T * d * 2 + 64 * d * 2 + T * 6 * 12)
+    assert _gb(work["router"][1]) == pytest.approx(0.0685, abs=5e-4)
+    # permute: each token row read once, written once per selected expert
+    assert _gb(work["permute"][1]) == pytest.approx(0.470, abs=1e-3)
+    # combine: u, the shared output, K' routed rows read, h written, slots and gates read
+    assert _gb(work["combine"][1]) == pytest.approx(0.604, abs=1e-3)
+
+
+def test_decode_sized_gemms_are_counted_as_weight_streams():
+    w = _shape("16b_decode")
+    work = bench.algorithmic_work(w, active_experts=64)
+    assert work["gate_up_gemm"][0] == "hbm" and work["down_gemm"][0] == "hbm"
+    d, I, n = 2048, 1408, 64 + 2
+    weights = n * 3 * I * d * 2   # gate, up and down of every expert that received tokens
+    streamed = work["gate_up_gemm"][1] + work["down_gemm"][1]
+    assert weights < streamed < weights * 1.01
+    # fewer active experts, fewer weight bytes
+    assert bench.algorithmic_work(w, active_experts=10)["gate_up_gemm"][1] < work["gate_up_gemm"][1]
+
+
+def test_source_digest_ignores_comments_and_whitespace_only():
+    code = "int f(int x) {\n  return x + 1;  // add one\n}\n/* block\n comment */"
+    same = "int f(int x){return x+1;}"
+    other = "int f(int x){return x+2;}"
+    assert bench._code_only(code) == bench._code_only(same)
+    assert bench._code_only(code) != bench._code_only(other)
+    assert len(bench.csrc_digest()) == 40
+
+
+def test_workload_description_names_the_layer_and_its_sizes():
+    desc = bench.workload_desc(_shape("16b_prefill"), 4)
+    assert desc["workload"].startswith("16b_prefill: T=16384 d=2048")
+    assert desc["global_batch"] == 4 * 16384 and desc["parallelism"] == "dp4"
