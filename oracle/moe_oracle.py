@@ -1,4 +1,4 @@
-"""Plain fp64 CPU oracle of the DeepSeekMoE layer forward pass.
+"""Plain fp64 CPU oracle of the DeepSeekMoE layer forward pass (and its gradients).
 
 TEST INFRASTRUCTURE ONLY.  Only the test suite, the package smoke check and the CPU
 baseline leg of the benchmark may import this module.  It shares no code with the CUDA
@@ -32,7 +32,8 @@ Readings where the pages are silent (each also listed in the design notes):
 
 All arithmetic is fp64.  bf16 inputs arrive as uint16 bit patterns and are widened
 exactly.  Parity is pinned by the CPU tests against brute force, closed forms, library
-routines (scipy softmax, transformers' LlamaMLP SwiGLU) and invariants.
+routines (scipy softmax, transformers' LlamaMLP SwiGLU) and invariants; the backward pass
+(moe_backward) against central finite differences of moe_forward and invariants.
 """
 from __future__ import annotations
 
@@ -44,7 +45,7 @@ import numpy as np
 __all__ = ["widen", "router_logits", "affinity_softmax", "select_topk", "route",
            "swiglu_hidden", "swiglu_ffn", "balance_stats", "moe_forward", "near_tie_tokens",
            "brute_force_layer", "Routing", "LayerOut", "E4M3_MAX", "e4m3_round",
-           "quantize_rows_e4m3"]
+           "quantize_rows_e4m3", "swiglu_ffn_backward", "moe_backward", "LayerGrads"]
 
 
 def widen(a) -> np.ndarray:
@@ -244,6 +245,93 @@ def near_tie_tokens(s: np.ndarray, top_k: int, eps: float = 1e-6) -> np.ndarray:
         return np.zeros(s.shape[0], dtype=bool)
     part = -np.sort(-s, axis=1)
     return (part[:, top_k - 1] - part[:, top_k]) < eps
+
+
+# ---------------------------------------------------------------- backward pass
+# Gradients of the layer for training (the full-precision layer only).  The scalar being
+# differentiated is L = sum_t dh_t . h_t + d_aux * aux, i.e. dh = dL/dh (the gradient
+# arriving from above) and d_aux = dL/daux (the weight of the balance loss in the training
+# objective, usually 1).  Readings, where the pages give the forward only:
+#   * the top-k choice is piecewise constant in u and the centroids, so no gradient flows
+#     through *which* experts are chosen; the chosen gates g_i = s_i ("Routing in a
+#     classic MoE layer") carry the gradient into the affinities and through the softmax;
+#   * f_i = count_i / T ("Expert-level balance loss") is a step function of the same
+#     choice and is held constant; P_i = mean_t s[t, i] carries the balance loss's
+#     gradient, d aux / d s[t, i] = alpha_1 * f_i / T;
+#   * shared experts have gate 1, so their output gradient is dh itself.
+def _sigmoid(z: np.ndarray) -> np.ndarray:
+    with np.errstate(over="ignore"):
+        return 1.0 / (1.0 + np.exp(-z))
+
+
+def swiglu_ffn_backward(x, w_gate, w_up, w_down, dy):
+    """Gradients of y = W_down (SiLU(W_gate x) * (W_up x)) over rows x [n, d], given
+    dy = dL/dy [n, d].  With a = W_gate x, b = W_up x and SiLU'(a) = sigma(a) (1 + a
+    (1 - sigma(a))): dhid = dy W_down, da = dhid * b * SiLU'(a), db = dhid * SiLU(a).
+    Returns (dx [n, d], dW_gate [I, d], dW_up [I, d], dW_down [d, I])."""
+    x = widen(x)
+    wg, wu, wd = widen(w_gate), widen(w_up), widen(w_down)
+    dy = np.asarray(dy, dtype=np.float64)
+    a = x @ wg.T
+    b = x @ wu.T
+    sg = _sigmoid(a)
+    silu = a * sg
+    dhid = dy @ wd
+    da = dhid * b * (sg * (1.0 + a * (1.0 - sg)))
+    db = dhid * silu
+    return da @ wg + db @ wu, da.T @ x, db.T @ x, dy.T @ (silu * b)
+
+
+@dataclasses.dataclass
+class LayerGrads:
+    du: np.ndarray            # [T, d]
+    d_centroids: np.ndarray   # [N_r, d]
+    d_bias: np.ndarray        # [N_r] (of the per-expert logit bias, zero or not)
+    d_w_gate: np.ndarray      # [n_shared + N_r, I, d]
+    d_w_up: np.ndarray        # [n_shared + N_r, I, d]
+    d_w_down: np.ndarray      # [n_shared + N_r, d, I]
+
+
+def moe_backward(u, centroids, w_gate, w_up, w_down, n_shared: int, top_k: int,
+                 alpha1: float, dh, d_aux: float = 0.0, bias=None) -> LayerGrads:
+    """Gradients of L = sum_t dh_t . h_t + d_aux * aux for the layer of moe_forward (same
+    argument layouts; dh [T, d]).  The routing is recomputed exactly as in the forward."""
+    x = widen(u)
+    T, d = x.shape
+    cen = widen(centroids)
+    n_routed = cen.shape[0]
+    dh = np.asarray(dh, dtype=np.float64)
+    r = route(x, centroids, top_k, bias)
+    counts, f, P, aux = balance_stats(r.s, r.topk_idx, n_routed, alpha1)
+    G = n_shared + n_routed
+    inter = np.asarray(w_gate).shape[1]
+    d_wg = np.zeros((G, inter, d))
+    d_wu = np.zeros((G, inter, d))
+    d_wd = np.zeros((G, d, inter))
+    du = dh.copy()                                        # the residual
+    for j in range(n_shared):                             # gate 1
+        dx, d_wg[j], d_wu[j], d_wd[j] = swiglu_ffn_backward(x, w_gate[j], w_up[j], w_down[j], dh)
+        du += dx
+    dg = np.zeros((T, top_k))                             # dL / d g[t, k]
+    for e in range(n_routed):
+        tok, slot = np.nonzero(r.topk_idx == e)
+        if tok.size == 0:
+            continue
+        ge = n_shared + e
+        xe = x[tok]
+        dg[tok, slot] = np.sum(dh[tok] * swiglu_ffn(xe, w_gate[ge], w_up[ge], w_down[ge]), axis=1)
+        dy = r.topk_w[tok, slot][:, None] * dh[tok]
+        dx, d_wg[ge], d_wu[ge], d_wd[ge] = swiglu_ffn_backward(xe, w_gate[ge], w_up[ge], w_down[ge], dy)
+        du[tok] += dx                                     # a token picks an expert once
+    # affinities: the chosen gates, and the balance loss through P_i
+    ds = np.zeros((T, n_routed))
+    ds[np.arange(T)[:, None], r.topk_idx] = dg
+    ds += float(d_aux) * float(alpha1) * f[None, :] / T
+    # softmax: dl = s * (ds - sum_i s_i ds_i), row by row
+    dl = r.s * (ds - np.sum(r.s * ds, axis=1, keepdims=True))
+    du += dl @ cen
+    return LayerGrads(du=du, d_centroids=dl.T @ x, d_bias=dl.sum(axis=0), d_w_gate=d_wg,
+                      d_w_up=d_wu, d_w_down=d_wd)
 
 
 # ---------------------------------------------------------------- brute force (tiny inputs)
