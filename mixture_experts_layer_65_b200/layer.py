@@ -90,12 +90,45 @@ class MoELayer:
             expert_counts=torch.empty(self.n_routed, dtype=torch.int32, device=dev),
             aux_loss=torch.empty(1, dtype=torch.float32, device=dev))
 
+    def _check_device_tensor(self, name: str, t: torch.Tensor, shape: tuple, dtype) -> None:
+        if not isinstance(t, torch.Tensor) or not t.is_cuda or t.device != self.device:
+            raise ValueError(f"{name} must be a CUDA tensor on {self.device}")
+        if tuple(t.shape) != shape or t.dtype != dtype or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous {list(shape)} {dtype} tensor")
+
+    def _check_outputs(self, out: MoEOutput) -> None:
+        """The library writes through these pointers: every output must be device memory of
+        the layer's device with the documented shape and dtype."""
+        self._check_device_tensor("h", out.h, (self.T, self.d), self.torch_dtype)
+        self._check_device_tensor("topk_idx", out.topk_idx, (self.T, self.top_k), torch.int32)
+        self._check_device_tensor("topk_w", out.topk_w, (self.T, self.top_k), torch.float32)
+        self._check_device_tensor("expert_counts", out.expert_counts, (self.n_routed,), torch.int32)
+        self._check_device_tensor("aux_loss", out.aux_loss, (1,), torch.float32)
+
+    def _check_host_outputs(self, out: MoEOutput) -> None:
+        """Host outputs are copied into whole: each must be a contiguous host tensor of the
+        documented shape and dtype (topk/counts/aux may be None: not copied back)."""
+        spec = (("h", (self.T, self.d), self.torch_dtype),
+                ("topk_idx", (self.T, self.top_k), torch.int32),
+                ("topk_w", (self.T, self.top_k), torch.float32),
+                ("expert_counts", (self.n_routed,), torch.int32),
+                ("aux_loss", (1,), torch.float32))
+        for name, shape, dtype in spec:
+            t = getattr(out, name)
+            if t is None and name != "h":
+                continue
+            if (not isinstance(t, torch.Tensor) or t.is_cuda or tuple(t.shape) != shape
+                    or t.dtype != dtype or not t.is_contiguous()):
+                raise ValueError(f"{name} must be a contiguous host {list(shape)} {dtype} tensor")
+
     def forward(self, u: torch.Tensor, out: MoEOutput | None = None,
                 stream: torch.cuda.Stream | None = None) -> MoEOutput:
         """Enqueue one forward pass on `stream` (default: the current stream)."""
-        if u.shape != (self.T, self.d) or u.dtype != self.torch_dtype or not u.is_contiguous():
-            raise ValueError(f"u must be a contiguous [{self.T}, {self.d}] {self.torch_dtype} tensor")
-        out = out or self.alloc_outputs()
+        self._check_device_tensor("u", u, (self.T, self.d), self.torch_dtype)
+        if out is None:
+            out = self.alloc_outputs()
+        else:
+            self._check_outputs(out)
         s = stream or torch.cuda.current_stream(self.device)
         check(lib().moe_forward(self._h, _ptr(u), _ptr(out.h), _ptr(out.topk_idx),
                                 _ptr(out.topk_w), _ptr(out.expert_counts), _ptr(out.aux_loss),
@@ -107,9 +140,12 @@ class MoELayer:
     def forward_host(self, u: torch.Tensor, out: MoEOutput | None = None,
                      stream: torch.cuda.Stream | None = None) -> MoEOutput:
         """Forward pass on HOST tensors (pinned for overlap); copies in and out, synchronises."""
-        if u.is_cuda or u.shape != (self.T, self.d) or u.dtype != self.torch_dtype:
-            raise ValueError("u must be a host tensor of the layer shape and dtype")
-        if out is None:
+        if (u.is_cuda or u.shape != (self.T, self.d) or u.dtype != self.torch_dtype
+                or not u.is_contiguous()):
+            raise ValueError("u must be a contiguous host tensor of the layer shape and dtype")
+        if out is not None:
+            self._check_host_outputs(out)
+        else:
             out = MoEOutput(
                 h=torch.empty(self.T, self.d, dtype=self.torch_dtype, pin_memory=True),
                 topk_idx=torch.empty(self.T, self.top_k, dtype=torch.int32, pin_memory=True),
@@ -136,8 +172,10 @@ class MoELayer:
         """Enqueue a forward on pinned HOST tensors without waiting (two calls in flight,
         copies overlapped with the neighbouring forwards).  `u` must stay unchanged and
         `out` unread until pipeline_wait() and a synchronisation of `stream`."""
-        if u.is_cuda or u.shape != (self.T, self.d) or u.dtype != self.torch_dtype:
-            raise ValueError("u must be a host tensor of the layer shape and dtype")
+        if (u.is_cuda or u.shape != (self.T, self.d) or u.dtype != self.torch_dtype
+                or not u.is_contiguous()):
+            raise ValueError("u must be a contiguous host tensor of the layer shape and dtype")
+        self._check_host_outputs(out)
         if not (u.is_pinned() and out.h.is_pinned()):
             raise ValueError("forward_host_pipelined needs pinned host tensors")
         s = stream or torch.cuda.current_stream(self.device)

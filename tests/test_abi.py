@@ -84,3 +84,34 @@ def test_wait_selftest_validates_arguments_before_touching_the_device():
     assert L.moe_selftest_wait_timeout(2, 50_000_000, ctypes.byref(code)) == _lib.MOE_ERR_INVALID_ARG
     assert L.moe_selftest_wait_timeout(0, 10, ctypes.byref(code)) == _lib.MOE_ERR_INVALID_ARG
     assert L.moe_selftest_wait_timeout(0, 50_000_000, None) == _lib.MOE_ERR_INVALID_ARG
+
+
+def _unbound_layer():
+    """A binding object with the sizes of a small layer but no library handle: argument
+    validation must reject bad tensors before anything reaches the library."""
+    import torch
+    from mixture_experts_layer_65_b200.layer import MoELayer
+    L = object.__new__(MoELayer)
+    L.T, L.d, L.top_k, L.n_routed = 8, 64, 2, 4
+    L.torch_dtype, L.device, L._h = torch.bfloat16, torch.device("cuda", 0), None
+    return L
+
+
+def test_binding_rejects_host_or_misshapen_tensors_before_the_library():
+    import torch
+    from mixture_experts_layer_65_b200.layer import MoEOutput
+    L = _unbound_layer()
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        L.forward(torch.zeros(8, 64, dtype=torch.bfloat16))          # host input
+    host = MoEOutput(h=torch.zeros(8, 64, dtype=torch.bfloat16),
+                     topk_idx=torch.zeros(8, 2, dtype=torch.int32),
+                     topk_w=torch.zeros(8, 2), expert_counts=torch.zeros(4, dtype=torch.int32),
+                     aux_loss=torch.zeros(1))
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        L._check_outputs(host)                                          # host outputs
+    short = host._replace(topk_w=torch.zeros(8, 1))
+    with pytest.raises(ValueError, match="topk_w"):
+        L._check_host_outputs(short)                                    # too small to copy into
+    L._check_host_outputs(host._replace(topk_idx=None, aux_loss=None))  # optional outputs
+    with pytest.raises(ValueError, match="contiguous host"):
+        L.forward_host(torch.zeros(64, 8, dtype=torch.bfloat16).t(), host)   # not contiguous
