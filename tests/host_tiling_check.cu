@@ -1,0 +1,72 @@
+// Host-side tiling rules of the kernels, checked exhaustively without a GPU (the program
+// makes no CUDA call).  Exit status 0 = every rule holds; the first violation is printed.
+#include <cstdio>
+
+#include "combine.cuh"
+#include "gemm_tc.cuh"
+#include "router.cuh"
+
+using namespace moe;
+
+static int fails = 0;
+#define CHECK(cond, ...)                                  \
+  do {                                                    \
+    if (!(cond)) {                                        \
+      if (fails++ < 10) {                                 \
+        std::printf("FAIL %s: ", #cond);                  \
+        std::printf(__VA_ARGS__);                         \
+        std::printf("\n");                                \
+      }                                                   \
+    }                                                     \
+  } while (0)
+
+int main() {
+  // router tiles: a multiple of 8 rows, at most the MMA's 128, and the tiles cover T with
+  // at most ceil(T / (SMs * 128)) tiles per SM
+  for (int n_sms : {132, 148, 160}) {
+    for (int T = 1; T <= 70000; T += (T < 4096 ? 1 : 97)) {
+      const int R = router_tile_rows(T, n_sms);
+      CHECK(R >= 8 && R <= kRouterBM && R % 8 == 0, "T=%d sms=%d R=%d", T, n_sms, R);
+      const long tiles = (T + R - 1) / R;
+      const long rounds = (T + (long)n_sms * kRouterBM - 1) / ((long)n_sms * kRouterBM);
+      CHECK(tiles <= (long)n_sms * rounds, "T=%d sms=%d R=%d tiles=%ld", T, n_sms, R, tiles);
+    }
+  }
+  // router stages: every padded expert count and tile height gets a ring of >= 2 stages
+  // inside the shared-memory budget; the M = 128 MMA reading 128 rows from a stage's last
+  // A block stays inside that stage; two accumulators fit the 512 TMEM columns
+  for (int n_pad = 16; n_pad <= kMaxRouted; n_pad += 16) {
+    for (int R = 8; R <= kRouterBM; R += 8) {
+      const RouterStages rs = router_stages(n_pad, R);
+      CHECK(rs.stages >= 2 && rs.stages <= kRouterMaxStages, "n_pad=%d R=%d stages=%d", n_pad, R, rs.stages);
+      CHECK(rs.kps == 1 || rs.kps == 2, "n_pad=%d R=%d kps=%d", n_pad, R, rs.kps);
+      CHECK(router_smem_bytes(n_pad, rs.kps, R, rs.stages) <= kRouterSmemBudget,
+            "n_pad=%d R=%d bytes=%zu", n_pad, R, router_smem_bytes(n_pad, rs.kps, R, rs.stages));
+      const uint32_t stage = router_stage_bytes(n_pad, rs.kps, R);
+      CHECK((uint32_t)(rs.kps - 1) * router_a_bytes(R) + kRouterBM * 128u <= stage,
+            "n_pad=%d R=%d MMA A read past the stage", n_pad, R);
+      CHECK((uint32_t)rs.kps * (router_a_bytes(R) + router_b_bytes(n_pad)) <= stage,
+            "n_pad=%d R=%d blocks past the stage", n_pad, R);
+      CHECK(router_a_bytes(R) % 1024 == 0 && router_b_bytes(n_pad) % 1024 == 0 && stage % 1024 == 0,
+            "n_pad=%d R=%d 1 KB alignment of the swizzled blocks", n_pad, R);
+      uint32_t cols = 32;
+      while (cols < 2u * (uint32_t)n_pad) cols <<= 1;
+      CHECK(cols <= 512, "n_pad=%d TMEM columns %u", n_pad, cols);
+      CHECK(router_maxc(n_pad) * kRouterGroup >= n_pad, "n_pad=%d maxc=%d", n_pad, router_maxc(n_pad));
+    }
+  }
+  // combine: warps per row between 1 and one lane-wide vector batch per part
+  for (int T = 1; T <= 70000; T += (T < 4096 ? 1 : 97)) {
+    for (int nvec : {4, 8, 16, 32, 33, 64, 100, 160, 256, 512}) {
+      const int p = combine_parts(T, nvec, 148);
+      CHECK(p >= 1 && (p == 1 || p <= nvec / 32), "T=%d nvec=%d parts=%d", T, nvec, p);
+      CHECK((long)T * p < (1L << 31), "T=%d parts=%d overflows the grid", T, p);
+    }
+  }
+  // the paired GEMM's ring and control block fit the opt-in shared memory
+  CHECK(kGemmSmemBytes <= kRouterSmemBudget, "GEMM smem %zu", kGemmSmemBytes);
+  CHECK(kGemmStageBytes % 1024 == 0, "GEMM stage %u", kGemmStageBytes);
+  if (fails) std::printf("%d rule violations\n", fails);
+  else std::printf("all tiling rules hold\n");
+  return fails ? 1 : 0;
+}
