@@ -44,6 +44,22 @@ struct SmallGemmArgs {
   int* err;
 };
 
+// Schedule of the small-batch GEMM: tiles go round-robin to the CTAs, so the first
+// total % grid CTAs get one tile more.  When the shared group's tiles are heavier (K =
+// n_shared * inter against inter), they are placed on CTAs that get one tile fewer:
+// position p of the round-robin order visits tile small_tile_at(p).  The map is a
+// bijection of [0, total) and keeps each CTA's tile indices increasing (the group search
+// relies on it); it applies only when the target positions r0 .. r0 + n_sh - 1 (r0 =
+// total % grid) exist and lie in the first round.
+__host__ __device__ inline bool small_rebalance(int total, int n_sh, int grid, bool shared_heavier) {
+  const int r0 = total % grid;
+  return n_sh > 0 && shared_heavier && r0 > 0 && n_sh <= grid - r0 && r0 + n_sh <= total;
+}
+__host__ __device__ inline int small_tile_at(int pos, int total, int n_sh, int grid, bool rebalance) {
+  const int r0 = total % grid;
+  return !rebalance ? pos : pos < r0 ? n_sh + pos : pos < r0 + n_sh ? pos - r0 : pos;
+}
+
 // smem: stages x (weights 16 KB + tokens n_tok x 128 B) | epilogue buffers | barriers
 __host__ __device__ constexpr uint32_t small_stage_bytes(int n_tok) {
   return kSmallBM * 128u + (((uint32_t)n_tok * 128u + 1023u) & ~1023u);
@@ -110,18 +126,12 @@ grouped_gemm_small_kernel(const __grid_constant__ CUtensorMap tmW_s,
   pdl_wait();   // the tile tables and operands come from the previous kernels
   const int total = __ldg(&a.ts[a.G]);
 
-  // tile -> (group g, weight tile m); GemmArgs-style decode with one token tile per group
-  // Tiles go round-robin to the CTAs, so the first total % gridDim.x CTAs get one tile
-  // more.  When the shared group's tiles are heavier (K = n_shared * inter), they are
-  // placed on CTAs that get one tile fewer: position p of the round-robin order visits
-  // tile remap(p).  Each CTA's tile indices stay increasing (the group search relies on it).
+  // tile -> (group g, weight tile m); GemmArgs-style decode with one token tile per group,
+  // in the order of small_tile_at
   const int n_sh = a.has_shared ? __ldg(&a.ts[1]) : 0;
-  const int r0 = total % (int)gridDim.x;
-  // (the remap needs the positions r0 .. r0 + n_sh - 1 to exist: r0 + n_sh <= total)
-  const bool rebalance = n_sh > 0 && a.kb_shared > a.kb_routed && r0 > 0 &&
-                         n_sh <= (int)gridDim.x - r0 && r0 + n_sh <= total;
+  const bool rebalance = small_rebalance(total, n_sh, (int)gridDim.x, a.kb_shared > a.kb_routed);
   auto decode = [&](int pos, int& g, int& m, int& e, bool& sh) {
-    const int tile = !rebalance ? pos : pos < r0 ? n_sh + pos : pos < r0 + n_sh ? pos - r0 : pos;
+    const int tile = small_tile_at(pos, total, n_sh, (int)gridDim.x, rebalance);
     while (g < a.G - 1 && tile >= __ldg(&a.ts[g + 1])) ++g;
     m = tile - __ldg(&a.ts[g]);
     sh = a.has_shared && g == 0;
