@@ -67,3 +67,41 @@ def test_workload_description_names_the_layer_and_its_sizes():
     desc = bench.workload_desc(_shape("16b_prefill"), 4)
     assert desc["workload"].startswith("16b_prefill: T=16384 d=2048")
     assert desc["global_batch"] == 4 * 16384 and desc["parallelism"] == "dp4"
+
+
+def _run_bench(args, env_extra=None):
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")}
+    env.update(env_extra or {})
+    p = subprocess.run([sys.executable, os.path.join(root, "bench.py"), *args], cwd=root,
+                       env=env, capture_output=True, text=True, timeout=600)
+    lines = [l for l in p.stdout.splitlines() if l.startswith("{")]
+    return p.returncode, [json.loads(l) for l in lines], p.stderr
+
+
+def test_reference_arm_prints_one_contract_line_on_the_host():
+    # the reference arm times the fp64 oracle on the host cores: no GPU involved
+    rc, lines, err = _run_bench(["--impl", "reference", "--config", "tiny", "--steps", "2",
+                                 "--warmup", "3"])
+    assert rc == 0, err
+    assert len(lines) == 1
+    j = lines[0]
+    assert j["impl"] == "reference" and j["unit"] == "tokens/s" and j["value"] > 0
+    assert j["steps"] == 2 and j["warmup"] == 3 and j["n_gpus"] == 1
+    assert j["higher_is_better"] is True and j["config"]["workload"].startswith("tiny:")
+    assert j["cpu_baseline"]["kind"] == "oracle" and j["cpu_baseline"]["cores"] >= 1
+    assert j["cpu_baseline"]["value"] == j["value"]
+    assert j["e2e"]["h2d_bytes_per_step"] == 0 and j["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_reference_arm_other_ranks_exit_quietly():
+    # under torchrun only rank 0 runs the oracle and prints
+    rc, lines, err = _run_bench(["--impl", "reference", "--config", "tiny", "--steps", "1",
+                                 "--warmup", "3"], {"RANK": "1", "WORLD_SIZE": "2",
+                                                    "LOCAL_RANK": "1"})
+    assert rc == 0, err
+    assert lines == []
