@@ -55,6 +55,8 @@ SMALL = [
     dict(T=100, d=256, n_shared=2, n_routed=16, inter=192, top_k=4, dtype="bf16"),
     # small-batch path at its largest token count, many experts without tokens
     dict(T=128, d=384, n_shared=1, n_routed=64, inter=128, top_k=6, dtype="bf16"),
+    # one token above the small-batch limit: the paired GEMMs with the fused row copy
+    dict(T=129, d=256, n_shared=1, n_routed=16, inter=128, top_k=4, dtype="bf16"),
     # fp32 path, ragged sizes
     dict(T=300, d=64, n_shared=2, n_routed=9, inter=48, top_k=3, dtype="fp32"),
     dict(T=1, d=32, n_shared=0, n_routed=4, inter=16, top_k=4, dtype="fp32"),
@@ -252,6 +254,8 @@ E4M3_SMALL = [
     # no shared expert: separate row-copy kernel; a token count of the decode size
     dict(T=1000, d=512, n_shared=0, n_routed=16, inter=256, top_k=2),
     dict(T=100, d=384, n_shared=1, n_routed=64, inter=128, top_k=6),
+    # the limits (256 routed experts, top-16) with two router tiles per CTA
+    dict(T=20000, d=256, n_shared=1, n_routed=256, inter=64, top_k=16),
 ]
 
 
