@@ -190,9 +190,13 @@ moe_status moe_timing_end(moe_handle* handle, double* kernel_ms, int32_t* n_forw
  *
  * Inputs (DEVICE, 16-byte aligned): u [T, d] bf16; centroids [n_routed, d] bf16;
  * logit_bias [n_routed] fp32 or NULL.  Outputs (DEVICE): topk_idx [T, top_k] int32,
- * topk_w [T, top_k] fp32, expert_counts [n_routed] int32, aux_loss [1] fp32 -- the same
- * values moe_forward returns for that layer -- and, if not NULL, device_error [1] int32
- * (0, or the code a kernel recorded, e.g. a bounded wait that ran out).
+ * topk_w [T, top_k] fp32, expert_counts [n_routed] int32, aux_loss [1] fp32 and, if not
+ * NULL, device_error [1] int32 (0, or the code a kernel recorded, e.g. a bounded wait that
+ * ran out).  For T > 128 (or d % 128 != 0) these are bit for bit the values moe_forward
+ * returns for that layer (the same kernels run).  For decode-sized batches (T <= 128,
+ * d % 128 == 0) moe_forward routes with a SIMT kernel that sums each logit in another
+ * order: the gates then agree to within fp32 rounding and the routed sets wherever the
+ * K'-th and (K'+1)-th affinities are further apart than that rounding.
  * Limits: 1 <= T <= MOE_NOALLOC_MAX_TOKENS, 1 <= n_routed <= MOE_NOALLOC_MAX_ROUTED,
  * 1 <= top_k <= min(MOE_NOALLOC_MAX_TOP_K, n_routed), d a multiple of 64; anything
  * larger returns MOE_ERR_UNSUPPORTED before touching the GPU.

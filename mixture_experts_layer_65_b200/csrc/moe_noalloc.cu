@@ -15,9 +15,9 @@ using namespace moe;
 
 namespace {
 
-// router tiles: the tiling moe_forward uses, or tiles of 128 tokens where that would need more
+// router tiles the scratch holds (moe_forward's tiling needs at most one per SM per round of
+// 128-token tiles: 148 at T = 16384 on a B200)
 constexpr int kNoAllocTiles = 320;
-static_assert(kNoAllocTiles * kRouterBM >= MOE_NOALLOC_MAX_TOKENS, "tiles of 128 must fit");
 // byte offsets inside the scratch array
 constexpr size_t kOffRank = 0;                                                      // [T, top_k] i32
 constexpr size_t kOffHist = kOffRank + (size_t)MOE_NOALLOC_MAX_TOKENS * kMaxTopK * 4;  // [tiles, N_r] i32
@@ -84,11 +84,22 @@ bool encode_rows(CUtensorMap* m, const void* ptr, uint64_t d, uint64_t rows, uin
 template <int MAXC>
 cudaError_t launch_router(const CUtensorMap& tmU, const CUtensorMap& tmE, const RouterTcArgs& ra,
                           int grid, size_t smem, cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute((const void*)router_tc_kernel<MAXC>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
   launch_pdl(router_tc_kernel<MAXC>, dim3(grid), dim3(kRouterThreads), smem, st, tmU, tmE, ra);
   return cudaGetLastError();
+}
+
+// The router instantiations may use up to the opt-in shared-memory budget: set once per
+// device, in the one-time set-up.
+cudaError_t set_router_smem_limits() {
+  const void* k[] = {(const void*)router_tc_kernel<2>, (const void*)router_tc_kernel<4>,
+                     (const void*)router_tc_kernel<8>, (const void*)router_tc_kernel<16>,
+                     (const void*)router_tc_kernel<32>};
+  for (const void* f : k) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRouterSmemBudget);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace
@@ -125,9 +136,11 @@ extern "C" moe_status moe_route_noalloc(const void* u, const void* centroids, co
       S.status = cudaDeviceGetAttribute(&S.n_sms, cudaDevAttrMultiProcessorCount, dev);
     if (S.status == cudaSuccess)
       S.status = cudaGetSymbolAddress(reinterpret_cast<void**>(&S.scratch), g_noalloc_scratch);
+    if (S.status == cudaSuccess && S.sm_major == 10 && S.sm_minor == 0)
+      S.status = set_router_smem_limits();
   });
   if (S.status != cudaSuccess || !S.scratch)
-    return nfail(MOE_ERR_CUDA, "moe_route_noalloc: cudaGetSymbolAddress of the scratch array failed");
+    return nfail(MOE_ERR_CUDA, "moe_route_noalloc: one-time set-up (scratch address, kernel attributes) failed");
   if (S.sm_major != 10 || S.sm_minor != 0)
     return nfail(MOE_ERR_UNSUPPORTED, "moe_route_noalloc: needs an sm_100a (B200) device");
 
@@ -141,9 +154,12 @@ extern "C" moe_status moe_route_noalloc(const void* u, const void* centroids, co
     return nfail(MOE_ERR_CUDA, "moe_route_noalloc: cudaMemsetAsync on the scratch failed");
 
   const int n_pad = (n_routed + 15) / 16 * 16;
-  int rows = router_tile_rows(T, S.n_sms);
-  if ((T + rows - 1) / rows > kNoAllocTiles) rows = kRouterBM;
+  // moe_forward's tiling: one tile of <= 128 tokens per SM and round, so the tile count is at
+  // most max(SMs, T / 128 + SMs), far below the scratch's capacity on a 148-SM part
+  const int rows = router_tile_rows(T, S.n_sms);
   const int n_tiles = (T + rows - 1) / rows;
+  if (n_tiles > kNoAllocTiles)
+    return nfail(MOE_ERR_UNSUPPORTED, "moe_route_noalloc: more router tiles than the scratch holds");
   CUtensorMap tmU, tmE;
   if (!encode_rows(&tmU, u, d, T, (uint32_t)rows) || !encode_rows(&tmE, centroids, d, n_routed, n_pad))
     return nfail(MOE_ERR_CUDA, "moe_route_noalloc: cuTensorMapEncodeTiled failed");

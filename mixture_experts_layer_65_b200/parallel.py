@@ -39,11 +39,17 @@ def all_reduce_balance_stats(counts: torch.Tensor, psum: torch.Tensor, n_tokens:
 
 
 def global_balance_loss(layer, out, psum_buf: torch.Tensor, counts_buf: torch.Tensor,
-                        aux_buf: torch.Tensor, group=None, n_global: int | None = None) -> torch.Tensor:
+                        aux_buf: torch.Tensor, group=None, n_global: int | None = None,
+                        loss_fn=None) -> torch.Tensor:
     """After `layer.forward(u, out)`: the balance loss of the global batch into `aux_buf`
-    (`n_global`: the global token count, if known -- see global_token_count)."""
-    from .layer import balance_loss
+    (`n_global`: the global token count, if known -- see global_token_count).
+
+    `loss_fn(counts, psum, n_tokens, alpha1, out)` computes the loss from the all-reduced
+    statistics; the default is the library's kernel (`layer.balance_loss`).  `layer` needs
+    `expert_psum(buf)`, `T` and `alpha1`; `out` needs `expert_counts`."""
+    if loss_fn is None:
+        from .layer import balance_loss as loss_fn
     layer.expert_psum(psum_buf)
     counts_buf.copy_(out.expert_counts)
     n_global = all_reduce_balance_stats(counts_buf, psum_buf, layer.T, group, n_global)
-    return balance_loss(counts_buf, psum_buf, n_global, layer.alpha1, aux_buf)
+    return loss_fn(counts_buf, psum_buf, n_global, layer.alpha1, aux_buf)

@@ -1,12 +1,16 @@
 """Host-side arithmetic of the benchmark (CPU only): the per-kernel algorithmic work that
 the roofline fractions divide by, pinned to figures computed independently from the layer
 shapes, and the source digest that decides whether the committed ncu traffic still applies."""
+import os
 import types
 
 import pytest
 
 import bench
 from mixture_experts_layer_65_b200 import workloads as W
+
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def _gb(x):
@@ -100,8 +104,65 @@ def test_reference_arm_prints_one_contract_line_on_the_host():
 
 def test_reference_arm_other_ranks_exit_quietly():
     # under torchrun only rank 0 runs the oracle and prints
-    rc, lines, err = _run_bench(["--impl", "reference", "--config", "tiny", "--steps", "1",
-                                 "--warmup", "3"], {"RANK": "1", "WORLD_SIZE": "2",
+    rc, lines, err = _run_bench(["--impl", "reference", "--gpus", "2", "--config", "tiny",
+                                 "--steps", "1", "--warmup", "3"], {"RANK": "1", "WORLD_SIZE": "2",
                                                     "LOCAL_RANK": "1"})
     assert rc == 0, err
     assert lines == []
+
+
+def _bench(*argv, env=None):
+    import subprocess
+    import sys
+    e = dict(os.environ)
+    e.pop("WORLD_SIZE", None)
+    e.update(env or {})
+    return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *argv], env=e,
+                          capture_output=True, text=True, timeout=240)
+
+
+def test_gpus_flag_launches_that_many_ranks():
+    """`--gpus 2` outside a launcher starts two ranks (torchrun); on CPU the dry run takes
+    the balance-loss exchange through gloo and rank 0 prints one line with n_gpus 2 and the
+    global loss of both ranks' statistics."""
+    import json
+
+    import numpy as np
+
+    from mixture_experts_layer_65_b200 import workloads as W
+    p = _bench("--gpus", "2", "--dry-run", "--steps", "3", "--warmup", "3")
+    assert p.returncode == 0, p.stderr[-2000:]
+    lines = [json.loads(l) for l in p.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, p.stdout
+    line = lines[0]
+    assert line["n_gpus"] == 2 and line["dry_run"] and line["value"] is None
+    spec = W.CONFIGS["16b_prefill"]
+    T, nr, K = spec["T"], spec["n_routed"], spec["top_k"]
+    c = np.zeros(nr)
+    ps = np.zeros(nr)
+    for rank in range(2):   # the ranks' synthetic statistics, as bench.py draws them
+        rng = np.random.default_rng(rank)
+        c += rng.multinomial(T * K, np.full(nr, 1.0 / nr))
+        ps += (rng.dirichlet(np.ones(nr)) * T).astype(np.float32)
+    n = 2 * T
+    assert line["global_tokens"] == n
+    assert line["aux_loss"] == pytest.approx(spec["alpha1"] * np.sum((c / n) * (ps / n)), rel=1e-5)
+
+
+def test_gpus_flag_must_match_the_launcher():
+    p = _bench("--gpus", "1", "--dry-run", env={"WORLD_SIZE": "2"})
+    assert p.returncode == 2
+    assert "must agree" in p.stderr
+
+
+def test_peak_regime_follows_the_sampled_clock():
+    """Tensor-bound kernels are held against the burst peak unless the run was power-capped
+    (sw_power_cap seen, median SM clock below 90% of the maximum, timed >= 0.5 s)."""
+    burst = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}
+    capped = {"sm_mhz": 1280.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    assert bench.peak_regime(burst, 0.04) == "burst"
+    assert bench.peak_regime(burst, 5.0) == "burst"
+    assert bench.peak_regime(capped, 5.0) == "sustained"
+    assert bench.peak_regime(capped, 0.04) == "burst"
+    assert bench.peak_regime(None, 5.0) == "burst"
+    assert bench.PEAK_KEY["burst"] == "bf16_tflops"

@@ -3,7 +3,11 @@
 Each rank routes its own shard of the tokens; the balance statistics are all-reduced with
 the same helper the GPU path uses (`parallel.all_reduce_balance_stats`), and the global
 loss and counts must equal those of the unsharded batch.  Uneven shards are included.
+`parallel.global_balance_loss` -- the call the benchmark makes after every forward on
+N > 1 GPUs -- is also run end to end, with the loss formula restated on the CPU in place
+of the library's kernel.
 """
+import types
 import os
 import socket
 
@@ -42,7 +46,27 @@ def _worker(rank, world, port, bounds, q):
         p2 = torch.from_numpy(r.s.sum(axis=0))
         n2 = parallel.all_reduce_balance_stats(c2, p2, hi - lo, n_global=n_once)
         assert n2 == n and torch.equal(c2, counts) and torch.equal(p2, psum)
-        q.put((rank, n, counts.numpy(), psum.numpy(), aux, r.topk_idx))
+        # the benchmark's per-step call, end to end: the layer's psum and counts buffers,
+        # the all-reduce, then the loss from the global statistics
+        layer = types.SimpleNamespace(T=hi - lo, alpha1=w.alpha1,
+                                      expert_psum=lambda buf: buf.copy_(torch.from_numpy(r.s.sum(axis=0))))
+        out = types.SimpleNamespace(expert_counts=torch.from_numpy(
+            np.bincount(r.topk_idx.reshape(-1), minlength=w.n_routed)))
+
+        def cpu_loss(c, p, n_tok, a1, o):
+            o.fill_(a1 * float(torch.sum((c / n_tok) * (p / n_tok))))
+            return o
+
+        aux_g = parallel.global_balance_loss(
+            layer, out, torch.empty(w.n_routed, dtype=torch.float64),
+            torch.empty(w.n_routed, dtype=torch.int64), torch.empty(1, dtype=torch.float64),
+            loss_fn=cpu_loss)
+        aux_g2 = parallel.global_balance_loss(
+            layer, out, torch.empty(w.n_routed, dtype=torch.float64),
+            torch.empty(w.n_routed, dtype=torch.int64), torch.empty(1, dtype=torch.float64),
+            n_global=n_once, loss_fn=cpu_loss)
+        assert float(aux_g) == float(aux_g2)
+        q.put((rank, n, counts.numpy(), psum.numpy(), aux, r.topk_idx, float(aux_g)))
     finally:
         dist.destroy_process_group()
 
@@ -57,8 +81,8 @@ def test_sharded_balance_statistics_match_the_full_batch(bounds):
         p.start()
     res = {}
     for _ in range(2):
-        rank, n, counts, psum, aux, idx = q.get(timeout=120)
-        res[rank] = (n, counts, psum, aux, idx)
+        rank, n, counts, psum, aux, idx, aux_g = q.get(timeout=120)
+        res[rank] = (n, counts, psum, aux, idx, aux_g)
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
@@ -66,10 +90,11 @@ def test_sharded_balance_statistics_match_the_full_batch(bounds):
     full = O.moe_forward(w.u, w.centroids, w.w_gate, w.w_up, w.w_down, w.n_shared, w.top_k,
                          w.alpha1, rows=[0])
     for rank in (0, 1):
-        n, counts, psum, aux, _ = res[rank]
+        n, counts, psum, aux, _, aux_g = res[rank]
         assert n == w.T
         np.testing.assert_array_equal(counts, full.counts)
         np.testing.assert_allclose(psum / n, full.P, rtol=1e-13)
         assert aux == pytest.approx(full.aux, rel=1e-12)
+        assert aux_g == pytest.approx(full.aux, rel=1e-12)
     # routing is per token: the shards' indices are the full batch's rows
     np.testing.assert_array_equal(np.concatenate([res[0][4], res[1][4]]), full.routing.topk_idx)

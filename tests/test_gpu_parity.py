@@ -286,3 +286,18 @@ def test_e4m3_gate_up_full_size_and_tolerance_study():
     # (a rounding step of up to 2^-4 of a value on both gate/up operands), measured 2.6e-2
     # on h and 5.6e-2 on the expert part at this size
     assert full <= 5e-2 and expert <= 1e-1
+
+
+# ------------------------------------------------------------------------ gate rounding
+@pytest.mark.parametrize("T", [4096, 64], ids=["tensor_core_router", "decode_simt_router"])
+@pytest.mark.parametrize("d", [256, 1280, 2048, 4096])
+def test_gate_error_within_its_derived_bound(d, T):
+    """The gates' rounding bound (tests/parity.gate_error_bound, derived from each router
+    kernel's accumulation order) against the measured error across hidden widths: every
+    gate inside its bound; the printed ratio error / bound shows how much of it is used."""
+    w = W.make_workload("16b_prefill", T=T, d=d, n_shared=0, n_routed=64, inter=64, top_k=6,
+                        alpha1=0.001)
+    g, *_ = run(w)
+    rep = P.compare(w, g)
+    print(f"gate pin d={d} T={T} path={P.router_path(w)}: max rel err {rep['gate_rel_err']:.3e}, "
+          f"max err/bound {rep['gate_err_over_bound']:.3f}")
