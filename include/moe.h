@@ -163,6 +163,36 @@ moe_status moe_balance_loss(const int32_t* counts, const float* psum, int32_t n_
                             int64_t n_tokens, float alpha1, float* aux_loss,
                             moe_stream_t stream);
 
+/* ---------------------------------------------------------------------------------
+ * Backward pass of the layer (for training).  The pages give the forward only; the
+ * gradients are those of L = sum_t dh_t . h_t + d_aux * aux for the layer above, with the
+ * top-k choice (and with it f_i = count_i / T) held fixed: the chosen gates g = s carry
+ * the gradient into the affinities and through the softmax ("Routing in a classic MoE
+ * layer", "Top-k routing, from affinities to gates"); the balance loss reaches them through
+ * P_i ("Expert-level balance loss"); shared experts pass dh to their FFN with gate 1.
+ *
+ * moe_backward_prepare: once per handle, synchronous; allocates the backward's workspace and
+ * transposed copies of the down, gate/up and centroid weights, and makes every later
+ * moe_forward on the handle also keep its logits.  bf16 layers on the paired-GEMM path only
+ * (MOE_ERR_UNSUPPORTED for fp32 layers, MOE_BF16_E4M3_GATEUP and T <= 128 with
+ * d % 128 == 0).
+ *
+ * moe_backward, on `stream`, after a moe_forward of the same handle on the same u (it reuses
+ * that forward's routing, grouped rows and expert outputs, so no other forward may run on the
+ * handle in between).  DEVICE pointers: u [T, d] bf16 and topk_idx, topk_w, expert_counts:
+ * that forward's input and outputs; dh [T, d] bf16, the incoming gradient of h; d_aux the
+ * weight of the balance loss in L.  Outputs: du [T, d] bf16; d_centroids [n_routed, d]
+ * fp32; d_bias [n_routed] fp32 (the gradient of a per-expert logit bias) or NULL; and
+ * either all or none (NULL) of the weight gradients, fp32 in the layouts of moe_cfg's
+ * weights: d_w_gate, d_w_up [n_shared + n_routed, inter, d], d_w_down [n_shared + n_routed,
+ * d, inter] (an expert without tokens gets zeros).  Rows of u, dh and du and the weight
+ * gradients 16-byte aligned.  Deterministic (fixed-order sums, no atomics). */
+moe_status moe_backward_prepare(moe_handle* handle);
+moe_status moe_backward(moe_handle* handle, const void* u, const int32_t* topk_idx,
+                        const float* topk_w, const int32_t* expert_counts, const void* dh,
+                        float d_aux, void* du, float* d_centroids, float* d_bias,
+                        float* d_w_gate, float* d_w_up, float* d_w_down, moe_stream_t stream);
+
 /* Per-kernel timing.  After moe_timing_begin(handle, n), each of the next n calls of
  * moe_forward on this handle records a CUDA event on its stream before each of its
  * kernels and after the last one (host-side event creation happens here, not in
@@ -172,6 +202,74 @@ moe_status moe_balance_loss(const int32_t* counts, const float* psum, int32_t n_
  * *n_forwards, and switches recording off. */
 moe_status moe_timing_begin(moe_handle* handle, int32_t max_forwards);
 moe_status moe_timing_end(moe_handle* handle, double* kernel_ms, int32_t* n_forwards);
+
+/* ---------------------------------------------------------------------------------
+ * Expert-parallel layer: the routed experts are split over `world` ranks (one GPU each),
+ * the tokens stay data-parallel.  Source: the deepforge.srivtx.xyz article, section "Where
+ * this sits" (experts spread over devices, whose computation the device-level balance loss
+ * keeps even); the arithmetic is the layer's above, and a token's output does not depend
+ * on the split.
+ *
+ * Rank r holds the n_shared shared experts and the routed experts [e0, e0 + n_local),
+ * n_local = n_routed / world, e0 = r * n_local.  One forward of T tokens on every rank:
+ *   1. moe_ep_dispatch(u) -> topk_idx, topk_w, expert_counts (this rank's tokens),
+ *      aux_loss (of this rank's batch), send_rows: the token row of every (token, slot),
+ *      T * top_k rows ordered by expert, tokens ascending within an expert -- i.e. the rows
+ *      for rank q are the contiguous block of q's experts.
+ *   2. caller: all-to-all the per-expert counts (n_local per rank), then the rows, so that
+ *      rank q receives from every source s the rows s routed to q's experts, in the order s
+ *      sent them: blocks (s, e) for s = 0..world-1, e = 0..n_local-1.
+ *   3. moe_ep_experts(recv_rows, recv_counts [world, n_local], n_recv) -> out_rows: each
+ *      received row through its expert's SwiGLU FFN, same row order.
+ *   4. caller: the reverse all-to-all (each rank gets back its send_rows' outputs).
+ *   5. moe_ep_combine(u, back_rows, topk_w) -> h = u + sum_shared FFN_j(u) +
+ *      sum_k g_k * back_rows[row of (t, k)].
+ * The global balance loss: all-reduce expert_counts and moe_ep_expert_psum's sums over
+ * the ranks, then moe_balance_loss with the global token count.
+ */
+typedef struct moe_ep_handle moe_ep_handle;
+
+/* cfg as for moe_create (bf16 layers only; n_routed % world == 0), except that w_gate,
+ * w_up and w_down hold [n_shared + n_local, ...] experts: the shared ones, then this rank's
+ * routed experts e0 .. e0 + n_local - 1; centroids and logit_bias cover all n_routed
+ * experts.  recv_capacity: the most rows moe_ep_experts will be given (0 = world * T *
+ * top_k: every rank's rows when all ranks route T tokens; pass the sum over the ranks of
+ * T_rank * top_k when their token counts differ).  Synchronous; *out = NULL on failure. */
+moe_status moe_ep_create(const moe_cfg* cfg, int32_t rank, int32_t world, int64_t recv_capacity,
+                         moe_ep_handle** out);
+
+/* Step 1 on `stream`.  DEVICE pointers: u [T, d] bf16 (16-byte aligned); outputs topk_idx,
+ * topk_w [T, top_k], expert_counts [n_routed] int32, aux_loss [1], send_rows [T * top_k, d]
+ * bf16 (16-byte aligned).  Row j of send_rows belongs to (token, slot) pairs in the order
+ * described above. */
+moe_status moe_ep_dispatch(moe_ep_handle* handle, const void* u, int32_t* topk_idx,
+                           float* topk_w, int32_t* expert_counts, float* aux_loss,
+                           void* send_rows, moe_stream_t stream);
+
+/* Step 3 on `stream`.  recv_rows [n_recv, d] bf16 and recv_counts [world, n_local] int32
+ * (DEVICE; sum = n_recv, which the caller also passes on the host), out_rows [n_recv, d]
+ * bf16 (DEVICE).  n_recv <= the handle's recv capacity (MOE_ERR_INVALID_ARG otherwise). */
+moe_status moe_ep_experts(moe_ep_handle* handle, const void* recv_rows,
+                          const int32_t* recv_counts, int64_t n_recv, void* out_rows,
+                          moe_stream_t stream);
+
+/* Step 5 on `stream`.  u [T, d] (the dispatch's input), back_rows [T * top_k, d] (step 4's
+ * result, in send_rows' order), topk_w [T, top_k] (the dispatch's gates), h [T, d]; all
+ * DEVICE, bf16 rows 16-byte aligned.  Uses the row order of the most recent dispatch. */
+moe_status moe_ep_combine(moe_ep_handle* handle, const void* u, const void* back_rows,
+                          const float* topk_w, void* h, moe_stream_t stream);
+
+/* Per-expert affinity sums [n_routed] (fp32, DEVICE) of the most recent dispatch. */
+moe_status moe_ep_expert_psum(moe_ep_handle* handle, float* psum, moe_stream_t stream);
+
+/* As moe_device_status, for the expert-parallel handle. */
+moe_status moe_ep_device_status(moe_ep_handle* handle, moe_stream_t stream);
+
+/* The received-row capacity fixed at create (0 for NULL). */
+int64_t moe_ep_recv_capacity(const moe_ep_handle* handle);
+
+/* Free everything the handle owns.  NULL-safe.  Synchronises the device first. */
+void moe_ep_destroy(moe_ep_handle* handle);
 
 /* ---------------------------------------------------------------------------------
  * Allocation-free router step.  (The DeepSeekMoE pages have no counterpart: this is a

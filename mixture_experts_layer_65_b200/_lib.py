@@ -52,6 +52,18 @@ _SIGS = {
     "moe_route_noalloc": (ctypes.c_int, [_P, _P, _P, ctypes.c_int32, ctypes.c_int32,
                                          ctypes.c_int32, ctypes.c_int32, ctypes.c_float,
                                          _P, _P, _P, _P, _P, _P]),
+    "moe_ep_create": (ctypes.c_int, [ctypes.POINTER(MoeCfg), ctypes.c_int32, ctypes.c_int32,
+                                     ctypes.c_int64, ctypes.POINTER(ctypes.c_void_p)]),
+    "moe_ep_dispatch": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_ep_experts": (ctypes.c_int, [_P, _P, _P, ctypes.c_int64, _P, _P]),
+    "moe_ep_combine": (ctypes.c_int, [_P, _P, _P, _P, _P, _P]),
+    "moe_ep_expert_psum": (ctypes.c_int, [_P, _P, _P]),
+    "moe_ep_device_status": (ctypes.c_int, [_P, _P]),
+    "moe_ep_recv_capacity": (ctypes.c_int64, [_P]),
+    "moe_ep_destroy": (None, [_P]),
+    "moe_backward_prepare": (ctypes.c_int, [_P]),
+    "moe_backward": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_float, _P, _P, _P, _P, _P, _P,
+                                    _P]),
     "moe_kernels_per_forward": (ctypes.c_int32, [_P]),
     "moe_device_bytes": (ctypes.c_size_t, [_P]),
     "moe_destroy": (None, [_P]),

@@ -14,7 +14,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmoe.so")
-SOURCES = [os.path.join(CSRC, "moe_api.cu"), os.path.join(CSRC, "moe_noalloc.cu")]
+SOURCES = [os.path.join(CSRC, "moe_api.cu"), os.path.join(CSRC, "moe_ep.cu"),
+           os.path.join(CSRC, "moe_noalloc.cu")]
 GENCODE = "arch=compute_100a,code=sm_100a"
 
 

@@ -25,10 +25,11 @@ struct CombineArgs {
   const T* ys;             // [>= T, d] shared-group output, or nullptr when K_s = 0
   const T* yr;             // [rows_cap, d] routed outputs (expert-contiguous rows)
   const int32_t* slot_row; // [T, top_k]
-  const float* topk_w;     // [T, top_k]
+  const float* topk_w;     // [T, top_k], or nullptr: every gate 1 (the backward's du)
   T* h;                    // [T, d]
   int T_, d, top_k;
   int parts;               // warps per token row, each a contiguous range of its vectors
+  const T* xtra;           // [>= T, d] added last, or nullptr (the backward's router term)
 };
 
 // Warps per token row: 1 for large batches; for small ones enough to give the SMs about
@@ -71,7 +72,7 @@ combine_bf16_kernel(CombineArgs<__nv_bfloat16> a) {
   __shared__ float s_w[kCombineWarps][kMaxTopK];
   if (lane < a.top_k) {
     s_row[warp][lane] = a.slot_row[(size_t)t * a.top_k + lane];
-    s_w[warp][lane] = a.topk_w[(size_t)t * a.top_k + lane];
+    s_w[warp][lane] = a.topk_w ? a.topk_w[(size_t)t * a.top_k + lane] : 1.0f;
   }
   __syncwarp();
   const uint4* yk[MAXK];
@@ -86,6 +87,7 @@ combine_bf16_kernel(CombineArgs<__nv_bfloat16> a) {
   combine_range(a.d >> 3, a.parts, gw - t * a.parts, v0, v1);
   const uint4* ur = reinterpret_cast<const uint4*>(a.u + (size_t)t * a.d);
   const uint4* sr = a.ys ? reinterpret_cast<const uint4*>(a.ys + (size_t)t * a.d) : nullptr;
+  const uint4* xr = a.xtra ? reinterpret_cast<const uint4*>(a.xtra + (size_t)t * a.d) : nullptr;
   uint4* hr = reinterpret_cast<uint4*>(a.h + (size_t)t * a.d);
   for (int v = v0 + lane; v < v1; v += 32) {
     uint4 x[MAXK];
@@ -102,6 +104,7 @@ combine_bf16_kernel(CombineArgs<__nv_bfloat16> a) {
 #pragma unroll
     for (int k = 0; k < MAXK; ++k)
       if (k < a.top_k) add8(acc, x[k], wk[k]);
+    if (xr) add8(acc, __ldg(xr + v), 1.0f);
     uint4 o;
     o.x = pack_bf16x2(acc[0], acc[1]);
     o.y = pack_bf16x2(acc[2], acc[3]);

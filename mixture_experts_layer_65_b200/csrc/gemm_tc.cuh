@@ -11,6 +11,16 @@
 //
 //   mode kGateUpSwiGLU:  Hmid[r, :] = SiLU(X W_gate^T) * (X W_up^T)      (K = d)
 //   mode kDown:          Y[r, :]    = Hmid W_down^T                        (K = I_g)
+//                        (also any plain D = A B^T with a bf16 output: the backward's
+//                        dHmid = dY W_down and dX = [da db] [W_gate; W_up] products)
+//   mode kGateUpBwd:     the gate/up products recomputed, a = X W_gate^T, b = X W_up^T, and
+//                        with the incoming dHmid the SwiGLU backward in the epilogue:
+//                        da = dHmid * b * SiLU'(a), db = dHmid * SiLU(a), stored interleaved
+//                        like the gate/up weight rows (K = d)
+//   mode kWgrad:         weight gradients dW[g] = A_g B_g^T with K = the group's (padded)
+//                        rows: A and B are transposed activations [width, rows] read at the
+//                        group's row offset; fp32 outputs, one matrix per group, gate/up rows
+//                        de-interleaved on the way out
 //
 // Design: persistent clusters of two CTAs (one per SM); each cluster computes 256 x 256
 // output tiles with the paired-SM MMA (tcgen05.mma.cta_group::2, M = 256, N = 256,
@@ -66,7 +76,7 @@ constexpr uint32_t kGemmStageBytes = kGemmKPS * (kGemmABytes + kGemmBBytes);
 constexpr uint32_t kGemmTmemCols = 512;
 constexpr size_t kGemmSmemBytes = 1024 + (size_t)kGemmStages * kGemmStageBytes + 256;
 
-enum GemmMode : int { kGateUpSwiGLU = 0, kDown = 1 };
+enum GemmMode : int { kGateUpSwiGLU = 0, kDown = 1, kGateUpBwd = 2, kWgrad = 3 };
 
 struct GemmArgs {
   const int32_t* grp_row;   // [G] first row of the group in A (and in the output)
@@ -98,6 +108,21 @@ struct GemmArgs {
   const float* sb_shared;
   const float* sb_routed;
   int64_t sb_routed_stride;
+  // kGateUpBwd: the incoming gradient of the SwiGLU activation, [rows, width] bf16 (shared
+  // group: width K_s * I; routed: I); the outputs (out_*) hold [rows, 2 * width]
+  const __nv_bfloat16* dh_shared;
+  const __nv_bfloat16* dh_routed;
+  int64_t ld_dh_shared, ld_dh_routed;
+  // kWgrad: K of a routed group = its rows rounded up to wg_bm (counts from the scan), of the
+  // shared group kb_shared; output rows_* = M, cols_* = N; fp32 outputs [M, N] per group
+  // (routed: + e * wg_stride), or with wg_split the interleaved gate/up rows of M = 2 I
+  // split into out0 (gate) and out1 (up), [I, N] each
+  const int32_t* wg_counts;
+  int wg_bm, wg_split;
+  int wg_colsplit;   // > 0: the shared group's output columns are side-by-side
+                     // [M, wg_colsplit] matrices (its K_s experts), each after the previous
+  float *wg_out0_shared, *wg_out1_shared, *wg_out0_routed, *wg_out1_routed;
+  int64_t wg_stride;
 };
 
 struct TileCoord {
@@ -114,6 +139,18 @@ __device__ __forceinline__ void gemm_decode(int tile, int& g, const GemmArgs& a,
   c.n = local - c.m * nt;
   c.e = g - a.has_shared;
   c.g = g;
+}
+
+// K-blocks of a tile: fixed per group kind, or (kWgrad, routed groups) the group's rows
+// rounded up to wg_bm, / 64 (0 for an expert without rows: the tile is written as zeros).
+template <int MODE>
+__device__ __forceinline__ int gemm_kblocks(const GemmArgs& a, const TileCoord& c) {
+  if (c.shared) return a.kb_shared;
+  if constexpr (MODE == kWgrad) {
+    const int n = __ldg(a.wg_counts + c.e);
+    return (n + a.wg_bm - 1) / a.wg_bm * (a.wg_bm / kGemmBK);
+  }
+  return a.kb_routed;
 }
 
 // F8: A and B are e4m3 (k-blocks of 128 elements = the same 128-byte rows), MMAs of kind
@@ -188,9 +225,12 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
           rows_ready = true;
         }
         const CUtensorMap* ta = c.shared ? &tmA_s : &tmA_r;
-        const int arow = __ldg(&a.grp_row[c.g]) + c.m * kPairBM + (int)rank * 128;
+        // weight gradients: rows of A are the output rows, the group's rows are K (at the
+        // group's column offset in the transposed routed activations)
+        const int kbase = (MODE == kWgrad && !c.shared) ? __ldg(&a.grp_row[c.g]) : 0;
+        const int arow = (MODE == kWgrad ? 0 : __ldg(&a.grp_row[c.g])) + c.m * kPairBM + (int)rank * 128;
         const int brow = c.n * kGemmBN + (int)rank * (kGemmBN / 2);
-        const int kbn = c.shared ? a.kb_shared : a.kb_routed;
+        const int kbn = gemm_kblocks<MODE>(a, c);
         for (int kb0 = 0; kb0 < kbn; kb0 += kGemmKPS) {
           ok = mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, a.err, kErrWaitProducer);
           if (!ok) break;
@@ -200,9 +240,10 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
           if (leader)
             mbar_arrive_expect_tx(smem_u32(&full[stage]), 2u * (uint32_t)nk * (kGemmABytes + kGemmBBytes));
           for (int j = 0; j < nk; ++j) {
-            const int kx = (kb0 + j) * (F8 ? 2 * kGemmBK : kGemmBK);   // elements
+            const int kx = kbase + (kb0 + j) * (F8 ? 2 * kGemmBK : kGemmBK);   // elements
             tma_load_2d_pair(sa + j * kGemmABytes, ta, fb, kx, arow);
-            if (c.shared) tma_load_2d_pair(sa + kGemmBOff + j * kGemmBBytes, &tmB_s, fb, kx, brow);
+            if (c.shared || MODE == kWgrad)
+              tma_load_2d_pair(sa + kGemmBOff + j * kGemmBBytes, c.shared ? &tmB_s : &tmB_r, fb, kx, brow);
             else tma_load_3d_pair(sa + kGemmBOff + j * kGemmBBytes, &tmB_r, fb, kx, brow, c.e);
           }
           if (++stage == kGemmStages) { stage = 0; phase ^= 1u; }
@@ -227,7 +268,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
       for (int tile = cid; tile < total && ok; tile += ncl, ++it) {
         TileCoord c;
         gemm_decode(tile, g, a, c);
-        const int kbn = c.shared ? a.kb_shared : a.kb_routed;
+        const int kbn = gemm_kblocks<MODE>(a, c);
         const int acc = it & 1;
         const uint32_t acc_par = (it >> 1) & 1;
         ok = mbar_wait(smem_u32(&acc_empty[acc]), acc_par ^ 1u, abort_flag, a.err, kErrWaitMma);
@@ -290,15 +331,106 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
       tc_fence_after();
       const uint32_t trow =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * kGemmBN);
-      const int64_t orow = (int64_t)__ldg(&a.grp_row[c.g]) + (int64_t)c.m * kPairBM +
-                           (int64_t)rank * 128 + rr;
+      // output row: in the group's rows of A, or (kWgrad) in the gradient matrix itself
+      const int64_t orow = (MODE == kWgrad ? 0 : (int64_t)__ldg(&a.grp_row[c.g])) +
+                           (int64_t)c.m * kPairBM + (int64_t)rank * 128 + rr;
       __nv_bfloat16* out = c.shared ? a.out_shared : a.out_routed;
       const int64_t ld = c.shared ? a.ld_shared : a.ld_routed;
       const int64_t rows = c.shared ? a.rows_shared : a.rows_routed;
       const int cols = c.shared ? a.cols_shared : a.cols_routed;
       const bool row_ok = orow < rows;
-      if (!row_ok) record_error(a.err, kErrOutRow);
-      if (MODE == kGateUpSwiGLU) {
+      // (a weight gradient's last row tile may reach past its M rows: those rows are skipped)
+      if (!row_ok && MODE != kWgrad) record_error(a.err, kErrOutRow);
+      if constexpr (MODE == kWgrad) {
+        // fp32 rows of the group's weight gradient; a group without rows gives zeros
+        const bool kzero = gemm_kblocks<MODE>(a, c) == 0;
+        const int64_t mrow = orow;
+        const bool mok = row_ok;
+        float* dst = nullptr;
+        if (mok) {
+          float* o0 = c.shared ? a.wg_out0_shared : a.wg_out0_routed + (int64_t)c.e * a.wg_stride;
+          float* o1 = c.shared ? a.wg_out1_shared : a.wg_out1_routed + (int64_t)c.e * a.wg_stride;
+          if (a.wg_split) {   // interleaved gate/up rows: blocks of 64, gate first
+            const int64_t blk = mrow >> 6;
+            dst = ((blk & 1) ? o1 : o0) + ((blk >> 1) * 64 + (mrow & 63)) * (int64_t)cols;
+          } else if (c.shared && a.wg_colsplit > 0) {
+            dst = o0 + mrow * (int64_t)a.wg_colsplit;   // column c: matrix c / colsplit
+          } else {
+            dst = o0 + mrow * (int64_t)cols;
+          }
+        }
+#pragma unroll 1
+        for (int cc = half * (kGemmBN / 2); cc < (half + 1) * (kGemmBN / 2); cc += 32) {
+          const int col = c.n * kGemmBN + cc;
+          if (col >= cols) break;
+          uint32_t v[32];
+          __syncwarp();
+          tmem_ld32(trow + static_cast<uint32_t>(cc), v);
+          tmem_ld_wait(v);
+          if (mok) {
+            // (with wg_colsplit, a 32-column chunk never straddles two matrices: the widths
+            // are multiples of 64)
+            float* dcol = (c.shared && a.wg_colsplit > 0)
+                              ? dst + (int64_t)(col / a.wg_colsplit) * rows * a.wg_colsplit + col % a.wg_colsplit
+                              : dst + col;
+            float4* d4 = reinterpret_cast<float4*>(dcol);
+#pragma unroll
+            for (int x = 0; x < 8; ++x)
+              d4[x] = kzero ? make_float4(0.f, 0.f, 0.f, 0.f)
+                            : make_float4(__uint_as_float(v[4 * x]), __uint_as_float(v[4 * x + 1]),
+                                          __uint_as_float(v[4 * x + 2]), __uint_as_float(v[4 * x + 3]));
+          }
+        }
+      } else if constexpr (MODE == kGateUpBwd) {
+        // SwiGLU backward on 16 outputs at a time: with a = gate, b = up, s = sigmoid(a),
+        // SiLU(a) = a s and SiLU'(a) = s (1 + a (1 - s)); the incoming dHmid of the same
+        // outputs is read from global memory; da and db go to the interleaved columns of the
+        // accumulator they came from (64 gate columns, then the 64 matching up columns)
+        const int hb = half;
+        const int col0 = c.n * (kGemmBN / 2) + hb * 64;   // activation column
+        const __nv_bfloat16* dhp = (c.shared ? a.dh_shared : a.dh_routed) +
+                                   orow * (c.shared ? a.ld_dh_shared : a.ld_dh_routed) + col0;
+        const int64_t ocol = (int64_t)c.n * kGemmBN + hb * 128;   // interleaved output column
+#pragma unroll 1
+        for (int j = 0; j < 64 && col0 < cols; j += 16) {
+          uint32_t gv[16], uv[16];
+          __syncwarp();
+          tmem_ld16(trow + static_cast<uint32_t>(hb * 128 + j), gv);
+          tmem_ld16(trow + static_cast<uint32_t>(hb * 128 + 64 + j), uv);
+          tmem_ld_wait16(gv);
+          tmem_ld_wait16(uv);
+          uint4 dv[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
+          if (row_ok) {
+            dv[0] = *reinterpret_cast<const uint4*>(dhp + j);
+            dv[1] = *reinterpret_cast<const uint4*>(dhp + j + 8);
+          }
+          float dh[16];
+          bf16x8_to_f32(dv[0], *reinterpret_cast<float(*)[8]>(&dh[0]));
+          bf16x8_to_f32(dv[1], *reinterpret_cast<float(*)[8]>(&dh[8]));
+          uint32_t pa[8], pb[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            float da2[2], db2[2];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+              const float av = __uint_as_float(gv[2 * i + k]);
+              const float bv = __uint_as_float(uv[2 * i + k]);
+              const float sg = __fdividef(1.0f, 1.0f + __expf(fminf(-av, 80.0f)));
+              da2[k] = dh[2 * i + k] * bv * (sg * (1.0f + av * (1.0f - sg)));
+              db2[k] = dh[2 * i + k] * (av * sg);
+            }
+            pa[i] = pack_bf16x2(da2[0], da2[1]);
+            pb[i] = pack_bf16x2(db2[0], db2[1]);
+          }
+          if (row_ok) {
+            __nv_bfloat16* orow_p = out + orow * ld + ocol + j;
+            reinterpret_cast<uint4*>(orow_p)[0] = make_uint4(pa[0], pa[1], pa[2], pa[3]);
+            reinterpret_cast<uint4*>(orow_p)[1] = make_uint4(pa[4], pa[5], pa[6], pa[7]);
+            reinterpret_cast<uint4*>(orow_p + 64)[0] = make_uint4(pb[0], pb[1], pb[2], pb[3]);
+            reinterpret_cast<uint4*>(orow_p + 64)[1] = make_uint4(pb[4], pb[5], pb[6], pb[7]);
+          }
+        }
+      } else if (MODE == kGateUpSwiGLU) {
         float sa = 1.f;                 // e4m3: the A row's scale, and the B rows' scales
         const float* sbv = nullptr;
         if (F8) {

@@ -4,22 +4,22 @@
 // Launch sequence of moe_forward (one stream, no host synchronisation, every launch with
 // programmatic dependent launch):
 //   1. router      logits -> softmax -> top-k, gates, per-tile histograms / ranks / sums
-//                  (tensor-core kernel; a SIMT kernel for decode-sized batches and fp32)
-//   2. scan        per-expert counts, padded offsets, tile tables, balance loss
+//                  (tensor-core kernel; a SIMT kernel for decode-sized batches and fp32);
+//                  its last CTA then runs the scan: per-expert counts, padded offsets,
+//                  tile tables, balance loss
 //   3. quantise    (e4m3 gate/up layers only) e4m3 token rows + per-row scales
 //   4. permute     token rows -> expert-contiguous rows (top_k copies per token); on bf16
 //                  layers with shared experts this copy runs inside step 5 instead
 //   5. gate/up     grouped GEMM + SwiGLU (shared group reads the token rows directly)
 //   6. down        grouped GEMM
 //   7. combine     h = u + shared + sum_k g_k * routed_k (fp32, fixed order)
-#include <cstdarg>
-#include <cstdio>
 #include <cstring>
 #include <string>
-#include <type_traits>
 #include <vector>
 
 #include "moe.h"
+#include "api_common.cuh"
+#include "backward.cuh"
 #include "combine.cuh"
 #include "gemm_simt.cuh"
 #include "gemm_small.cuh"
@@ -33,98 +33,6 @@ using namespace moe;
 namespace {
 
 thread_local std::string g_last_error;
-
-moe_status fail(moe_status st, const char* fmt, ...) {
-  char buf[512];
-  va_list ap;
-  va_start(ap, fmt);
-  vsnprintf(buf, sizeof(buf), fmt, ap);
-  va_end(ap);
-  g_last_error = buf;
-  return st;
-}
-
-#define MOE_CUDA(expr)                                                                     \
-  do {                                                                                     \
-    cudaError_t e_ = (expr);                                                               \
-    if (e_ != cudaSuccess)                                                                 \
-      return fail(MOE_ERR_CUDA, "%s: %s (%s:%d)", #expr, cudaGetErrorString(e_), __FILE__, \
-                  __LINE__);                                                               \
-  } while (0)
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn get_encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
-}
-
-// bf16 row-major [outer, inner] matrix, box = box_outer rows x 64 columns, 128 B swizzle.
-bool encode_2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer,
-               uint32_t box_outer) {
-  EncodeTiledFn fn = get_encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {inner * 2};
-  cuuint32_t box[2] = {64, box_outer};
-  cuuint32_t es[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
-            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// bf16 [depth, outer, inner], box = box_outer rows x 64 columns of one matrix.
-bool encode_3d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t depth,
-               uint32_t box_outer) {
-  EncodeTiledFn fn = get_encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[3] = {inner, outer, depth};
-  cuuint64_t strides[2] = {inner * 2, inner * outer * 2};
-  cuuint32_t box[3] = {64, box_outer, 1};
-  cuuint32_t es[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
-            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// e4m3 bytes: row-major [outer, inner] matrix, box = box_outer rows x 128 columns (128 B).
-bool encode_2d_e4m3(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer,
-                    uint32_t box_outer) {
-  EncodeTiledFn fn = get_encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {inner};
-  cuuint32_t box[2] = {128, box_outer};
-  cuuint32_t es[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// e4m3 bytes [depth, outer, inner], box = box_outer rows x 128 columns of one matrix.
-bool encode_3d_e4m3(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer,
-                    uint64_t depth, uint32_t box_outer) {
-  EncodeTiledFn fn = get_encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[3] = {inner, outer, depth};
-  cuuint64_t strides[2] = {inner, inner * outer};
-  cuuint32_t box[3] = {128, box_outer, 1};
-  cuuint32_t es[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 // Quantise `rows` bf16 rows of `cols` values to e4m3 with per-row scales, on `st`.
 cudaError_t launch_quant(const void* src, int64_t rows, int cols, void* dst, float* scale,
@@ -164,30 +72,6 @@ __global__ void balance_loss_kernel(const int32_t* counts, const float* psum, in
 }
 
 constexpr int kKernelsPerForward = 6;
-
-// Call f(std::integral_constant<int, MAXC>{}) for the router's columns per thread bound.
-template <class F>
-auto with_maxc(int maxc, F&& f) {
-  switch (maxc) {
-    case 2: return f(std::integral_constant<int, 2>{});
-    case 4: return f(std::integral_constant<int, 4>{});
-    case 8: return f(std::integral_constant<int, 8>{});
-    case 16: return f(std::integral_constant<int, 16>{});
-    default: return f(std::integral_constant<int, 32>{});
-  }
-}
-
-// Call f(std::integral_constant<int, MAXK>{}) for the combine's bound on top_k.
-template <class F>
-auto with_maxk(int maxk, F&& f) {
-  switch (maxk) {
-    case 4: return f(std::integral_constant<int, 4>{});
-    case 6: return f(std::integral_constant<int, 6>{});
-    case 8: return f(std::integral_constant<int, 8>{});
-    case 12: return f(std::integral_constant<int, 12>{});
-    default: return f(std::integral_constant<int, 16>{});
-  }
-}
 
 }  // namespace
 
@@ -232,6 +116,7 @@ struct moe_handle {
   void *xp = nullptr, *hs = nullptr, *hr = nullptr, *ys = nullptr, *yr = nullptr;
   int* err = nullptr;
   int* copy_done = nullptr;   // counter of the fused permute (paired bf16 path with a shared group)
+  int* done_ctas = nullptr;   // router CTAs finished (the last one runs the scan, resets it)
   // e4m3 gate/up: quantised weights (interleaved rows), per-row scales, quantised tokens
   void *w8_gu_s = nullptr, *w8_gu_r = nullptr, *u8 = nullptr;
   float *sw_s = nullptr, *sw_r = nullptr, *su = nullptr, *su_p = nullptr;
@@ -256,6 +141,28 @@ struct moe_handle {
   PipeSlot pslot[2];
   int64_t p_calls = 0;
   bool p_ready = false;
+  // backward (moe_backward_prepare): the forward's logits, transposed weight copies and the
+  // backward's workspace
+  bool bwd = false;
+  bool bwd_forward = false;                // a forward ran since moe_backward_prepare
+  int kpad = 0;                            // n_pad rounded up to 64: K of the e-product GEMM
+  float* logits = nullptr;                 // [T, n_routed]
+  int32_t* ts3 = nullptr;                  // [G + 1] dHmid GEMM tiles (N = I at 256 per tile)
+  void *w_dT_s = nullptr, *w_dT_r = nullptr;     // [Is, d], [n_routed, I, d]
+  void *w_guT_s = nullptr, *w_guT_r = nullptr;   // [d, 2 Is], [n_routed, d, 2 I] (interleaved K)
+  void* e_T = nullptr;                            // [d, kpad] centroids transposed (zero-padded)
+  void *dyr = nullptr, *dhr = nullptr, *dhs = nullptr, *dabr = nullptr, *dabs = nullptr;
+  void *dxr = nullptr, *dxs = nullptr, *dur = nullptr, *dlb = nullptr;
+  float *dg = nullptr, *dl = nullptr, *cen_part = nullptr;
+  int32_t *r_grp = nullptr, *r_ts = nullptr;      // one-group tables of the e-product GEMM
+  // weight gradients: transposed activations [width, rows] (padding rows zero) and the
+  // (static) tile tables of the dW_gate/up and dW_down GEMMs
+  void *xpT = nullptr, *dyrT = nullptr, *hrT = nullptr, *dabrT = nullptr;
+  void *uT = nullptr, *dhT = nullptr, *hsT = nullptr, *dabsT = nullptr;
+  int32_t *wts1 = nullptr, *wts2 = nullptr;
+  CUtensorMap tmXpT, tmDyrT, tmHrT, tmDabrT, tmUT, tmDhT, tmHsT, tmDabsT;
+  int cen_chunks = 0;
+  CUtensorMap tmDyr, tmWdTs, tmWdTr, tmDabs, tmDabr, tmWguTs, tmWguTr, tmDlb, tmEt;
   // per-kernel timing (moe_timing_begin / moe_timing_end)
   std::vector<cudaEvent_t> events;   // kKernelsPerForward + 1 per recorded call
   int timing_cap = 0, timing_used = 0;
@@ -279,12 +186,6 @@ moe_status dalloc(moe_handle* H, void** p, size_t bytes) {
   return MOE_OK;
 }
 
-#define MOE_TRY(expr)              \
-  do {                             \
-    moe_status s_ = (expr);        \
-    if (s_ != MOE_OK) return s_;   \
-  } while (0)
-
 void free_handle(moe_handle* H) {
   if (!H) return;
   for (cudaEvent_t e : H->events) cudaEventDestroy(e);
@@ -297,8 +198,6 @@ void free_handle(moe_handle* H) {
   for (void* p : H->allocs) cudaFree(p);
   delete H;
 }
-
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 moe_status validate(const moe_cfg* c) {
   if (!c) return fail(MOE_ERR_INVALID_ARG, "cfg is NULL");
@@ -342,7 +241,9 @@ int32_t moe_abi_version(void) { return MOE_ABI_VERSION; }
 const char* moe_last_error(void) { return g_last_error.c_str(); }
 
 int32_t moe_kernels_per_forward(const moe_handle* handle) {
-  return handle ? kKernelsPerForward - (handle->fuse_permute ? 1 : 0) + (handle->e4m3 ? 1 : 0) : 0;
+  // six timing slots; the scan has none of its own (router's last CTA), the permute none
+  // when the gate/up GEMM copies the rows, and e4m3 layers add the token quantisation
+  return handle ? kKernelsPerForward - 1 - (handle->fuse_permute ? 1 : 0) + (handle->e4m3 ? 1 : 0) : 0;
 }
 
 size_t moe_device_bytes(const moe_handle* handle) { return handle ? handle->bytes : 0; }
@@ -466,6 +367,8 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
   MOE_CUDA(cudaMemsetAsync(H->err, 0, 256, st));
   MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->copy_done), 256));
   MOE_CUDA(cudaMemsetAsync(H->copy_done, 0, 256, st));
+  MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->done_ctas), 256));
+  MOE_CUDA(cudaMemsetAsync(H->done_ctas, 0, 256, st));
   const size_t rc = (size_t)H->rows_cap, tp = (size_t)H->T_pad;
   MOE_TRY(dalloc(H, &H->xp, rc * d * (H->e4m3 ? 1 : es)));   // e4m3 rows on that path
   if (H->e4m3) {
@@ -623,7 +526,15 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
   const moe_cfg& c = H->cfg;
   const int T = c.T, d = c.d, K = c.top_k, nr = c.n_routed;
 
-  RouterOut ro{topk_idx, topk_w, H->topk_rank, H->tile_hist, H->tile_psum, H->err};
+  const int bn1 = H->small ? 64 : (H->bf16 ? kGemmBN / 2 : kSimtBN);
+  const int bn2 = H->small ? kSmallBM : (H->bf16 ? kGemmBN : kSimtBN);
+  ScanArgs sa{H->tile_hist, H->tile_psum, H->n_tiles, nr, T, H->has_shared, H->inter_shared,
+              c.inter, d, H->bm, H->tile_rows, bn1, bn2, c.alpha1, expert_counts, aux_loss,
+              H->psum_total,
+              H->tile_base, H->grp_row, H->ts1, H->ts2,
+              H->fuse_permute ? H->copy_done : nullptr, H->done_ctas, H->bwd ? H->ts3 : nullptr};
+  RouterOut ro{topk_idx, topk_w, H->topk_rank, H->tile_hist, H->tile_psum, H->err, sa,
+               H->bwd ? H->logits : nullptr};
   CUtensorMap tmU, tmUr;
   tick(H, stream, 0);
   if (H->small) {
@@ -655,16 +566,7 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
   }
   MOE_CUDA(cudaGetLastError());
 
-  const int bn1 = H->small ? 64 : (H->bf16 ? kGemmBN / 2 : kSimtBN);
-  const int bn2 = H->small ? kSmallBM : (H->bf16 ? kGemmBN : kSimtBN);
-  ScanArgs sa{H->tile_hist, H->tile_psum, H->n_tiles, nr, T, H->has_shared, H->inter_shared,
-              c.inter, d, H->bm, H->tile_rows, bn1, bn2, c.alpha1, expert_counts, aux_loss,
-              H->psum_total,
-              H->tile_base, H->grp_row, H->ts1, H->ts2,
-              H->fuse_permute ? H->copy_done : nullptr};
-  tick(H, stream, 1);
-  launch_pdl(scan_kernel, dim3(1), dim3(kScanThreads), 0, stream, sa);
-  MOE_CUDA(cudaGetLastError());
+  tick(H, stream, 1);   // (the scan runs in the router's last CTA: an empty slot)
 
   PermuteArgs pa{static_cast<const uint8_t*>(u), topk_idx, H->topk_rank, H->tile_base, H->slot_row,
                  static_cast<uint8_t*>(H->xp), T, K, nr, (int)H->rows_cap, H->router_rows,
@@ -816,6 +718,311 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
     tick(H, stream, kKernelsPerForward);
     ++H->timing_used;
   }
+  if (H->bwd) H->bwd_forward = true;
+  return MOE_OK;
+}
+
+
+moe_status moe_backward_prepare(moe_handle* H) {
+  if (!H) return fail(MOE_ERR_INVALID_ARG, "handle is NULL");
+  if (H->bwd) return MOE_OK;
+  if (!H->bf16 || H->e4m3 || H->small)
+    return fail(MOE_ERR_UNSUPPORTED, "the backward runs bf16 layers on the paired-GEMM path "
+                                     "(not fp32, not e4m3 gate/up, not T <= 128 decode-sized)");
+  int dev = -1;
+  MOE_CUDA(cudaGetDevice(&dev));
+  if (dev != H->device)
+    return fail(MOE_ERR_INVALID_ARG, "current device %d is not the handle's device %d", dev, H->device);
+  const moe_cfg& c = H->cfg;
+  const size_t d = c.d, I = c.inter, Is = H->inter_shared, nr = c.n_routed, T = c.T, K = c.top_k;
+  const size_t rc = (size_t)H->rows_cap, tp = (size_t)H->T_pad, np = (size_t)H->n_pad, es = 2;
+  const bool ks = H->has_shared;
+  cudaStream_t st;
+  MOE_CUDA(cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking));
+  struct StreamGuard {
+    cudaStream_t s;
+    ~StreamGuard() { cudaStreamDestroy(s); }
+  } guard{st};
+  H->kpad = (H->n_pad + 63) / 64 * 64;
+  const size_t kp = (size_t)H->kpad;
+  MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->logits), T * nr * 4));
+  MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->ts3), (size_t)(H->G + 1) * 4));
+  MOE_CUDA(cudaMemsetAsync(H->ts3, 0, (size_t)(H->G + 1) * 4, st));   // no tiles before a forward
+  // transposed weights: down [d, I] -> [I, d]; interleaved gate/up [2I, d] -> [d, 2I]
+  MOE_TRY(dalloc(H, &H->w_dT_r, nr * I * d * es));
+  MOE_TRY(dalloc(H, &H->w_guT_r, nr * 2 * I * d * es));
+  MOE_TRY(dalloc(H, &H->e_T, d * kp * es));
+  void* e_pad = nullptr;   // the centroids with zero rows up to kpad, transposed below
+  MOE_TRY(dalloc(H, &e_pad, kp * d * es));
+  MOE_CUDA(cudaMemsetAsync(e_pad, 0, kp * d * es, st));
+  MOE_CUDA(cudaMemcpyAsync(e_pad, H->centroids, np * d * es, cudaMemcpyDeviceToDevice, st));
+  auto tr = [&](const void* src, void* dst, size_t R, size_t C, size_t batch) {
+    transpose_bf16_kernel<<<dim3((unsigned)((C + kTrTile - 1) / kTrTile), (unsigned)((R + kTrTile - 1) / kTrTile),
+                              (unsigned)batch), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(src),
+                                                              static_cast<__nv_bfloat16*>(dst), (int)R, (int)C);
+    return cudaGetLastError();
+  };
+  MOE_CUDA(tr(H->w_d_r, H->w_dT_r, d, I, nr));
+  MOE_CUDA(tr(H->w_gu_r, H->w_guT_r, 2 * I, d, nr));
+  MOE_CUDA(tr(e_pad, H->e_T, kp, d, 1));
+  if (ks) {
+    MOE_TRY(dalloc(H, &H->w_dT_s, Is * d * es));
+    MOE_TRY(dalloc(H, &H->w_guT_s, 2 * Is * d * es));
+    MOE_CUDA(tr(H->w_d_s, H->w_dT_s, d, Is, 1));
+    MOE_CUDA(tr(H->w_gu_s, H->w_guT_s, 2 * Is, d, 1));
+    MOE_TRY(dalloc(H, &H->dhs, tp * Is * es));
+    MOE_TRY(dalloc(H, &H->dabs, tp * 2 * Is * es));
+    MOE_TRY(dalloc(H, &H->dxs, tp * d * es));
+  }
+  MOE_TRY(dalloc(H, &H->dyr, rc * d * es));
+  MOE_TRY(dalloc(H, &H->dhr, rc * I * es));
+  MOE_TRY(dalloc(H, &H->dabr, rc * 2 * I * es));
+  MOE_TRY(dalloc(H, &H->dxr, rc * d * es));
+  MOE_TRY(dalloc(H, &H->dur, tp * d * es));
+  MOE_TRY(dalloc(H, &H->dlb, tp * kp * es));
+  MOE_CUDA(cudaMemsetAsync(H->dlb, 0, tp * kp * es, st));   // rows past T, columns past n_pad: 0
+  MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->dg), T * K * 4));
+  MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->dl), T * np * 4));
+  H->cen_chunks = (int)((T + kCenChunk - 1) / kCenChunk);
+  MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->cen_part), (size_t)H->cen_chunks * nr * (d + 1) * 4));
+  MOE_TRY(dalloc(H, &H->xpT, d * rc * es));
+  MOE_TRY(dalloc(H, &H->dyrT, d * rc * es));
+  MOE_TRY(dalloc(H, &H->hrT, I * rc * es));
+  MOE_TRY(dalloc(H, &H->dabrT, 2 * I * rc * es));
+  if (ks) {
+    MOE_TRY(dalloc(H, &H->uT, d * tp * es));
+    MOE_TRY(dalloc(H, &H->dhT, d * tp * es));
+    MOE_TRY(dalloc(H, &H->hsT, Is * tp * es));
+    MOE_TRY(dalloc(H, &H->dabsT, 2 * Is * tp * es));
+  }
+  {
+    // static tile tables: group g of dW_gate/up has (2 I_g / 256) x (d / 256) tiles, of
+    // dW_down (d / 256) x ceil(I_g / 256), I_g = K_s I for the shared group
+    std::vector<int32_t> w1(H->G + 1, 0), w2(H->G + 1, 0);
+    for (int g = 0; g < H->G; ++g) {
+      const size_t Ig = (H->has_shared && g == 0) ? Is : I;
+      w1[g + 1] = w1[g] + (int)((2 * Ig + kPairBM - 1) / kPairBM) * (int)((d + kGemmBN - 1) / kGemmBN);
+      w2[g + 1] = w2[g] + (int)((d + kPairBM - 1) / kPairBM) * (int)((Ig + kGemmBN - 1) / kGemmBN);
+    }
+    MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->wts1), (size_t)(H->G + 1) * 4));
+    MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->wts2), (size_t)(H->G + 1) * 4));
+    MOE_CUDA(cudaMemcpyAsync(H->wts1, w1.data(), w1.size() * 4, cudaMemcpyHostToDevice, st));
+    MOE_CUDA(cudaMemcpyAsync(H->wts2, w2.data(), w2.size() * 4, cudaMemcpyHostToDevice, st));
+    MOE_CUDA(cudaStreamSynchronize(st));   // the host tables above go out of scope
+  }
+  MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->r_grp), 4));
+  MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->r_ts), 8));
+  const int32_t grp0 = 0;
+  const int32_t rts[2] = {0, (int)(tp / kPairBM) * (int)((d + kGemmBN - 1) / kGemmBN)};
+  MOE_CUDA(cudaMemcpyAsync(H->r_grp, &grp0, 4, cudaMemcpyHostToDevice, st));
+  MOE_CUDA(cudaMemcpyAsync(H->r_ts, rts, 8, cudaMemcpyHostToDevice, st));
+  MOE_CUDA(cudaStreamSynchronize(st));
+  bool ok = encode_2d(&H->tmDyr, H->dyr, d, rc, 128) &&
+            encode_3d(&H->tmWdTr, H->w_dT_r, d, I, nr, kGemmBN / 2) &&
+            encode_2d(&H->tmDabr, H->dabr, 2 * I, rc, 128) &&
+            encode_3d(&H->tmWguTr, H->w_guT_r, 2 * I, d, nr, kGemmBN / 2) &&
+            encode_2d(&H->tmDlb, H->dlb, kp, tp, 128) && encode_2d(&H->tmEt, H->e_T, kp, d, kGemmBN / 2);
+  if (ks)
+    ok = ok && encode_2d(&H->tmWdTs, H->w_dT_s, d, Is, kGemmBN / 2) &&
+         encode_2d(&H->tmDabs, H->dabs, 2 * Is, tp, 128) &&
+         encode_2d(&H->tmWguTs, H->w_guT_s, 2 * Is, d, kGemmBN / 2);
+  else {
+    H->tmWdTs = H->tmWdTr;
+    H->tmDabs = H->tmDabr;
+    H->tmWguTs = H->tmWguTr;
+  }
+  ok = ok && encode_2d(&H->tmXpT, H->xpT, rc, d, 128) && encode_2d(&H->tmDyrT, H->dyrT, rc, d, 128) &&
+       encode_2d(&H->tmHrT, H->hrT, rc, I, 128) && encode_2d(&H->tmDabrT, H->dabrT, rc, 2 * I, 128);
+  if (ks)
+    ok = ok && encode_2d(&H->tmUT, H->uT, tp, d, 128) && encode_2d(&H->tmDhT, H->dhT, tp, d, 128) &&
+         encode_2d(&H->tmHsT, H->hsT, tp, Is, 128) && encode_2d(&H->tmDabsT, H->dabsT, tp, 2 * Is, 128);
+  else {
+    H->tmUT = H->tmXpT;
+    H->tmDhT = H->tmDyrT;
+    H->tmHsT = H->tmHrT;
+    H->tmDabsT = H->tmDabrT;
+  }
+  if (!ok) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for a backward operand");
+  MOE_CUDA(cudaFuncSetAttribute((const void*)grouped_gemm_tc_kernel<kWgrad>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmemBytes));
+  MOE_CUDA(cudaFuncSetAttribute((const void*)grouped_gemm_tc_kernel<kGateUpBwd>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmemBytes));
+  H->bwd = true;
+  H->bwd_forward = false;
+  return MOE_OK;
+}
+
+moe_status moe_backward(moe_handle* H, const void* u, const int32_t* topk_idx, const float* topk_w,
+                        const int32_t* expert_counts, const void* dh, float d_aux, void* du,
+                        float* d_centroids, float* d_bias, float* d_w_gate, float* d_w_up,
+                        float* d_w_down, moe_stream_t stream_) {
+  if (!H) return fail(MOE_ERR_INVALID_ARG, "handle is NULL");
+  if (!H->bwd || !H->bwd_forward)
+    return fail(MOE_ERR_INVALID_ARG, "call moe_backward_prepare and then moe_forward first");
+  if (!u || !topk_idx || !topk_w || !expert_counts || !dh || !du || !d_centroids)
+    return fail(MOE_ERR_INVALID_ARG, "an input/output pointer is NULL");
+  if (!aligned16(u) || !aligned16(dh) || !aligned16(du))
+    return fail(MOE_ERR_INVALID_ARG, "u, dh and du must be 16-byte aligned");
+  const bool wgrad = d_w_gate || d_w_up || d_w_down;
+  if (wgrad && !(d_w_gate && d_w_up && d_w_down))
+    return fail(MOE_ERR_INVALID_ARG, "d_w_gate, d_w_up and d_w_down are all given or all NULL");
+  if (wgrad && (!aligned16(d_w_gate) || !aligned16(d_w_up) || !aligned16(d_w_down)))
+    return fail(MOE_ERR_INVALID_ARG, "the weight gradients must be 16-byte aligned");
+  int dev = -1;
+  MOE_CUDA(cudaGetDevice(&dev));
+  if (dev != H->device)
+    return fail(MOE_ERR_INVALID_ARG, "current device %d is not the handle's device %d", dev, H->device);
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const moe_cfg& c = H->cfg;
+  const int T = c.T, d = c.d, K = c.top_k, nr = c.n_routed, I = c.inter, Is = H->inter_shared;
+  // 1. dY rows of the routed experts (g dh) and the gates' gradients (dh . Y)
+  BwdRowsArgs ba{static_cast<const __nv_bfloat16*>(dh), topk_w, H->slot_row,
+                 static_cast<const __nv_bfloat16*>(H->yr), static_cast<__nv_bfloat16*>(H->dyr), H->dg,
+                 T, d, K, H->rows_cap, H->err};
+  launch_pdl(bwd_rows_kernel, dim3((T + kBwdWarps - 1) / kBwdWarps), dim3(kBwdWarps * 32), 0, stream, ba);
+  MOE_CUDA(cudaGetLastError());
+  CUtensorMap tmDh, tmU;
+  if (!encode_2d(&tmDh, dh, d, T, 128) || !encode_2d(&tmU, u, d, T, 128))
+    return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for u or dh");
+  // 2. dHmid = dY W_down (shared group: dY = dh)
+  GemmArgs g{};
+  g.grp_row = H->grp_row; g.ts = H->ts3; g.G = H->G; g.has_shared = H->has_shared;
+  g.kb_shared = d / kGemmBK; g.kb_routed = d / kGemmBK;
+  g.nt_shared = (Is + kGemmBN - 1) / kGemmBN; g.nt_routed = (I + kGemmBN - 1) / kGemmBN;
+  g.out_shared = static_cast<__nv_bfloat16*>(H->dhs); g.ld_shared = Is; g.rows_shared = H->T_pad;
+  g.cols_shared = Is;
+  g.out_routed = static_cast<__nv_bfloat16*>(H->dhr); g.ld_routed = I; g.rows_routed = H->rows_cap;
+  g.cols_routed = I;
+  g.err = H->err;
+  launch_pdl(grouped_gemm_tc_kernel<kDown>, dim3(H->gemm_grid), dim3(kGemmThreads), kGemmSmemBytes, stream,
+             tmDh, H->tmDyr, H->tmWdTs, H->tmWdTr, g);
+  MOE_CUDA(cudaGetLastError());
+  // 3. gate/up recomputed with the SwiGLU backward: (da, db) interleaved like W_gu's rows
+  GemmArgs g1{};
+  g1.grp_row = H->grp_row; g1.ts = H->ts1; g1.G = H->G; g1.has_shared = H->has_shared;
+  g1.kb_shared = d / kGemmBK; g1.kb_routed = d / kGemmBK;
+  g1.nt_shared = (Is + kGemmBN / 2 - 1) / (kGemmBN / 2); g1.nt_routed = (I + kGemmBN / 2 - 1) / (kGemmBN / 2);
+  g1.out_shared = static_cast<__nv_bfloat16*>(H->dabs); g1.ld_shared = 2 * (int64_t)Is;
+  g1.rows_shared = H->T_pad; g1.cols_shared = Is;
+  g1.out_routed = static_cast<__nv_bfloat16*>(H->dabr); g1.ld_routed = 2 * (int64_t)I;
+  g1.rows_routed = H->rows_cap; g1.cols_routed = I;
+  g1.dh_shared = static_cast<const __nv_bfloat16*>(H->dhs); g1.ld_dh_shared = Is;
+  g1.dh_routed = static_cast<const __nv_bfloat16*>(H->dhr); g1.ld_dh_routed = I;
+  g1.err = H->err;
+  launch_pdl(grouped_gemm_tc_kernel<kGateUpBwd>, dim3(H->gemm_grid), dim3(kGemmThreads), kGemmSmemBytes,
+             stream, tmU, H->tmXp, H->tmWguS, H->tmWguR, g1);
+  MOE_CUDA(cudaGetLastError());
+  // 4. dX = [da db] [W_gate; W_up]
+  GemmArgs g2{};
+  g2.grp_row = H->grp_row; g2.ts = H->ts2; g2.G = H->G; g2.has_shared = H->has_shared;
+  g2.kb_shared = 2 * Is / kGemmBK; g2.kb_routed = 2 * I / kGemmBK;
+  g2.nt_shared = g2.nt_routed = (d + kGemmBN - 1) / kGemmBN;
+  g2.out_shared = static_cast<__nv_bfloat16*>(H->dxs); g2.ld_shared = d; g2.rows_shared = H->T_pad;
+  g2.cols_shared = d;
+  g2.out_routed = static_cast<__nv_bfloat16*>(H->dxr); g2.ld_routed = d; g2.rows_routed = H->rows_cap;
+  g2.cols_routed = d;
+  g2.err = H->err;
+  launch_pdl(grouped_gemm_tc_kernel<kDown>, dim3(H->gemm_grid), dim3(kGemmThreads), kGemmSmemBytes, stream,
+             H->tmDabs, H->tmDabr, H->tmWguTs, H->tmWguTr, g2);
+  MOE_CUDA(cudaGetLastError());
+  // 5. router: dl = s (ds - sum s ds), then dl e (one-group GEMM, K = n_pad)
+  BwdRouterArgs ra{H->logits, topk_idx, H->dg, expert_counts, T, nr, K, H->n_pad, H->kpad,
+                   (float)((double)d_aux * (double)c.alpha1 / ((double)T * (double)T)), H->dl,
+                   static_cast<__nv_bfloat16*>(H->dlb)};
+  with_maxc(H->maxc, [&](auto m) {
+    launch_pdl(bwd_router_kernel<m()>, dim3((T + kBwdWarps - 1) / kBwdWarps), dim3(kBwdWarps * 32), 0, stream, ra);
+    return 0;
+  });
+  MOE_CUDA(cudaGetLastError());
+  GemmArgs g3{};
+  g3.grp_row = H->r_grp; g3.ts = H->r_ts; g3.G = 1; g3.has_shared = 1;
+  g3.kb_shared = g3.kb_routed = H->kpad / kGemmBK;
+  g3.nt_shared = g3.nt_routed = (d + kGemmBN - 1) / kGemmBN;
+  g3.out_shared = g3.out_routed = static_cast<__nv_bfloat16*>(H->dur);
+  g3.ld_shared = g3.ld_routed = d;
+  g3.rows_shared = g3.rows_routed = H->T_pad;
+  g3.cols_shared = g3.cols_routed = d;
+  g3.err = H->err;
+  launch_pdl(grouped_gemm_tc_kernel<kDown>, dim3(H->gemm_grid), dim3(kGemmThreads), kGemmSmemBytes, stream,
+             H->tmDlb, H->tmDlb, H->tmEt, H->tmEt, g3);
+  MOE_CUDA(cudaGetLastError());
+  // 6. du = dh + dX_shared + sum_k dX_k + dl e (fixed order, one rounding)
+  const int parts = combine_parts(T, d / 8, H->n_sms);
+  CombineArgs<__nv_bfloat16> ca{static_cast<const __nv_bfloat16*>(dh),
+                                H->has_shared ? static_cast<const __nv_bfloat16*>(H->dxs) : nullptr,
+                                static_cast<const __nv_bfloat16*>(H->dxr), H->slot_row, nullptr,
+                                static_cast<__nv_bfloat16*>(du), T, d, K, parts,
+                                static_cast<const __nv_bfloat16*>(H->dur)};
+  const int cgrid = (int)(((int64_t)T * parts + kCombineWarps - 1) / kCombineWarps);
+  with_maxk(H->maxk, [&](auto m) {
+    launch_pdl(combine_bf16_kernel<m()>, dim3(cgrid), dim3(kCombineWarps * 32), 0, stream, ca);
+    return 0;
+  });
+  MOE_CUDA(cudaGetLastError());
+  // 7. centroid and bias gradients: chunk partials, then their fixed-order sum
+  BwdCentroidArgs cp{H->dl, static_cast<const __nv_bfloat16*>(u), T, d, nr, H->n_pad, H->cen_chunks,
+                     H->cen_part};
+  launch_pdl(bwd_centroid_partial_kernel, dim3((d + kCenCols - 1) / kCenCols, H->cen_chunks), dim3(256), 0,
+             stream, cp);
+  MOE_CUDA(cudaGetLastError());
+  const int rgrid = (int)(((size_t)nr * (d + 1) + 255) / 256);
+  launch_pdl(bwd_centroid_reduce_kernel, dim3(rgrid < 4 * H->n_sms ? rgrid : 4 * H->n_sms), dim3(256), 0,
+             stream, (const float*)H->cen_part, H->cen_chunks, nr, d, d_centroids, d_bias);
+  MOE_CUDA(cudaGetLastError());
+  if (!wgrad) return MOE_OK;
+  // 8. weight gradients: transposed activations (padding rows zero), then per group
+  //    dW_gate/up = [da db]^T X (rows interleaved like W_gu, split on the way out) and
+  //    dW_down = dY^T Hmid, K = the group's rows
+  const int64_t rc = H->rows_cap, tp = H->T_pad;
+  auto mtr = [&](const void* src, void* dst, int64_t rows, int C, int64_t ld_src, int64_t ld_dst,
+                 bool routed) {
+    MaskedTransposeArgs ma{static_cast<const __nv_bfloat16*>(src), static_cast<__nv_bfloat16*>(dst), rows, C,
+                           ld_src, ld_dst, routed ? H->grp_row + H->has_shared : nullptr, expert_counts,
+                           nr, 0, T, routed ? rows : (int64_t)T};
+    launch_pdl(masked_transpose_kernel, dim3((unsigned)((C + kTrTile - 1) / kTrTile),
+                                             (unsigned)((rows + kTrTile - 1) / kTrTile)),
+               dim3(256), 0, stream, ma);
+    return cudaGetLastError();
+  };
+  MOE_CUDA(mtr(H->xp, H->xpT, rc, d, d, rc, true));
+  MOE_CUDA(mtr(H->dyr, H->dyrT, rc, d, d, rc, true));
+  MOE_CUDA(mtr(H->hr, H->hrT, rc, I, I, rc, true));
+  MOE_CUDA(mtr(H->dabr, H->dabrT, rc, 2 * I, 2 * I, rc, true));
+  if (H->has_shared) {
+    MOE_CUDA(mtr(u, H->uT, tp, d, d, tp, false));
+    MOE_CUDA(mtr(dh, H->dhT, tp, d, d, tp, false));
+    MOE_CUDA(mtr(H->hs, H->hsT, tp, Is, Is, tp, false));
+    MOE_CUDA(mtr(H->dabs, H->dabsT, tp, 2 * Is, 2 * Is, tp, false));
+  }
+  const size_t ks = c.n_shared;
+  GemmArgs w1{};
+  w1.grp_row = H->grp_row; w1.ts = H->wts1; w1.G = H->G; w1.has_shared = H->has_shared;
+  w1.kb_shared = (int)(tp / kGemmBK); w1.kb_routed = 0;
+  w1.nt_shared = w1.nt_routed = (d + kGemmBN - 1) / kGemmBN;
+  w1.rows_shared = 2 * (int64_t)Is; w1.rows_routed = 2 * (int64_t)I;
+  w1.cols_shared = w1.cols_routed = d;
+  w1.err = H->err;
+  w1.wg_counts = expert_counts; w1.wg_bm = H->bm; w1.wg_split = 1;
+  w1.wg_out0_shared = d_w_gate; w1.wg_out1_shared = d_w_up;
+  w1.wg_out0_routed = d_w_gate + ks * (size_t)I * d; w1.wg_out1_routed = d_w_up + ks * (size_t)I * d;
+  w1.wg_stride = (int64_t)I * d;
+  launch_pdl(grouped_gemm_tc_kernel<kWgrad>, dim3(H->gemm_grid), dim3(kGemmThreads), kGemmSmemBytes, stream,
+             H->tmDabsT, H->tmDabrT, H->tmUT, H->tmXpT, w1);
+  MOE_CUDA(cudaGetLastError());
+  GemmArgs w2{};
+  w2.grp_row = H->grp_row; w2.ts = H->wts2; w2.G = H->G; w2.has_shared = H->has_shared;
+  w2.kb_shared = (int)(tp / kGemmBK); w2.kb_routed = 0;
+  w2.nt_shared = (Is + kGemmBN - 1) / kGemmBN; w2.nt_routed = (I + kGemmBN - 1) / kGemmBN;
+  w2.rows_shared = w2.rows_routed = d;
+  w2.cols_shared = Is; w2.cols_routed = I;
+  w2.err = H->err;
+  w2.wg_counts = expert_counts; w2.wg_bm = H->bm; w2.wg_split = 0;
+  w2.wg_out0_shared = d_w_down; w2.wg_out0_routed = d_w_down + ks * (size_t)d * I;
+  w2.wg_stride = (int64_t)d * I;
+  w2.wg_colsplit = I;   // the shared group's K_s experts sit side by side along I
+  launch_pdl(grouped_gemm_tc_kernel<kWgrad>, dim3(H->gemm_grid), dim3(kGemmThreads), kGemmSmemBytes, stream,
+             H->tmDhT, H->tmDyrT, H->tmHsT, H->tmHrT, w2);
+  MOE_CUDA(cudaGetLastError());
   return MOE_OK;
 }
 

@@ -1,6 +1,6 @@
 // router.cuh -- fused router: centroid GEMM, softmax over the routed experts, top-k with
 // lower-index tie-break, gates, per-tile expert histograms / within-tile ranks and
-// per-tile affinity sums.
+// per-tile affinity sums; the last CTA then runs the scan (scan.cuh).
 //
 // DeepSeekMoE (deepforge.srivtx.xyz article), "Routing in a classic MoE layer":
 // s_i = softmax_i(u^T e_i), g_i = s_i for the top-K affinities, else 0; "Top-k routing,
@@ -9,34 +9,34 @@
 // loss": counts and mean affinities per routed expert.
 //
 // Tiles of R <= 128 tokens, as many as there are SMs, so that each SM streams the centroid
-// matrix once per tile and issues the fewest MMAs: at the layer sizes of interest the
-// tile loads run close to HBM bandwidth and the per-instruction MMA cost does not shrink
-// below N = 256, so smaller tiles only add centroid traffic and MMA instructions.  The bf16
-// kernel computes the 128 x N_pad logit tile with tcgen05.mma into one of two
-// tensor-memory accumulators (A = the tile's token rows streamed by TMA, B = the padded
-// centroid matrix; accumulator rows past R are never read back); a CTA with several tiles
-// (large T) overlaps the next tile's loads with the epilogue.  Sixteen epilogue warps copy
-// the logits (+ bias) to shared memory in passes of 64 rows and work on each pass with
-// eight threads per token row: row max and softmax denominator by shuffles, the top-k by
-// a bitonic sort of each thread's keys and three bitonic merges across the row's threads
-// (or, for top_k > 8 or wide rows, top_k rounds of a group-wide maximum).  The fp32 kernel
-// computes the same logits with FMA into the same shared-memory layout and shares the rest.
+// matrix once per tile and issues the fewest MMAs.  The bf16 kernel computes the 128 x N_pad
+// logit tile with tcgen05.mma into one of two tensor-memory accumulators (A = the tile's
+// token rows streamed by TMA, B = the padded centroid matrix; accumulator rows past R are
+// never read back); a CTA with several tiles (large T) overlaps the next tile's loads with
+// the epilogue.  Sixteen epilogue warps copy the logits (+ bias) to shared memory in passes
+// of 64 rows and route each row with one warp: the lanes hold the row's columns, the row
+// max and the top-k come from warp-wide redux max / min on 32-bit order-preserving keys
+// (max key, then the lowest index carrying it: exactly the stable ranking), the softmax
+// denominator from a fixed butterfly of shuffles.  The fp32 kernel and the decode-sized
+// bf16 kernel compute the same logits with FMA into the same shared-memory layout and share
+// the rest.
 #pragma once
 
 #include <climits>
 
-#include "ptx.cuh"
+#include "scan.cuh"
 
 namespace moe {
 
-constexpr int kMaxTopK = 16;
-constexpr int kMaxRouted = 256;
 constexpr int kRouterBM = 128;          // MMA rows = largest token tile
 constexpr int kRouterPass = 64;         // token rows per epilogue pass
-constexpr int kRouterGroup = 8;         // threads per token row in the epilogue
-constexpr int kRouterEpiThreads = 512;  // kRouterPass * kRouterGroup
+constexpr int kRouterEpiThreads = 512;  // 16 warps, one token row at a time each
 constexpr int kRouterThreads = 64 + kRouterEpiThreads;   // warp 0 TMA, warp 1 MMA
 constexpr int kRouterMaxStages = 8;
+#ifndef MOE_ROUTER_MAX_KPS
+#define MOE_ROUTER_MAX_KPS 4
+#endif
+constexpr int kRouterMaxKps = MOE_ROUTER_MAX_KPS;   // 64-wide k-blocks per pipeline stage, at most
 constexpr size_t kRouterSmemBudget = 232448;   // opt-in dynamic shared memory per block
 constexpr size_t kRouterCtlBytes = 512;        // mbarriers, TMEM slot, abort flag
 
@@ -47,16 +47,22 @@ struct RouterOut {
   int32_t* tile_hist;   // [n_tiles, n_routed]
   float* tile_psum;     // [n_tiles, n_routed]  sum over the tile's tokens of s[t, i]
   int* err;
+  ScanArgs scan;        // run by the last CTA (scan.cuh)
+  float* logits;        // [T, n_routed] the logits (bias added) for the backward, or nullptr
 };
 
-struct RouterEpiSmem {
+// 16-byte aligned size: the logit rows that follow it take float4 stores.
+struct alignas(16) RouterEpiSmem {
   float bias[kMaxRouted];
   uint32_t mask[kMaxRouted][4];            // bit r of mask[e][r/32]: token r of the tile chose e
   int32_t sel[kRouterBM][kMaxTopK];        // chosen experts of each row, in rank order
   float gsel[kRouterBM][kMaxTopK];         // their gates s[t, e]
   float inv_sum[kRouterPass];              // 1 / softmax denominator (0 for rows past T)
   float ppart[8][kMaxRouted];              // per-expert sums over row parts of the tile
+  int last;                                // router_finish: this CTA finished last
 };
+static_assert(sizeof(RouterEpiSmem) >= sizeof(ScanSmem), "the scan reuses the epilogue scratch");
+static_assert(sizeof(RouterEpiSmem) % 16 == 0, "the logit rows after the scratch need 16-byte alignment");
 
 // Epilogue scratch: RouterEpiSmem, then the logit rows of one pass lg[64][ld] (fp32, bias
 // added), overwritten in place by exp(l - max).  ld = N_pad + 4 keeps the float4 row
@@ -65,7 +71,8 @@ __host__ __device__ constexpr int router_ld(int n_pad) { return n_pad + 4; }
 __host__ __device__ constexpr size_t router_epi_bytes(int n_pad) {
   return sizeof(RouterEpiSmem) + (size_t)kRouterPass * router_ld(n_pad) * 4;
 }
-// Columns per epilogue thread, N_pad / 8, rounded up to the compile-time bound.
+// Compile-time bound on N_pad / 8 (the kernels are instantiated per bound); each lane of a
+// routing warp holds up to MAXC / 4 = ceil(N_pad / 32) columns of a row.
 __host__ __device__ constexpr int router_maxc(int n_pad) {
   return n_pad <= 16 ? 2 : n_pad <= 32 ? 4 : n_pad <= 64 ? 8 : n_pad <= 128 ? 16 : 32;
 }
@@ -81,47 +88,124 @@ __host__ __device__ constexpr int router_psum_parts(int n_pad) {
   return kRouterEpiThreads / n_pad > 8 ? 8 : kRouterEpiThreads / n_pad;
 }
 
-// Total order on (logit, expert): larger logit first; on equal logits the lower index.
-// NaN ranks as -inf and -0 as +0, so every slot gets a real index and equal values tie.
-__device__ __forceinline__ uint64_t route_key(float l, int i) {
+// Order-preserving 32-bit key of a logit: a larger logit gets a larger key; NaN ranks as
+// -inf and -0 as +0, so every expert gets a real rank and equal values tie.  Key 0 is below
+// every logit (unused columns, experts already chosen).
+__device__ __forceinline__ uint32_t logit_key(float l) {
   uint32_t b = (l != l) ? 0xFF800000u : __float_as_uint(l);
   if (b == 0x80000000u) b = 0u;
-  const uint32_t ord = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-  return (static_cast<uint64_t>(ord) << 32) | static_cast<uint64_t>(0xFFFFFFFFu - (uint32_t)i);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
-__device__ __forceinline__ int key_index(uint64_t key) {
-  return (int)(0xFFFFFFFFu - (uint32_t)key);
+// The logit of a key (inverse of logit_key for keys >= 1).
+__device__ __forceinline__ float key_logit(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
-// Descending bitonic sort of N keys held in registers.
-template <int N>
-__device__ __forceinline__ void bitonic_sort_desc(uint64_t (&k)[N]) {
+constexpr int kRouteRows = 2;   // rows a routing warp works on together (independent chains)
+
+// Route kRouteRows rows of the pass with one warp.  rr[j]: the rows (in the pass; -1 = none);
+// their logits (bias added) are lg[rr][c] for c < N_pad.  Lane l holds columns l + 32 m.
+// Per row: the max (redux max of the keys), exp(l - max) written back in place, the
+// denominator (each lane's columns in order, then a butterfly of xor-shuffles 16, 8, 4, 2, 1,
+// so every lane holds the same sum), and top_k rounds of "largest key, then the lowest
+// column carrying it" (redux max, redux min), whose winner's key is then cleared.  Lane p
+// records round p: sel/gsel/mask of the tile row.  Rows past the tile or past T get zero
+// exp values and inv_sum 0.
+template <int MAXC>
+__device__ __forceinline__ void route_rows_warp(const int (&rr)[kRouteRows], int lane, int pass,
+                                                int tile, int R, int T, int n_routed, int n_pad,
+                                                int top_k, uint8_t* epi, const RouterOut& o) {
+  constexpr int MC = (MAXC + 3) / 4;   // columns per lane
+  RouterEpiSmem& S = *reinterpret_cast<RouterEpiSmem*>(epi);
+  float* lg = reinterpret_cast<float*>(epi + sizeof(RouterEpiSmem));
+  const int ld = router_ld(n_pad);
+  uint32_t key[kRouteRows][MC];
+  float ex[kRouteRows][MC];
+  bool valid[kRouteRows];
+  float inv[kRouteRows];
 #pragma unroll
-  for (int size = 2; size <= N; size <<= 1) {
+  for (int j = 0; j < kRouteRows; ++j) {
+    const int tr = pass * kRouterPass + rr[j];
+    valid[j] = rr[j] >= 0 && tile * R + tr < T;
+    const float* row = lg + (size_t)(rr[j] < 0 ? 0 : rr[j]) * ld;
+    uint32_t kmax = 0u;
 #pragma unroll
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+    for (int m = 0; m < MC; ++m) {
+      const int c = lane + 32 * m;
+      const bool in = valid[j] && c < n_routed;
+      ex[j][m] = in ? row[c] : 0.f;
+      key[j][m] = in ? logit_key(ex[j][m]) : 0u;
+      kmax = max(kmax, key[j][m]);
+      if (in && o.logits) o.logits[(size_t)(tile * R + tr) * n_routed + c] = ex[j][m];
+    }
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    const float lmax = key_logit(kmax);
+    float part = 0.f;
 #pragma unroll
-      for (int i = 0; i < N; ++i) {
-        const int l = i ^ stride;
-        if (l > i) {
-          const bool desc = (i & size) == 0;
-          const uint64_t x = k[i], y = k[l];
-          const bool sw = desc ? (x < y) : (x > y);
-          k[i] = sw ? y : x;
-          k[l] = sw ? x : y;
-        }
+    for (int m = 0; m < MC; ++m) {
+      const int c = lane + 32 * m;
+      ex[j][m] = (valid[j] && c < n_routed) ? __expf(ex[j][m] - lmax) : 0.f;
+      part += ex[j][m];
+    }
+#pragma unroll
+    for (int o2 = 16; o2 > 0; o2 >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o2);
+    inv[j] = valid[j] ? 1.0f / part : 0.f;
+  }
+  int my_e[kRouteRows];
+  float my_g[kRouteRows];
+#pragma unroll
+  for (int j = 0; j < kRouteRows; ++j) { my_e[j] = 0; my_g[j] = 0.f; }
+#pragma unroll 1
+  for (int p = 0; p < top_k; ++p) {
+#pragma unroll
+    for (int j = 0; j < kRouteRows; ++j) {
+      uint32_t bk = 0u;
+      int bc = 0x7fffffff;
+#pragma unroll
+      for (int m = 0; m < MC; ++m) {
+        if (key[j][m] > bk) { bk = key[j][m]; bc = lane + 32 * m; }   // ascending columns
       }
+      const uint32_t gk = __reduce_max_sync(0xffffffffu, bk);
+      const int gc = (int)__reduce_min_sync(0xffffffffu, bk == gk ? (uint32_t)bc : 0x7fffffffu);
+      float eg = 0.f;
+#pragma unroll
+      for (int m = 0; m < MC; ++m) {
+        if (lane + 32 * m == gc) { eg = ex[j][m]; key[j][m] = 0u; }
+      }
+      eg = __shfl_sync(0xffffffffu, eg, gc & 31);
+      if (lane == p) { my_e[j] = gc; my_g[j] = eg * inv[j]; }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < kRouteRows; ++j) {
+    if (rr[j] < 0) continue;
+    float* row = lg + (size_t)rr[j] * ld;
+#pragma unroll
+    for (int m = 0; m < MC; ++m) {
+      const int c = lane + 32 * m;
+      if (c < n_pad) row[c] = ex[j][m];
+    }
+    if (lane == 0) S.inv_sum[rr[j]] = inv[j];
+    if (valid[j] && lane < top_k) {
+      const int tr = pass * kRouterPass + rr[j];
+      int e = my_e[j];
+      if (e < 0 || e >= n_routed) {
+        record_error(o.err, kErrRouteIndex);
+        e = 0;
+      }
+      S.sel[tr][lane] = e;
+      S.gsel[tr][lane] = my_g[j];
+      atomicOr(&S.mask[e][tr >> 5], 1u << (tr & 31));
     }
   }
 }
 
 // One epilogue pass: the pass's logit rows (bias added) are in lg[r][i] for r < rows,
-// i < N_pad, and the masks are zero (first pass) or hold the earlier passes' choices.
-// Thread tid (of 512) works on row r = tid / 8 of the pass (tile row 64 * pass + r) with
-// the eight threads of its row owning consecutive column blocks of C = N_pad / 8.  Writes
-// sel/gsel/mask for its rows and adds the pass's per-expert affinity sums into ppart.
-// `sync()` synchronises the 512 threads; returns with the scratch still in use.
+// i < N_pad, and the masks are zero (first pass) or hold the earlier passes' choices.  The
+// 16 warps route rows w, w + 16, ... of the pass, kRouteRows at a time; then the pass's
+// per-expert affinity sums are added to the earlier passes' parts.  `sync()` synchronises
+// the 512 threads.
 template <int MAXC, class Sync>
 __device__ __forceinline__ void router_pass(int tid, int pass, int tile, int R, int T,
                                             int n_routed, int n_pad, int top_k, uint8_t* epi,
@@ -129,120 +213,15 @@ __device__ __forceinline__ void router_pass(int tid, int pass, int tile, int R, 
   RouterEpiSmem& S = *reinterpret_cast<RouterEpiSmem*>(epi);
   float* lg = reinterpret_cast<float*>(epi + sizeof(RouterEpiSmem));
   const int ld = router_ld(n_pad);
-  const int r = tid >> 3, j = tid & 7;
-  const int tr = pass * kRouterPass + r;                  // row in the tile
   const int rows = min(kRouterPass, R - pass * kRouterPass);
-  const int C = n_pad >> 3;              // even: N_pad is a multiple of 16
-  const int c0 = j * C;
-  const int t = tile * R + tr;
-  const bool valid = r < rows && t < T;
-  float* row = lg + (size_t)r * ld;
-
-  // warps whose four rows all lie past the pass skip the per-row work (they still take
-  // part in every barrier)
-  if ((tid >> 5) * 4 < rows) {
-  // keys and the row max; rows past the tile or past T are treated as zeros
-  uint64_t key[MAXC];
-  float lmax = -INFINITY;
+  const int warp = tid >> 5, lane = tid & 31;
+  constexpr int kWarps = kRouterEpiThreads / 32;
+  for (int r0 = warp; r0 < rows; r0 += kWarps * kRouteRows) {
+    int rr[kRouteRows];
 #pragma unroll
-  for (int k = 0; k < MAXC; k += 2) {
-    float2 x = make_float2(0.f, 0.f);
-    if (k < C && valid) x = *reinterpret_cast<const float2*>(row + c0 + k);
-    const bool in0 = k < C && c0 + k < n_routed, in1 = k < C && c0 + k + 1 < n_routed;
-    key[k] = in0 ? route_key(x.x, c0 + k) : 0ull;
-    key[k + 1] = in1 ? route_key(x.y, c0 + k + 1) : 0ull;
-    if (in0) lmax = fmaxf(lmax, x.x);
-    if (in1) lmax = fmaxf(lmax, x.y);
+    for (int j = 0; j < kRouteRows; ++j) rr[j] = r0 + j * kWarps < rows ? r0 + j * kWarps : -1;
+    route_rows_warp<MAXC>(rr, lane, pass, tile, R, T, n_routed, n_pad, top_k, epi, o);
   }
-#pragma unroll
-  for (int m = 1; m < kRouterGroup; m <<= 1)
-    lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, m));
-
-  // exp(l - max) in place, denominator: column order within a thread, then a fixed tree
-  float part = 0.f;
-#pragma unroll
-  for (int k = 0; k < MAXC; k += 2) {
-    if (k < C) {
-      const float2 x = *reinterpret_cast<const float2*>(row + c0 + k);
-      const float e0 = (valid && c0 + k < n_routed) ? __expf(x.x - lmax) : 0.f;
-      const float e1 = (valid && c0 + k + 1 < n_routed) ? __expf(x.y - lmax) : 0.f;
-      part += e0;
-      part += e1;
-      *reinterpret_cast<float2*>(row + c0 + k) = make_float2(e0, e1);
-    }
-  }
-#pragma unroll
-  for (int m = 1; m < kRouterGroup; m <<= 1) part += __shfl_xor_sync(0xffffffffu, part, m);
-  const float inv_sum = 1.0f / part;
-  if (j == 0) S.inv_sum[r] = valid ? inv_sum : 0.f;
-  __syncwarp();   // the row's exp values (written by the eight threads of a warp) are read below
-
-  auto record = [&](int p, uint64_t g) {
-    int e = key_index(g);
-    if (e < 0 || e >= n_routed) {
-      record_error(o.err, kErrRouteIndex);
-      e = 0;
-    }
-    if (valid) {
-      S.sel[tr][p] = e;
-      S.gsel[tr][p] = row[e] * inv_sum;
-      atomicOr(&S.mask[e][tr >> 5], 1u << (tr & 31));
-    }
-  };
-
-  if (MAXC <= 8 && top_k <= 8) {
-    // sort the thread's keys (padded to 8 with zeros), then three bitonic merges with the
-    // partner threads: every thread of the row ends up with the row's 8 largest keys
-    uint64_t kk[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) kk[i] = i < MAXC ? key[i < MAXC ? i : 0] : 0ull;
-    bitonic_sort_desc<8>(kk);
-#pragma unroll
-    for (int m = 1; m < kRouterGroup; m <<= 1) {
-      uint64_t pk[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) pk[i] = __shfl_xor_sync(0xffffffffu, kk[i], m);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) kk[i] = kk[i] > pk[7 - i] ? kk[i] : pk[7 - i];   // bitonic
-#pragma unroll
-      for (int stride = 4; stride > 0; stride >>= 1) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int l = i ^ stride;
-          if (l > i) {
-            const uint64_t x = kk[i], y = kk[l];
-            kk[i] = x > y ? x : y;
-            kk[l] = x > y ? y : x;
-          }
-        }
-      }
-    }
-    // thread j of the row records rank j
-    uint64_t mine = 0ull;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) mine = i == j ? kk[i] : mine;
-    if (j < top_k) record(j, mine);
-  } else {
-    // top_k rounds: the group's largest remaining key; its owner records it and drops it
-#pragma unroll 1
-    for (int p = 0; p < top_k; ++p) {
-      uint64_t best = key[0];
-#pragma unroll
-      for (int k = 1; k < MAXC; ++k) best = key[k] > best ? key[k] : best;
-      uint64_t g = best;
-#pragma unroll
-      for (int m = 1; m < kRouterGroup; m <<= 1) {
-        const uint64_t y = __shfl_xor_sync(0xffffffffu, g, m);
-        g = y > g ? y : g;
-      }
-      if (best == g) {   // keys are distinct (distinct indices): exactly one owner
-        record(p, g);
-#pragma unroll
-        for (int k = 0; k < MAXC; ++k) key[k] = key[k] == g ? 0ull : key[k];
-      }
-    }
-  }
-  }   // warps with rows
   sync();
 
   // the pass's per-expert affinity sums: row parts, added to the earlier passes' parts
@@ -252,7 +231,7 @@ __device__ __forceinline__ void router_pass(int tid, int pass, int tile, int R, 
     const int pp = idx / n_pad, c = idx - pp * n_pad;
     const int r0 = pp * RP, r1 = min(rows, r0 + RP);
     float a = 0.f;
-    for (int rr = r0; rr < r1; ++rr) a += lg[(size_t)rr * ld + c] * S.inv_sum[rr];
+    for (int r = r0; r < r1; ++r) a += lg[(size_t)r * ld + c] * S.inv_sum[r];
     S.ppart[pp][c] = pass == 0 ? a : S.ppart[pp][c] + a;
   }
 }
@@ -310,7 +289,7 @@ __device__ __forceinline__ void tmem_ld_wait16(uint32_t (&r)[16]) {
 // ------------------------------------------------------------------------ bf16, tcgen05
 struct RouterTcArgs {
   int T, d, n_routed, n_pad, top_k;
-  int kps, stages;     // k-blocks per stage (1 or 2), stages in the ring
+  int kps, stages;     // k-blocks per stage (1 .. 4), stages in the ring
   int tile_rows;       // R: tokens per tile (<= 128, multiple of 8); the U map's box height
   int n_tiles;         // tiles, handed out round-robin over the CTAs
   uint32_t tmem_cols;  // power of two >= 2 * n_pad: two accumulators
@@ -318,14 +297,14 @@ struct RouterTcArgs {
   RouterOut out;
 };
 
-// A stage holds kps (1 or 2) 64-wide k-blocks: A_0 .. A_{kps-1} (the tile's R token rows of
+// A stage holds kps (1 .. 4) 64-wide k-blocks: A_0 .. A_{kps-1} (the tile's R token rows of
 // 128 B, rounded up to 1 KB) then B_0 .. B_{kps-1} (n_pad centroid rows of 128 B each, also
 // rounded up).  A barrier round trip (the producer's wait on `empty`, the MMA issuer's
 // wait on `full`) costs a few hundred cycles, about as long as the four N <= 64 MMAs of
-// one k-block, so a stage carries two where three stages of that size fit.  The M = 128
-// MMA reads 128 A rows; rows R..127 fall on the next block of the same stage (or the tail
-// padding), which the same TMA batch has filled: they only produce accumulator rows that
-// are never read.
+// one k-block, so a stage carries as many k-blocks as keep the most of them in flight.  The
+// M = 128 MMA reads 128 A rows; rows R..127 fall on the next block of the same stage (or the
+// tail padding), which the same TMA batch has filled: they only produce accumulator rows
+// that are never read.
 __host__ __device__ constexpr uint32_t router_a_bytes(int R) { return ((uint32_t)R * 128u + 1023u) & ~1023u; }
 __host__ __device__ constexpr uint32_t router_b_bytes(int n_pad) { return ((uint32_t)n_pad * 128u + 1023u) & ~1023u; }
 __host__ __device__ constexpr uint32_t router_stage_bytes(int n_pad, int kps, int R) {
@@ -339,17 +318,20 @@ __host__ __device__ constexpr size_t router_smem_bytes(int n_pad, int kps, int R
   return 1024 + (size_t)stages * router_stage_bytes(n_pad, kps, R) + router_epi_bytes(n_pad) +
          kRouterCtlBytes;
 }
-// Stage shape: {k-blocks per stage, stages} that fit kRouterSmemBudget; stages < 2 when
-// nothing does.
+// Stage shape: the {k-blocks per stage, stages} (at least two stages) that fits
+// kRouterSmemBudget with the most k-blocks in flight, the larger stage on a tie (fewer
+// barrier round trips); stages < 2 when nothing fits.
 struct RouterStages { int kps, stages; };
 inline RouterStages router_stages(int n_pad, int R) {
-  for (int kps = 2; kps >= 1; --kps) {
+  RouterStages best{1, 0};
+  for (int kps = 1; kps <= kRouterMaxKps; ++kps) {
     long st = ((long)kRouterSmemBudget - (long)router_smem_bytes(n_pad, kps, R, 0)) /
               (long)router_stage_bytes(n_pad, kps, R);
     if (st > kRouterMaxStages) st = kRouterMaxStages;
-    if (st >= 3 || kps == 1) return RouterStages{kps, (int)st};
+    if (st < 2) continue;
+    if (best.stages < 2 || st * kps >= (long)best.stages * best.kps) best = RouterStages{kps, (int)st};
   }
-  return RouterStages{1, 0};
+  return best;
 }
 
 // Persistent: CTA b handles tiles b, b + gridDim.x, ...  With several tiles per CTA the
@@ -526,6 +508,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant_
       router_tile_outputs(tid, tile, a.tile_rows, a.T, a.n_routed, a.n_pad, a.top_k, epi, a.out);
       sync();   // scratch free for the next tile
     }
+    router_finish(a.out.scan, tid, &SM.last, epi, sync);
   }
 
   tc_fence_before();
@@ -580,6 +563,7 @@ __global__ void __launch_bounds__(kRouterEpiThreads) router_simt_kernel(RouterSi
                     sync);
   __syncthreads();
   router_tile_outputs(tid, tile, kRouterPass, a.T, a.n_routed, n_pad, a.top_k, smem_raw, a.out);
+  router_finish(a.out.scan, tid, &SM.last, smem_raw, sync);
 }
 
 // ------------------------------------------------------------------------ bf16, few tokens
@@ -666,6 +650,7 @@ __global__ void __launch_bounds__(kRouterEpiThreads) router_small_kernel(RouterS
   router_pass<MAXC>(tid, 0, tile, R, a.T, a.n_routed, n_pad, a.top_k, smem_raw, a.out, sync);
   __syncthreads();
   router_tile_outputs(tid, tile, R, a.T, a.n_routed, n_pad, a.top_k, smem_raw, a.out);
+  router_finish(a.out.scan, tid, &SM.last, smem_raw, sync);
 }
 
 }  // namespace moe

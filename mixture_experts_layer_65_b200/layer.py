@@ -189,6 +189,38 @@ class MoELayer:
         s = stream or torch.cuda.current_stream(self.device)
         check(lib().moe_pipeline_wait(self._h, s.cuda_stream))
 
+    def backward_prepare(self) -> None:
+        """Allocate the backward's workspace and transposed weights (once; later forwards also
+        keep their logits).  bf16 layers on the paired-GEMM path only."""
+        with torch.cuda.device(self.device):
+            check(lib().moe_backward_prepare(self._h))
+
+    def backward(self, u: torch.Tensor, out: MoEOutput, dh: torch.Tensor, d_aux: float = 0.0,
+                 weights: bool = True, stream: torch.cuda.Stream | None = None):
+        """Gradients of sum(dh * h) + d_aux * aux after `forward(u, out)` on this layer (no
+        other forward in between): (du [T, d] bf16, d_centroids [n_routed, d] fp32,
+        d_bias [n_routed] fp32, d_w_gate, d_w_up [G, inter, d] fp32, d_w_down [G, d, inter]
+        fp32), G = n_shared + n_routed; the last three are None with weights=False."""
+        self._check_device_tensor("u", u, (self.T, self.d), self.torch_dtype)
+        self._check_device_tensor("dh", dh, (self.T, self.d), self.torch_dtype)
+        self._check_outputs(out)
+        dev = self.device
+        du = torch.empty(self.T, self.d, dtype=self.torch_dtype, device=dev)
+        d_cen = torch.empty(self.n_routed, self.d, dtype=torch.float32, device=dev)
+        d_bias = torch.empty(self.n_routed, dtype=torch.float32, device=dev)
+        G = self.n_shared + self.n_routed
+        dwg = dwu = dwd = None
+        if weights:
+            dwg = torch.empty(G, self.inter, self.d, dtype=torch.float32, device=dev)
+            dwu = torch.empty(G, self.inter, self.d, dtype=torch.float32, device=dev)
+            dwd = torch.empty(G, self.d, self.inter, dtype=torch.float32, device=dev)
+        s = stream or torch.cuda.current_stream(dev)
+        check(lib().moe_backward(self._h, _ptr(u), _ptr(out.topk_idx), _ptr(out.topk_w),
+                                 _ptr(out.expert_counts), _ptr(dh), float(d_aux), _ptr(du),
+                                 _ptr(d_cen), _ptr(d_bias), _ptr(dwg), _ptr(dwu), _ptr(dwd),
+                                 s.cuda_stream))
+        return du, d_cen, d_bias, dwg, dwu, dwd
+
     DEBUG_BUFFERS = {"slot_row": 0, "xp": 1, "hr": 2, "yr": 3, "hs": 4, "ys": 5, "grp_row": 6}
 
     def debug_buffer(self, name: str) -> torch.Tensor:

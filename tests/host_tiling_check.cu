@@ -42,7 +42,7 @@ int main() {
     for (int R = 8; R <= kRouterBM; R += 8) {
       const RouterStages rs = router_stages(n_pad, R);
       CHECK(rs.stages >= 2 && rs.stages <= kRouterMaxStages, "n_pad=%d R=%d stages=%d", n_pad, R, rs.stages);
-      CHECK(rs.kps == 1 || rs.kps == 2, "n_pad=%d R=%d kps=%d", n_pad, R, rs.kps);
+      CHECK(rs.kps >= 1 && rs.kps <= kRouterMaxKps, "n_pad=%d R=%d kps=%d", n_pad, R, rs.kps);
       CHECK(router_smem_bytes(n_pad, rs.kps, R, rs.stages) <= kRouterSmemBudget,
             "n_pad=%d R=%d bytes=%zu", n_pad, R, router_smem_bytes(n_pad, rs.kps, R, rs.stages));
       const uint32_t stage = router_stage_bytes(n_pad, rs.kps, R);
@@ -52,10 +52,28 @@ int main() {
             "n_pad=%d R=%d blocks past the stage", n_pad, R);
       CHECK(router_a_bytes(R) % 1024 == 0 && router_b_bytes(n_pad) % 1024 == 0 && stage % 1024 == 0,
             "n_pad=%d R=%d 1 KB alignment of the swizzled blocks", n_pad, R);
+      // the epilogue's logit rows (float4 stores) and the control block (mbarriers) after
+      // the 1 KB-aligned ring stay 16-byte aligned
+      CHECK(sizeof(RouterEpiSmem) % 16 == 0 && (router_ld(n_pad) * 4) % 16 == 0 &&
+                router_epi_bytes(n_pad) % 16 == 0,
+            "n_pad=%d epilogue scratch alignment", n_pad);
       uint32_t cols = 32;
       while (cols < 2u * (uint32_t)n_pad) cols <<= 1;
       CHECK(cols <= 512, "n_pad=%d TMEM columns %u", n_pad, cols);
-      CHECK(router_maxc(n_pad) * kRouterGroup >= n_pad, "n_pad=%d maxc=%d", n_pad, router_maxc(n_pad));
+      // a routing warp's 32 lanes hold ceil(MAXC / 4) columns each: all N_pad of them
+      CHECK((router_maxc(n_pad) + 3) / 4 * 32 >= n_pad, "n_pad=%d maxc=%d", n_pad, router_maxc(n_pad));
+    }
+  }
+  // the scan in the router's last CTA: (segment, expert) pairs fit its 512 threads and the
+  // segments cover every tile
+  for (int nr = 1; nr <= kMaxRouted; ++nr) {
+    for (int n_tiles = 1; n_tiles <= 700; ++n_tiles) {
+      int nseg = kScanThreads / nr;
+      if (nseg > n_tiles) nseg = n_tiles;
+      if (nseg < 1) nseg = 1;
+      const int seg_len = (n_tiles + nseg - 1) / nseg;
+      CHECK(nseg * nr <= kScanThreads && (long)nseg * seg_len >= n_tiles,
+            "nr=%d n_tiles=%d nseg=%d seg_len=%d", nr, n_tiles, nseg, seg_len);
     }
   }
   // combine: warps per row between 1 and one lane-wide vector batch per part

@@ -1,0 +1,81 @@
+"""Backward pass on the GPU against the oracle's pinned moe_backward (fp64).
+
+The library's gradients of L = sum_t dh_t . h_t + d_aux * aux -- du, d_centroids and d_bias
+-- element by element against the oracle on the same bf16-valued inputs and dh.  Tolerance,
+the forward's form: max|x - x_ref| <= 2e-2 max|x_ref| for each output, and the same for the
+expert part of du (du - dh).  Derivation: the GPU path rounds to bf16 (relative 2^-9) at
+most four times on any path into du (dY, dHmid, [da db], dX) with fp32 accumulation in
+between, about 4 * 2^-9 = 0.8 % of the expert part; d_centroids and d_bias are fp32 sums of
+dl, whose inputs (the gates' gradients dh . Y) carry one bf16 rounding of Y.
+"""
+import numpy as np
+import pytest
+import torch
+
+from mixture_experts_layer_65_b200 import build
+from mixture_experts_layer_65_b200 import workloads as W
+from mixture_experts_layer_65_b200.layer import MoELayer, to_device_tensor
+from oracle import moe_oracle as O
+
+pytestmark = pytest.mark.gpu
+TOL = 2e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib_ready():
+    build.build()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+
+
+def _err(got, ref):
+    return float(np.abs(got - ref).max()) / max(float(np.abs(ref).max()), 1e-30)
+
+
+SPECS = [
+    ("shared2_r16", dict(T=333, d=256, n_shared=2, n_routed=16, inter=192, top_k=4), 0.0),
+    ("no_shared", dict(T=700, d=256, n_shared=0, n_routed=16, inter=128, top_k=2), 1.0),
+    ("zipf_bias", dict(T=1000, d=256, n_shared=1, n_routed=16, inter=128, top_k=4, zipf_s=1.1), 1.0),
+    ("n63_top7", dict(T=520, d=320, n_shared=1, n_routed=63, inter=128, top_k=7), 1.0),
+    ("16b_shape", dict(T=2048, d=2048, n_shared=2, n_routed=64, inter=1408, top_k=6), 1.0),
+]
+
+
+@pytest.mark.parametrize("name,spec,d_aux", SPECS, ids=[s[0] for s in SPECS])
+def test_backward_matches_the_oracle(name, spec, d_aux):
+    w = W.make_workload("16b_prefill", alpha1=0.001, **spec)
+    rng = np.random.default_rng(11)
+    dh_bits = W.f32_to_bf16_bits(rng.standard_normal((w.T, w.d), dtype=np.float32))
+    layer = MoELayer.from_workload(w)
+    layer.backward_prepare()
+    u = to_device_tensor(w.u, "cuda")
+    out = layer.forward(u)
+    dh = to_device_tensor(dh_bits, "cuda")
+    grads = [layer.backward(u, out, dh, d_aux) for _ in range(2)]
+    torch.cuda.synchronize()
+    layer.device_status()
+    # deterministic: the second backward is bit for bit the first
+    for a, b in zip(grads[0], grads[1]):
+        assert torch.equal(a, b)
+    du, dcen, dbias = (g.float().cpu().numpy().astype(np.float64) for g in grads[0])
+    ref = O.moe_backward(w.u, w.centroids, w.w_gate, w.w_up, w.w_down, w.n_shared, w.top_k,
+                         w.alpha1, O.widen(dh_bits), d_aux=d_aux, bias=w.logit_bias)
+    dh64 = O.widen(dh_bits)
+    e_du = _err(du, ref.du)
+    slack = 2.0 ** -8 * np.maximum(np.abs(du), np.abs(ref.du))   # du's own bf16 rounding
+    e_part = float(np.maximum(np.abs(du - ref.du) - slack, 0).max()) / float(np.abs(ref.du - dh64).max())
+    e_cen, e_bias = _err(dcen, ref.d_centroids), _err(dbias, ref.d_bias)
+    print(f"{name}: du {e_du:.2e}, du expert part {e_part:.2e}, d_centroids {e_cen:.2e}, "
+          f"d_bias {e_bias:.2e}")
+    assert e_du <= TOL and e_part <= TOL
+    assert e_cen <= TOL and e_bias <= TOL
+    layer.close()
+
+
+def test_backward_refuses_unsupported_layers():
+    from mixture_experts_layer_65_b200 import _lib
+    w = W.make_workload("tiny")   # fp32 layer
+    layer = MoELayer.from_workload(w)
+    with pytest.raises(_lib.MoeError) as e:
+        layer.backward_prepare()
+    assert e.value.status == _lib.MOE_ERR_UNSUPPORTED
+    layer.close()

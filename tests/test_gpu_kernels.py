@@ -102,3 +102,56 @@ def test_intermediates_match_the_oracle(spec, e4m3):
         _close(ys, y_ref, "shared output")
     else:
         assert layer.debug_buffer("hs").numel() == 0
+
+
+@pytest.mark.parametrize("name", ["16b_prefill", "145b"])
+def test_full_size_intermediates_on_sampled_rows_of_every_expert(name):
+    """At full size (the launch configuration the benchmark times): for every routed expert,
+    its first and last rows and six random ones (the 145B layer's Zipf-skewed expert 0 holds
+    ~32 K rows, the longest tile chains), the SwiGLU activation and the expert output
+    against the oracle; the shared group's activations and summed output on sampled tokens;
+    the row copy byte for byte on those rows."""
+    w = W.make_workload(name)
+    layer = MoELayer.from_workload(w)
+    out = layer.forward(to_device_tensor(w.u, "cuda"))
+    torch.cuda.synchronize()
+    layer.device_status()
+    T, d, I, K, ks, nr = w.T, w.d, w.inter, w.top_k, w.n_shared, w.n_routed
+    idx = out.topk_idx.cpu().numpy()
+    slot = layer.debug_buffer("slot_row").cpu().numpy().reshape(T, K)
+    rng = np.random.default_rng(7)
+    picks = []                                  # (token, slot) pairs to check
+    for e in range(nr):
+        ts, kk = np.nonzero(idx == e)
+        if ts.size == 0:
+            continue
+        order = np.argsort(slot[ts, kk])
+        sel = np.unique(np.concatenate([[0, ts.size - 1], rng.integers(0, ts.size, 6)]))
+        picks += [(ts[order[i]], kk[order[i]], e) for i in sel]
+    picks = np.array(picks)
+    rows = torch.from_numpy(slot[picks[:, 0], picks[:, 1]].astype(np.int64)).cuda()
+    xp = layer.debug_buffer("xp").view(-1, d)[rows].cpu().view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(xp, w.u[picks[:, 0]])
+    hr = _f64(layer.debug_buffer("hr").view(-1, I)[rows])
+    yr = _f64(layer.debug_buffer("yr").view(-1, d)[rows])
+    worst_h = worst_y = 0.0
+    for e in np.unique(picks[:, 2]):
+        m = picks[:, 2] == e
+        x = w.u[picks[m, 0]]
+        g = ks + e
+        worst_h = max(worst_h, _close(hr[m], O.swiglu_hidden(x, w.w_gate[g], w.w_up[g]), f"hidden {e}"))
+        worst_y = max(worst_y, _close(yr[m], O.swiglu_ffn(x, w.w_gate[g], w.w_up[g], w.w_down[g]),
+                                      f"output {e}"))
+    toks = np.unique(np.concatenate([[0, T - 1], rng.integers(0, T, 30)]))
+    tt = torch.from_numpy(toks).cuda()
+    hs = _f64(layer.debug_buffer("hs").view(-1, ks * I)[tt])
+    ys = _f64(layer.debug_buffer("ys").view(-1, d)[tt])
+    y_ref = np.zeros((toks.size, d))
+    for j in range(ks):
+        _close(hs[:, j * I:(j + 1) * I], O.swiglu_hidden(w.u[toks], w.w_gate[j], w.w_up[j]),
+               f"hidden of shared expert {j}")
+        y_ref += O.swiglu_ffn(w.u[toks], w.w_gate[j], w.w_up[j], w.w_down[j])
+    _close(ys, y_ref, "shared output")
+    print(name, f"{len(picks)} routed rows of {len(np.unique(picks[:, 2]))} experts: "
+                f"hidden err {worst_h:.2e}, output err {worst_y:.2e}")
+    layer.close()
