@@ -400,9 +400,7 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
     H->router_kps = rs.kps;
     H->router_stages = rs.stages;
     H->router_smem = router_smem_bytes(H->n_pad, rs.kps, H->router_rows, rs.stages);
-    uint32_t cols = 32;
-    while (cols < 2u * (uint32_t)H->n_pad) cols <<= 1;
-    H->router_tmem_cols = cols;
+    H->router_tmem_cols = router_tmem_cols(H->n_pad);
     const void* rk = with_maxc(H->maxc, [](auto m) { return (const void*)router_tc_kernel<m()>; });
     MOE_CUDA(cudaFuncSetAttribute(rk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)H->router_smem));
     MOE_CUDA(cudaFuncSetAttribute((const void*)grouped_gemm_tc_kernel<kGateUpSwiGLU>,

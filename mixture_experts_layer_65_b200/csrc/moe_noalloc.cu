@@ -169,8 +169,7 @@ extern "C" moe_status moe_route_noalloc(const void* u, const void* centroids, co
   const RouterStages rs = router_stages(n_pad, rows);
   if (rs.stages < 2) return nfail(MOE_ERR_UNSUPPORTED, "moe_route_noalloc: router stages do not fit");
   const size_t smem = router_smem_bytes(n_pad, rs.kps, rows, rs.stages);
-  uint32_t cols = 32;
-  while (cols < 2u * (uint32_t)n_pad) cols <<= 1;
+  const uint32_t cols = router_tmem_cols(n_pad);
 
   ScanArgs sa{reinterpret_cast<int32_t*>(sc + kOffHist), reinterpret_cast<float*>(sc + kOffPsum),
               n_tiles, n_routed, T, /*has_shared=*/0,

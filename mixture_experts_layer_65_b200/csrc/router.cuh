@@ -14,12 +14,12 @@
 // token rows streamed by TMA, B = the padded centroid matrix; accumulator rows past R are
 // never read back); a CTA with several tiles (large T) overlaps the next tile's loads with
 // the epilogue.  Sixteen epilogue warps copy the logits (+ bias) to shared memory in passes
-// of 64 rows and route each row with one warp: the lanes hold the row's columns, the row
-// max and the top-k come from warp-wide redux max / min on 32-bit order-preserving keys
-// (max key, then the lowest index carrying it: exactly the stable ranking), the softmax
-// denominator from a fixed butterfly of shuffles.  The fp32 kernel and the decode-sized
-// bf16 kernel compute the same logits with FMA into the same shared-memory layout and share
-// the rest.
+// of 64 rows and work on each pass with eight threads per token row: row max and softmax
+// denominator by shuffles, the top-k by a bitonic sort of each thread's 64-bit (logit,
+// index) keys and three bitonic merges across the row's threads (or, for top_k > 8 or wide
+// rows, top_k rounds of a group-wide maximum).  The fp32 kernel and the decode-sized bf16
+// kernel compute the same logits with FMA into the same shared-memory layout and share the
+// rest.
 #pragma once
 
 #include <climits>
@@ -30,7 +30,8 @@ namespace moe {
 
 constexpr int kRouterBM = 128;          // MMA rows = largest token tile
 constexpr int kRouterPass = 64;         // token rows per epilogue pass
-constexpr int kRouterEpiThreads = 512;  // 16 warps, one token row at a time each
+constexpr int kRouterGroup = 8;         // threads per token row in the epilogue
+constexpr int kRouterEpiThreads = 512;  // kRouterPass * kRouterGroup
 constexpr int kRouterThreads = 64 + kRouterEpiThreads;   // warp 0 TMA, warp 1 MMA
 constexpr int kRouterMaxStages = 8;
 #ifndef MOE_ROUTER_MAX_KPS
@@ -83,6 +84,12 @@ inline int router_tile_rows(int T, int n_sms) {
   const int k = (per_sm + kRouterBM - 1) / kRouterBM;
   return (((per_sm + k - 1) / k) + 7) / 8 * 8;
 }
+// TMEM columns of the tc router: two tiles' accumulators (N_pad each) in flight, a power of
+// two >= 32.
+__host__ __device__ constexpr uint32_t router_tmem_cols(int n_pad) {
+  return 2u * (uint32_t)n_pad <= 32u ? 32u : 2u * (uint32_t)n_pad <= 64u ? 64u
+         : 2u * (uint32_t)n_pad <= 128u ? 128u : 2u * (uint32_t)n_pad <= 256u ? 256u : 512u;
+}
 // Parts the rows of a pass are split into for the per-expert sums.
 __host__ __device__ constexpr int router_psum_parts(int n_pad) {
   return kRouterEpiThreads / n_pad > 8 ? 8 : kRouterEpiThreads / n_pad;
@@ -102,110 +109,47 @@ __device__ __forceinline__ float key_logit(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
-constexpr int kRouteRows = 2;   // rows a routing warp works on together (independent chains)
+// Total order on (logit, expert): larger logit first; on equal logits the lower index.
+// NaN ranks as -inf and -0 as +0, so every slot gets a real index and equal values tie.
+__device__ __forceinline__ uint64_t route_key(float l, int i) {
+  uint32_t b = (l != l) ? 0xFF800000u : __float_as_uint(l);
+  if (b == 0x80000000u) b = 0u;
+  const uint32_t ord = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+  return (static_cast<uint64_t>(ord) << 32) | static_cast<uint64_t>(0xFFFFFFFFu - (uint32_t)i);
+}
 
-// Route kRouteRows rows of the pass with one warp.  rr[j]: the rows (in the pass; -1 = none);
-// their logits (bias added) are lg[rr][c] for c < N_pad.  Lane l holds columns l + 32 m.
-// Per row: the max (redux max of the keys), exp(l - max) written back in place, the
-// denominator (each lane's columns in order, then a butterfly of xor-shuffles 16, 8, 4, 2, 1,
-// so every lane holds the same sum), and top_k rounds of "largest key, then the lowest
-// column carrying it" (redux max, redux min), whose winner's key is then cleared.  Lane p
-// records round p: sel/gsel/mask of the tile row.  Rows past the tile or past T get zero
-// exp values and inv_sum 0.
-template <int MAXC>
-__device__ __forceinline__ void route_rows_warp(const int (&rr)[kRouteRows], int lane, int pass,
-                                                int tile, int R, int T, int n_routed, int n_pad,
-                                                int top_k, uint8_t* epi, const RouterOut& o) {
-  constexpr int MC = (MAXC + 3) / 4;   // columns per lane
-  RouterEpiSmem& S = *reinterpret_cast<RouterEpiSmem*>(epi);
-  float* lg = reinterpret_cast<float*>(epi + sizeof(RouterEpiSmem));
-  const int ld = router_ld(n_pad);
-  uint32_t key[kRouteRows][MC];
-  float ex[kRouteRows][MC];
-  bool valid[kRouteRows];
-  float inv[kRouteRows];
+__device__ __forceinline__ int key_index(uint64_t key) {
+  return (int)(0xFFFFFFFFu - (uint32_t)key);
+}
+
+// Descending bitonic sort of N keys held in registers.
+template <int N>
+__device__ __forceinline__ void bitonic_sort_desc(uint64_t (&k)[N]) {
 #pragma unroll
-  for (int j = 0; j < kRouteRows; ++j) {
-    const int tr = pass * kRouterPass + rr[j];
-    valid[j] = rr[j] >= 0 && tile * R + tr < T;
-    const float* row = lg + (size_t)(rr[j] < 0 ? 0 : rr[j]) * ld;
-    uint32_t kmax = 0u;
+  for (int size = 2; size <= N; size <<= 1) {
 #pragma unroll
-    for (int m = 0; m < MC; ++m) {
-      const int c = lane + 32 * m;
-      const bool in = valid[j] && c < n_routed;
-      ex[j][m] = in ? row[c] : 0.f;
-      key[j][m] = in ? logit_key(ex[j][m]) : 0u;
-      kmax = max(kmax, key[j][m]);
-      if (in && o.logits) o.logits[(size_t)(tile * R + tr) * n_routed + c] = ex[j][m];
-    }
-    kmax = __reduce_max_sync(0xffffffffu, kmax);
-    const float lmax = key_logit(kmax);
-    float part = 0.f;
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
 #pragma unroll
-    for (int m = 0; m < MC; ++m) {
-      const int c = lane + 32 * m;
-      ex[j][m] = (valid[j] && c < n_routed) ? __expf(ex[j][m] - lmax) : 0.f;
-      part += ex[j][m];
-    }
-#pragma unroll
-    for (int o2 = 16; o2 > 0; o2 >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o2);
-    inv[j] = valid[j] ? 1.0f / part : 0.f;
-  }
-  int my_e[kRouteRows];
-  float my_g[kRouteRows];
-#pragma unroll
-  for (int j = 0; j < kRouteRows; ++j) { my_e[j] = 0; my_g[j] = 0.f; }
-#pragma unroll 1
-  for (int p = 0; p < top_k; ++p) {
-#pragma unroll
-    for (int j = 0; j < kRouteRows; ++j) {
-      uint32_t bk = 0u;
-      int bc = 0x7fffffff;
-#pragma unroll
-      for (int m = 0; m < MC; ++m) {
-        if (key[j][m] > bk) { bk = key[j][m]; bc = lane + 32 * m; }   // ascending columns
+      for (int i = 0; i < N; ++i) {
+        const int l = i ^ stride;
+        if (l > i) {
+          const bool desc = (i & size) == 0;
+          const uint64_t x = k[i], y = k[l];
+          const bool sw = desc ? (x < y) : (x > y);
+          k[i] = sw ? y : x;
+          k[l] = sw ? x : y;
+        }
       }
-      const uint32_t gk = __reduce_max_sync(0xffffffffu, bk);
-      const int gc = (int)__reduce_min_sync(0xffffffffu, bk == gk ? (uint32_t)bc : 0x7fffffffu);
-      float eg = 0.f;
-#pragma unroll
-      for (int m = 0; m < MC; ++m) {
-        if (lane + 32 * m == gc) { eg = ex[j][m]; key[j][m] = 0u; }
-      }
-      eg = __shfl_sync(0xffffffffu, eg, gc & 31);
-      if (lane == p) { my_e[j] = gc; my_g[j] = eg * inv[j]; }
-    }
-  }
-#pragma unroll
-  for (int j = 0; j < kRouteRows; ++j) {
-    if (rr[j] < 0) continue;
-    float* row = lg + (size_t)rr[j] * ld;
-#pragma unroll
-    for (int m = 0; m < MC; ++m) {
-      const int c = lane + 32 * m;
-      if (c < n_pad) row[c] = ex[j][m];
-    }
-    if (lane == 0) S.inv_sum[rr[j]] = inv[j];
-    if (valid[j] && lane < top_k) {
-      const int tr = pass * kRouterPass + rr[j];
-      int e = my_e[j];
-      if (e < 0 || e >= n_routed) {
-        record_error(o.err, kErrRouteIndex);
-        e = 0;
-      }
-      S.sel[tr][lane] = e;
-      S.gsel[tr][lane] = my_g[j];
-      atomicOr(&S.mask[e][tr >> 5], 1u << (tr & 31));
     }
   }
 }
 
 // One epilogue pass: the pass's logit rows (bias added) are in lg[r][i] for r < rows,
-// i < N_pad, and the masks are zero (first pass) or hold the earlier passes' choices.  The
-// 16 warps route rows w, w + 16, ... of the pass, kRouteRows at a time; then the pass's
-// per-expert affinity sums are added to the earlier passes' parts.  `sync()` synchronises
-// the 512 threads.
+// i < N_pad, and the masks are zero (first pass) or hold the earlier passes' choices.
+// Thread tid (of 512) works on row r = tid / 8 of the pass (tile row 64 * pass + r) with
+// the eight threads of its row owning consecutive column blocks of C = N_pad / 8.  Writes
+// sel/gsel/mask for its rows and adds the pass's per-expert affinity sums into ppart.
+// `sync()` synchronises the 512 threads; returns with the scratch still in use.
 template <int MAXC, class Sync>
 __device__ __forceinline__ void router_pass(int tid, int pass, int tile, int R, int T,
                                             int n_routed, int n_pad, int top_k, uint8_t* epi,
@@ -213,15 +157,124 @@ __device__ __forceinline__ void router_pass(int tid, int pass, int tile, int R, 
   RouterEpiSmem& S = *reinterpret_cast<RouterEpiSmem*>(epi);
   float* lg = reinterpret_cast<float*>(epi + sizeof(RouterEpiSmem));
   const int ld = router_ld(n_pad);
+  const int r = tid >> 3, j = tid & 7;
+  const int tr = pass * kRouterPass + r;                  // row in the tile
   const int rows = min(kRouterPass, R - pass * kRouterPass);
-  const int warp = tid >> 5, lane = tid & 31;
-  constexpr int kWarps = kRouterEpiThreads / 32;
-  for (int r0 = warp; r0 < rows; r0 += kWarps * kRouteRows) {
-    int rr[kRouteRows];
+  const int C = n_pad >> 3;              // even: N_pad is a multiple of 16
+  const int c0 = j * C;
+  const int t = tile * R + tr;
+  const bool valid = r < rows && t < T;
+  float* row = lg + (size_t)r * ld;
+
+  // warps whose four rows all lie past the pass skip the per-row work (they still take
+  // part in every barrier)
+  if ((tid >> 5) * 4 < rows) {
+  // keys and the row max; rows past the tile or past T are treated as zeros
+  uint64_t key[MAXC];
+  float lmax = -INFINITY;
 #pragma unroll
-    for (int j = 0; j < kRouteRows; ++j) rr[j] = r0 + j * kWarps < rows ? r0 + j * kWarps : -1;
-    route_rows_warp<MAXC>(rr, lane, pass, tile, R, T, n_routed, n_pad, top_k, epi, o);
+  for (int k = 0; k < MAXC; k += 2) {
+    float2 x = make_float2(0.f, 0.f);
+    if (k < C && valid) x = *reinterpret_cast<const float2*>(row + c0 + k);
+    const bool in0 = k < C && c0 + k < n_routed, in1 = k < C && c0 + k + 1 < n_routed;
+    key[k] = in0 ? route_key(x.x, c0 + k) : 0ull;
+    key[k + 1] = in1 ? route_key(x.y, c0 + k + 1) : 0ull;
+    if (valid && o.logits) {   // the logits (bias added), kept for the backward
+      if (in0) o.logits[(size_t)t * n_routed + c0 + k] = x.x;
+      if (in1) o.logits[(size_t)t * n_routed + c0 + k + 1] = x.y;
+    }
+    if (in0) lmax = fmaxf(lmax, x.x);
+    if (in1) lmax = fmaxf(lmax, x.y);
   }
+#pragma unroll
+  for (int m = 1; m < kRouterGroup; m <<= 1)
+    lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, m));
+
+  // exp(l - max) in place, denominator: column order within a thread, then a fixed tree
+  float part = 0.f;
+#pragma unroll
+  for (int k = 0; k < MAXC; k += 2) {
+    if (k < C) {
+      const float2 x = *reinterpret_cast<const float2*>(row + c0 + k);
+      const float e0 = (valid && c0 + k < n_routed) ? __expf(x.x - lmax) : 0.f;
+      const float e1 = (valid && c0 + k + 1 < n_routed) ? __expf(x.y - lmax) : 0.f;
+      part += e0;
+      part += e1;
+      *reinterpret_cast<float2*>(row + c0 + k) = make_float2(e0, e1);
+    }
+  }
+#pragma unroll
+  for (int m = 1; m < kRouterGroup; m <<= 1) part += __shfl_xor_sync(0xffffffffu, part, m);
+  const float inv_sum = 1.0f / part;
+  if (j == 0) S.inv_sum[r] = valid ? inv_sum : 0.f;
+  __syncwarp();   // the row's exp values (written by the eight threads of a warp) are read below
+
+  auto record = [&](int p, uint64_t g) {
+    int e = key_index(g);
+    if (e < 0 || e >= n_routed) {
+      record_error(o.err, kErrRouteIndex);
+      e = 0;
+    }
+    if (valid) {
+      S.sel[tr][p] = e;
+      S.gsel[tr][p] = row[e] * inv_sum;
+      atomicOr(&S.mask[e][tr >> 5], 1u << (tr & 31));
+    }
+  };
+
+  if (MAXC <= 8 && top_k <= 8) {
+    // sort the thread's keys (padded to 8 with zeros), then three bitonic merges with the
+    // partner threads: every thread of the row ends up with the row's 8 largest keys
+    uint64_t kk[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) kk[i] = i < MAXC ? key[i < MAXC ? i : 0] : 0ull;
+    bitonic_sort_desc<8>(kk);
+#pragma unroll
+    for (int m = 1; m < kRouterGroup; m <<= 1) {
+      uint64_t pk[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) pk[i] = __shfl_xor_sync(0xffffffffu, kk[i], m);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) kk[i] = kk[i] > pk[7 - i] ? kk[i] : pk[7 - i];   // bitonic
+#pragma unroll
+      for (int stride = 4; stride > 0; stride >>= 1) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int l = i ^ stride;
+          if (l > i) {
+            const uint64_t x = kk[i], y = kk[l];
+            kk[i] = x > y ? x : y;
+            kk[l] = x > y ? y : x;
+          }
+        }
+      }
+    }
+    // thread j of the row records rank j
+    uint64_t mine = 0ull;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mine = i == j ? kk[i] : mine;
+    if (j < top_k) record(j, mine);
+  } else {
+    // top_k rounds: the group's largest remaining key; its owner records it and drops it
+#pragma unroll 1
+    for (int p = 0; p < top_k; ++p) {
+      uint64_t best = key[0];
+#pragma unroll
+      for (int k = 1; k < MAXC; ++k) best = key[k] > best ? key[k] : best;
+      uint64_t g = best;
+#pragma unroll
+      for (int m = 1; m < kRouterGroup; m <<= 1) {
+        const uint64_t y = __shfl_xor_sync(0xffffffffu, g, m);
+        g = y > g ? y : g;
+      }
+      if (best == g) {   // keys are distinct (distinct indices): exactly one owner
+        record(p, g);
+#pragma unroll
+        for (int k = 0; k < MAXC; ++k) key[k] = key[k] == g ? 0ull : key[k];
+      }
+    }
+  }
+  }   // warps with rows
   sync();
 
   // the pass's per-expert affinity sums: row parts, added to the earlier passes' parts
@@ -231,7 +284,7 @@ __device__ __forceinline__ void router_pass(int tid, int pass, int tile, int R, 
     const int pp = idx / n_pad, c = idx - pp * n_pad;
     const int r0 = pp * RP, r1 = min(rows, r0 + RP);
     float a = 0.f;
-    for (int r = r0; r < r1; ++r) a += lg[(size_t)r * ld + c] * S.inv_sum[r];
+    for (int rr = r0; rr < r1; ++rr) a += lg[(size_t)rr * ld + c] * S.inv_sum[rr];
     S.ppart[pp][c] = pass == 0 ? a : S.ppart[pp][c] + a;
   }
 }
@@ -292,7 +345,7 @@ struct RouterTcArgs {
   int kps, stages;     // k-blocks per stage (1 .. 4), stages in the ring
   int tile_rows;       // R: tokens per tile (<= 128, multiple of 8); the U map's box height
   int n_tiles;         // tiles, handed out round-robin over the CTAs
-  uint32_t tmem_cols;  // power of two >= 2 * n_pad: two accumulators
+  uint32_t tmem_cols;  // router_tmem_cols(n_pad): two tiles' accumulators in flight
   const float* bias;   // [>= n_routed] (zeros where no bias)
   RouterOut out;
 };

@@ -59,7 +59,7 @@ struct ScanSmem {
   double aux[kMaxRouted];
 };
 
-constexpr int kScanBatch = 8;   // independent loads in flight per thread
+constexpr int kScanBatch = 16;  // independent loads in flight per thread
 
 // Threads tid < 512 of the last router CTA; `sync()` synchronises exactly those threads.
 // The tiles' histograms and sums were written by other CTAs (published with a fence before

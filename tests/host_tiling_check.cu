@@ -57,11 +57,11 @@ int main() {
       CHECK(sizeof(RouterEpiSmem) % 16 == 0 && (router_ld(n_pad) * 4) % 16 == 0 &&
                 router_epi_bytes(n_pad) % 16 == 0,
             "n_pad=%d epilogue scratch alignment", n_pad);
-      uint32_t cols = 32;
-      while (cols < 2u * (uint32_t)n_pad) cols <<= 1;
-      CHECK(cols <= 512, "n_pad=%d TMEM columns %u", n_pad, cols);
-      // a routing warp's 32 lanes hold ceil(MAXC / 4) columns each: all N_pad of them
-      CHECK((router_maxc(n_pad) + 3) / 4 * 32 >= n_pad, "n_pad=%d maxc=%d", n_pad, router_maxc(n_pad));
+      // two tiles' accumulators fit the 512 TMEM columns (a power of two >= 32)
+      const uint32_t cols = router_tmem_cols(n_pad);
+      CHECK(cols <= 512 && cols >= 2u * n_pad && (cols & (cols - 1)) == 0,
+            "n_pad=%d TMEM columns %u", n_pad, cols);
+      CHECK(router_maxc(n_pad) * kRouterGroup >= n_pad, "n_pad=%d maxc=%d", n_pad, router_maxc(n_pad));
     }
   }
   // the scan in the router's last CTA: (segment, expert) pairs fit its 512 threads and the

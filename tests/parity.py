@@ -137,9 +137,9 @@ def gate_error_bound(w, logits: np.ndarray, idx: np.ndarray, path: str | None = 
     perturbation of x_i plus the largest perturbation of any x_j (each: the accumulation
     bound of the logit, the bias add and the subtraction, half an ulp each), plus the error
     of the fast exponential at x_i and at the worst x_j (2 + 1.2 |x| ulp, its documented
-    accuracy), plus N_pad/8 + 5 roundings: the denominator's sum (each of 8 threads adds its
-    N_pad/8 columns, then a tree of three adds), its reciprocal and the product.  First
-    order; the factor 1.01 covers the higher-order terms.
+    accuracy), plus N_pad/8 + 5 roundings: the denominator's sum (each of the row's 8
+    threads adds its N_pad/8 columns, then a tree of three adds), its reciprocal and the
+    product.  First order; the factor 1.01 covers the higher-order terms.
     """
     B = logit_error_bound(w, path)
     x = logits - logits.max(axis=1, keepdims=True)

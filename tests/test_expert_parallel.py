@@ -144,15 +144,24 @@ def _run_ep(w, bounds, comm_for_rank):
 
 
 def _check(w, bounds, res, full):
+    # bit for bit moe_forward's outputs when every rank routes on the same kernel as the
+    # full batch (a rank of <= 128 tokens uses the SIMT router, which sums the logits in
+    # another order); the oracle comparison below holds either way
+    import types
+    same = all(P.router_path(types.SimpleNamespace(dtype=w.dtype, T=hi - lo, d=w.d)) ==
+               P.router_path(w) for lo, hi in zip(bounds[:-1], bounds[1:]))
     for call in range(2):
         h = torch.cat([r[call].h for r in res])
         idx = torch.cat([r[call].topk_idx for r in res])
         gates = torch.cat([r[call].topk_w for r in res])
-        assert torch.equal(idx, full.topk_idx), f"call {call}: routed indices differ"
-        assert torch.equal(gates, full.topk_w), f"call {call}: gates differ"
-        assert torch.equal(h, full.h), f"call {call}: h differs from moe_forward"
-        for r in res:
-            assert torch.equal(r[call].expert_counts, full.expert_counts)
+        if same:
+            assert torch.equal(idx, full.topk_idx), f"call {call}: routed indices differ"
+            assert torch.equal(gates, full.topk_w), f"call {call}: gates differ"
+            assert torch.equal(h, full.h), f"call {call}: h differs from moe_forward"
+            for r in res:
+                assert torch.equal(r[call].expert_counts, full.expert_counts)
+        for r in res:   # every rank holds the same global counts
+            assert torch.equal(r[call].expert_counts, res[0][call].expert_counts)
         g = P.GpuOut(h=h.float().cpu().numpy().astype(np.float64),
                      topk_idx=idx.cpu().numpy().astype(np.int64),
                      topk_w=gates.cpu().numpy().astype(np.float64),

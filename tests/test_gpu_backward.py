@@ -1,12 +1,15 @@
 """Backward pass on the GPU against the oracle's pinned moe_backward (fp64).
 
-The library's gradients of L = sum_t dh_t . h_t + d_aux * aux -- du, d_centroids and d_bias
--- element by element against the oracle on the same bf16-valued inputs and dh.  Tolerance,
+The library's gradients of L = sum_t dh_t . h_t + d_aux * aux -- du, d_centroids, d_bias and
+the expert weight gradients -- element by element against the oracle on the same
+bf16-valued inputs and dh.  Tolerance,
 the forward's form: max|x - x_ref| <= 2e-2 max|x_ref| for each output, and the same for the
 expert part of du (du - dh).  Derivation: the GPU path rounds to bf16 (relative 2^-9) at
 most four times on any path into du (dY, dHmid, [da db], dX) with fp32 accumulation in
 between, about 4 * 2^-9 = 0.8 % of the expert part; d_centroids and d_bias are fp32 sums of
-dl, whose inputs (the gates' gradients dh . Y) carry one bf16 rounding of Y.
+dl, whose inputs (the gates' gradients dh . Y) carry one bf16 rounding of Y; a weight
+gradient is an fp32-accumulated sum over the expert's rows of products of two bf16 factors
+that carry at most three such roundings, compared against each expert's own maximum.
 """
 import numpy as np
 import pytest
@@ -56,7 +59,7 @@ def test_backward_matches_the_oracle(name, spec, d_aux):
     # deterministic: the second backward is bit for bit the first
     for a, b in zip(grads[0], grads[1]):
         assert torch.equal(a, b)
-    du, dcen, dbias = (g.float().cpu().numpy().astype(np.float64) for g in grads[0])
+    du, dcen, dbias, dwg, dwu, dwd = (g.float().cpu().numpy().astype(np.float64) for g in grads[0])
     ref = O.moe_backward(w.u, w.centroids, w.w_gate, w.w_up, w.w_down, w.n_shared, w.top_k,
                          w.alpha1, O.widen(dh_bits), d_aux=d_aux, bias=w.logit_bias)
     dh64 = O.widen(dh_bits)
@@ -64,8 +67,19 @@ def test_backward_matches_the_oracle(name, spec, d_aux):
     slack = 2.0 ** -8 * np.maximum(np.abs(du), np.abs(ref.du))   # du's own bf16 rounding
     e_part = float(np.maximum(np.abs(du - ref.du) - slack, 0).max()) / float(np.abs(ref.du - dh64).max())
     e_cen, e_bias = _err(dcen, ref.d_centroids), _err(dbias, ref.d_bias)
+    # weight gradients per expert (an expert's own scale: routed experts see few tokens)
+    e_w = 0.0
+    for name_w, got, want in (("d_w_gate", dwg, ref.d_w_gate), ("d_w_up", dwu, ref.d_w_up),
+                              ("d_w_down", dwd, ref.d_w_down)):
+        for g in range(got.shape[0]):
+            if not np.any(want[g]):   # an expert without tokens: exactly zero
+                assert not np.any(got[g]), (name_w, g)
+                continue
+            eg = _err(got[g], want[g])
+            e_w = max(e_w, eg)
+            assert eg <= TOL, (name_w, g, eg)
     print(f"{name}: du {e_du:.2e}, du expert part {e_part:.2e}, d_centroids {e_cen:.2e}, "
-          f"d_bias {e_bias:.2e}")
+          f"d_bias {e_bias:.2e}, weight gradients (worst expert) {e_w:.2e}")
     assert e_du <= TOL and e_part <= TOL
     assert e_cen <= TOL and e_bias <= TOL
     layer.close()

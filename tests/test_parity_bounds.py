@@ -66,6 +66,7 @@ def _emulate_gates(w, logits32: np.ndarray, idx: np.ndarray) -> np.ndarray:
 
 CASES = [
     ("mma16", dict(T=48, d=512, n_routed=64, top_k=6, dtype="bf16"), False),
+    ("mma16", dict(T=16, d=512, n_routed=200, top_k=8, dtype="bf16"), True),    # wide rows
     ("mma16", dict(T=48, d=512, n_routed=64, top_k=6, dtype="bf16"), True),
     ("mma16", dict(T=32, d=1024, n_routed=16, top_k=2, dtype="bf16", zipf_s=1.1), True),
     ("lanes", dict(T=16, d=384, n_routed=64, top_k=6, dtype="bf16"), False),
