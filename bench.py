@@ -87,7 +87,7 @@ PEAK_KEY = {"burst": "bf16_tflops", "sustained": "bf16_tflops_sustained"}
 def workload_desc(w, n_gpus: int) -> dict:
     return {"workload": f"{w.name}: T={w.T} d={w.d} shared={w.n_shared} routed={w.n_routed} "
                         f"inter={w.inter} top_k={w.top_k} {w.dtype}"
-                        f"{' (gate/up e4m3)' if getattr(w, 'gate_up_e4m3', False) else ''}",
+                        f"{(' (gate/up and down e4m3)' if getattr(w, 'down_e4m3', False) else ' (gate/up e4m3)') if getattr(w, 'gate_up_e4m3', False) else ''}",
             "T_per_gpu": w.T, "d": w.d, "n_shared": w.n_shared, "n_routed": w.n_routed,
             "inter": w.inter, "top_k": w.top_k, "global_batch": w.T * n_gpus,
             "parallelism": f"dp{n_gpus}"}
@@ -215,7 +215,8 @@ def oracle_tokens_per_s(w, seconds: float) -> tuple[float, dict]:
     def run(n):
         t0 = time.perf_counter()
         O.moe_forward(w.u[:n], w.centroids, w.w_gate, w.w_up, w.w_down, w.n_shared, w.top_k,
-                      w.alpha1, bias=w.logit_bias, gate_up_e4m3=w.gate_up_e4m3)
+                      w.alpha1, bias=w.logit_bias, gate_up_e4m3=w.gate_up_e4m3,
+                      down_e4m3=w.down_e4m3)
         return time.perf_counter() - t0
 
     # grow the sample until one call takes about `seconds` (the oracle has a per-call cost
@@ -247,7 +248,8 @@ def run_reference(args, rank: int, world: int):
 
     t0 = time.perf_counter()
     O.moe_forward(w.u[:16], w.centroids, w.w_gate, w.w_up, w.w_down, w.n_shared, w.top_k,
-                  w.alpha1, bias=w.logit_bias, gate_up_e4m3=w.gate_up_e4m3)
+                  w.alpha1, bias=w.logit_bias, gate_up_e4m3=w.gate_up_e4m3,
+                      down_e4m3=w.down_e4m3)
     per_tok = (time.perf_counter() - t0) / 16
     n = int(max(1, min(w.T, budget / max(per_tok, 1e-9))))
     times = []
@@ -255,7 +257,8 @@ def run_reference(args, rank: int, world: int):
         s = (i * n) % max(1, w.T - n + 1)
         t0 = time.perf_counter()
         O.moe_forward(w.u[s:s + n], w.centroids, w.w_gate, w.w_up, w.w_down, w.n_shared,
-                      w.top_k, w.alpha1, bias=w.logit_bias, gate_up_e4m3=w.gate_up_e4m3)
+                      w.top_k, w.alpha1, bias=w.logit_bias, gate_up_e4m3=w.gate_up_e4m3,
+                      down_e4m3=w.down_e4m3)
         if i >= args.warmup:
             times.append(time.perf_counter() - t0)
     tot = sum(times)
@@ -436,20 +439,20 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     # dense e4m3 : bf16 ratio (4.5 : 2.25 PFLOP/s), and the token rows are quantised (one
     # extra kernel, timed in the permute slot)
     e4m3 = bool(getattr(w, "gate_up_e4m3", False))
-    tensor_ratio = {k: (2.0 if (e4m3 and k == "gate_up_gemm") else 1.0) for k in KERNELS}
+    e4m3_down = bool(getattr(w, "down_e4m3", False))
+    tensor_ratio = {k: (2.0 if ((e4m3 and k == "gate_up_gemm") or (e4m3_down and k == "down_gemm"))
+                        else 1.0) for k in KERNELS}
     if e4m3:
         work["permute"] = ("hbm", w.T * w.d * 3 + w.T * 4)   # quantise: bf16 in, e4m3 + scale out
     # with a shared group the paired bf16 GEMM copies the routed rows itself (its copy
     # warps run beside the shared group's tiles): no permute kernel is launched
-    # the scan runs in the router's last CTA: its slot is the empty gap between the two
-    fused_permute = layer.kernels_per_forward - (1 if e4m3 else 0) == len(KERNELS) - 2
+    fused_permute = (layer.kernels_per_forward - (1 if e4m3 else 0) -
+                     ((1 + (w.n_shared > 0)) if e4m3_down else 0)) == len(KERNELS) - 1
     for k in KERNELS:
         kind, amount = work[k]
         avg_ms = kernel_ms[k] / max(1, n_rec)
         ent = {"avg_ms": avg_ms, "share": kernel_ms[k] / max(1e-12, sum(kernel_ms.values()))}
-        if k == "scan":
-            ent.update(fused_into="router")
-        elif k == "permute" and fused_permute and not e4m3:
+        if k == "permute" and fused_permute and not e4m3:
             ent.update(fused_into="gate_up_gemm")
         elif kind == "tensor":
             ach = amount / (avg_ms * 1e-3) / 1e12
@@ -459,6 +462,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                        frac_of_sustained=ach / (tensor_ratio[k] * peaks["bf16_tflops_sustained"]))
             if tensor_ratio[k] != 1.0:
                 ent.update(operands="e4m3", peak_note="measured bf16 peak x 2 (nominal dense e4m3/bf16)")
+            if k == "down_gemm" and e4m3_down:
+                ent.update(slot_includes="the activations' e4m3 quantisation before the GEMM")
         elif kind == "hbm":
             ach = amount / (avg_ms * 1e-3) / 1e9
             ent.update(bound="hbm", achieved=ach, unit="GB/s", frac=ach / peaks["hbm_gbs"])
@@ -493,7 +498,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16 (gate/up GEMM on e4m3 operands)" if e4m3 else w.dtype,
+        "dtype": ("bf16 (expert GEMMs on e4m3 operands)" if e4m3_down else
+                  "bf16 (gate/up GEMM on e4m3 operands)" if e4m3 else w.dtype),
         "data": "synthetic (seeded N(0,1) tokens, N(0,0.02) random-init experts, no trained weights)",
         "config": dict(workload_desc(w, world),
                        l2=f"inputs rotate over {n_buf} token buffers "

@@ -58,7 +58,13 @@ typedef enum {
  * scale = fp32(a / 448).  The gate/up products are computed on q with fp32 accumulation
  * and multiplied by the two row scales; the router, the down projection, the residual and
  * the combine are those of MOE_BF16.  Needs d % 128 == 0. */
-typedef enum { MOE_FP32 = 0, MOE_BF16 = 1, MOE_BF16_E4M3_GATEUP = 2 } moe_dtype;
+/* MOE_BF16_E4M3: MOE_BF16_E4M3_GATEUP whose down projection runs on e4m3 operands too, with
+ * the same per-row rule: each row of the SwiGLU activations (as the layer stores them, in
+ * bf16) and each W_down row (one output channel) gets its own scale; the K_s shared
+ * experts, which run as one group, quantise the concatenation of their activations and of
+ * their W_down rows (one scale per concatenated row).  Needs d % 128 == 0 and
+ * inter % 128 == 0. */
+typedef enum { MOE_FP32 = 0, MOE_BF16 = 1, MOE_BF16_E4M3_GATEUP = 2, MOE_BF16_E4M3 = 3 } moe_dtype;
 
 /* Layer description.  All weight pointers are DEVICE pointers in `dtype`, read only
  * during moe_create (the library keeps its own re-laid-out copy; the caller may free
@@ -75,8 +81,9 @@ typedef enum { MOE_FP32 = 0, MOE_BF16 = 1, MOE_BF16_E4M3_GATEUP = 2 } moe_dtype;
  *   w_up       [n_shared + n_routed, inter, d]
  *   w_down     [n_shared + n_routed, d, inter]
  * bf16 layers need d % 64 == 0 and inter % 64 == 0 (MOE_ERR_UNSUPPORTED otherwise);
- * MOE_BF16_E4M3_GATEUP layers also d % 128 == 0; fp32 layers need d % 4 == 0.  The
- * weights of MOE_BF16_E4M3_GATEUP layers are given in bf16 and quantised by moe_create. */
+ * MOE_BF16_E4M3_GATEUP layers also d % 128 == 0, MOE_BF16_E4M3 layers d % 128 == 0 and
+ * inter % 128 == 0; fp32 layers need d % 4 == 0.  The weights of the e4m3 variants are
+ * given in bf16 and quantised by moe_create. */
 typedef struct {
   int32_t T;
   int32_t d;

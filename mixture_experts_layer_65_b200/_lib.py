@@ -11,7 +11,7 @@ HEADER = os.path.join(os.path.dirname(_HERE), "include", "moe.h")
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_OOM, \
     MOE_ERR_DEVICE_CHECK = range(6)
-MOE_FP32, MOE_BF16, MOE_BF16_E4M3_GATEUP = 0, 1, 2
+MOE_FP32, MOE_BF16, MOE_BF16_E4M3_GATEUP, MOE_BF16_E4M3 = 0, 1, 2, 3
 STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
                 3: "MOE_ERR_CUDA", 4: "MOE_ERR_OOM", 5: "MOE_ERR_DEVICE_CHECK"}
 

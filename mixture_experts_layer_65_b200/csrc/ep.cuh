@@ -24,7 +24,7 @@ struct EpLayoutArgs {
   ScanArgs scan;                // tile_hist = recv_counts (tiles = source ranks)
 };
 
-// One CTA of 512 threads (world * n_local <= 256 blocks): the blocks' offsets in the
+// One CTA of kScanThreads threads (world * n_local <= 256 blocks): the blocks' offsets in the
 // received buffer (an exclusive prefix in (s, e) order), then the group layout of the local
 // experts (scan_tail: group starts, tile tables, each block's destination row).
 static __global__ void __launch_bounds__(kScanThreads, 1) ep_layout_kernel(EpLayoutArgs a) {

@@ -10,7 +10,8 @@
 // expert K_s times as wide).
 //
 //   mode kGateUpSwiGLU:  Hmid[r, :] = SiLU(X W_gate^T) * (X W_up^T)      (K = d)
-//   mode kDown:          Y[r, :]    = Hmid W_down^T                        (K = I_g)
+//   mode kDown:          Y[r, :]    = Hmid W_down^T                        (K = I_g; with
+//                        e4m3 operands, scaled by the A row's and W_down row's scales)
 //                        (also any plain D = A B^T with a bf16 output: the backward's
 //                        dHmid = dY W_down and dX = [da db] [W_gate; W_up] products)
 //   mode kGateUpBwd:     the gate/up products recomputed, a = X W_gate^T, b = X W_up^T, and
@@ -503,23 +504,56 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
           }
         }
       } else {
+        // plain D = A B^T, bf16 out: each of the quadrant's WPQ warps takes kGemmBN / WPQ
+        // columns; with e4m3 operands every accumulator is first multiplied by its A row's
+        // and B row's scales (16 columns at a time, within the smaller register budget)
+        constexpr int CW = kGemmBN / WPQ;
+        if constexpr (F8) {
+          const float sa = row_ok ? __ldg((c.shared ? a.sa_shared : a.sa_routed) + orow) : 0.f;
+          const float* sbv = c.shared ? a.sb_shared : a.sb_routed + (int64_t)c.e * a.sb_routed_stride;
 #pragma unroll 1
-        for (int cc = half * (kGemmBN / 2); cc < (half + 1) * (kGemmBN / 2); cc += 32) {
-          const int col = c.n * kGemmBN + cc;
-          if (col >= cols) break;
-          uint32_t v[32];
-          __syncwarp();
-          tmem_ld32(trow + static_cast<uint32_t>(cc), v);
-          tmem_ld_wait(v);
-          uint32_t pk[16];
+          for (int cc = part * CW; cc < (part + 1) * CW; cc += 16) {
+            const int col = c.n * kGemmBN + cc;
+            if (col >= cols) break;
+            uint32_t v[16];
+            __syncwarp();
+            tmem_ld16(trow + static_cast<uint32_t>(cc), v);
+            tmem_ld_wait16(v);
+            const float4* sb4 = reinterpret_cast<const float4*>(sbv + col);
+            uint32_t pk[8];
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-          if (row_ok) {
-            uint4* dst = reinterpret_cast<uint4*>(out + orow * ld + col);
+            for (int q4 = 0; q4 < 4; ++q4) {
+              const float4 b4 = __ldg(sb4 + q4);
+              pk[2 * q4] = pack_bf16x2(__uint_as_float(v[4 * q4]) * sa * b4.x,
+                                       __uint_as_float(v[4 * q4 + 1]) * sa * b4.y);
+              pk[2 * q4 + 1] = pack_bf16x2(__uint_as_float(v[4 * q4 + 2]) * sa * b4.z,
+                                           __uint_as_float(v[4 * q4 + 3]) * sa * b4.w);
+            }
+            if (row_ok) {
+              uint4* dst = reinterpret_cast<uint4*>(out + orow * ld + col);
+              dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            }
+          }
+        } else {
+#pragma unroll 1
+          for (int cc = part * CW; cc < (part + 1) * CW; cc += 32) {
+            const int col = c.n * kGemmBN + cc;
+            if (col >= cols) break;
+            uint32_t v[32];
+            __syncwarp();
+            tmem_ld32(trow + static_cast<uint32_t>(cc), v);
+            tmem_ld_wait(v);
+            uint32_t pk[16];
 #pragma unroll
-            for (int x = 0; x < 4; ++x)
-              dst[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+            for (int i = 0; i < 16; ++i)
+              pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+            if (row_ok) {
+              uint4* dst = reinterpret_cast<uint4*>(out + orow * ld + col);
+#pragma unroll
+              for (int x = 0; x < 4; ++x)
+                dst[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+            }
           }
         }
       }

@@ -4,9 +4,8 @@
 // Launch sequence of moe_forward (one stream, no host synchronisation, every launch with
 // programmatic dependent launch):
 //   1. router      logits -> softmax -> top-k, gates, per-tile histograms / ranks / sums
-//                  (tensor-core kernel; a SIMT kernel for decode-sized batches and fp32);
-//                  its last CTA then runs the scan: per-expert counts, padded offsets,
-//                  tile tables, balance loss
+//                  (tensor-core kernel; a SIMT kernel for decode-sized batches and fp32)
+//   2. scan        per-expert counts, padded offsets, tile tables, balance loss
 //   3. quantise    (e4m3 gate/up layers only) e4m3 token rows + per-row scales
 //   4. permute     token rows -> expert-contiguous rows (top_k copies per token); on bf16
 //                  layers with shared experts this copy runs inside step 5 instead
@@ -83,7 +82,8 @@ struct moe_handle {
   moe_cfg cfg;
   int device = 0, n_sms = 0;
   bool bf16 = true;        // bf16 storage (MOE_BF16 and MOE_BF16_E4M3_GATEUP)
-  bool e4m3 = false;       // gate/up GEMM on e4m3 operands (MOE_BF16_E4M3_GATEUP)
+  bool e4m3 = false;       // gate/up GEMM on e4m3 operands (MOE_BF16_E4M3_GATEUP, MOE_BF16_E4M3)
+  bool e4m3_down = false;  // down GEMM on e4m3 operands too (MOE_BF16_E4M3)
   int es = 2;              // element size
   int G = 0, has_shared = 0, inter_shared = 0;
   int n_tiles = 0;         // router tiles
@@ -116,11 +116,14 @@ struct moe_handle {
   void *xp = nullptr, *hs = nullptr, *hr = nullptr, *ys = nullptr, *yr = nullptr;
   int* err = nullptr;
   int* copy_done = nullptr;   // counter of the fused permute (paired bf16 path with a shared group)
-  int* done_ctas = nullptr;   // router CTAs finished (the last one runs the scan, resets it)
   // e4m3 gate/up: quantised weights (interleaved rows), per-row scales, quantised tokens
   void *w8_gu_s = nullptr, *w8_gu_r = nullptr, *u8 = nullptr;
   float *sw_s = nullptr, *sw_r = nullptr, *su = nullptr, *su_p = nullptr;
   CUtensorMap tmU8, tmXp8, tmW8guS, tmW8guR;
+  // e4m3 down projection: quantised W_down rows and activation rows, their scales
+  void *w8_d_s = nullptr, *w8_d_r = nullptr, *h8s = nullptr, *h8r = nullptr;
+  float *sw_d_s = nullptr, *sw_d_r = nullptr, *sh_s = nullptr, *sh_r = nullptr;
+  CUtensorMap tmH8s, tmH8r, tmW8dS, tmW8dR;
   bool fuse_permute = false;
   // staging for moe_forward_host
   void *u_dev = nullptr, *h_dev = nullptr;
@@ -211,13 +214,16 @@ moe_status validate(const moe_cfg* c) {
     return fail(MOE_ERR_INVALID_ARG, "top_k=%d outside [1, n_routed=%d]", c->top_k, c->n_routed);
   if (c->top_k > kMaxTopK)
     return fail(MOE_ERR_UNSUPPORTED, "top_k=%d above %d", c->top_k, kMaxTopK);
-  if (c->dtype != MOE_FP32 && c->dtype != MOE_BF16 && c->dtype != MOE_BF16_E4M3_GATEUP)
-    return fail(MOE_ERR_INVALID_ARG, "dtype=%d is not MOE_FP32, MOE_BF16 or MOE_BF16_E4M3_GATEUP",
-                c->dtype);
+  if (c->dtype != MOE_FP32 && c->dtype != MOE_BF16 && c->dtype != MOE_BF16_E4M3_GATEUP &&
+      c->dtype != MOE_BF16_E4M3)
+    return fail(MOE_ERR_INVALID_ARG,
+                "dtype=%d is not MOE_FP32, MOE_BF16, MOE_BF16_E4M3_GATEUP or MOE_BF16_E4M3", c->dtype);
   if (!c->centroids || !c->w_gate || !c->w_up || !c->w_down)
     return fail(MOE_ERR_INVALID_ARG, "a weight pointer is NULL");
-  if (c->dtype == MOE_BF16_E4M3_GATEUP && c->d % 128)
-    return fail(MOE_ERR_UNSUPPORTED, "e4m3 gate/up layers need d %% 128 == 0 (d=%d)", c->d);
+  if ((c->dtype == MOE_BF16_E4M3_GATEUP || c->dtype == MOE_BF16_E4M3) && c->d % 128)
+    return fail(MOE_ERR_UNSUPPORTED, "e4m3 layers need d %% 128 == 0 (d=%d)", c->d);
+  if (c->dtype == MOE_BF16_E4M3 && c->inter % 128)
+    return fail(MOE_ERR_UNSUPPORTED, "e4m3 down projections need inter %% 128 == 0 (inter=%d)", c->inter);
   if (c->dtype != MOE_FP32) {
     if (c->d % 64 || c->inter % 64)
       return fail(MOE_ERR_UNSUPPORTED, "bf16 layers need d %% 64 == 0 and inter %% 64 == 0 (d=%d inter=%d)",
@@ -241,9 +247,11 @@ int32_t moe_abi_version(void) { return MOE_ABI_VERSION; }
 const char* moe_last_error(void) { return g_last_error.c_str(); }
 
 int32_t moe_kernels_per_forward(const moe_handle* handle) {
-  // six timing slots; the scan has none of its own (router's last CTA), the permute none
-  // when the gate/up GEMM copies the rows, and e4m3 layers add the token quantisation
-  return handle ? kKernelsPerForward - 1 - (handle->fuse_permute ? 1 : 0) + (handle->e4m3 ? 1 : 0) : 0;
+  // six timing slots; the permute has no kernel when the gate/up GEMM copies the rows, and
+  // e4m3 layers add the token quantisation
+  return handle ? kKernelsPerForward - (handle->fuse_permute ? 1 : 0) + (handle->e4m3 ? 1 : 0) +
+                      (handle->e4m3_down ? 1 + handle->has_shared : 0)
+                : 0;
 }
 
 size_t moe_device_bytes(const moe_handle* handle) { return handle ? handle->bytes : 0; }
@@ -263,7 +271,8 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
   H->cfg.centroids = H->cfg.w_gate = H->cfg.w_up = H->cfg.w_down = nullptr;
   H->cfg.logit_bias = nullptr;
   H->bf16 = c.dtype != MOE_FP32;
-  H->e4m3 = c.dtype == MOE_BF16_E4M3_GATEUP;
+  H->e4m3 = c.dtype == MOE_BF16_E4M3_GATEUP || c.dtype == MOE_BF16_E4M3;
+  H->e4m3_down = c.dtype == MOE_BF16_E4M3;
   H->es = H->bf16 ? 2 : 4;
   H->has_shared = c.n_shared > 0 ? 1 : 0;
   H->inter_shared = c.n_shared * c.inter;
@@ -351,6 +360,18 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
     MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->sw_r), 2 * nr * I * 4));
     MOE_CUDA(launch_quant(H->w_gu_r, (int64_t)(2 * nr * I), (int)d, H->w8_gu_r, H->sw_r, H->n_sms, st));
   }
+  if (H->e4m3_down) {
+    // e4m3 copies of the W_down rows (output channels), one fp32 scale per row; the shared
+    // group's rows are the K_s experts' rows side by side
+    if (ks) {
+      MOE_TRY(dalloc(H, &H->w8_d_s, d * Is));
+      MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->sw_d_s), d * 4));
+      MOE_CUDA(launch_quant(H->w_d_s, (int64_t)d, (int)Is, H->w8_d_s, H->sw_d_s, H->n_sms, st));
+    }
+    MOE_TRY(dalloc(H, &H->w8_d_r, nr * d * I));
+    MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->sw_d_r), nr * d * 4));
+    MOE_CUDA(launch_quant(H->w_d_r, (int64_t)(nr * d), (int)I, H->w8_d_r, H->sw_d_r, H->n_sms, st));
+  }
 
   // ---- workspace
   const size_t T = c.T, K = c.top_k, nt = H->n_tiles;
@@ -367,8 +388,6 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
   MOE_CUDA(cudaMemsetAsync(H->err, 0, 256, st));
   MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->copy_done), 256));
   MOE_CUDA(cudaMemsetAsync(H->copy_done, 0, 256, st));
-  MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->done_ctas), 256));
-  MOE_CUDA(cudaMemsetAsync(H->done_ctas, 0, 256, st));
   const size_t rc = (size_t)H->rows_cap, tp = (size_t)H->T_pad;
   MOE_TRY(dalloc(H, &H->xp, rc * d * (H->e4m3 ? 1 : es)));   // e4m3 rows on that path
   if (H->e4m3) {
@@ -381,6 +400,14 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
   }
   MOE_TRY(dalloc(H, &H->hr, rc * I * es));
   MOE_TRY(dalloc(H, &H->yr, rc * d * es));
+  if (H->e4m3_down) {
+    MOE_TRY(dalloc(H, &H->h8r, rc * I));
+    MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->sh_r), rc * 4));
+    if (ks) {
+      MOE_TRY(dalloc(H, &H->h8s, tp * Is));
+      MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->sh_s), tp * 4));
+    }
+  }
   if (ks) {
     MOE_TRY(dalloc(H, &H->hs, tp * Is * es));
     MOE_TRY(dalloc(H, &H->ys, tp * d * es));
@@ -428,6 +455,8 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
       if (H->e4m3) {
         MOE_CUDA(cudaFuncSetAttribute((const void*)grouped_gemm_tc_kernel<kGateUpSwiGLU, true>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmemBytes));
+        MOE_CUDA(cudaFuncSetAttribute((const void*)grouped_gemm_tc_kernel<kDown, true>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmemBytes));
         lc.blockDim = dim3(gemm_threads(true), 1, 1);
         MOE_CUDA(cudaOccupancyMaxActiveClusters(
             &clusters, (const void*)grouped_gemm_tc_kernel<kGateUpSwiGLU, true>, &lc));
@@ -456,6 +485,17 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
            encode_3d_e4m3(&H->tmW8guR, H->w8_gu_r, d, 2 * I, nr, kGemmBN / 2);
       if (ks) ok = ok && encode_2d_e4m3(&H->tmW8guS, H->w8_gu_s, d, 2 * Is, kGemmBN / 2);
       else H->tmW8guS = H->tmW8guR;
+    }
+    if (H->e4m3_down) {
+      ok = ok && encode_2d_e4m3(&H->tmH8r, H->h8r, I, rc, 128) &&
+           encode_3d_e4m3(&H->tmW8dR, H->w8_d_r, I, d, nr, kGemmBN / 2);
+      if (ks)
+        ok = ok && encode_2d_e4m3(&H->tmH8s, H->h8s, Is, tp, 128) &&
+             encode_2d_e4m3(&H->tmW8dS, H->w8_d_s, Is, d, kGemmBN / 2);
+      else {
+        H->tmH8s = H->tmH8r;
+        H->tmW8dS = H->tmW8dR;
+      }
     }
     if (!ok) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for a weight/workspace tensor");
     if (H->small) {
@@ -530,8 +570,8 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
               c.inter, d, H->bm, H->tile_rows, bn1, bn2, c.alpha1, expert_counts, aux_loss,
               H->psum_total,
               H->tile_base, H->grp_row, H->ts1, H->ts2,
-              H->fuse_permute ? H->copy_done : nullptr, H->done_ctas, H->bwd ? H->ts3 : nullptr};
-  RouterOut ro{topk_idx, topk_w, H->topk_rank, H->tile_hist, H->tile_psum, H->err, sa,
+              H->fuse_permute ? H->copy_done : nullptr, H->bwd ? H->ts3 : nullptr};
+  RouterOut ro{topk_idx, topk_w, H->topk_rank, H->tile_hist, H->tile_psum, H->err,
                H->bwd ? H->logits : nullptr};
   CUtensorMap tmU, tmUr;
   tick(H, stream, 0);
@@ -564,7 +604,9 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
   }
   MOE_CUDA(cudaGetLastError());
 
-  tick(H, stream, 1);   // (the scan runs in the router's last CTA: an empty slot)
+  tick(H, stream, 1);
+  launch_pdl(scan_kernel, dim3(1), dim3(kScanThreads), 0, stream, sa);
+  MOE_CUDA(cudaGetLastError());
 
   PermuteArgs pa{static_cast<const uint8_t*>(u), topk_idx, H->topk_rank, H->tile_base, H->slot_row,
                  static_cast<uint8_t*>(H->xp), T, K, nr, (int)H->rows_cap, H->router_rows,
@@ -648,7 +690,25 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
     g2.cols_routed = d;
     g2.err = H->err;
     tick(H, stream, 4);
-    launch_pdl(grouped_gemm_tc_kernel<kDown>, dim3(H->gemm_grid), dim3(kGemmThreads), kGemmSmemBytes, stream,  H->tmHs, H->tmHr, H->tmWdS, H->tmWdR, g2);
+    if (H->e4m3_down) {
+      // the activations' rows to e4m3 (the shared group's rows span its K_s experts), then the
+      // down GEMM on e4m3 operands with the row scales applied in its epilogue
+      if (H->has_shared)
+        MOE_CUDA(launch_quant(H->hs, H->T_pad, Is, H->h8s, H->sh_s, H->n_sms, stream));
+      MOE_CUDA(launch_quant(H->hr, H->rows_cap, I, H->h8r, H->sh_r, H->n_sms, stream));
+      g2.kb_shared = Is / (2 * kGemmBK);   // k-blocks of 128 e4m3 values
+      g2.kb_routed = I / (2 * kGemmBK);
+      g2.sa_shared = H->sh_s;
+      g2.sa_routed = H->sh_r;
+      g2.sb_shared = H->sw_d_s;
+      g2.sb_routed = H->sw_d_r;
+      g2.sb_routed_stride = d;
+      launch_pdl(grouped_gemm_tc_kernel<kDown, true>, dim3(H->gemm_grid_f8), dim3(gemm_threads(true)),
+                 kGemmSmemBytes, stream, H->tmH8s, H->tmH8r, H->tmW8dS, H->tmW8dR, g2);
+    } else {
+      launch_pdl(grouped_gemm_tc_kernel<kDown>, dim3(H->gemm_grid), dim3(kGemmThreads), kGemmSmemBytes,
+                 stream, H->tmHs, H->tmHr, H->tmWdS, H->tmWdR, g2);
+    }
     MOE_CUDA(cudaGetLastError());
   } else {
     const size_t ks = c.n_shared;

@@ -7,8 +7,7 @@
 // (NCCL).  The arithmetic is the layer's: the same router, grouped GEMMs and combine
 // kernels as moe_forward, so a token's output does not depend on how the experts are split.
 //
-//   moe_ep_dispatch  router (+ scan, in its last CTA) with unpadded expert offsets, then the
-//                    row copy: every (token, slot) row in expert order = destination-rank
+//   moe_ep_dispatch  router and scan (unpadded expert offsets), then the row copy: every (token, slot) row in expert order = destination-rank
 //                    order, which is what the caller's all-to-all sends
 //   moe_ep_experts   layout scan of the received blocks, rows into padded expert groups,
 //                    gate/up + SwiGLU and down GEMMs of the local experts, rows back into the
@@ -44,7 +43,7 @@ struct moe_ep_handle {
   void *w_gu_s = nullptr, *w_gu_r = nullptr, *w_d_s = nullptr, *w_d_r = nullptr;
   // dispatch
   int32_t *topk_rank = nullptr, *slot_row = nullptr, *tile_hist = nullptr, *tile_base = nullptr;
-  int32_t *disp_grp = nullptr, *disp_ts1 = nullptr, *disp_ts2 = nullptr, *done_ctas = nullptr;
+  int32_t *disp_grp = nullptr, *disp_ts1 = nullptr, *disp_ts2 = nullptr;
   int* err = nullptr;
   float *tile_psum = nullptr, *psum_total = nullptr;
   // local experts
@@ -164,8 +163,6 @@ moe_status ep_create_impl(const moe_cfg& c, int32_t rank, int32_t world, int64_t
   MOE_TRY(M.alloc_t(&H->disp_grp, nr * 4));
   MOE_TRY(M.alloc_t(&H->disp_ts1, (nr + 1) * 4));
   MOE_TRY(M.alloc_t(&H->disp_ts2, (nr + 1) * 4));
-  MOE_TRY(M.alloc_t(&H->done_ctas, 256));
-  MOE_CUDA(cudaMemsetAsync(H->done_ctas, 0, 256, st));
   MOE_TRY(M.alloc_t(&H->err, 256));
   MOE_CUDA(cudaMemsetAsync(H->err, 0, 256, st));
   // ---- local experts
@@ -294,8 +291,8 @@ moe_status moe_ep_dispatch(moe_ep_handle* H, const void* u, int32_t* topk_idx, f
   ScanArgs sa{H->tile_hist, H->tile_psum, H->n_tiles, nr, T, /*has_shared=*/0, /*inter_shared=*/0,
               c.inter, d, /*bm=*/1, /*tile_rows=*/kPairBM, kGemmBN / 2, kGemmBN, c.alpha1,
               expert_counts, aux_loss, H->psum_total, H->tile_base, H->disp_grp, H->disp_ts1,
-              H->disp_ts2, /*copy_done=*/nullptr, H->done_ctas};
-  RouterOut ro{topk_idx, topk_w, H->topk_rank, H->tile_hist, H->tile_psum, H->err, sa};
+              H->disp_ts2, /*copy_done=*/nullptr};
+  RouterOut ro{topk_idx, topk_w, H->topk_rank, H->tile_hist, H->tile_psum, H->err};
   if (H->small_router) {
     RouterSmallArgs ra{static_cast<const __nv_bfloat16*>(u),
                        static_cast<const __nv_bfloat16*>(H->centroids), H->bias, T, d, nr, K, 1, ro};
@@ -317,6 +314,8 @@ moe_status moe_ep_dispatch(moe_ep_handle* H, const void* u, int32_t* topk_idx, f
       return 0;
     });
   }
+  MOE_CUDA(cudaGetLastError());
+  launch_pdl(scan_kernel, dim3(1), dim3(kScanThreads), 0, stream, sa);
   MOE_CUDA(cudaGetLastError());
   PermuteArgs pa{static_cast<const uint8_t*>(u), topk_idx, H->topk_rank, H->tile_base, H->slot_row,
                  static_cast<uint8_t*>(send_rows), T, K, nr, T * K, H->router_rows, d * 2, H->err};
@@ -344,7 +343,7 @@ moe_status moe_ep_experts(moe_ep_handle* H, const void* recv_rows, const int32_t
                   ScanArgs{recv_counts, /*tile_psum=*/nullptr, H->world, H->n_local, /*T=*/1,
                            /*has_shared=*/0, /*inter_shared=*/0, I, d, kPairBM, kPairBM, kGemmBN / 2,
                            kGemmBN, 0.f, H->local_counts, /*aux_loss=*/nullptr, /*psum_total=*/nullptr,
-                           H->block_dst, H->grp_row, H->ts1, H->ts2, nullptr, nullptr}};
+                           H->block_dst, H->grp_row, H->ts1, H->ts2, nullptr}};
   launch_pdl(ep_layout_kernel, dim3(1), dim3(kScanThreads), 0, stream, la);
   MOE_CUDA(cudaGetLastError());
   const unsigned mgrid = (unsigned)((n_recv + kEpMoveWarps - 1) / kEpMoveWarps);

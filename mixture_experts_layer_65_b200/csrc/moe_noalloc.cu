@@ -1,9 +1,9 @@
 // moe_noalloc.cu -- moe_route_noalloc: the router step (routing, gates, expert counts,
 // balance loss) for callers that cannot allocate device memory.
 //
-// It launches the same bf16 tcgen05 router kernel as moe_forward (whose last CTA runs the
-// scan); the per-tile histograms, ranks and affinity sums, the scan's tables and the CTA
-// counter live in one fixed file-scope device array instead of a handle's workspace.  The array exists once per
+// It launches the same bf16 tcgen05 router kernel and scan kernel as moe_forward; the
+// per-tile histograms, ranks and affinity sums and the scan's tables live in one fixed
+// file-scope device array instead of a handle's workspace.  The array exists once per
 // GPU that loads this library and stays there until the process exits.
 #include <mutex>
 
@@ -27,8 +27,7 @@ constexpr size_t kOffGrp = kOffPsumTot + kMaxRouted * 4;                        
 constexpr size_t kOffTs1 = kOffGrp + (kMaxRouted + 64) * 4;                             // [N_r + 1] i32
 constexpr size_t kOffTs2 = kOffTs1 + (kMaxRouted + 64) * 4;                             // [N_r + 1] i32
 constexpr size_t kOffErr = kOffTs2 + (kMaxRouted + 64) * 4;                             // error word
-constexpr size_t kOffDone = kOffErr + 256;                                             // router CTA counter
-constexpr size_t kOffZeroBias = kOffDone + 256;                                        // [N_r] f32 zeros
+constexpr size_t kOffZeroBias = kOffErr + 256;                                         // [N_r] f32 zeros
 constexpr size_t kScratchBytes = kOffZeroBias + kMaxRouted * 4;
 static_assert(kScratchBytes <= MOE_NOALLOC_SCRATCH_BYTES, "scratch layout exceeds the stated size");
 
@@ -147,12 +146,9 @@ extern "C" moe_status moe_route_noalloc(const void* u, const void* centroids, co
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream_);
   unsigned char* sc = S.scratch;
   int32_t* err = reinterpret_cast<int32_t*>(sc + kOffErr);
-  int32_t* done = reinterpret_cast<int32_t*>(sc + kOffDone);
   float* zero_bias = reinterpret_cast<float*>(sc + kOffZeroBias);
-  // the array keeps the previous call's contents: clear what must start at zero (the error
-  // word, the router's CTA counter -- its last CTA also resets it -- and the zero bias)
+  // the array keeps the previous call's contents: clear what must start at zero
   if (cudaMemsetAsync(err, 0, sizeof(int32_t), st) != cudaSuccess ||
-      cudaMemsetAsync(done, 0, sizeof(int32_t), st) != cudaSuccess ||
       (!logit_bias && cudaMemsetAsync(zero_bias, 0, (size_t)n_routed * 4, st) != cudaSuccess))
     return nfail(MOE_ERR_CUDA, "moe_route_noalloc: cudaMemsetAsync on the scratch failed");
 
@@ -179,10 +175,9 @@ extern "C" moe_status moe_route_noalloc(const void* u, const void* centroids, co
               aux_loss, reinterpret_cast<float*>(sc + kOffPsumTot),
               reinterpret_cast<int32_t*>(sc + kOffBase), reinterpret_cast<int32_t*>(sc + kOffGrp),
               reinterpret_cast<int32_t*>(sc + kOffTs1), reinterpret_cast<int32_t*>(sc + kOffTs2),
-              /*copy_done=*/nullptr, done};
+              /*copy_done=*/nullptr};
   RouterOut ro{topk_idx, topk_w, reinterpret_cast<int32_t*>(sc + kOffRank),
-               reinterpret_cast<int32_t*>(sc + kOffHist), reinterpret_cast<float*>(sc + kOffPsum), err,
-               sa};
+               reinterpret_cast<int32_t*>(sc + kOffHist), reinterpret_cast<float*>(sc + kOffPsum), err};
   RouterTcArgs ra{T, d, n_routed, n_pad, top_k, rs.kps, rs.stages, rows, n_tiles, cols,
                   logit_bias ? logit_bias : zero_bias, ro};
   const int grid = n_tiles < S.n_sms ? n_tiles : S.n_sms;
@@ -193,6 +188,8 @@ extern "C" moe_status moe_route_noalloc(const void* u, const void* centroids, co
                  : mc == 16 ? launch_router<16>(tmU, tmE, ra, grid, smem, st)
                             : launch_router<32>(tmU, tmE, ra, grid, smem, st);
   if (e != cudaSuccess) return nfail(MOE_ERR_CUDA, "moe_route_noalloc: router launch failed");
+  launch_pdl(scan_kernel, dim3(1), dim3(kScanThreads), 0, st, sa);
+  if (cudaGetLastError() != cudaSuccess) return nfail(MOE_ERR_CUDA, "moe_route_noalloc: scan launch failed");
   if (device_error &&
       cudaMemcpyAsync(device_error, err, sizeof(int32_t), cudaMemcpyDeviceToDevice, st) != cudaSuccess)
     return nfail(MOE_ERR_CUDA, "moe_route_noalloc: copying the device error word failed");

@@ -1,6 +1,6 @@
 // router.cuh -- fused router: centroid GEMM, softmax over the routed experts, top-k with
 // lower-index tie-break, gates, per-tile expert histograms / within-tile ranks and
-// per-tile affinity sums; the last CTA then runs the scan (scan.cuh).
+// per-tile affinity sums (the scan kernel of scan.cuh turns them into the layer's totals).
 //
 // DeepSeekMoE (deepforge.srivtx.xyz article), "Routing in a classic MoE layer":
 // s_i = softmax_i(u^T e_i), g_i = s_i for the top-K affinities, else 0; "Top-k routing,
@@ -48,7 +48,6 @@ struct RouterOut {
   int32_t* tile_hist;   // [n_tiles, n_routed]
   float* tile_psum;     // [n_tiles, n_routed]  sum over the tile's tokens of s[t, i]
   int* err;
-  ScanArgs scan;        // run by the last CTA (scan.cuh)
   float* logits;        // [T, n_routed] the logits (bias added) for the backward, or nullptr
 };
 
@@ -60,9 +59,7 @@ struct alignas(16) RouterEpiSmem {
   float gsel[kRouterBM][kMaxTopK];         // their gates s[t, e]
   float inv_sum[kRouterPass];              // 1 / softmax denominator (0 for rows past T)
   float ppart[8][kMaxRouted];              // per-expert sums over row parts of the tile
-  int last;                                // router_finish: this CTA finished last
 };
-static_assert(sizeof(RouterEpiSmem) >= sizeof(ScanSmem), "the scan reuses the epilogue scratch");
 static_assert(sizeof(RouterEpiSmem) % 16 == 0, "the logit rows after the scratch need 16-byte alignment");
 
 // Epilogue scratch: RouterEpiSmem, then the logit rows of one pass lg[64][ld] (fp32, bias
@@ -561,7 +558,6 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant_
       router_tile_outputs(tid, tile, a.tile_rows, a.T, a.n_routed, a.n_pad, a.top_k, epi, a.out);
       sync();   // scratch free for the next tile
     }
-    router_finish(a.out.scan, tid, &SM.last, epi, sync);
   }
 
   tc_fence_before();
@@ -616,7 +612,6 @@ __global__ void __launch_bounds__(kRouterEpiThreads) router_simt_kernel(RouterSi
                     sync);
   __syncthreads();
   router_tile_outputs(tid, tile, kRouterPass, a.T, a.n_routed, n_pad, a.top_k, smem_raw, a.out);
-  router_finish(a.out.scan, tid, &SM.last, smem_raw, sync);
 }
 
 // ------------------------------------------------------------------------ bf16, few tokens
@@ -703,7 +698,6 @@ __global__ void __launch_bounds__(kRouterEpiThreads) router_small_kernel(RouterS
   router_pass<MAXC>(tid, 0, tile, R, a.T, a.n_routed, n_pad, a.top_k, smem_raw, a.out, sync);
   __syncthreads();
   router_tile_outputs(tid, tile, R, a.T, a.n_routed, n_pad, a.top_k, smem_raw, a.out);
-  router_finish(a.out.scan, tid, &SM.last, smem_raw, sync);
 }
 
 }  // namespace moe

@@ -10,8 +10,9 @@
 // aux = alpha_1 * sum_i (count_i / T) * (psum_i / T).  Every sum runs in a fixed order, so the
 // results do not depend on scheduling.
 //
-// It runs inside the router kernels: the last router CTA to finish (counted with one atomic
-// per CTA, no waiting) runs scan_tail with 512 threads.
+// It runs as a kernel of its own, one CTA of 1024 threads, launched right after the router
+// (programmatic dependent launch hides its launch); the expert-parallel layout kernel runs
+// the same scan over received blocks.
 #pragma once
 
 #include "ptx.cuh"
@@ -20,7 +21,7 @@ namespace moe {
 
 constexpr int kMaxTopK = 16;
 constexpr int kMaxRouted = 256;
-constexpr int kScanThreads = 512;   // threads that run scan_tail
+constexpr int kScanThreads = 1024;  // threads that run scan_tail (one CTA)
 
 struct ScanArgs {
   const int32_t* tile_hist;   // [n_tiles, n_routed]
@@ -42,8 +43,6 @@ struct ScanArgs {
   int32_t* ts1;               // [G + 1] tile prefix of the gate/up GEMM
   int32_t* ts2;               // [G + 1] tile prefix of the down GEMM
   int32_t* copy_done;         // counter of the fused GEMM's copy warps, zeroed here; or nullptr
-  int32_t* done_ctas;         // router CTAs finished so far (the last one runs the scan and
-                              // resets it to 0 for the next forward)
   int32_t* ts3;               // [G + 1] tile prefix of a GEMM with N = the group's
                               // intermediate width at bn2 columns per tile (the backward's
                               // dHmid GEMM), or nullptr
@@ -61,9 +60,8 @@ struct ScanSmem {
 
 constexpr int kScanBatch = 16;  // independent loads in flight per thread
 
-// Threads tid < 512 of the last router CTA; `sync()` synchronises exactly those threads.
-// The tiles' histograms and sums were written by other CTAs (published with a fence before
-// their count), so they are read through L2.
+// The kScanThreads threads of one CTA; `sync()` synchronises them.  The tiles' histograms
+// and sums were written by the previous kernel; they are read through L2.
 template <class Sync>
 __device__ void scan_tail(const ScanArgs& a, int tid, uint8_t* smem, Sync sync) {
   ScanSmem& S = *reinterpret_cast<ScanSmem*>(smem);
@@ -205,25 +203,12 @@ __device__ void scan_tail(const ScanArgs& a, int tid, uint8_t* smem, Sync sync) 
   }
 }
 
-// Called once per router CTA by its 512 epilogue threads after its last tile's outputs are
-// written: publish them, count the CTA, and if it is the last one, run the scan and reset
-// the counter.  `flag` is a shared-memory word; `scratch` holds a ScanSmem (free by now).
-template <class Sync>
-__device__ __forceinline__ void router_finish(const ScanArgs& a, int tid, int* flag,
-                                              uint8_t* scratch, Sync sync) {
-  __threadfence();   // this thread's tile outputs, visible GPU-wide before the count
-  sync();
-  if (tid == 0) {
-    const int prev = atomicAdd(a.done_ctas, 1);
-    *flag = prev == (int)(gridDim.x * gridDim.y * gridDim.z) - 1;
-  }
-  sync();
-  const bool last = *flag != 0;
-  sync();   // everyone has read the flag before the scratch is reused
-  if (!last) return;
-  __threadfence();   // acquire side: the other CTAs' outputs, read through L2 below
-  scan_tail(a, tid, scratch, sync);
-  if (tid == 0) *a.done_ctas = 0;
+// One CTA of kScanThreads threads, launched after the router.
+static __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a) {
+  pdl_launch_dependents();
+  pdl_wait();
+  __shared__ __align__(16) uint8_t smem[sizeof(ScanSmem)];
+  scan_tail(a, threadIdx.x, smem, [] { __syncthreads(); });
 }
 
 }  // namespace moe

@@ -2,7 +2,7 @@
 //
 // DeepSeekMoE (deepforge.srivtx.xyz article), "Top-k routing, from affinities to gates":
 // a production layer groups the tokens of each expert so that every expert runs one
-// dense GEMM chain over its rows.  After the scan (scan.cuh, run by the router's last CTA)
+// dense GEMM chain over its rows.  After the scan (scan.cuh)
 // has placed every (router tile, expert) in the expert-contiguous row space, the permute
 // copies each token row to its top_k destinations (order inside an expert = ascending token
 // id): as a kernel of its own, or inside the copy warps of the gate/up GEMM.

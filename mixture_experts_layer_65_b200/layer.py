@@ -42,12 +42,16 @@ class MoELayer:
     def __init__(self, *, T: int, d: int, n_routed: int, n_shared: int, top_k: int, inter: int,
                  dtype: str, alpha1: float, centroids: torch.Tensor, w_gate: torch.Tensor,
                  w_up: torch.Tensor, w_down: torch.Tensor, logit_bias: torch.Tensor | None = None,
-                 gate_up_e4m3: bool = False):
+                 gate_up_e4m3: bool = False, down_e4m3: bool = False):
         """gate_up_e4m3 (bf16 layers): the gate/up GEMM runs on per-row scaled e4m3
-        operands (MOE_BF16_E4M3_GATEUP in include/moe.h); the weights are still given in bf16."""
+        operands (MOE_BF16_E4M3_GATEUP in include/moe.h); down_e4m3 (with gate_up_e4m3): the
+        down GEMM too (MOE_BF16_E4M3).  The weights are still given in bf16."""
         if gate_up_e4m3 and dtype != "bf16":
             raise ValueError("gate_up_e4m3 needs a bf16 layer")
+        if down_e4m3 and not gate_up_e4m3:
+            raise ValueError("down_e4m3 comes with gate_up_e4m3 (the MOE_BF16_E4M3 layer)")
         self.gate_up_e4m3 = gate_up_e4m3
+        self.down_e4m3 = down_e4m3
         self.T, self.d, self.n_routed, self.n_shared = T, d, n_routed, n_shared
         self.top_k, self.inter, self.alpha1 = top_k, inter, alpha1
         self.dtype = dtype
@@ -60,6 +64,7 @@ class MoELayer:
             raise ValueError("logit_bias must be a float32 CUDA tensor")
         cfg = MoeCfg(T=T, d=d, n_routed=n_routed, n_shared=n_shared, top_k=top_k, inter=inter,
                      dtype=(_lib.MOE_FP32 if dtype != "bf16" else
+                            _lib.MOE_BF16_E4M3 if down_e4m3 else
                             _lib.MOE_BF16_E4M3_GATEUP if gate_up_e4m3 else _lib.MOE_BF16),
                      alpha1=alpha1,
                      centroids=_ptr(centroids), logit_bias=_ptr(logit_bias), w_gate=_ptr(w_gate),
@@ -78,7 +83,8 @@ class MoELayer:
                    centroids=to_device_tensor(w.centroids, dev),
                    w_gate=to_device_tensor(w.w_gate, dev), w_up=to_device_tensor(w.w_up, dev),
                    w_down=to_device_tensor(w.w_down, dev), logit_bias=bias,
-                   gate_up_e4m3=getattr(w, "gate_up_e4m3", False))
+                   gate_up_e4m3=getattr(w, "gate_up_e4m3", False),
+                   down_e4m3=getattr(w, "down_e4m3", False))
 
     # -------------------------------------------------------------------------- calls
     def alloc_outputs(self) -> MoEOutput:

@@ -55,6 +55,10 @@ CONFIGS: dict[str, dict] = {
     # reduced-precision variant; same draws as "16b_prefill")
     "16b_prefill_e4m3": dict(T=16384, d=2048, n_shared=2, n_routed=64, inter=1408, top_k=6,
                              dtype="bf16", alpha1=0.001, zipf_s=None, gate_up_e4m3=True),
+    # the same layer with both expert GEMMs on e4m3 operands
+    "16b_prefill_e4m3_experts": dict(T=16384, d=2048, n_shared=2, n_routed=64, inter=1408,
+                                     top_k=6, dtype="bf16", alpha1=0.001, zipf_s=None,
+                                     gate_up_e4m3=True, down_e4m3=True),
 }
 
 _STREAMS = ("u", "centroids", "w_gate", "w_up", "w_down")
@@ -110,6 +114,7 @@ class Workload:
     w_down: np.ndarray
     logit_bias: np.ndarray | None
     gate_up_e4m3: bool = False     # bf16 layer whose gate/up products take e4m3 operands
+    down_e4m3: bool = False        # ... and whose down products too (needs gate_up_e4m3)
 
     @property
     def n_experts(self) -> int:
@@ -118,7 +123,7 @@ class Workload:
     def spec(self) -> dict:
         return dict(T=self.T, d=self.d, n_shared=self.n_shared, n_routed=self.n_routed,
                     inter=self.inter, top_k=self.top_k, dtype=self.dtype, alpha1=self.alpha1,
-                    gate_up_e4m3=self.gate_up_e4m3)
+                    gate_up_e4m3=self.gate_up_e4m3, down_e4m3=self.down_e4m3)
 
 
 def _draw(seed_seq, shape, std: float, dtype: str) -> np.ndarray:
@@ -179,4 +184,5 @@ def make_workload(name: str = "tiny", seed: int = 0, threads: int | None = None,
     return Workload(name=name, T=T, d=d, n_shared=ks, n_routed=nr, inter=inter, top_k=top_k,
                     dtype=dtype, alpha1=float(spec["alpha1"]), u=u, centroids=cen,
                     w_gate=w_gate, w_up=w_up, w_down=w_down, logit_bias=bias,
-                    gate_up_e4m3=bool(spec.get("gate_up_e4m3", False)))
+                    gate_up_e4m3=bool(spec.get("gate_up_e4m3", False)),
+                    down_e4m3=bool(spec.get("down_e4m3", False)))

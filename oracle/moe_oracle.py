@@ -45,7 +45,8 @@ import numpy as np
 __all__ = ["widen", "router_logits", "affinity_softmax", "select_topk", "route",
            "swiglu_hidden", "swiglu_ffn", "balance_stats", "moe_forward", "near_tie_tokens",
            "brute_force_layer", "Routing", "LayerOut", "E4M3_MAX", "e4m3_round",
-           "quantize_rows_e4m3", "swiglu_ffn_backward", "moe_backward", "LayerGrads"]
+           "quantize_rows_e4m3", "bf16_round", "swiglu_ffn_backward", "moe_backward",
+           "LayerGrads"]
 
 
 def widen(a) -> np.ndarray:
@@ -120,9 +121,16 @@ def swiglu_hidden(x, w_gate, w_up, gate_up_e4m3: bool = False) -> np.ndarray:
     return _silu(a) * b
 
 
-def swiglu_ffn(x, w_gate, w_up, w_down, gate_up_e4m3: bool = False) -> np.ndarray:
-    """FFN(x) = W_down (SiLU(W_gate x) * (W_up x)); x [n, d], W_gate/W_up [I, d], W_down [d, I]."""
-    return swiglu_hidden(x, w_gate, w_up, gate_up_e4m3) @ widen(w_down).T
+def swiglu_ffn(x, w_gate, w_up, w_down, gate_up_e4m3: bool = False,
+               down_e4m3: bool = False) -> np.ndarray:
+    """FFN(x) = W_down (SiLU(W_gate x) * (W_up x)); x [n, d], W_gate/W_up [I, d], W_down [d, I].
+
+    down_e4m3: the e4m3 down variant -- the hidden rows (rounded to bf16) and W_down's rows
+    are replaced by their scaled e4m3 approximations in the down product."""
+    hid = swiglu_hidden(x, w_gate, w_up, gate_up_e4m3)
+    if down_e4m3:
+        return _dequantized(bf16_round(hid)) @ _dequantized(w_down).T
+    return hid @ widen(w_down).T
 
 
 # ---------------------------------------------------------------- e4m3 gate/up variant
@@ -171,6 +179,20 @@ def _dequantized(x) -> np.ndarray:
     return q * scale[:, None]
 
 
+# The e4m3 down variant (also not on the pages) quantises the down product's operands the
+# same way: each hidden row SiLU(W_gate x) * (W_up x), first rounded to bf16 (the precision
+# the layer stores it in), and each W_down row (one output channel) get their own scale.
+# For the shared experts, which run as one group, the row is the concatenation of the K_s
+# experts' hidden rows and the W_down row the concatenation of theirs (one scale each).
+def bf16_round(y) -> np.ndarray:
+    """Nearest bfloat16 value of each entry (ties to even; fp64 values go through fp32,
+    whose rounding cannot change a bf16 decision except for exact ties)."""
+    y32 = np.ascontiguousarray(np.asarray(y, dtype=np.float64), dtype=np.float32)
+    b = y32.view(np.uint32).astype(np.uint64)
+    b = (b + 0x7FFF + ((b >> 16) & 1)) & 0xFFFF0000
+    return b.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
 # ---------------------------------------------------------------- balance statistics
 def balance_stats(s: np.ndarray, topk_idx: np.ndarray, n_routed: int, alpha1: float):
     """Expert-level balance statistics (deepforge, "Expert-level balance loss").
@@ -199,7 +221,8 @@ class LayerOut:
 
 
 def moe_forward(u, centroids, w_gate, w_up, w_down, n_shared: int, top_k: int,
-                alpha1: float, bias=None, rows=None, gate_up_e4m3: bool = False) -> LayerOut:
+                alpha1: float, bias=None, rows=None, gate_up_e4m3: bool = False,
+                down_e4m3: bool = False) -> LayerOut:
     """h = u + sum_{j shared} FFN_j(u) + sum_{i routed, selected} g_i FFN_i(u).
 
     Weights: w_gate/w_up [n_shared + N_r, I, d], w_down [n_shared + N_r, d, I], shared
@@ -207,8 +230,9 @@ def moe_forward(u, centroids, w_gate, w_up, w_down, n_shared: int, top_k: int,
     all T tokens; `rows` (token ids) restricts only which output rows are computed.
     Per routed expert the selecting tokens are gathered and run as one fp64 GEMM chain
     (the grouping the deepforge article names for production implementations).
-    gate_up_e4m3 selects the e4m3 gate/up variant (quantize_rows_e4m3); routing, the
-    residual and the down projection use the unquantised values either way.
+    gate_up_e4m3 selects the e4m3 gate/up variant (quantize_rows_e4m3), down_e4m3 the e4m3
+    down variant (quantised bf16 hidden rows and W_down rows; the shared experts' rows
+    concatenated); routing and the residual use the unquantised values either way.
     """
     u64 = widen(u)
     T = u64.shape[0]
@@ -219,8 +243,14 @@ def moe_forward(u, centroids, w_gate, w_up, w_down, n_shared: int, top_k: int,
     rows = np.arange(T) if rows is None else np.asarray(rows, dtype=np.int64)
     x = u64[rows]
     h = x.copy()                                          # residual
-    for j in range(n_shared):                             # shared experts, gate 1
-        h += swiglu_ffn(x, w_gate[j], w_up[j], w_down[j], gate_up_e4m3)
+    if down_e4m3 and n_shared:                            # shared experts as one group
+        hid = np.concatenate([swiglu_hidden(x, w_gate[j], w_up[j], gate_up_e4m3)
+                              for j in range(n_shared)], axis=1)
+        wd = np.concatenate([widen(w_down[j]) for j in range(n_shared)], axis=1)
+        h += _dequantized(bf16_round(hid)) @ _dequantized(wd).T
+    else:
+        for j in range(n_shared):                         # shared experts, gate 1
+            h += swiglu_ffn(x, w_gate[j], w_up[j], w_down[j], gate_up_e4m3)
     sel = r.topk_idx[rows]                                # [n, K']
     gate = r.topk_w[rows]
     for e in range(n_routed):
@@ -228,7 +258,7 @@ def moe_forward(u, centroids, w_gate, w_up, w_down, n_shared: int, top_k: int,
         if hit_r.size == 0:
             continue
         y = swiglu_ffn(x[hit_r], w_gate[n_shared + e], w_up[n_shared + e],
-                       w_down[n_shared + e], gate_up_e4m3)
+                       w_down[n_shared + e], gate_up_e4m3, down_e4m3)
         h[hit_r] += gate[hit_r, hit_k][:, None] * y
     return LayerOut(h=h, rows=rows, routing=r, counts=counts, f=f, P=P, aux=aux)
 

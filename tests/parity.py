@@ -199,7 +199,8 @@ def compare(w, g: GpuOut, rows=None, report: dict | None = None) -> dict:
     """Assert parity of every output; returns a report dict (excluded tokens, errors)."""
     ref = O.moe_forward(w.u, w.centroids, w.w_gate, w.w_up, w.w_down, w.n_shared, w.top_k,
                         w.alpha1, bias=w.logit_bias, rows=rows,
-                        gate_up_e4m3=getattr(w, "gate_up_e4m3", False))
+                        gate_up_e4m3=getattr(w, "gate_up_e4m3", False),
+                        down_e4m3=getattr(w, "down_e4m3", False))
     rep = report if report is not None else {}
     keep = compare_routing(w, ref.routing, g.topk_idx, g.topk_w, g.counts, g.aux, ref.P, rep)
     rep["aux_ref"] = ref.aux

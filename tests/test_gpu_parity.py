@@ -79,11 +79,10 @@ def test_full_size_layer(name):
     rows = None if w.T <= 512 else P.sample_rows(w.T)
     rep = P.compare(w, g, rows=rows)
     print(name, rep)
-    # the router's last CTA runs the scan (no kernel of its own); the paired bf16 GEMM path
-    # with a shared group fuses the row permute into the gate/up GEMM; decode-sized layers
-    # and layers without shared experts launch it
+    # the paired bf16 GEMM path with a shared group fuses the row permute into the gate/up
+    # GEMM; decode-sized layers and layers without shared experts launch it
     fused = w.dtype == "bf16" and w.T > 128 and w.n_shared > 0
-    assert layer.kernels_per_forward == (4 if fused else 5)
+    assert layer.kernels_per_forward == (5 if fused else 6)
 
 
 # ------------------------------------------------------------------------ the limits
@@ -184,9 +183,9 @@ def test_nan_row_propagates_without_hang():
     assert err <= P.TOL["bf16"]
 
 
-@pytest.mark.parametrize("e4m3", [False, True], ids=["bf16", "e4m3_gate_up"])
+@pytest.mark.parametrize("e4m3", [False, True, "experts"], ids=["bf16", "e4m3_gate_up", "e4m3_experts"])
 def test_bitwise_deterministic(e4m3):
-    w = W.make_workload("16b_prefill", T=3000, gate_up_e4m3=e4m3)
+    w = W.make_workload("16b_prefill", T=3000, gate_up_e4m3=bool(e4m3), down_e4m3=e4m3 == "experts")
     layer = MoELayer.from_workload(w)
     u = to_device_tensor(w.u, "cuda")
     a = layer.forward(u)
@@ -266,11 +265,32 @@ def test_e4m3_gate_up_layers(spec):
     g, layer, *_ = run(w)
     rep = P.compare(w, g)       # against the oracle's e4m3 variant, the bf16 tolerance
     print(spec, rep)
-    assert layer.kernels_per_forward == (5 if spec["n_shared"] else 6)
+    assert layer.kernels_per_forward == (6 if spec["n_shared"] else 7)
 
 
-def test_e4m3_gate_up_full_size_and_tolerance_study():
-    w = W.make_workload("16b_prefill_e4m3")
+# both expert GEMMs on e4m3 operands (intermediate widths a multiple of 128)
+E4M3_DOWN_SMALL = [
+    dict(T=333, d=256, n_shared=2, n_routed=16, inter=256, top_k=4),
+    dict(T=1000, d=512, n_shared=0, n_routed=16, inter=256, top_k=2),
+    dict(T=100, d=384, n_shared=1, n_routed=64, inter=128, top_k=6),
+    dict(T=20000, d=256, n_shared=1, n_routed=256, inter=128, top_k=16),
+]
+
+
+@pytest.mark.parametrize("spec", E4M3_DOWN_SMALL, ids=lambda s: "T{T}_d{d}_s{n_shared}_r{n_routed}_i{inter}_k{top_k}".format(**s))
+def test_e4m3_expert_layers(spec):
+    w = W.make_workload("16b_prefill", alpha1=0.001, dtype="bf16", gate_up_e4m3=True,
+                        down_e4m3=True, **spec)
+    g, layer, *_ = run(w)
+    rep = P.compare(w, g)       # against the oracle's e4m3 variant, the bf16 tolerance
+    print(spec, rep)
+    # the e4m3 down GEMM adds the activations' quantisation (shared group and routed rows)
+    assert layer.kernels_per_forward == (6 if spec["n_shared"] else 7) + 1 + (spec["n_shared"] > 0)
+
+
+@pytest.mark.parametrize("name", ["16b_prefill_e4m3", "16b_prefill_e4m3_experts"])
+def test_e4m3_gate_up_full_size_and_tolerance_study(name):
+    w = W.make_workload(name)
     g, layer, *_ = run(w)
     rows = P.sample_rows(w.T)
     rep = P.compare(w, g, rows=rows)
@@ -281,11 +301,12 @@ def test_e4m3_gate_up_full_size_and_tolerance_study():
     h = g.h[rows].astype(np.float64)
     full = np.abs(h - ref.h).max() / np.abs(ref.h).max()
     expert = np.abs((h - u) - (ref.h - u)).max() / np.abs(ref.h - u).max()
-    print("e4m3 gate/up vs e4m3 oracle:", rep)
-    print(f"e4m3 gate/up vs full-precision oracle: h {full:.3e}, expert part {expert:.3e}")
+    print(f"{name} vs its e4m3 oracle:", rep)
+    print(f"{name} vs full-precision oracle: h {full:.3e}, expert part {expert:.3e}")
     # the variant's own bound against the full-precision layer: e4m3 keeps 3 mantissa bits
-    # (a rounding step of up to 2^-4 of a value on both gate/up operands), measured 2.6e-2
-    # on h and 5.6e-2 on the expert part at this size
+    # (a rounding step of up to 2^-4 of a value on both operands of every quantised product);
+    # gate/up only: measured 2.6e-2 on h and 5.6e-2 on the expert part at this size; with the
+    # down products quantised as well the rounding enters twice over
     assert full <= 5e-2 and expert <= 1e-1
 
 

@@ -373,3 +373,92 @@ def test_e4m3_variant_changes_only_the_expert_part_and_by_little():
     u = O.widen(w.u)
     rel = np.abs((b.h - u) - (a.h - u)).max() / np.abs(a.h - u).max()
     assert 1e-4 < rel < 0.1, rel                                           # quantised, not broken
+
+
+# ---------------------------------------------------------------- e4m3 down variant
+def test_bf16_round_matches_torch_and_ties_to_even():
+    import torch
+    rng = np.random.default_rng(5)
+    x = np.concatenate([rng.standard_normal(20000) * 10.0 ** rng.integers(-6, 6, 20000),
+                        [0.0, -0.0, 1.0, -3.5, 1e-40]])
+    want = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(O.bf16_round(x), want)
+    # exact ties between neighbouring bf16 values go to the even mantissa
+    base = np.array([1.0, 1.0 + 2 ** -7, 3.0, 3.0 + 2 ** -6])
+    ties = base + np.array([2 ** -8, 2 ** -8, 2 ** -7, 2 ** -7])
+    np.testing.assert_array_equal(O.bf16_round(ties), [1.0, 1.0 + 2 ** -6, 3.0, 3.0 + 2 ** -5])
+    bf = O.bf16_round(x)
+    np.testing.assert_array_equal(O.bf16_round(bf), bf)   # bf16 values stay
+
+
+def _e4m3_err_bound(x, scale):
+    """|deq(x) - x| per entry: half a step of 3 mantissa bits (2^-4 relative) for normal
+    e4m3 values, half the subnormal step (2^-10) times the row scale below them."""
+    return np.abs(x) * 2.0 ** -4 + 2.0 ** -10 * scale[:, None]
+
+
+def test_e4m3_down_output_within_the_quantisation_bound():
+    """Each routed expert's output with the down product on quantised bf16 hidden rows and
+    quantised W_down rows differs from the plain product by at most the sum of the entries'
+    rounding bounds (bf16: 2^-9 relative; e4m3: the bound above)."""
+    w = W.make_workload("tiny", T=64)
+    for e in range(3):
+        g = w.n_shared + e
+        x = w.u[:32]
+        hid = O.swiglu_hidden(x, w.w_gate[g], w.w_up[g])
+        wd = O.widen(w.w_down[g])
+        y_plain = hid @ wd.T
+        y_var = O.swiglu_ffn(x, w.w_gate[g], w.w_up[g], w.w_down[g], down_e4m3=True)
+        hb = O.bf16_round(hid)
+        _, sh = O.quantize_rows_e4m3(hb)
+        _, sw = O.quantize_rows_e4m3(w.w_down[g])
+        eh = np.abs(hb - hid) + _e4m3_err_bound(hb, sh)          # hidden entries
+        ew = _e4m3_err_bound(wd, sw)                             # weight entries
+        bound = eh @ np.abs(wd).T + np.abs(hid) @ ew.T + eh @ ew.T
+        err = np.abs(y_var - y_plain)
+        assert np.all(err <= bound * (1 + 1e-9))
+        assert err.max() > 0                                     # the variant does round
+        # a forgotten scale would break it by orders of magnitude
+        q, s = O.quantize_rows_e4m3(O.bf16_round(hid))
+        assert np.any(np.abs(q @ wd.T - y_plain) > bound)
+
+
+def test_e4m3_down_quantises_rows_of_w_down():
+    """W_down rows that are e4m3 values times a power-of-two row scale quantise without
+    loss per row (row maximum 448 * 2^-j); the variant then equals the product of the
+    quantised hidden rows with W_down itself.  Quantising per column instead would not be
+    lossless here (the columns mix rows of different scales)."""
+    rng = np.random.default_rng(9)
+    grid = np.array([v for v in np.unique(np.abs(O.e4m3_round(rng.standard_normal(5000) * 100))) if v > 0])
+    d, I = 8, 16
+    wd = rng.choice(grid, (d, I)) * rng.choice([-1.0, 1.0], (d, I))
+    wd[:, 0] = 448.0
+    wd = wd * 2.0 ** -rng.integers(3, 12, d)[:, None]
+    np.testing.assert_array_equal(O._dequantized(wd), wd)
+    assert not np.array_equal(O._dequantized(wd.T).T, wd)
+    hid = rng.standard_normal((5, I))
+    want = O._dequantized(O.bf16_round(hid)) @ wd.T
+    x_rows = O._dequantized(O.bf16_round(hid))
+    np.testing.assert_allclose(x_rows @ O._dequantized(wd).T, want, rtol=0, atol=0)
+
+
+def test_e4m3_down_shared_experts_form_one_group():
+    """With the down product quantised, the K_s shared experts run as one group: their part
+    of the layer is the quantised concatenation of their bf16 hidden rows times the
+    quantised W_down matrices side by side (one scale per row of each concatenation), so
+    that the layer equals its routed part (no shared expert) plus that group.  Per-expert
+    scales differ from it once the experts' magnitudes do."""
+    w = W.make_workload("tiny", T=40, n_shared=2)
+    w.w_gate[1] *= 8    # the second shared expert's hidden values are much larger
+    a = O.moe_forward(w.u, w.centroids, w.w_gate, w.w_up, w.w_down, 2, w.top_k, w.alpha1,
+                      down_e4m3=True)
+    routed_only = O.moe_forward(w.u, w.centroids, w.w_gate[2:], w.w_up[2:], w.w_down[2:], 0,
+                                w.top_k, w.alpha1, down_e4m3=True)
+    x = O.widen(w.u)
+    hid = np.concatenate([O.swiglu_hidden(x, w.w_gate[j], w.w_up[j]) for j in range(2)], axis=1)
+    wd_joint = np.concatenate([O.widen(w.w_down[0]), O.widen(w.w_down[1])], axis=1)
+    shared = O._dequantized(O.bf16_round(hid)) @ O._dequantized(wd_joint).T
+    np.testing.assert_allclose(a.h, routed_only.h + shared, rtol=0, atol=1e-12)
+    per_expert = sum(O._dequantized(O.bf16_round(O.swiglu_hidden(x, w.w_gate[j], w.w_up[j])))
+                     @ O._dequantized(w.w_down[j]).T for j in range(2))
+    assert np.abs(per_expert - shared).max() > 1e-6
