@@ -79,6 +79,9 @@ constexpr size_t kGemmSmemBytes = 1024 + (size_t)kGemmStages * kGemmStageBytes +
 
 enum GemmMode : int { kGateUpSwiGLU = 0, kDown = 1, kGateUpBwd = 2, kWgrad = 3 };
 
+// bf16 outputs are written 32 bytes per thread (st.global.v8): out_* must be 32-byte aligned
+// and ld_* a multiple of 16 elements (the library's buffers: cudaMalloc'd, d and the
+// intermediate widths multiples of 64).
 struct GemmArgs {
   const int32_t* grp_row;   // [G] first row of the group in A (and in the output)
   const int32_t* ts;        // [G + 1] tile prefix (256-row tiles)
@@ -425,10 +428,9 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
           }
           if (row_ok) {
             __nv_bfloat16* orow_p = out + orow * ld + ocol + j;
-            reinterpret_cast<uint4*>(orow_p)[0] = make_uint4(pa[0], pa[1], pa[2], pa[3]);
-            reinterpret_cast<uint4*>(orow_p)[1] = make_uint4(pa[4], pa[5], pa[6], pa[7]);
-            reinterpret_cast<uint4*>(orow_p + 64)[0] = make_uint4(pb[0], pb[1], pb[2], pb[3]);
-            reinterpret_cast<uint4*>(orow_p + 64)[1] = make_uint4(pb[4], pb[5], pb[6], pb[7]);
+            st_global_v8(orow_p, make_uint4(pa[0], pa[1], pa[2], pa[3]), make_uint4(pa[4], pa[5], pa[6], pa[7]));
+            st_global_v8(orow_p + 64, make_uint4(pb[0], pb[1], pb[2], pb[3]),
+                         make_uint4(pb[4], pb[5], pb[6], pb[7]));
           }
         }
       } else if (MODE == kGateUpSwiGLU) {
@@ -459,10 +461,10 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
               pk[i] = pack_bf16x2(h0, h1);
             }
             if (row_ok) {
-              uint4* dst = reinterpret_cast<uint4*>(out + orow * ld + col0 + j);
-#pragma unroll
-              for (int v = 0; v < 4; ++v)
-                dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+              __nv_bfloat16* dst = out + orow * ld + col0 + j;
+              st_global_v8(dst, make_uint4(pk[0], pk[1], pk[2], pk[3]), make_uint4(pk[4], pk[5], pk[6], pk[7]));
+              st_global_v8(dst + 16, make_uint4(pk[8], pk[9], pk[10], pk[11]),
+                           make_uint4(pk[12], pk[13], pk[14], pk[15]));
             }
           }
         } else {
@@ -496,11 +498,9 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
               pk[2 * v] = pack_bf16x2(hv[0], hv[1]);
               pk[2 * v + 1] = pack_bf16x2(hv[2], hv[3]);
             }
-            if (row_ok) {
-              uint4* dst = reinterpret_cast<uint4*>(out + orow * ld + col0 + j);
-              dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-              dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-            }
+            if (row_ok)
+              st_global_v8(out + orow * ld + col0 + j, make_uint4(pk[0], pk[1], pk[2], pk[3]),
+                           make_uint4(pk[4], pk[5], pk[6], pk[7]));
           }
         }
       } else {
@@ -529,11 +529,9 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
               pk[2 * q4 + 1] = pack_bf16x2(__uint_as_float(v[4 * q4 + 2]) * sa * b4.z,
                                            __uint_as_float(v[4 * q4 + 3]) * sa * b4.w);
             }
-            if (row_ok) {
-              uint4* dst = reinterpret_cast<uint4*>(out + orow * ld + col);
-              dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-              dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-            }
+            if (row_ok)
+              st_global_v8(out + orow * ld + col, make_uint4(pk[0], pk[1], pk[2], pk[3]),
+                           make_uint4(pk[4], pk[5], pk[6], pk[7]));
           }
         } else {
 #pragma unroll 1
@@ -549,10 +547,10 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
             for (int i = 0; i < 16; ++i)
               pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
             if (row_ok) {
-              uint4* dst = reinterpret_cast<uint4*>(out + orow * ld + col);
-#pragma unroll
-              for (int x = 0; x < 4; ++x)
-                dst[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+              __nv_bfloat16* dst = out + orow * ld + col;
+              st_global_v8(dst, make_uint4(pk[0], pk[1], pk[2], pk[3]), make_uint4(pk[4], pk[5], pk[6], pk[7]));
+              st_global_v8(dst + 16, make_uint4(pk[8], pk[9], pk[10], pk[11]),
+                           make_uint4(pk[12], pk[13], pk[14], pk[15]));
             }
           }
         }
