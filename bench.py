@@ -445,7 +445,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     if e4m3:
         work["permute"] = ("hbm", w.T * w.d * 3 + w.T * 4)   # quantise: bf16 in, e4m3 + scale out
     # with a shared group the paired bf16 GEMM copies the routed rows itself (its copy
-    # warps run beside the shared group's tiles): no permute kernel is launched
+    # warps run beside the shared group's tiles), and so does the decode-sized gate/up GEMM
+    # (its epilogue warps, after the scan has placed the rows): no permute kernel is launched
     fused_permute = (layer.kernels_per_forward - (1 if e4m3 else 0) -
                      ((1 + (w.n_shared > 0)) if e4m3_down else 0)) == len(KERNELS) - 1
     for k in KERNELS:
@@ -453,7 +454,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         avg_ms = kernel_ms[k] / max(1, n_rec)
         ent = {"avg_ms": avg_ms, "share": kernel_ms[k] / max(1e-12, sum(kernel_ms.values()))}
         if k == "permute" and fused_permute and not e4m3:
-            ent.update(fused_into="gate_up_gemm")
+            # paired path: the gate/up GEMM's copy warps; decode-sized layers: the scan places
+            # the rows and the gate/up GEMM's epilogue warps copy them
+            ent.update(fused_into="gate_up_gemm" if w.T > 128 else "scan + gate_up_gemm")
         elif kind == "tensor":
             ach = amount / (avg_ms * 1e-3) / 1e12
             ent.update(bound="tensor", achieved=ach, unit="TFLOP/s",

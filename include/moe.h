@@ -342,6 +342,8 @@ moe_status moe_selftest_wait_timeout(int32_t kind, int64_t limit_ns, int32_t* de
  *   4 hs  [T_pad, n_shared*inter]  shared experts' activations, experts side by side
  *   5 ys  [T_pad, d]       sum of the shared experts' outputs
  *   6 grp_row [G] int32    first row of each group (shared group first when n_shared > 0)
+ *   7 row_tok [rows_cap] int32  token of each routed row (decode-sized path: T <= 128
+ *                          bf16 layers with d % 128 == 0; else empty)
  * Buffers 4 and 5 are empty (size 0) when n_shared == 0. */
 moe_status moe_debug_copy(const moe_handle* handle, int32_t which, void* dst, size_t bytes,
                           size_t* size, moe_stream_t stream);

@@ -42,6 +42,17 @@ struct SmallGemmArgs {
   __nv_bfloat16* out_routed;
   int64_t ld_routed;
   int* err;
+  // Fused row copy (gate/up GEMM): with copy_done != nullptr the epilogue warps, before
+  // their first tile, copy token row row_tok[r] of u to row r of xp for every routed row
+  // r < n_rows (16-byte vectors, copy_vecs per row), then each adds 1 to *copy_done; a
+  // CTA's producer waits for all gridDim.x * 4 of them before loading its first routed
+  // token tile (the shared group reads u itself).  The wait relies on the whole grid being
+  // resident at once (one CTA per SM).
+  const int32_t* row_tok;
+  const __nv_bfloat16* u;
+  __nv_bfloat16* xp;
+  int n_rows, copy_vecs;
+  int* copy_done;
 };
 
 // Schedule of the small-batch GEMM: tiles go round-robin to the CTAs, so the first
@@ -143,10 +154,17 @@ grouped_gemm_small_kernel(const __grid_constant__ CUtensorMap tmW_s,
       int stage = 0, g = 0;
       uint32_t phase = 0, issued = 0, last_par = 0;
       bool ok = true;
+      bool rows_ready = MODE != kGateUpSwiGLU || a.copy_done == nullptr;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         int m, e;
         bool sh;
         decode(tile, g, m, e, sh);
+        if (!sh && !rows_ready) {   // the routed token rows are copied by the epilogue warps
+          ok = counter_wait(a.copy_done, (int)gridDim.x * 4, abort_flag, a.err, kErrWaitCopy);
+          if (!ok) break;
+          fence_proxy_async_global();   // the copied rows, seen by the TMA loads below
+          rows_ready = true;
+        }
         const int xrow = __ldg(&a.grp_row[g]);
         const int kbn = sh ? a.kb_shared : a.kb_routed;
         for (int kb = 0; kb < kbn; ++kb) {
@@ -210,6 +228,37 @@ grouped_gemm_small_kernel(const __grid_constant__ CUtensorMap tmW_s,
     const int q = warp & 3;              // TMEM lane quadrant
     const int L = q * 32 + lane;         // TMEM lane = weight row of the tile
     const int et = threadIdx.x - 64;     // 0..127
+    if (MODE == kGateUpSwiGLU && a.copy_done != nullptr) {
+      // the routed token rows, one warp per row (eight 16-byte vectors per lane in flight)
+      constexpr int kV = 8;
+      const int nw = (int)gridDim.x * 4;
+      for (int r = (int)blockIdx.x * 4 + (et >> 5); r < a.n_rows; r += nw) {
+        const int t = __ldg(a.row_tok + r);
+        if (t < 0 || t >= a.T) {
+          record_error(a.err, kErrPermuteRow);
+          continue;
+        }
+        const uint4* src = reinterpret_cast<const uint4*>(a.u + (size_t)t * a.copy_vecs * 8);
+        uint4* dst = reinterpret_cast<uint4*>(a.xp + (size_t)r * a.copy_vecs * 8);
+        for (int v0 = 0; v0 < a.copy_vecs; v0 += 32 * kV) {
+          uint4 buf[kV];
+#pragma unroll
+          for (int j = 0; j < kV; ++j) {
+            const int v = v0 + j * 32 + lane;
+            if (v < a.copy_vecs) buf[j] = __ldg(src + v);
+          }
+#pragma unroll
+          for (int j = 0; j < kV; ++j) {
+            const int v = v0 + j * 32 + lane;
+            if (v < a.copy_vecs) dst[v] = buf[j];
+          }
+        }
+      }
+      fence_proxy_async_global();
+      __threadfence();
+      __syncwarp();
+      if (lane == 0) atomicAdd(a.copy_done, 1);
+    }
     int g = 0, it = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
       int m, e;

@@ -87,6 +87,7 @@ struct moe_handle {
   int es = 2;              // element size
   int G = 0, has_shared = 0, inter_shared = 0;
   int n_tiles = 0;         // router tiles
+  int router_cluster = 1;  // CTAs per token of the decode-sized router
   int router_rows = 0;     // tokens per router tile
   int64_t T_pad = 0, rows_cap = 0;   // padded to bm, the GEMM row tile
   int bm = 0, tile_rows = 0;
@@ -116,6 +117,8 @@ struct moe_handle {
   void *xp = nullptr, *hs = nullptr, *hr = nullptr, *ys = nullptr, *yr = nullptr;
   int* err = nullptr;
   int* copy_done = nullptr;   // counter of the fused permute (paired bf16 path with a shared group)
+  int32_t* row_tok = nullptr; // [rows_cap] token of each routed row (decode-sized path: the
+                              // scan places the rows, the gate/up GEMM's epilogue warps copy them)
   // e4m3 gate/up: quantised weights (interleaved rows), per-row scales, quantised tokens
   void *w8_gu_s = nullptr, *w8_gu_r = nullptr, *u8 = nullptr;
   float *sw_s = nullptr, *sw_r = nullptr, *su = nullptr, *su_p = nullptr;
@@ -247,9 +250,11 @@ int32_t moe_abi_version(void) { return MOE_ABI_VERSION; }
 const char* moe_last_error(void) { return g_last_error.c_str(); }
 
 int32_t moe_kernels_per_forward(const moe_handle* handle) {
-  // six timing slots; the permute has no kernel when the gate/up GEMM copies the rows, and
-  // e4m3 layers add the token quantisation
-  return handle ? kKernelsPerForward - (handle->fuse_permute ? 1 : 0) + (handle->e4m3 ? 1 : 0) +
+  // six timing slots; the permute has no kernel when the gate/up GEMM copies the rows (on
+  // decode-sized layers after the scan has placed them), and e4m3 layers add the token
+  // quantisation
+  return handle ? kKernelsPerForward - (handle->fuse_permute || handle->small ? 1 : 0) +
+                      (handle->e4m3 ? 1 : 0) +
                       (handle->e4m3_down ? 1 + handle->has_shared : 0)
                 : 0;
 }
@@ -284,6 +289,7 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
   if (H->small) {
     H->router_rows = 1;
     H->n_tiles = c.T;
+    H->router_cluster = router_small_cluster(c.T, H->n_sms);
   }
   H->n_tok = (c.T + 15) / 16 * 16;
   H->bm = H->small ? 1 : (H->bf16 ? kPairBM : kSimtBM);
@@ -390,6 +396,7 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
   MOE_CUDA(cudaMemsetAsync(H->copy_done, 0, 256, st));
   const size_t rc = (size_t)H->rows_cap, tp = (size_t)H->T_pad;
   MOE_TRY(dalloc(H, &H->xp, rc * d * (H->e4m3 ? 1 : es)));   // e4m3 rows on that path
+  if (H->small) MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->row_tok), rc * 4));
   if (H->e4m3) {
     MOE_TRY(dalloc(H, &H->u8, tp * d));
     MOE_CUDA(cudaMemsetAsync(H->u8, 0, tp * d, st));
@@ -570,7 +577,12 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
               c.inter, d, H->bm, H->tile_rows, bn1, bn2, c.alpha1, expert_counts, aux_loss,
               H->psum_total,
               H->tile_base, H->grp_row, H->ts1, H->ts2,
-              H->fuse_permute ? H->copy_done : nullptr, H->bwd ? H->ts3 : nullptr};
+              H->fuse_permute || H->small ? H->copy_done : nullptr, H->bwd ? H->ts3 : nullptr};
+  if (H->small) {   // the scan places the routed rows; the gate/up GEMM copies them
+    sa.topk_idx = topk_idx; sa.topk_rank = H->topk_rank;
+    sa.slot_row = H->slot_row; sa.row_tok = H->row_tok;
+    sa.top_k = K; sa.router_rows = H->router_rows; sa.rows_cap = (int)H->rows_cap; sa.err = H->err;
+  }
   RouterOut ro{topk_idx, topk_w, H->topk_rank, H->tile_hist, H->tile_psum, H->err,
                H->bwd ? H->logits : nullptr};
   CUtensorMap tmU, tmUr;
@@ -580,8 +592,8 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
                        static_cast<const __nv_bfloat16*>(H->centroids), H->bias, T, d, nr, K,
                        H->router_rows, ro};
     with_maxc(H->maxc, [&](auto m) {
-      launch_pdl(router_small_kernel<m()>, dim3(H->n_tiles), dim3(kRouterEpiThreads),
-                 H->simt_router_smem, stream, ra);
+      launch_pdl_cluster(router_small_kernel<m()>, dim3(H->n_tiles * H->router_cluster), dim3(kRouterEpiThreads),
+                         H->simt_router_smem, stream, (unsigned)H->router_cluster, ra);
       return 0;
     });
   } else if (H->bf16) {
@@ -620,7 +632,7 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
     pa.scale_src = H->su;
     pa.scale_dst = H->su_p;
   }
-  if (!H->fuse_permute) {
+  if (!H->fuse_permute && !H->small) {
     launch_pdl(permute_kernel, dim3((T + kPermuteWarps - 1) / kPermuteWarps), dim3(kPermuteWarps * 32), 0, stream, pa);
     MOE_CUDA(cudaGetLastError());
   }
@@ -638,10 +650,15 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
     s1.out_shared = static_cast<__nv_bfloat16*>(H->hs); s1.ld_shared = Is;
     s1.out_routed = static_cast<__nv_bfloat16*>(H->hr); s1.ld_routed = I;
     s1.err = H->err;
+    // the routed rows (placed by the scan) are copied by the gate/up GEMM's epilogue warps
+    s1.row_tok = H->row_tok; s1.u = static_cast<const __nv_bfloat16*>(u);
+    s1.xp = static_cast<__nv_bfloat16*>(H->xp); s1.n_rows = T * K; s1.copy_vecs = d / 8;
+    s1.copy_done = H->copy_done;
     tick(H, stream, 3);
     launch_pdl(grouped_gemm_small_kernel<kGateUpSwiGLU>, dim3(H->n_sms), dim3(kSmallThreads), H->small_smem, stream,  H->tmWguS, H->tmWguR, tmUN, H->tmXpN, s1);
     MOE_CUDA(cudaGetLastError());
     SmallGemmArgs s2 = s1;
+    s2.copy_done = nullptr;   // no row copy: the activations are expert-contiguous rows
     s2.ts = H->ts2;
     s2.kb_shared = Is / 64; s2.kb_routed = I / 64;
     s2.mt_shared = d / kSmallBM; s2.mt_routed = d / kSmallBM;
@@ -1261,7 +1278,8 @@ moe_status moe_debug_copy(const moe_handle* H, int32_t which, void* dst, size_t 
     case 4: src = H->hs; n = H->hs ? tp * (size_t)H->inter_shared * es : 0; break;
     case 5: src = H->ys; n = H->ys ? tp * d * es : 0; break;
     case 6: src = H->grp_row; n = (size_t)H->G * 4; break;
-    default: return fail(MOE_ERR_INVALID_ARG, "which=%d outside [0, 6]", which);
+    case 7: src = H->row_tok; n = H->row_tok ? rc * 4 : 0; break;
+    default: return fail(MOE_ERR_INVALID_ARG, "which=%d outside [0, 7]", which);
   }
   *size = n;
   if (!dst) return MOE_OK;

@@ -35,6 +35,7 @@ struct moe_ep_handle {
   int n_pad = 0, maxc = 32, maxk = 16, has_shared = 0, inter_shared = 0;
   bool small_router = false;
   int router_rows = 0, n_tiles = 0, router_stages = 0, router_kps = 1, gemm_grid = 0;
+  int router_cluster = 1;   // CTAs per token of the decode-sized router
   uint32_t router_tmem_cols = 0;
   size_t router_smem = 0, simt_router_smem = 0;
   // weights: all centroids (padded), this rank's routed experts and the shared group
@@ -113,6 +114,7 @@ moe_status ep_create_impl(const moe_cfg& c, int32_t rank, int32_t world, int64_t
   H->small_router = c.T <= kSmallMaxTok && c.d % kSmallBM == 0;
   H->router_rows = H->small_router ? 1 : router_tile_rows(c.T, H->n_sms);
   H->n_tiles = (c.T + H->router_rows - 1) / H->router_rows;
+  if (H->small_router) H->router_cluster = router_small_cluster(c.T, H->n_sms);
 
   const size_t d = c.d, I = c.inter, Is = H->inter_shared, ks = c.n_shared, nl = H->n_local;
   const size_t nr = c.n_routed, T = c.T, K = c.top_k, nt = H->n_tiles, es = 2;
@@ -297,8 +299,8 @@ moe_status moe_ep_dispatch(moe_ep_handle* H, const void* u, int32_t* topk_idx, f
     RouterSmallArgs ra{static_cast<const __nv_bfloat16*>(u),
                        static_cast<const __nv_bfloat16*>(H->centroids), H->bias, T, d, nr, K, 1, ro};
     with_maxc(H->maxc, [&](auto m) {
-      launch_pdl(router_small_kernel<m()>, dim3(H->n_tiles), dim3(kRouterEpiThreads), H->simt_router_smem,
-                 stream, ra);
+      launch_pdl_cluster(router_small_kernel<m()>, dim3(H->n_tiles * H->router_cluster), dim3(kRouterEpiThreads),
+                         H->simt_router_smem, stream, (unsigned)H->router_cluster, ra);
       return 0;
     });
   } else {

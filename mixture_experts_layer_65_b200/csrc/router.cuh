@@ -615,22 +615,34 @@ __global__ void __launch_bounds__(kRouterEpiThreads) router_simt_kernel(RouterSi
 }
 
 // ------------------------------------------------------------------------ bf16, few tokens
-constexpr int kSmallPairs = 4;   // (token, expert) dot products a warp computes together
+constexpr int kSmallPairs = 2;   // (token, expert) dot products a warp computes together
+constexpr int kSmallVecSteps = 4;   // 16-byte vector steps of each whose loads are in flight together
 
 struct RouterSmallArgs {
   const __nv_bfloat16* u;     // [T, d]
   const __nv_bfloat16* cen;   // [n_routed, d]
   const float* bias;          // [>= n_routed]
   int T, d, n_routed, top_k;
-  int tile_rows;              // tokens per CTA (1..64)
+  int tile_rows;              // tokens per cluster (1..64)
   RouterOut out;
 };
 
 // For decode-sized batches (a handful of tokens), where the tensor-core router would
 // stream the whole centroid matrix through its TMA ring for a tile of a few rows: each
-// CTA takes tile_rows tokens, each warp one (token, expert) dot product at a time with
-// the lanes splitting d (16-byte vectors) and a fixed shuffle tree, then the shared
-// epilogue.  512 threads; dynamic smem router_epi_bytes(n_pad).
+// cluster of C CTAs (router_small_cluster: as many as the SMs allow for a single wave, at
+// most kRouterSmallCluster) takes tile_rows tokens, and CTA q of it the logits of experts
+// [q E, (q + 1) E), E = ceil(N_r / C), so that each SM streams only its share of the
+// centroid matrix.  Each warp computes kSmallPairs (token, expert)
+// dot products at a time with the lanes splitting d (16-byte vectors, kSmallVecSteps steps
+// of loads in flight) and a fixed shuffle tree; the logits (bias added) go straight into the leader CTA's logit rows through
+// distributed shared memory, and after a cluster barrier the leader runs the shared
+// epilogue.  512 threads per CTA; dynamic smem router_epi_bytes(n_pad).
+constexpr int kRouterSmallCluster = 4;
+// CTAs per token cluster for T tokens on n_sms SMs (one CTA of 512 threads per SM).
+inline int router_small_cluster(int T, int n_sms) {
+  const int c = T > 0 ? n_sms / T : 1;
+  return c < 1 ? 1 : (c > kRouterSmallCluster ? kRouterSmallCluster : c);
+}
 template <int MAXC>
 __global__ void __launch_bounds__(kRouterEpiThreads) router_small_kernel(RouterSmallArgs a) {
   pdl_launch_dependents();
@@ -639,46 +651,63 @@ __global__ void __launch_bounds__(kRouterEpiThreads) router_small_kernel(RouterS
   RouterEpiSmem& SM = *reinterpret_cast<RouterEpiSmem*>(smem_raw);
   float* lg = reinterpret_cast<float*>(smem_raw + sizeof(RouterEpiSmem));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int tile = blockIdx.x, R = a.tile_rows;
+  const uint32_t q = cluster_ctarank();
+  const int C = (int)cluster_nctarank();
+  const int tile = (int)blockIdx.x / C, R = a.tile_rows;
   const int n_pad = (a.n_routed + 15) & ~15;
   const int ld = router_ld(n_pad);
   const int nv = a.d >> 3;
-  for (int e = tid; e < 4 * kMaxRouted; e += kRouterEpiThreads) (&SM.mask[0][0])[e] = 0u;
-  // each warp takes kSmallPairs consecutive (token, expert) pairs at once, so that their
+  const int E = (a.n_routed + C - 1) / C;
+  const int e0 = (int)q * E;
+  const int ne = a.n_routed - e0 < E ? (a.n_routed - e0 > 0 ? a.n_routed - e0 : 0) : E;
+  if (q == 0)
+    for (int e = tid; e < 4 * kMaxRouted; e += kRouterEpiThreads) (&SM.mask[0][0])[e] = 0u;
+  const uint32_t lg_leader = mapa_shared(smem_u32(lg), 0);
+  cluster_sync_all();   // every CTA of the cluster is running before the first remote store
+  // round by round, warp w takes pairs w, w + 16, ... (kSmallPairs of them) so that their
   // loads are in flight together; every dot product keeps its own order of operations
-  const int npairs = R * a.n_routed;
-  for (int p0 = warp * kSmallPairs; p0 < npairs; p0 += (kRouterEpiThreads / 32) * kSmallPairs) {
+  constexpr int kWarps = kRouterEpiThreads / 32;
+  const int npairs = R * ne;
+  for (int p0 = 0; p0 < npairs; p0 += kWarps * kSmallPairs) {
     const uint4* ur[kSmallPairs];
     const uint4* er[kSmallPairs];
     bool on[kSmallPairs];
     float acc[kSmallPairs];
 #pragma unroll
     for (int j = 0; j < kSmallPairs; ++j) {
-      const int p = p0 + j < npairs ? p0 + j : npairs - 1;
-      const int r = p / a.n_routed, i = p - r * a.n_routed;
+      const int pj = p0 + j * kWarps + warp;
+      const int p = pj < npairs ? pj : npairs - 1;
+      const int r = p / ne, i = e0 + (p - r * ne);
       const int t = tile * R + r;
-      on[j] = p0 + j < npairs && t < a.T;
+      on[j] = pj < npairs && t < a.T;
       ur[j] = reinterpret_cast<const uint4*>(a.u + (size_t)(t < a.T ? t : 0) * a.d);
       er[j] = reinterpret_cast<const uint4*>(a.cen + (size_t)i * a.d);
       acc[j] = 0.f;
     }
-    for (int v = lane; v < nv; v += 32) {
-      uint4 xu[kSmallPairs], xe[kSmallPairs];
+    for (int v0 = lane; v0 < nv; v0 += 32 * kSmallVecSteps) {
+      uint4 xu[kSmallVecSteps][kSmallPairs], xe[kSmallVecSteps][kSmallPairs];
 #pragma unroll
-      for (int j = 0; j < kSmallPairs; ++j) {
-        if (on[j]) {
-          xu[j] = __ldg(ur[j] + v);
-          xe[j] = __ldg(er[j] + v);
+      for (int b = 0; b < kSmallVecSteps; ++b) {
+#pragma unroll
+        for (int j = 0; j < kSmallPairs; ++j) {
+          if (on[j] && v0 + 32 * b < nv) {
+            xu[b][j] = __ldg(ur[j] + v0 + 32 * b);
+            xe[b][j] = __ldg(er[j] + v0 + 32 * b);
+          }
         }
       }
+      // each pair's products in ascending vector order, as one FMA chain
 #pragma unroll
-      for (int j = 0; j < kSmallPairs; ++j) {
-        if (on[j]) {
-          float x[8], y[8];
-          bf16x8_to_f32(xu[j], x);
-          bf16x8_to_f32(xe[j], y);
+      for (int b = 0; b < kSmallVecSteps; ++b) {
 #pragma unroll
-          for (int k = 0; k < 8; ++k) acc[j] = fmaf(x[k], y[k], acc[j]);
+        for (int j = 0; j < kSmallPairs; ++j) {
+          if (on[j] && v0 + 32 * b < nv) {
+            float x[8], y[8];
+            bf16x8_to_f32(xu[b][j], x);
+            bf16x8_to_f32(xe[b][j], y);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) acc[j] = fmaf(x[k], y[k], acc[j]);
+          }
         }
       }
     }
@@ -686,14 +715,15 @@ __global__ void __launch_bounds__(kRouterEpiThreads) router_small_kernel(RouterS
     for (int j = 0; j < kSmallPairs; ++j) {
 #pragma unroll
       for (int m = 16; m > 0; m >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], m);
-      const int p = p0 + j;
+      const int p = p0 + j * kWarps + warp;
       if (lane == 0 && p < npairs) {
-        const int r = p / a.n_routed, i = p - r * a.n_routed;
-        lg[(size_t)r * ld + i] = acc[j] + a.bias[i];
+        const int r = p / ne, i = e0 + (p - r * ne);
+        st_shared_cluster_f32(lg_leader + 4u * (uint32_t)(r * ld + i), acc[j] + a.bias[i]);
       }
     }
   }
-  __syncthreads();
+  cluster_sync_all();   // the cluster's logits are in the leader's rows
+  if (q != 0) return;
   auto sync = [] { __syncthreads(); };
   router_pass<MAXC>(tid, 0, tile, R, a.T, a.n_routed, n_pad, a.top_k, smem_raw, a.out, sync);
   __syncthreads();

@@ -46,6 +46,15 @@ struct ScanArgs {
   int32_t* ts3;               // [G + 1] tile prefix of a GEMM with N = the group's
                               // intermediate width at bn2 columns per tile (the backward's
                               // dHmid GEMM), or nullptr
+  // Routed-row indices (decode-sized layers, whose gate/up GEMM copies the token rows
+  // itself): with slot_row != nullptr the scan ends by placing every (token, slot) —
+  // slot_row[t, k] = its destination row, row_tok[row] = t — as the permute would.
+  const int32_t* topk_idx;    // [T, top_k]
+  const int32_t* topk_rank;   // [T, top_k]
+  int32_t* slot_row;          // [T, top_k], or nullptr
+  int32_t* row_tok;           // [rows_cap]
+  int top_k, router_rows, rows_cap;
+  int* err;
 };
 
 struct ScanSmem {
@@ -199,6 +208,28 @@ __device__ void scan_tail(const ScanArgs& a, int tid, uint8_t* smem, Sync sync) 
           run += hv[j];
         }
       }
+    }
+  }
+  // 5. (decode-sized layers) the destination row of every (token, slot) and the token of
+  //    every destination row
+  if (a.slot_row) {
+    sync();   // the tile bases above, written by other threads
+    const int n = a.T * a.top_k;
+    for (int idx = tid; idx < n; idx += kScanThreads) {
+      const int t = idx / a.top_k;
+      const int ex = a.topk_idx[idx];
+      int dst = -1;
+      if (ex >= 0 && ex < nr) {
+        dst = a.tile_base[(size_t)(t / a.router_rows) * nr + ex] + a.topk_rank[idx];
+        if (dst < 0 || dst >= a.rows_cap) {
+          record_error(a.err, kErrPermuteRow);
+          dst = -1;
+        }
+      } else {
+        record_error(a.err, kErrRouteIndex);
+      }
+      a.slot_row[idx] = dst < 0 ? 0 : dst;
+      if (dst >= 0) a.row_tok[dst] = t;
     }
   }
 }

@@ -227,17 +227,19 @@ class MoELayer:
                                  s.cuda_stream))
         return du, d_cen, d_bias, dwg, dwu, dwd
 
-    DEBUG_BUFFERS = {"slot_row": 0, "xp": 1, "hr": 2, "yr": 3, "hs": 4, "ys": 5, "grp_row": 6}
+    DEBUG_BUFFERS = {"slot_row": 0, "xp": 1, "hr": 2, "yr": 3, "hs": 4, "ys": 5, "grp_row": 6,
+                     "row_tok": 7}
 
     def debug_buffer(self, name: str) -> torch.Tensor:
         """A copy (flat, device) of a workspace buffer as the last forward left it: for
-        per-kernel tests.  int32 for slot_row/grp_row, uint8 bytes for xp of e4m3 gate/up
-        layers, else the layer dtype."""
+        per-kernel tests.  int32 for slot_row/grp_row/row_tok, uint8 bytes for xp of e4m3
+        gate/up layers, else the layer dtype.  row_tok is empty except on decode-sized
+        layers."""
         which = self.DEBUG_BUFFERS[name]
         size = ctypes.c_size_t(0)
         s = torch.cuda.current_stream(self.device)
         check(lib().moe_debug_copy(self._h, which, None, 0, ctypes.byref(size), s.cuda_stream))
-        if name in ("slot_row", "grp_row"):
+        if name in ("slot_row", "grp_row", "row_tok"):
             dt = torch.int32
         elif name == "xp" and self.gate_up_e4m3:
             dt = torch.uint8

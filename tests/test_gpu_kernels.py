@@ -25,6 +25,7 @@ pytestmark = pytest.mark.gpu
 SPECS = [
     dict(T=333, d=256, n_shared=2, n_routed=16, inter=192, top_k=4),   # row copy in the GEMM
     dict(T=700, d=256, n_shared=0, n_routed=16, inter=128, top_k=2),   # permute kernel
+    dict(T=96, d=256, n_shared=2, n_routed=16, inter=128, top_k=4),    # decode-sized: copy in the GEMM
 ]
 
 
@@ -67,6 +68,9 @@ def test_intermediates_match_the_oracle(spec, e4m3):
     xp = layer.debug_buffer("xp").cpu()
     rows = slot.reshape(-1)
     toks = np.repeat(np.arange(T), K)
+    row_tok = layer.debug_buffer("row_tok").cpu().numpy()
+    if row_tok.size:   # decode-sized layer: the scan recorded the token of every routed row
+        np.testing.assert_array_equal(row_tok[rows], toks)
     if e4m3:
         xp8 = xp.view(-1, d)[torch.from_numpy(rows)]
         got = xp8.view(torch.float8_e4m3fn).to(torch.float64).numpy()
