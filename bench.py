@@ -54,6 +54,10 @@ def parse_args():
     p.add_argument("--sustained-seconds", type=float, default=3.0,
                    help="after the timed steps, run forwards back to back this long and report "
                         "the power-capped (sustained) throughput beside the value; 0 skips it")
+    p.add_argument("--backward", type=int, default=0, metavar="K",
+                   help="also time K forward + backward steps (input, router and weight "
+                        "gradients) after the forward measurements and add a 'backward' "
+                        "object to the line; bf16 prefill-sized layers only")
     p.add_argument("--dry-run", action="store_true",
                    help="CPU check of the multi-rank plumbing (gloo): rank discovery, the "
                         "global balance loss's exchange on synthetic per-rank statistics and "
@@ -426,10 +430,20 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             e2e_ms = float(t.item())
         layer.device_status()
 
+    bwd = None
+    if args.backward > 0:
+        bwd = time_backward(args, layer, ubufs, out, stream, dev, world, local_rank, rank)
+
     if rank != 0:
         return
     del graphs
     peaks, peak_src = load_peaks()
+    if bwd is not None:
+        regime_b = peak_regime(bwd.pop("_clk"), bwd["seconds"])
+        peak_b = peaks[PEAK_KEY[regime_b]]
+        bwd.update(peak_regime=regime_b, frac=bwd["gemm_tflops"] / peak_b,
+                   frac_of_burst=bwd["gemm_tflops"] / peaks["bf16_tflops"],
+                   frac_of_sustained=bwd["gemm_tflops"] / peaks["bf16_tflops_sustained"])
     # the kernels were timed right after the timed steps: hold tensor-bound kernels against
     # the peak of the clock regime that run was in
     regime = peak_regime(clk, ms * 1e-3 + sum(kernel_ms.values()) * 1e-3)
@@ -528,10 +542,71 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "clocks": clk,
         "sustained": sustained,
     }
+    if bwd is not None:
+        line["backward"] = bwd
     if world == 1 and not args.no_cpu_baseline:
         _, desc = oracle_tokens_per_s(w, args.cpu_seconds)
         line["cpu_baseline"] = desc
     print(json.dumps(line), flush=True)
+
+
+def time_backward(args, layer, ubufs, out, stream, dev, world, local_rank, rank):
+    """K forward + backward steps (eager forwards: the captured graphs predate the backward's
+    bookkeeping), each on the next token buffer with a fixed seeded upstream gradient dh and
+    d_aux = 1; CUDA events on the launching stream around each backward and around the
+    whole loop, max over ranks.  The backward's GEMM work is 16·T·d·I·(K_s + K') FLOPs:
+    dHmid (2), the recomputed gate/up (4), dX (4), dW_gate/up (4) and dW_down (2), selected
+    experts only; the router's dl·e GEMM and the SIMT kernels are not counted."""
+    import torch
+    import torch.distributed as dist
+
+    layer.backward_prepare()
+    g = torch.Generator(device=dev).manual_seed(1234 + rank)
+    dh = (torch.randn(layer.T, layer.d, device=dev, generator=g) * 0.01).to(layer.torch_dtype)
+    n_buf = len(ubufs)
+
+    def one(i, evs=None):
+        layer.forward(ubufs[i % n_buf], out)
+        if evs is not None:
+            evs[0].record(stream)
+        grads = layer.backward(ubufs[i % n_buf], out, dh, d_aux=1.0)
+        if evs is not None:
+            evs[1].record(stream)
+        return grads
+
+    for i in range(3):
+        one(i)
+    torch.cuda.synchronize()
+    layer.device_status()
+    if world > 1:
+        dist.barrier()
+    k = args.backward
+    clocks = ClockSampler(device=local_rank) if rank == 0 else None
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(k)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ts = ClockSampler.now()
+    t0.record(stream)
+    for i in range(k):
+        one(i, evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop((ts, ClockSampler.now())) if clocks else None
+    total_ms = t0.elapsed_time(t1)
+    bwd_ms = sum(a.elapsed_time(b) for a, b in evs)
+    if world > 1:
+        t = torch.tensor([total_ms, bwd_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, bwd_ms = (float(x) for x in t.tolist())
+    layer.device_status()
+    flops = 16.0 * layer.T * layer.d * layer.inter * (layer.n_shared + layer.top_k)
+    return {"steps": k, "seconds": total_ms * 1e-3,
+            "fwd_bwd_ms_per_step": total_ms / k, "bwd_ms_per_step": bwd_ms / k,
+            "fwd_bwd_tokens_per_s": world * layer.T * k / (total_ms * 1e-3),
+            "bwd_gemm_tflop_per_step": flops / 1e12,
+            "gemm_tflops": flops / (bwd_ms / k * 1e-3) / 1e12,
+            "gradients": "du, d_centroids, d_bias, d_w_gate, d_w_up, d_w_down (fp32)",
+            "timing": "CUDA events around each backward call (eager forwards in between)",
+            "clocks": clk, "_clk": clk}
 
 
 def relaunch_under_torchrun(args) -> int:

@@ -182,9 +182,14 @@ struct BwdCentroidArgs {
   float* part;                 // [n_chunks, n_routed, d + 1]: column d holds the bias part
 };
 
-// 256 threads: thread (i, q) accumulates expert i (i < n_routed, in steps of 256 / 16) over
-// 4 of the CTA's 64 columns (q), plus, for q == 0, the bias sum; tokens in ascending order.
-static __global__ void __launch_bounds__(256) bwd_centroid_partial_kernel(BwdCentroidArgs a) {
+// 256 threads: thread (i, q) accumulates experts i0, i0 + 16, ... (at most MAXPER of them,
+// MAXPER = ceil(n_routed / 16) rounded up to a power of two) over 4 of the CTA's 64 columns
+// (q), plus, for q == 0, the bias sums; tokens in ascending order.
+__host__ __device__ constexpr int centroid_maxper(int n_routed) {
+  return n_routed <= 16 ? 1 : n_routed <= 32 ? 2 : n_routed <= 64 ? 4 : n_routed <= 128 ? 8 : 16;
+}
+template <int MAXPER>
+__global__ void __launch_bounds__(256) bwd_centroid_partial_kernel(BwdCentroidArgs a) {
   pdl_launch_dependents();
   pdl_wait();
   __shared__ float s_u[kCenStep][kCenCols];
@@ -194,7 +199,7 @@ static __global__ void __launch_bounds__(256) bwd_centroid_partial_kernel(BwdCen
   const int t0 = chunk * kCenChunk, t1 = min(a.T, t0 + kCenChunk);
   const int q = threadIdx.x & 15;           // columns col0 + 4 q .. + 3
   const int i0 = threadIdx.x >> 4;          // experts i0, i0 + 16, ...
-  constexpr int kMaxPer = kMaxRouted / 16;
+  constexpr int kMaxPer = MAXPER;
   float acc[kMaxPer][4];
   float bacc[kMaxPer];
 #pragma unroll
@@ -294,26 +299,45 @@ __device__ __forceinline__ bool masked_row_valid(const MaskedTransposeArgs& a, i
   return r - __ldg(a.grp_row + lo) < n;
 }
 
+// 64 x 64 tiles, 16-byte vectors both ways: 256 threads load the tile's 64 source rows
+// (eight vectors each, coalesced) into shared memory, where each 128-byte row stores its
+// vectors XOR-permuted by (row / 8) mod 8, then write 64 destination rows of eight vectors,
+// each vector gathering one column of eight source rows; eight consecutive threads write one
+// destination row's 128 bytes, and the gathers of a warp hit distinct banks.  C and the
+// strides must be multiples of 8 elements (the library's widths are multiples of 64).
+constexpr int kMtTile = 64;
 static __global__ void __launch_bounds__(256) masked_transpose_kernel(MaskedTransposeArgs a) {
   pdl_launch_dependents();
   pdl_wait();
-  __shared__ __nv_bfloat16 tile[kTrTile][kTrTile + 2];
-  __shared__ bool valid[kTrTile];
-  const int c0 = blockIdx.x * kTrTile;
-  const int64_t r0 = (int64_t)blockIdx.y * kTrTile;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  if (threadIdx.x < kTrTile) valid[threadIdx.x] = r0 + threadIdx.x < a.rows && masked_row_valid(a, r0 + threadIdx.x);
+  __shared__ __align__(16) __nv_bfloat16 tile[kMtTile][kMtTile];
+  __shared__ bool valid[kMtTile];
+  const int c0 = blockIdx.x * kMtTile;
+  const int64_t r0 = (int64_t)blockIdx.y * kMtTile;
+  const int t = threadIdx.x;
+  if (t < kMtTile) valid[t] = r0 + t < a.rows && masked_row_valid(a, r0 + t);
   __syncthreads();
-  for (int i = ty; i < kTrTile; i += 8) {
-    const int64_t r = r0 + i;
-    const int c = c0 + tx;
-    if (c < a.C) tile[i][tx] = valid[i] ? a.src[r * a.ld_src + c] : __float2bfloat16_rn(0.f);
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int row = t / 8 + 32 * i, vec = t % 8;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (valid[row] && c0 + vec * 8 < a.C)
+      v = __ldg(reinterpret_cast<const uint4*>(a.src + (r0 + row) * a.ld_src + c0 + vec * 8));
+    *reinterpret_cast<uint4*>(&tile[row][(vec ^ ((row >> 3) & 7)) * 8]) = v;
   }
   __syncthreads();
-  for (int i = ty; i < kTrTile; i += 8) {
-    const int c = c0 + i;
-    const int64_t r = r0 + tx;
-    if (c < a.C && r < a.rows) a.dst[(int64_t)c * a.ld_dst + r] = tile[tx][i];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int c = t / 8 + 32 * i, rv = t % 8;   // destination row c0 + c, vector rv
+    if (c0 + c >= a.C || r0 + rv * 8 >= a.rows) continue;
+    const int ch = ((c >> 3) ^ rv) * 8 + (c & 7);   // column c of source rows 8 rv .. 8 rv + 7
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const __nv_bfloat16 lo = tile[rv * 8 + 2 * j][ch], hi = tile[rv * 8 + 2 * j + 1][ch];
+      w[j] = (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
+    }
+    *reinterpret_cast<uint4*>(a.dst + (int64_t)(c0 + c) * a.ld_dst + r0 + rv * 8) =
+        make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
 

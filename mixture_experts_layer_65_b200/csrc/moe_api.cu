@@ -12,6 +12,7 @@
 //   5. gate/up     grouped GEMM + SwiGLU (shared group reads the token rows directly)
 //   6. down        grouped GEMM
 //   7. combine     h = u + shared + sum_k g_k * routed_k (fp32, fixed order)
+#include <algorithm>
 #include <cstring>
 #include <string>
 #include <vector>
@@ -96,6 +97,7 @@ struct moe_handle {
   // small-batch (decode) path: token counts <= n_tok, weights on the MMA's M dimension
   bool small = false;
   int n_tok = 0, small_stages = 0;
+  int small_grid2 = 0;     // CTAs of the small-batch down GEMM
   size_t small_smem = 0;
   int n_pad = 0, maxk = 16, maxc = 32;
   int router_stages = 0, router_kps = 1;
@@ -515,6 +517,17 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
       int stages = (int)((200u * 1024u - epi) / sb);
       stages = stages > kSmallMaxStages ? kSmallMaxStages : (stages < 2 ? 2 : stages);
       H->small_stages = stages;
+      // The down GEMM's grid: the fewest CTAs that still give each the same work when every
+      // routed expert receives tokens (a tile of the shared group counts as n_shared routed
+      // tiles: its K is n_shared * inter), so that no CTA runs a last tile alone.
+      {
+        const int64_t mt = d / kSmallBM;
+        const int64_t act = std::min<int64_t>((int64_t)nr, (int64_t)c.T * c.top_k);
+        const int64_t units = act * mt + (ks ? mt * (int64_t)ks : 0);
+        const int64_t per = (units + H->n_sms - 1) / H->n_sms;
+        const int64_t g2 = per > 0 ? (units + per - 1) / per : H->n_sms;
+        H->small_grid2 = (int)std::min<int64_t>(H->n_sms, std::max<int64_t>(1, g2));
+      }
       H->small_smem = 1024 + (size_t)stages * sb + epi + 256;
       MOE_CUDA(cudaFuncSetAttribute((const void*)grouped_gemm_small_kernel<kGateUpSwiGLU>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)H->small_smem));
@@ -665,7 +678,7 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
     s2.out_shared = static_cast<__nv_bfloat16*>(H->ys); s2.ld_shared = d;
     s2.out_routed = static_cast<__nv_bfloat16*>(H->yr); s2.ld_routed = d;
     tick(H, stream, 4);
-    launch_pdl(grouped_gemm_small_kernel<kDown>, dim3(H->n_sms), dim3(kSmallThreads), H->small_smem, stream,  H->tmWdS, H->tmWdR, H->tmHsN, H->tmHrN, s2);
+    launch_pdl(grouped_gemm_small_kernel<kDown>, dim3(H->small_grid2), dim3(kSmallThreads), H->small_smem, stream,  H->tmWdS, H->tmWdR, H->tmHsN, H->tmHrN, s2);
     MOE_CUDA(cudaGetLastError());
   } else if (H->bf16) {
     GemmArgs g1{};
@@ -1037,8 +1050,16 @@ moe_status moe_backward(moe_handle* H, const void* u, const int32_t* topk_idx, c
   // 7. centroid and bias gradients: chunk partials, then their fixed-order sum
   BwdCentroidArgs cp{H->dl, static_cast<const __nv_bfloat16*>(u), T, d, nr, H->n_pad, H->cen_chunks,
                      H->cen_part};
-  launch_pdl(bwd_centroid_partial_kernel, dim3((d + kCenCols - 1) / kCenCols, H->cen_chunks), dim3(256), 0,
-             stream, cp);
+  {
+    const dim3 cg((d + kCenCols - 1) / kCenCols, H->cen_chunks);
+    switch (centroid_maxper(nr)) {
+      case 1: launch_pdl(bwd_centroid_partial_kernel<1>, cg, dim3(256), 0, stream, cp); break;
+      case 2: launch_pdl(bwd_centroid_partial_kernel<2>, cg, dim3(256), 0, stream, cp); break;
+      case 4: launch_pdl(bwd_centroid_partial_kernel<4>, cg, dim3(256), 0, stream, cp); break;
+      case 8: launch_pdl(bwd_centroid_partial_kernel<8>, cg, dim3(256), 0, stream, cp); break;
+      default: launch_pdl(bwd_centroid_partial_kernel<16>, cg, dim3(256), 0, stream, cp); break;
+    }
+  }
   MOE_CUDA(cudaGetLastError());
   const int rgrid = (int)(((size_t)nr * (d + 1) + 255) / 256);
   launch_pdl(bwd_centroid_reduce_kernel, dim3(rgrid < 4 * H->n_sms ? rgrid : 4 * H->n_sms), dim3(256), 0,
@@ -1054,8 +1075,8 @@ moe_status moe_backward(moe_handle* H, const void* u, const int32_t* topk_idx, c
     MaskedTransposeArgs ma{static_cast<const __nv_bfloat16*>(src), static_cast<__nv_bfloat16*>(dst), rows, C,
                            ld_src, ld_dst, routed ? H->grp_row + H->has_shared : nullptr, expert_counts,
                            nr, 0, T, routed ? rows : (int64_t)T};
-    launch_pdl(masked_transpose_kernel, dim3((unsigned)((C + kTrTile - 1) / kTrTile),
-                                             (unsigned)((rows + kTrTile - 1) / kTrTile)),
+    launch_pdl(masked_transpose_kernel, dim3((unsigned)((C + kMtTile - 1) / kMtTile),
+                                             (unsigned)((rows + kMtTile - 1) / kMtTile)),
                dim3(256), 0, stream, ma);
     return cudaGetLastError();
   };
