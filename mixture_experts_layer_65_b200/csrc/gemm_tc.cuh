@@ -127,6 +127,7 @@ struct GemmArgs {
                      // [M, wg_colsplit] matrices (its K_s experts), each after the previous
   float *wg_out0_shared, *wg_out1_shared, *wg_out0_routed, *wg_out1_routed;
   int64_t wg_stride;
+  int wg_v8;         // the fp32 outputs are 32-byte aligned: 32-byte stores
 };
 
 struct TileCoord {
@@ -377,12 +378,20 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA_s,
             float* dcol = (c.shared && a.wg_colsplit > 0)
                               ? dst + (int64_t)(col / a.wg_colsplit) * rows * a.wg_colsplit + col % a.wg_colsplit
                               : dst + col;
-            float4* d4 = reinterpret_cast<float4*>(dcol);
+            if (kzero) {
 #pragma unroll
-            for (int x = 0; x < 8; ++x)
-              d4[x] = kzero ? make_float4(0.f, 0.f, 0.f, 0.f)
-                            : make_float4(__uint_as_float(v[4 * x]), __uint_as_float(v[4 * x + 1]),
-                                          __uint_as_float(v[4 * x + 2]), __uint_as_float(v[4 * x + 3]));
+              for (int x = 0; x < 32; ++x) v[x] = 0u;
+            }
+            if (a.wg_v8) {
+#pragma unroll
+              for (int x = 0; x < 4; ++x)
+                st_global_v8(dcol + 8 * x, make_uint4(v[8 * x], v[8 * x + 1], v[8 * x + 2], v[8 * x + 3]),
+                             make_uint4(v[8 * x + 4], v[8 * x + 5], v[8 * x + 6], v[8 * x + 7]));
+            } else {
+              uint4* d4 = reinterpret_cast<uint4*>(dcol);
+#pragma unroll
+              for (int x = 0; x < 8; ++x) d4[x] = make_uint4(v[4 * x], v[4 * x + 1], v[4 * x + 2], v[4 * x + 3]);
+            }
           }
         }
       } else if constexpr (MODE == kGateUpBwd) {

@@ -1102,6 +1102,11 @@ moe_status moe_backward(moe_handle* H, const void* u, const int32_t* topk_idx, c
   w1.wg_out0_shared = d_w_gate; w1.wg_out1_shared = d_w_up;
   w1.wg_out0_routed = d_w_gate + ks * (size_t)I * d; w1.wg_out1_routed = d_w_up + ks * (size_t)I * d;
   w1.wg_stride = (int64_t)I * d;
+  // 32-byte stores when the caller's gradient buffers allow them (16-byte alignment is
+  // all the interface requires)
+  const bool al32 = ((reinterpret_cast<uintptr_t>(d_w_gate) | reinterpret_cast<uintptr_t>(d_w_up) |
+                      reinterpret_cast<uintptr_t>(d_w_down)) & 31u) == 0;
+  w1.wg_v8 = al32;
   launch_pdl(grouped_gemm_tc_kernel<kWgrad>, dim3(H->gemm_grid), dim3(kGemmThreads), kGemmSmemBytes, stream,
              H->tmDabsT, H->tmDabrT, H->tmUT, H->tmXpT, w1);
   MOE_CUDA(cudaGetLastError());
@@ -1115,6 +1120,7 @@ moe_status moe_backward(moe_handle* H, const void* u, const int32_t* topk_idx, c
   w2.wg_counts = expert_counts; w2.wg_bm = H->bm; w2.wg_split = 0;
   w2.wg_out0_shared = d_w_down; w2.wg_out0_routed = d_w_down + ks * (size_t)d * I;
   w2.wg_stride = (int64_t)d * I;
+  w2.wg_v8 = al32;
   w2.wg_colsplit = I;   // the shared group's K_s experts sit side by side along I
   launch_pdl(grouped_gemm_tc_kernel<kWgrad>, dim3(H->gemm_grid), dim3(kGemmThreads), kGemmSmemBytes, stream,
              H->tmDhT, H->tmDyrT, H->tmHsT, H->tmHrT, w2);

@@ -85,6 +85,40 @@ def test_backward_matches_the_oracle(name, spec, d_aux):
     layer.close()
 
 
+def test_weight_gradients_into_16_byte_aligned_buffers():
+    """The interface asks 16-byte alignment of the gradient buffers; the weight-gradient
+    epilogue stores 32 bytes per thread only when all three are 32-byte aligned.  Buffers
+    offset by 16 bytes take the other path and must get the same bits."""
+    from mixture_experts_layer_65_b200._lib import check, lib
+    from mixture_experts_layer_65_b200.layer import _ptr
+    w = W.make_workload("16b_prefill", alpha1=0.001, **SPECS[0][1])
+    rng = np.random.default_rng(5)
+    layer = MoELayer.from_workload(w)
+    layer.backward_prepare()
+    u = to_device_tensor(w.u, "cuda")
+    out = layer.forward(u)
+    dh = to_device_tensor(W.f32_to_bf16_bits(rng.standard_normal((w.T, w.d), dtype=np.float32)), "cuda")
+    du, dcen, dbias, dwg, dwu, dwd = layer.backward(u, out, dh, 1.0)
+    assert all(t.data_ptr() % 32 == 0 for t in (dwg, dwu, dwd))
+
+    def off16(t):   # same shape, storage starting 16 bytes past a 256-byte boundary
+        buf = torch.empty(t.numel() + 4, dtype=t.dtype, device=t.device)
+        return buf[4:].view(t.shape)
+
+    du2, dcen2, dbias2 = torch.empty_like(du), torch.empty_like(dcen), torch.empty_like(dbias)
+    dwg2, dwu2, dwd2 = off16(dwg), off16(dwu), off16(dwd)
+    assert all(t.data_ptr() % 32 == 16 for t in (dwg2, dwu2, dwd2))
+    s = torch.cuda.current_stream()
+    check(lib().moe_backward(layer._h, _ptr(u), _ptr(out.topk_idx), _ptr(out.topk_w),
+                             _ptr(out.expert_counts), _ptr(dh), 1.0, _ptr(du2), _ptr(dcen2),
+                             _ptr(dbias2), _ptr(dwg2), _ptr(dwu2), _ptr(dwd2), s.cuda_stream))
+    torch.cuda.synchronize()
+    layer.device_status()
+    for a, b in ((du, du2), (dcen, dcen2), (dbias, dbias2), (dwg, dwg2), (dwu, dwu2), (dwd, dwd2)):
+        assert torch.equal(a, b)
+    layer.close()
+
+
 def test_backward_refuses_unsupported_layers():
     from mixture_experts_layer_65_b200 import _lib
     w = W.make_workload("tiny")   # fp32 layer
