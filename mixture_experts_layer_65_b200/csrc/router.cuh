@@ -206,8 +206,7 @@ __device__ __forceinline__ void router_pass(int tid, int pass, int tile, int R, 
   if (j == 0) S.inv_sum[r] = valid ? inv_sum : 0.f;
   __syncwarp();   // the row's exp values (written by the eight threads of a warp) are read below
 
-  auto record = [&](int p, uint64_t g) {
-    int e = key_index(g);
+  auto record_e = [&](int p, int e) {
     if (e < 0 || e >= n_routed) {
       record_error(o.err, kErrRouteIndex);
       e = 0;
@@ -218,8 +217,74 @@ __device__ __forceinline__ void router_pass(int tid, int pass, int tile, int R, 
       atomicOr(&S.mask[e][tr >> 5], 1u << (tr & 31));
     }
   };
+  auto record = [&](int p, uint64_t g) { record_e(p, key_index(g)); };
 
-  if (MAXC <= 8 && top_k <= 8) {
+  // Fast path (top_k <= 7, the bitonic network below on 32-bit keys): the logit's order
+  // key with its low ib bits replaced by the inverted expert index, ib = bits of N_pad - 1.
+  // It ranks as the exact (logit, index) order except among logits whose keys agree above
+  // those bits; so when ranks 0 .. top_k hold no such pair the chosen experts and their
+  // ranks are exactly those of the 64-bit order, and otherwise the warp redoes its rows
+  // with 64-bit keys.
+  bool done = false;
+  if (MAXC <= 8 && top_k <= 7) {
+    const int ib = 32 - __clz(n_pad - 1);
+    const uint32_t mk = (1u << ib) - 1u;
+    uint32_t kk[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint64_t k64 = i < MAXC ? key[i < MAXC ? i : 0] : 0ull;
+      kk[i] = k64 ? (((uint32_t)(k64 >> 32) & ~mk) | (mk - (uint32_t)key_index(k64))) : 0u;
+    }
+#pragma unroll
+    for (int size = 2; size <= 8; size <<= 1) {
+#pragma unroll
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int l = i ^ stride;
+          if (l > i) {
+            const uint32_t x = kk[i], y = kk[l];
+            const bool desc = (i & size) == 0;
+            kk[i] = desc ? max(x, y) : min(x, y);
+            kk[l] = desc ? min(x, y) : max(x, y);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int m = 1; m < kRouterGroup; m <<= 1) {
+      uint32_t pk[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) pk[i] = __shfl_xor_sync(0xffffffffu, kk[i], m);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) kk[i] = max(kk[i], pk[7 - i]);
+#pragma unroll
+      for (int stride = 4; stride > 0; stride >>= 1) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int l = i ^ stride;
+          if (l > i) {
+            const uint32_t x = kk[i], y = kk[l];
+            kk[i] = max(x, y);
+            kk[l] = min(x, y);
+          }
+        }
+      }
+    }
+    bool tie = false;   // the same for the row's eight threads (they hold the same list)
+#pragma unroll
+    for (int r = 0; r < 7; ++r)
+      tie |= r < top_k && kk[r + 1] != 0u && ((kk[r] ^ kk[r + 1]) & ~mk) == 0u;
+    if (!__any_sync(0xffffffffu, tie)) {
+      uint32_t mine = 0u;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mine = i == j ? kk[i] : mine;
+      if (j < top_k) record_e(j, mine ? (int)(mk - (mine & mk)) : -1);
+      done = true;
+    }
+  }
+  if (done) {
+  } else if (MAXC <= 8 && top_k <= 8) {
     // sort the thread's keys (padded to 8 with zeros), then three bitonic merges with the
     // partner threads: every thread of the row ends up with the row's 8 largest keys
     uint64_t kk[8];
