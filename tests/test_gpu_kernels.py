@@ -159,3 +159,28 @@ def test_full_size_intermediates_on_sampled_rows_of_every_expert(name):
     print(name, f"{len(picks)} routed rows of {len(np.unique(picks[:, 2]))} experts: "
                 f"hidden err {worst_h:.2e}, output err {worst_y:.2e}")
     layer.close()
+
+
+@pytest.mark.parametrize("name,spec", [
+    ("paired_shared", dict(T=333, d=256, n_shared=2, n_routed=16, inter=192, top_k=4)),
+    ("paired_no_shared", dict(T=700, d=256, n_shared=0, n_routed=16, inter=128, top_k=2)),
+    ("decode_sized", dict(T=96, d=256, n_shared=2, n_routed=16, inter=128, top_k=4)),
+])
+def test_per_kernel_timing_records_every_slot(name, spec):
+    """moe_timing_begin / moe_timing_end (the benchmark's per-kernel slots) on every launch
+    path: each slot of each recorded forward is recorded, whether or not a kernel runs in it
+    (the permute and, on decode-sized layers, the combine run inside other kernels)."""
+    w = W.make_workload("16b_prefill", alpha1=0.001, **spec)
+    layer = MoELayer.from_workload(w)
+    u = to_device_tensor(w.u, "cuda")
+    out = layer.alloc_outputs()
+    layer.forward(u, out)
+    layer.timing_begin(3)
+    for _ in range(3):
+        layer.forward(u, out)
+    ms, n = layer.timing_end()
+    layer.device_status()
+    assert n == 3
+    assert all(np.isfinite(v) and v >= 0.0 for v in ms.values()), ms
+    assert ms["gate_up_gemm"] > 0.0 and ms["down_gemm"] > 0.0
+    layer.close()
