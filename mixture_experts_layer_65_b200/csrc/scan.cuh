@@ -65,6 +65,7 @@ struct ScanSmem {
   int32_t w_off[kScanThreads / 32], w_t1[kScanThreads / 32], w_t2[kScanThreads / 32];
   int32_t w_t3[kScanThreads / 32];
   double aux[kMaxRouted];
+  float ps_tot[kMaxRouted];   // per-expert affinity totals (step 2), read again in step 3
 };
 
 constexpr int kScanBatch = 16;  // independent loads in flight per thread
@@ -85,7 +86,10 @@ __device__ void scan_tail(const ScanArgs& a, int tid, uint8_t* smem, Sync sync) 
   const int t1 = min(a.n_tiles, t0 + seg_len);
   if (tid == 0 && a.copy_done) *a.copy_done = 0;
 
-  // 1. per-segment sums, tiles in ascending order (loads batched, adds in order)
+  // 1. per-segment sums, tiles in ascending order (loads batched, adds in order); a
+  //    segment of at most kScanBatch tiles keeps its histogram entries for step 4
+  int hkeep[kScanBatch];
+  const bool keep = t1 - t0 <= kScanBatch;
   if (active) {
     int c = 0;
     float p = 0.f;
@@ -104,6 +108,7 @@ __device__ void scan_tail(const ScanArgs& a, int tid, uint8_t* smem, Sync sync) 
           c += hv[j];
           p += pv[j];
         }
+        hkeep[j] = hv[j];   // (the first and, when kept, only batch)
       }
     }
     S.cnt[tid] = c;
@@ -121,6 +126,7 @@ __device__ void scan_tail(const ScanArgs& a, int tid, uint8_t* smem, Sync sync) 
     }
     a.expert_counts[tid] = run;
     if (a.psum_total) a.psum_total[tid] = ps;
+    S.ps_tot[tid] = ps;
     S.off[tid] = run;   // count for now, offset after step 3
   }
   sync();
@@ -145,7 +151,7 @@ __device__ void scan_tail(const ScanArgs& a, int tid, uint8_t* smem, Sync sync) 
       t2c = mt * nt2;
       t3c = mt * nt3;
       const double invT = 1.0 / (double)a.T;
-      S.aux[tid] = a.psum_total ? ((double)cnt * invT) * ((double)a.psum_total[tid] * invT) : 0.0;
+      S.aux[tid] = a.psum_total ? ((double)cnt * invT) * ((double)S.ps_tot[tid] * invT) : 0.0;
     } else if (tid < kMaxRouted) {
       S.aux[tid] = 0.0;
     }
@@ -200,7 +206,7 @@ __device__ void scan_tail(const ScanArgs& a, int tid, uint8_t* smem, Sync sync) 
       int hv[kScanBatch];
 #pragma unroll
       for (int j = 0; j < kScanBatch; ++j)
-        hv[j] = tb + j < t1 ? __ldcg(a.tile_hist + (size_t)(tb + j) * nr + e) : 0;
+        hv[j] = keep ? hkeep[j] : tb + j < t1 ? __ldcg(a.tile_hist + (size_t)(tb + j) * nr + e) : 0;
 #pragma unroll
       for (int j = 0; j < kScanBatch; ++j) {
         if (tb + j < t1) {
