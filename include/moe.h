@@ -43,7 +43,7 @@ typedef struct CUstream_st* moe_stream_t; /* identical to cudaStream_t */
 typedef enum {
   MOE_OK = 0,
   MOE_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, inconsistent sizes            */
-  MOE_ERR_UNSUPPORTED = 2,  /* a valid layer this build does not handle (see create)  */
+  MOE_ERR_UNSUPPORTED = 2,  /* a valid layer the library does not handle (see create) */
   MOE_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed                      */
   MOE_ERR_OOM = 4,          /* device allocation failed                               */
   MOE_ERR_DEVICE_CHECK = 5  /* a kernel recorded an error (bounded wait ran out, ...) */
