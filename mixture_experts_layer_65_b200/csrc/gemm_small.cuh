@@ -27,6 +27,10 @@ constexpr int kSmallBM = 128;
 constexpr int kSmallThreads = 192;
 constexpr int kSmallMaxTok = 128;
 constexpr int kSmallMaxStages = 8;
+#ifndef MOE_SMALL_SMEM_BUDGET
+#define MOE_SMALL_SMEM_BUDGET (200u * 1024u)
+#endif
+constexpr uint32_t kSmallSmemBudget = MOE_SMALL_SMEM_BUDGET;   // stage ring + epilogue buffers
 
 struct SmallGemmArgs {
   const int32_t* grp_row;   // [G] first token row of each group in the token operand / output

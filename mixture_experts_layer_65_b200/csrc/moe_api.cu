@@ -514,7 +514,7 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
                                     (int)H->simt_router_smem));
       const size_t epi = (small_epi_bytes(H->n_tok) + 15) & ~size_t(15);
       const uint32_t sb = small_stage_bytes(H->n_tok);
-      int stages = (int)((200u * 1024u - epi) / sb);
+      int stages = (int)((kSmallSmemBudget - epi) / sb);
       stages = stages > kSmallMaxStages ? kSmallMaxStages : (stages < 2 ? 2 : stages);
       H->small_stages = stages;
       // The down GEMM's grid: the fewest CTAs that still give each the same work when every
