@@ -512,10 +512,7 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
       const void* rk = with_maxc(H->maxc, [](auto m) { return (const void*)router_small_kernel<m()>; });
       MOE_CUDA(cudaFuncSetAttribute(rk, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)H->simt_router_smem));
-      const size_t epi = (small_epi_bytes(H->n_tok) + 15) & ~size_t(15);
-      const uint32_t sb = small_stage_bytes(H->n_tok);
-      int stages = (int)((kSmallSmemBudget - epi) / sb);
-      stages = stages > kSmallMaxStages ? kSmallMaxStages : (stages < 2 ? 2 : stages);
+      const int stages = small_stages(H->n_tok);
       H->small_stages = stages;
       // The down GEMM's grid: the fewest CTAs that still give each the same work when every
       // routed expert receives tokens (a tile of the shared group counts as n_shared routed
@@ -528,7 +525,7 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
         const int64_t g2 = per > 0 ? (units + per - 1) / per : H->n_sms;
         H->small_grid2 = (int)std::min<int64_t>(H->n_sms, std::max<int64_t>(1, g2));
       }
-      H->small_smem = 1024 + (size_t)stages * sb + epi + 256;
+      H->small_smem = small_smem_bytes(H->n_tok, stages);
       MOE_CUDA(cudaFuncSetAttribute((const void*)grouped_gemm_small_kernel<kGateUpSwiGLU>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)H->small_smem));
       MOE_CUDA(cudaFuncSetAttribute((const void*)grouped_gemm_small_kernel<kDown>,

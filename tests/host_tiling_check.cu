@@ -114,6 +114,14 @@ int main() {
       }
     }
   }
+  // small-batch GEMM: for every token width a ring of 2 .. kSmallMaxStages stages that fits
+  // the opt-in shared memory with the epilogue buffers and the control block
+  for (int nt = 16; nt <= kSmallMaxTok; nt += 16) {
+    const int st = small_stages(nt);
+    CHECK(st >= 2 && st <= kSmallMaxStages, "n_tok=%d stages=%d", nt, st);
+    CHECK(small_smem_bytes(nt, st) <= kRouterSmemBudget, "n_tok=%d bytes=%zu", nt, small_smem_bytes(nt, st));
+    CHECK(small_stage_bytes(nt) % 1024 == 0, "n_tok=%d stage %u", nt, small_stage_bytes(nt));
+  }
   // the paired GEMM's ring and control block fit the opt-in shared memory
   CHECK(kGemmSmemBytes <= kRouterSmemBudget, "GEMM smem %zu", kGemmSmemBytes);
   CHECK(kGemmStageBytes % 1024 == 0, "GEMM stage %u", kGemmStageBytes);
