@@ -7,23 +7,32 @@
 // from HBM once and the tensor cores do almost no padding work, which makes the kernel a
 // weight-streaming one, as a decode step is.  Groups without tokens get no tiles.
 //
-//   mode kGateUpSwiGLU: a 128-row tile of the interleaved gate/up weights is one block of
-//                       64 gate rows followed by the 64 matching up rows; TMEM lane L < 64
-//                       holds gate values, lane L + 64 the up values of the same column.
-//   mode kDown:         a 128-row tile of W_down gives 128 output features.
+// A tile is two 128-row weight blocks that share the token operand: per k-block two MMAs
+// (M = 128, N = n_tok) write the two halves of one accumulator, columns [0, n_tok) and
+// [n_tok, 2 n_tok).
+//   mode kGateUpSwiGLU: the gate rows and the up rows of 128 intermediate features (the
+//                       interleaved weight layout keeps 64-row gate and up blocks, so each
+//                       half is two 64-row loads); TMEM lane L then holds gate and up of
+//                       feature L side by side and the SwiGLU needs no exchange.
+//   mode kDown:         W_down rows of 256 output features, 128 per half.
+// Rows past a group's width (its last tile) are outside the weight tensor map's box range
+// and arrive as zeros; their outputs are not stored.
 //
-// One CTA per SM (persistent), 192 threads: warp 0 issues TMA loads (weights 128 x 64 and
-// tokens n_tok x 64, 128-byte swizzle) into a multi-stage ring; warp 1 allocates TMEM (two
-// n_tok-column fp32 accumulators) and one thread issues tcgen05.mma (M = 128, N = n_tok);
-// warps 2..5 drain the accumulator, transpose through shared memory and store whole token
-// rows (coalesced).
+// One CTA per SM (persistent), 192 threads: warp 0 issues TMA loads (weights 2 x 128 x 64
+// and tokens n_tok x 64, 128-byte swizzle) into a multi-stage ring; warp 1 allocates TMEM
+// (two 2 n_tok-column fp32 accumulators) and one thread issues tcgen05.mma; warps 2..5
+// drain the accumulator (one TMEM lane = one output feature per thread) and store each
+// token's features straight from registers (a warp writes 32 consecutive features, 64
+// bytes, per token).  No shared memory besides the ring, so the ring holds as many stages
+// as fit: the kernel's speed follows the weight bytes in flight per SM.
 #pragma once
 
 #include "gemm_tc.cuh"
 
 namespace moe {
 
-constexpr int kSmallBM = 128;
+constexpr int kSmallBM = 128;               // weight rows per MMA (M)
+constexpr uint32_t kSmallWBytes = kSmallBM * 128u;   // one 128-row weight block per k-block
 constexpr int kSmallThreads = 192;
 constexpr int kSmallMaxTok = 128;
 constexpr int kSmallMaxStages = 8;
@@ -36,7 +45,8 @@ struct SmallGemmArgs {
   int n_tok;                // N of the MMA: multiple of 16, >= every group's token count
   int stages;
   int kb_shared, kb_routed; // K / 64
-  int mt_shared, mt_routed; // weight-row tiles per group
+  int cols_shared, cols_routed;   // output features of a group (its tiles cover them in
+                                  // steps of 128 (gate/up) or 256 (down))
   __nv_bfloat16* out_shared;
   int64_t ld_shared;
   __nv_bfloat16* out_routed;
@@ -71,26 +81,26 @@ __host__ __device__ inline int small_tile_at(int pos, int total, int n_sh, int g
   return !rebalance ? pos : pos < r0 ? n_sh + pos : pos < r0 + n_sh ? pos - r0 : pos;
 }
 
-// smem: stages x (weights 16 KB + tokens n_tok x 128 B) | epilogue buffers | barriers
+// smem: stages x (weights 2 x 16 KB + tokens n_tok x 128 B) | barriers
 __host__ __device__ constexpr uint32_t small_stage_bytes(int n_tok) {
-  return kSmallBM * 128u + (((uint32_t)n_tok * 128u + 1023u) & ~1023u);
+  return 2u * kSmallWBytes + (((uint32_t)n_tok * 128u + 1023u) & ~1023u);
 }
-__host__ __device__ constexpr size_t small_epi_bytes(int n_tok) {
-  // up values [64][n_tok + 1] fp32 and the transposed output tile [n_tok][128] bf16
-  return (size_t)64 * (n_tok + 1) * 4 + (size_t)n_tok * kSmallBM * 2;
-}
-
-// dynamic shared memory: alignment slack, stage ring, epilogue buffers, control block
+// dynamic shared memory: alignment slack, stage ring, control block
 __host__ __device__ constexpr size_t small_smem_bytes(int n_tok, int stages) {
-  return 1024 + (size_t)stages * small_stage_bytes(n_tok) + ((small_epi_bytes(n_tok) + 15) & ~size_t(15)) +
-         256;
+  return 1024 + (size_t)stages * small_stage_bytes(n_tok) + 256;
 }
 // The ring takes as many stages as the opt-in shared memory holds (at most kSmallMaxStages,
-// at least 2): the kernel streams weights, and each stage more keeps another 16 KB of them
-// in flight per SM (six stages -> eight: 215.1 -> 211.6 us per 16B decode forward).
+// at least 2): the kernel streams weights, and the more weight bytes it keeps in flight per
+// SM the faster it streams them (16B decode: 96 -> 128 KB in flight, 215.1 -> 211.6 us per
+// forward).
 __host__ __device__ constexpr int small_stages(int n_tok) {
   const long st = ((long)kRouterSmemBudget - (long)small_smem_bytes(n_tok, 0)) / (long)small_stage_bytes(n_tok);
   return st > kSmallMaxStages ? kSmallMaxStages : (st < 2 ? 2 : (int)st);
+}
+// TMEM columns: two accumulators of 2 n_tok columns, a power of two >= 32
+__host__ __device__ constexpr uint32_t small_tmem_cols(int n_tok) {
+  return 4u * (uint32_t)n_tok <= 32u ? 32u : 4u * (uint32_t)n_tok <= 64u ? 64u
+         : 4u * (uint32_t)n_tok <= 128u ? 128u : 4u * (uint32_t)n_tok <= 256u ? 256u : 512u;
 }
 
 template <int MODE>
@@ -107,9 +117,7 @@ grouped_gemm_small_kernel(const __grid_constant__ CUtensorMap tmW_s,
   const int nt = a.n_tok;
   const uint32_t stage_bytes = small_stage_bytes(nt);
   const uint32_t x_bytes = (uint32_t)nt * 128u;
-  float* upbuf = reinterpret_cast<float*>(base + (size_t)S * stage_bytes);
-  __nv_bfloat16* obuf = reinterpret_cast<__nv_bfloat16*>(upbuf + 64 * (nt + 1));
-  uint8_t* ctl = base + (size_t)S * stage_bytes + ((small_epi_bytes(nt) + 15) & ~size_t(15));
+  uint8_t* ctl = base + (size_t)S * stage_bytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(ctl);
   uint64_t* empty = full + kSmallMaxStages;
   uint64_t* acc_full = empty + kSmallMaxStages;
@@ -119,8 +127,7 @@ grouped_gemm_small_kernel(const __grid_constant__ CUtensorMap tmW_s,
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  uint32_t tmem_cols = 32;
-  while (tmem_cols < 2u * (uint32_t)nt) tmem_cols <<= 1;
+  const uint32_t tmem_cols = small_tmem_cols(nt);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -185,14 +192,20 @@ grouped_gemm_small_kernel(const __grid_constant__ CUtensorMap tmW_s,
           if (!ok) break;
           const uint32_t sa = smem_u32(base + (size_t)stage * stage_bytes);
           const uint32_t fb = smem_u32(&full[stage]);
-          mbar_arrive_expect_tx(fb, kSmallBM * 128u + x_bytes);
-          if (sh) {
-            tma_load_2d(sa, &tmW_s, fb, kb * 64, m * kSmallBM);
-            tma_load_2d(sa + kSmallBM * 128u, &tmX_s, fb, kb * 64, 0);
-          } else {
-            tma_load_3d(sa, &tmW_r, fb, kb * 64, m * kSmallBM, e);
-            tma_load_2d(sa + kSmallBM * 128u, &tmX_r, fb, kb * 64, xrow);
+          mbar_arrive_expect_tx(fb, 2u * kSmallWBytes + x_bytes);
+          // weight halves: gate/up -- half 0 the gate rows, half 1 the up rows of features
+          // [128 m, 128 m + 128), each from the 64-row blocks 2m and 2m + 1 of the
+          // interleaved layout (rows 256 m + 128 h + 64 half); down -- rows 256 m + 128 half
+          for (int half = 0; half < 2; ++half) {
+            for (int h = 0; h < (MODE == kGateUpSwiGLU ? 2 : 1); ++h) {
+              const uint32_t dst = sa + (uint32_t)half * kSmallWBytes + (uint32_t)h * (kSmallWBytes / 2);
+              const int row = MODE == kGateUpSwiGLU ? 256 * m + 128 * h + 64 * half : 256 * m + 128 * half;
+              if (sh) tma_load_2d(dst, &tmW_s, fb, kb * 64, row);
+              else tma_load_3d(dst, &tmW_r, fb, kb * 64, row, e);
+            }
           }
+          if (sh) tma_load_2d(sa + 2u * kSmallWBytes, &tmX_s, fb, kb * 64, 0);
+          else tma_load_2d(sa + 2u * kSmallWBytes, &tmX_r, fb, kb * 64, xrow);
           issued |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (phase << stage);
           if (++stage == S) { stage = 0; phase ^= 1u; }
@@ -218,16 +231,19 @@ grouped_gemm_small_kernel(const __grid_constant__ CUtensorMap tmW_s,
         ok = mbar_wait(smem_u32(&acc_empty[acc]), acc_par ^ 1u, abort_flag, a.err, kErrWaitMma);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t dt = tmem_base + (uint32_t)(acc * nt);
+        const uint32_t dt = tmem_base + (uint32_t)(acc * 2 * nt);
         for (int kb = 0; kb < kbn; ++kb) {
           ok = mbar_wait(smem_u32(&full[stage]), phase, abort_flag, a.err, kErrWaitMma);
           if (!ok) break;
           tc_fence_after();
           const uint32_t sa = smem_u32(base + (size_t)stage * stage_bytes);
-          const uint64_t adesc = sdesc_k_sw128(sa), bdesc = sdesc_k_sw128(sa + kSmallBM * 128u);
+          const uint64_t a0 = sdesc_k_sw128(sa), a1 = sdesc_k_sw128(sa + kSmallWBytes);
+          const uint64_t bdesc = sdesc_k_sw128(sa + 2u * kSmallWBytes);
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            tc_mma_f16(dt, adesc + 2u * k, bdesc + 2u * k, idesc, (kb | k) != 0);
+          for (int k = 0; k < 4; ++k) {
+            tc_mma_f16(dt, a0 + 2u * k, bdesc + 2u * k, idesc, (kb | k) != 0);
+            tc_mma_f16(dt + (uint32_t)nt, a1 + 2u * k, bdesc + 2u * k, idesc, (kb | k) != 0);
+          }
           tc_commit(smem_u32(&empty[stage]));
           if (++stage == S) { stage = 0; phase ^= 1u; }
         }
@@ -239,7 +255,7 @@ grouped_gemm_small_kernel(const __grid_constant__ CUtensorMap tmW_s,
     __syncwarp();
   } else {
     const int q = warp & 3;              // TMEM lane quadrant
-    const int L = q * 32 + lane;         // TMEM lane = weight row of the tile
+    const int L = q * 32 + lane;         // TMEM lane = weight row of each half
     const int et = threadIdx.x - 64;     // 0..127
     if (MODE == kGateUpSwiGLU && a.copy_done != nullptr) {
       // the routed token rows, one warp per row (eight 16-byte vectors per lane in flight)
@@ -279,70 +295,49 @@ grouped_gemm_small_kernel(const __grid_constant__ CUtensorMap tmW_s,
       decode(tile, g, m, e, sh);
       const int acc = it & 1;
       const uint32_t acc_par = (it >> 1) & 1;
-      bool ok = true;
-      if (et == 0) ok = mbar_wait(smem_u32(&acc_full[acc]), acc_par, abort_flag, a.err, kErrWaitEpilogue);
-      if (named_bar_any(2, 128, !ok)) break;
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(smem_u32(&acc_full[acc]), acc_par, abort_flag, a.err, kErrWaitEpilogue);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;   // warp-uniform decision
       tc_fence_after();
-      const uint32_t trow = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + (uint32_t)(acc * nt);
+      const uint32_t trow = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + (uint32_t)(acc * 2 * nt);
       const int rows = sh ? a.T : __ldg(&a.counts[e]);
       const int64_t row0 = __ldg(&a.grp_row[g]);
       __nv_bfloat16* out = sh ? a.out_shared : a.out_routed;
       const int64_t ld = sh ? a.ld_shared : a.ld_routed;
-      if (MODE == kGateUpSwiGLU) {
-        if (L >= 64) {   // up rows: park them in shared memory for their gate partners
-          for (int c = 0; c < nt; c += 16) {
-            uint32_t v[16];
-            __syncwarp();
-            tmem_ld16(trow + (uint32_t)c, v);
-            tmem_ld_wait16(v);
+      const int cols = sh ? a.cols_shared : a.cols_routed;
+      // this thread's output features: gate/up -- feature 128 m + L (gate in the first half
+      // of the accumulator, up in the second); down -- 256 m + L and 256 m + 128 + L
+      const int f0 = (MODE == kGateUpSwiGLU ? 128 : 256) * m + L;
+      const int f1 = f0 + 128;
+      for (int c = 0; c < rows; c += 16) {
+        uint32_t v0[16], v1[16];
+        __syncwarp();
+        tmem_ld16(trow + (uint32_t)c, v0);
+        tmem_ld16(trow + (uint32_t)(nt + c), v1);
+        tmem_ld_wait16(v0);
+        tmem_ld_wait16(v1);
+        __nv_bfloat16* o = out + (row0 + c) * ld;
+        const int nj = rows - c < 16 ? rows - c : 16;
+        if (MODE == kGateUpSwiGLU) {
+          if (f0 < cols) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) upbuf[(L - 64) * (nt + 1) + c + j] = __uint_as_float(v[j]);
+            for (int j = 0; j < 16; ++j)
+              if (j < nj)
+                o[(int64_t)j * ld + f0] = __float2bfloat16_rn(silu_fast(__uint_as_float(v0[j])) *
+                                                              __uint_as_float(v1[j]));
           }
-        }
-        named_bar_sync(2, 128);
-        if (L < 64) {    // gate rows: SiLU(gate) * up, token-major into the output tile
-          for (int c = 0; c < nt; c += 16) {
-            uint32_t v[16];
-            __syncwarp();
-            tmem_ld16(trow + (uint32_t)c, v);
-            tmem_ld_wait16(v);
+        } else {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const float h = silu_fast(__uint_as_float(v[j])) * upbuf[L * (nt + 1) + c + j];
-              obuf[(size_t)(c + j) * 64 + L] = __float2bfloat16_rn(h);
+          for (int j = 0; j < 16; ++j) {
+            if (j < nj) {
+              if (f0 < cols) o[(int64_t)j * ld + f0] = __float2bfloat16_rn(__uint_as_float(v0[j]));
+              if (f1 < cols) o[(int64_t)j * ld + f1] = __float2bfloat16_rn(__uint_as_float(v1[j]));
             }
           }
         }
-        tc_fence_before();
-        named_bar_sync(2, 128);
-        // rows of 64 outputs (128 B = 8 vectors) per token
-        const int col0 = m * 64;
-        for (int idx = et; idx < rows * 8; idx += 128) {
-          const int n = idx >> 3, v8 = idx & 7;
-          *reinterpret_cast<uint4*>(out + (row0 + n) * ld + col0 + v8 * 8) =
-              *reinterpret_cast<const uint4*>(obuf + (size_t)n * 64 + v8 * 8);
-        }
-      } else {
-        for (int c = 0; c < nt; c += 16) {
-          uint32_t v[16];
-          __syncwarp();
-          tmem_ld16(trow + (uint32_t)c, v);
-          tmem_ld_wait16(v);
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            obuf[(size_t)(c + j) * kSmallBM + L] = __float2bfloat16_rn(__uint_as_float(v[j]));
-        }
-        tc_fence_before();
-        named_bar_sync(2, 128);
-        // rows of 128 outputs (256 B = 16 vectors) per token
-        const int col0 = m * kSmallBM;
-        for (int idx = et; idx < rows * 16; idx += 128) {
-          const int n = idx >> 4, v16 = idx & 15;
-          *reinterpret_cast<uint4*>(out + (row0 + n) * ld + col0 + v16 * 8) =
-              *reinterpret_cast<const uint4*>(obuf + (size_t)n * kSmallBM + v16 * 8);
-        }
       }
-      named_bar_sync(2, 128);   // output tile and up buffer are reused by the next tile
+      tc_fence_before();
+      __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&acc_empty[acc]));
     }
   }

@@ -136,6 +136,7 @@ struct moe_handle {
   float *w_dev = nullptr, *aux_dev = nullptr;
   CUtensorMap tmE, tmXp, tmWguS, tmWguR, tmHs, tmHr, tmWdS, tmWdR;
   CUtensorMap tmXpN, tmHsN, tmHrN;   // token operands of the small-batch GEMMs (n_tok rows)
+  CUtensorMap tmWguS64, tmWguR64;    // gate/up weights in 64-row boxes (small-batch gate/up GEMM)
   // moe_forward_host_pipelined: copy-in / forward / copy-out streams, two staging slots
   struct PipeSlot {
     void *u = nullptr, *h = nullptr;
@@ -518,7 +519,7 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
       // routed expert receives tokens (a tile of the shared group counts as n_shared routed
       // tiles: its K is n_shared * inter), so that no CTA runs a last tile alone.
       {
-        const int64_t mt = d / kSmallBM;
+        const int64_t mt = (d + 2 * kSmallBM - 1) / (2 * kSmallBM);   // 256 features per tile
         const int64_t act = std::min<int64_t>((int64_t)nr, (int64_t)c.T * c.top_k);
         const int64_t units = act * mt + (ks ? mt * (int64_t)ks : 0);
         const int64_t per = (units + H->n_sms - 1) / H->n_sms;
@@ -531,9 +532,15 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
       MOE_CUDA(cudaFuncSetAttribute((const void*)grouped_gemm_small_kernel<kDown>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)H->small_smem));
       bool okn = encode_2d(&H->tmXpN, H->xp, d, rc, (uint32_t)H->n_tok) &&
-           encode_2d(&H->tmHrN, H->hr, I, rc, (uint32_t)H->n_tok);
-      if (ks) okn = okn && encode_2d(&H->tmHsN, H->hs, Is, tp, (uint32_t)H->n_tok);
-      else H->tmHsN = H->tmHrN;
+           encode_2d(&H->tmHrN, H->hr, I, rc, (uint32_t)H->n_tok) &&
+           encode_3d(&H->tmWguR64, H->w_gu_r, d, 2 * I, nr, 64);
+      if (ks)
+        okn = okn && encode_2d(&H->tmHsN, H->hs, Is, tp, (uint32_t)H->n_tok) &&
+              encode_2d(&H->tmWguS64, H->w_gu_s, d, 2 * Is, 64);
+      else {
+        H->tmHsN = H->tmHrN;
+        H->tmWguS64 = H->tmWguR64;
+      }
       if (!okn) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for a small-batch operand");
     }
   } else {
@@ -581,8 +588,8 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
   const moe_cfg& c = H->cfg;
   const int T = c.T, d = c.d, K = c.top_k, nr = c.n_routed;
 
-  const int bn1 = H->small ? 64 : (H->bf16 ? kGemmBN / 2 : kSimtBN);
-  const int bn2 = H->small ? kSmallBM : (H->bf16 ? kGemmBN : kSimtBN);
+  const int bn1 = H->small ? kSmallBM : (H->bf16 ? kGemmBN / 2 : kSimtBN);
+  const int bn2 = H->small ? 2 * kSmallBM : (H->bf16 ? kGemmBN : kSimtBN);
   ScanArgs sa{H->tile_hist, H->tile_psum, H->n_tiles, nr, T, H->has_shared, H->inter_shared,
               c.inter, d, H->bm, H->tile_rows, bn1, bn2, c.alpha1, expert_counts, aux_loss,
               H->psum_total,
@@ -656,7 +663,7 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
     s1.grp_row = H->grp_row; s1.ts = H->ts1; s1.counts = expert_counts; s1.G = H->G;
     s1.has_shared = H->has_shared; s1.T = T; s1.n_tok = H->n_tok; s1.stages = H->small_stages;
     s1.kb_shared = d / 64; s1.kb_routed = d / 64;
-    s1.mt_shared = Is / 64; s1.mt_routed = I / 64;
+    s1.cols_shared = Is; s1.cols_routed = I;
     s1.out_shared = static_cast<__nv_bfloat16*>(H->hs); s1.ld_shared = Is;
     s1.out_routed = static_cast<__nv_bfloat16*>(H->hr); s1.ld_routed = I;
     s1.err = H->err;
@@ -665,13 +672,13 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
     s1.xp = static_cast<__nv_bfloat16*>(H->xp); s1.n_rows = T * K; s1.copy_vecs = d / 8;
     s1.copy_done = H->copy_done;
     tick(H, stream, 3);
-    launch_pdl(grouped_gemm_small_kernel<kGateUpSwiGLU>, dim3(H->n_sms), dim3(kSmallThreads), H->small_smem, stream,  H->tmWguS, H->tmWguR, tmUN, H->tmXpN, s1);
+    launch_pdl(grouped_gemm_small_kernel<kGateUpSwiGLU>, dim3(H->n_sms), dim3(kSmallThreads), H->small_smem, stream,  H->tmWguS64, H->tmWguR64, tmUN, H->tmXpN, s1);
     MOE_CUDA(cudaGetLastError());
     SmallGemmArgs s2 = s1;
     s2.copy_done = nullptr;   // no row copy: the activations are expert-contiguous rows
     s2.ts = H->ts2;
     s2.kb_shared = Is / 64; s2.kb_routed = I / 64;
-    s2.mt_shared = d / kSmallBM; s2.mt_routed = d / kSmallBM;
+    s2.cols_shared = d; s2.cols_routed = d;
     s2.out_shared = static_cast<__nv_bfloat16*>(H->ys); s2.ld_shared = d;
     s2.out_routed = static_cast<__nv_bfloat16*>(H->yr); s2.ld_routed = d;
     tick(H, stream, 4);
