@@ -1,4 +1,5 @@
-// gemm_small.cuh -- grouped expert GEMMs for small token counts (decode), weights on M.
+// gemm_small.cuh -- the expert FFN for small token counts (decode): both grouped GEMMs,
+// weights on M, in one persistent kernel (decode_ffn_kernel).
 //
 // Same FFN as gemm_tc.cuh (SwiGLU experts, K_s shared experts as one always-on group), for
 // layers whose groups hold few tokens (every group's token count <= n_tok <= 128).  The
@@ -37,49 +38,40 @@ constexpr int kSmallThreads = 192;
 constexpr int kSmallMaxTok = 128;
 constexpr int kSmallMaxStages = 8;
 
-struct SmallGemmArgs {
-  const int32_t* grp_row;   // [G] first token row of each group in the token operand / output
-  const int32_t* ts;        // [G + 1] tile prefix (a group has tiles only if it has tokens)
-  const int32_t* counts;    // [n_routed] tokens of each routed group (shared group: T)
-  int G, has_shared, T;
-  int n_tok;                // N of the MMA: multiple of 16, >= every group's token count
-  int stages;
-  int kb_shared, kb_routed; // K / 64
+// One of the decode FFN kernel's two GEMMs.
+struct SmallPhase {
+  const int32_t* ts;              // [G + 1] tile prefix (a group has tiles only if it has tokens)
+  int kb_shared, kb_routed;       // K / 64
   int cols_shared, cols_routed;   // output features of a group (its tiles cover them in
                                   // steps of 128 (gate/up) or 256 (down))
   __nv_bfloat16* out_shared;
   int64_t ld_shared;
   __nv_bfloat16* out_routed;
   int64_t ld_routed;
+};
+
+struct SmallGemmArgs {
+  const int32_t* grp_row;   // [G] first token row of each group in the token operands / outputs
+  const int32_t* counts;    // [n_routed] tokens of each routed group (shared group: T)
+  int G, has_shared, T;
+  int n_tok;                // N of the MMA: multiple of 16, >= every group's token count
+  int stages;
+  SmallPhase ph[2];         // 0: gate/up + SwiGLU -> Hmid, 1: down -> Y
   int* err;
-  // Fused row copy (gate/up GEMM): with copy_done != nullptr the epilogue warps, before
-  // their first tile, copy token row row_tok[r] of u to row r of xp for every routed row
-  // r < n_rows (16-byte vectors, copy_vecs per row), then each adds 1 to *copy_done; a
-  // CTA's producer waits for all gridDim.x * 4 of them before loading its first routed
-  // token tile (the shared group reads u itself).  The wait relies on the whole grid being
-  // resident at once (one CTA per SM).
+  // Row copy: the epilogue warps, before their first tile, copy token row row_tok[r] of u
+  // to row r of xp for every routed row r < n_rows (16-byte vectors, copy_vecs per row),
+  // then each adds 1 to sync[0]; a CTA's producer waits for all gridDim.x * 4 of them
+  // before loading its first routed token tile (the shared group reads u itself).
   const int32_t* row_tok;
   const __nv_bfloat16* u;
   __nv_bfloat16* xp;
   int n_rows, copy_vecs;
-  int* copy_done;
+  // Counters, zeroed by the scan: sync[0] the row copies; sync[1 + g] the epilogue warps
+  // that have stored group g's activations (four per gate/up tile), which a producer waits
+  // for before loading one of g's down tiles.  Both waits rely on the whole grid being
+  // resident at once (one CTA per SM, at most one CTA per SM launched).
+  int* sync;
 };
-
-// Schedule of the small-batch GEMM: tiles go round-robin to the CTAs, so the first
-// total % grid CTAs get one tile more.  When the shared group's tiles are heavier (K =
-// n_shared * inter against inter), they are placed on CTAs that get one tile fewer:
-// position p of the round-robin order visits tile small_tile_at(p).  The map is a
-// bijection of [0, total) and keeps each CTA's tile indices increasing (the group search
-// relies on it); it applies only when the target positions r0 .. r0 + n_sh - 1 (r0 =
-// total % grid) exist and lie in the first round.
-__host__ __device__ inline bool small_rebalance(int total, int n_sh, int grid, bool shared_heavier) {
-  const int r0 = total % grid;
-  return n_sh > 0 && shared_heavier && r0 > 0 && n_sh <= grid - r0 && r0 + n_sh <= total;
-}
-__host__ __device__ inline int small_tile_at(int pos, int total, int n_sh, int grid, bool rebalance) {
-  const int r0 = total % grid;
-  return !rebalance ? pos : pos < r0 ? n_sh + pos : pos < r0 + n_sh ? pos - r0 : pos;
-}
 
 // smem: stages x (weights 2 x 16 KB + tokens n_tok x 128 B) | barriers
 __host__ __device__ constexpr uint32_t small_stage_bytes(int n_tok) {
@@ -103,12 +95,17 @@ __host__ __device__ constexpr uint32_t small_tmem_cols(int n_tok) {
          : 4u * (uint32_t)n_tok <= 128u ? 128u : 4u * (uint32_t)n_tok <= 256u ? 256u : 512u;
 }
 
-template <int MODE>
-__global__ void __launch_bounds__(kSmallThreads, 1)
-grouped_gemm_small_kernel(const __grid_constant__ CUtensorMap tmW_s,
-                          const __grid_constant__ CUtensorMap tmW_r,
-                          const __grid_constant__ CUtensorMap tmX_s,
-                          const __grid_constant__ CUtensorMap tmX_r, SmallGemmArgs a) {
+// The decode FFN: both GEMMs in one persistent kernel.  The gate/up tiles (phase 0) and then
+// the down tiles (phase 1) are handed out round-robin over one list, so the down tiles fill
+// the gaps the gate/up tiles leave and the weights stream without a break between the two
+// GEMMs.  A down tile of group g waits (bounded) until every gate/up tile of g has stored
+// its activations.
+static __global__ void __launch_bounds__(kSmallThreads, 1)
+decode_ffn_kernel(const __grid_constant__ CUtensorMap tmW0_s, const __grid_constant__ CUtensorMap tmW0_r,
+                  const __grid_constant__ CUtensorMap tmX0_s, const __grid_constant__ CUtensorMap tmX0_r,
+                  const __grid_constant__ CUtensorMap tmW1_s, const __grid_constant__ CUtensorMap tmW1_r,
+                  const __grid_constant__ CUtensorMap tmX1_s, const __grid_constant__ CUtensorMap tmX1_r,
+                  SmallGemmArgs a) {
   pdl_launch_dependents();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -141,10 +138,14 @@ grouped_gemm_small_kernel(const __grid_constant__ CUtensorMap tmW_s,
     mbar_init(smem_u32(drain), 1);
     *abort_flag = 0;
     fence_mbar_init();
-    tma_prefetch_desc(&tmW_s);
-    tma_prefetch_desc(&tmW_r);
-    tma_prefetch_desc(&tmX_s);
-    tma_prefetch_desc(&tmX_r);
+    tma_prefetch_desc(&tmW0_s);
+    tma_prefetch_desc(&tmW0_r);
+    tma_prefetch_desc(&tmX0_s);
+    tma_prefetch_desc(&tmX0_r);
+    tma_prefetch_desc(&tmW1_s);
+    tma_prefetch_desc(&tmW1_r);
+    tma_prefetch_desc(&tmX1_s);
+    tma_prefetch_desc(&tmX1_r);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), tmem_cols);
@@ -155,38 +156,52 @@ grouped_gemm_small_kernel(const __grid_constant__ CUtensorMap tmW_s,
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   pdl_wait();   // the tile tables and operands come from the previous kernels
-  const int total = __ldg(&a.ts[a.G]);
+  const int total0 = __ldg(&a.ph[0].ts[a.G]);
+  const int total = total0 + __ldg(&a.ph[1].ts[a.G]);
 
-  // tile -> (group g, weight tile m); GemmArgs-style decode with one token tile per group,
-  // in the order of small_tile_at
-  const int n_sh = a.has_shared ? __ldg(&a.ts[1]) : 0;
-  const bool rebalance = small_rebalance(total, n_sh, (int)gridDim.x, a.kb_shared > a.kb_routed);
-  auto decode = [&](int pos, int& g, int& m, int& e, bool& sh) {
-    const int tile = small_tile_at(pos, total, n_sh, (int)gridDim.x, rebalance);
-    while (g < a.G - 1 && tile >= __ldg(&a.ts[g + 1])) ++g;
-    m = tile - __ldg(&a.ts[g]);
-    sh = a.has_shared && g == 0;
-    e = g - a.has_shared;
+  // position -> (phase, group g, weight tile m of the group, routed expert e, shared?);
+  // each role walks its positions in increasing order with a group cursor that restarts
+  // when the phase changes
+  struct Cursor { int phase = 0, g = 0; };
+  auto decode = [&](int pos, Cursor& cu, int& m, int& e, bool& sh) {
+    const int ph = pos < total0 ? 0 : 1;
+    if (ph != cu.phase) { cu.phase = ph; cu.g = 0; }
+    const int tile = ph ? pos - total0 : pos;
+    const int32_t* ts = a.ph[ph].ts;
+    while (cu.g < a.G - 1 && tile >= __ldg(&ts[cu.g + 1])) ++cu.g;
+    m = tile - __ldg(&ts[cu.g]);
+    sh = a.has_shared && cu.g == 0;
+    e = cu.g - a.has_shared;
   };
 
   if (warp == 0) {
     if (lane == 0) {
-      int stage = 0, g = 0;
+      int stage = 0;
+      Cursor cu;
       uint32_t phase = 0, issued = 0, last_par = 0;
       bool ok = true;
-      bool rows_ready = MODE != kGateUpSwiGLU || a.copy_done == nullptr;
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      bool rows_ready = false;
+      for (int pos = blockIdx.x; pos < total && ok; pos += gridDim.x) {
         int m, e;
         bool sh;
-        decode(tile, g, m, e, sh);
-        if (!sh && !rows_ready) {   // the routed token rows are copied by the epilogue warps
-          ok = counter_wait(a.copy_done, (int)gridDim.x * 4, abort_flag, a.err, kErrWaitCopy);
+        decode(pos, cu, m, e, sh);
+        const int ph = cu.phase, g = cu.g;
+        if (ph == 0 && !sh && !rows_ready) {   // the routed token rows, copied by the epilogue warps
+          ok = counter_wait(a.sync, (int)gridDim.x * 4, abort_flag, a.err, kErrWaitCopy);
           if (!ok) break;
           fence_proxy_async_global();   // the copied rows, seen by the TMA loads below
           rows_ready = true;
         }
-        const int xrow = __ldg(&a.grp_row[g]);
-        const int kbn = sh ? a.kb_shared : a.kb_routed;
+        if (ph == 1) {   // the group's activations, stored by the epilogues of its gate/up tiles
+          const int need = 4 * (__ldg(&a.ph[0].ts[g + 1]) - __ldg(&a.ph[0].ts[g]));
+          ok = counter_wait(a.sync + 1 + g, need, abort_flag, a.err, kErrWaitHidden);
+          if (!ok) break;
+          fence_proxy_async_global();
+        }
+        const CUtensorMap* tw = ph == 0 ? (sh ? &tmW0_s : &tmW0_r) : (sh ? &tmW1_s : &tmW1_r);
+        const CUtensorMap* tx = ph == 0 ? (sh ? &tmX0_s : &tmX0_r) : (sh ? &tmX1_s : &tmX1_r);
+        const int xrow = sh ? 0 : __ldg(&a.grp_row[g]);
+        const int kbn = sh ? a.ph[ph].kb_shared : a.ph[ph].kb_routed;
         for (int kb = 0; kb < kbn; ++kb) {
           ok = mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, a.err, kErrWaitProducer);
           if (!ok) break;
@@ -197,15 +212,14 @@ grouped_gemm_small_kernel(const __grid_constant__ CUtensorMap tmW_s,
           // [128 m, 128 m + 128), each from the 64-row blocks 2m and 2m + 1 of the
           // interleaved layout (rows 256 m + 128 h + 64 half); down -- rows 256 m + 128 half
           for (int half = 0; half < 2; ++half) {
-            for (int h = 0; h < (MODE == kGateUpSwiGLU ? 2 : 1); ++h) {
+            for (int h = 0; h < (ph == 0 ? 2 : 1); ++h) {
               const uint32_t dst = sa + (uint32_t)half * kSmallWBytes + (uint32_t)h * (kSmallWBytes / 2);
-              const int row = MODE == kGateUpSwiGLU ? 256 * m + 128 * h + 64 * half : 256 * m + 128 * half;
-              if (sh) tma_load_2d(dst, &tmW_s, fb, kb * 64, row);
-              else tma_load_3d(dst, &tmW_r, fb, kb * 64, row, e);
+              const int row = ph == 0 ? 256 * m + 128 * h + 64 * half : 256 * m + 128 * half;
+              if (sh) tma_load_2d(dst, tw, fb, kb * 64, row);
+              else tma_load_3d(dst, tw, fb, kb * 64, row, e);
             }
           }
-          if (sh) tma_load_2d(sa + 2u * kSmallWBytes, &tmX_s, fb, kb * 64, 0);
-          else tma_load_2d(sa + 2u * kSmallWBytes, &tmX_r, fb, kb * 64, xrow);
+          tma_load_2d(sa + 2u * kSmallWBytes, tx, fb, kb * 64, xrow);
           issued |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (phase << stage);
           if (++stage == S) { stage = 0; phase ^= 1u; }
@@ -218,14 +232,15 @@ grouped_gemm_small_kernel(const __grid_constant__ CUtensorMap tmW_s,
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(kSmallBM, nt);
-      int stage = 0, g = 0, it = 0;
+      int stage = 0, it = 0;
+      Cursor cu;
       uint32_t phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++it) {
+      for (int pos = blockIdx.x; pos < total && ok; pos += gridDim.x, ++it) {
         int m, e;
         bool sh;
-        decode(tile, g, m, e, sh);
-        const int kbn = sh ? a.kb_shared : a.kb_routed;
+        decode(pos, cu, m, e, sh);
+        const int kbn = sh ? a.ph[cu.phase].kb_shared : a.ph[cu.phase].kb_routed;
         const int acc = it & 1;
         const uint32_t acc_par = (it >> 1) & 1;
         ok = mbar_wait(smem_u32(&acc_empty[acc]), acc_par ^ 1u, abort_flag, a.err, kErrWaitMma);
@@ -257,7 +272,7 @@ grouped_gemm_small_kernel(const __grid_constant__ CUtensorMap tmW_s,
     const int q = warp & 3;              // TMEM lane quadrant
     const int L = q * 32 + lane;         // TMEM lane = weight row of each half
     const int et = threadIdx.x - 64;     // 0..127
-    if (MODE == kGateUpSwiGLU && a.copy_done != nullptr) {
+    {
       // the routed token rows, one warp per row (eight 16-byte vectors per lane in flight)
       constexpr int kV = 8;
       const int nw = (int)gridDim.x * 4;
@@ -286,13 +301,15 @@ grouped_gemm_small_kernel(const __grid_constant__ CUtensorMap tmW_s,
       fence_proxy_async_global();
       __threadfence();
       __syncwarp();
-      if (lane == 0) atomicAdd(a.copy_done, 1);
+      if (lane == 0) atomicAdd(a.sync, 1);
     }
-    int g = 0, it = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+    int it = 0;
+    Cursor cu;
+    for (int pos = blockIdx.x; pos < total; pos += gridDim.x, ++it) {
       int m, e;
       bool sh;
-      decode(tile, g, m, e, sh);
+      decode(pos, cu, m, e, sh);
+      const int ph = cu.phase;
       const int acc = it & 1;
       const uint32_t acc_par = (it >> 1) & 1;
       int ok = 1;
@@ -300,14 +317,15 @@ grouped_gemm_small_kernel(const __grid_constant__ CUtensorMap tmW_s,
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;   // warp-uniform decision
       tc_fence_after();
       const uint32_t trow = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + (uint32_t)(acc * 2 * nt);
+      const SmallPhase& P = a.ph[ph];
       const int rows = sh ? a.T : __ldg(&a.counts[e]);
-      const int64_t row0 = __ldg(&a.grp_row[g]);
-      __nv_bfloat16* out = sh ? a.out_shared : a.out_routed;
-      const int64_t ld = sh ? a.ld_shared : a.ld_routed;
-      const int cols = sh ? a.cols_shared : a.cols_routed;
+      const int64_t row0 = sh ? 0 : __ldg(&a.grp_row[cu.g]);
+      __nv_bfloat16* out = sh ? P.out_shared : P.out_routed;
+      const int64_t ld = sh ? P.ld_shared : P.ld_routed;
+      const int cols = sh ? P.cols_shared : P.cols_routed;
       // this thread's output features: gate/up -- feature 128 m + L (gate in the first half
       // of the accumulator, up in the second); down -- 256 m + L and 256 m + 128 + L
-      const int f0 = (MODE == kGateUpSwiGLU ? 128 : 256) * m + L;
+      const int f0 = (ph == 0 ? 128 : 256) * m + L;
       const int f1 = f0 + 128;
       for (int c = 0; c < rows; c += 16) {
         uint32_t v0[16], v1[16];
@@ -318,7 +336,7 @@ grouped_gemm_small_kernel(const __grid_constant__ CUtensorMap tmW_s,
         tmem_ld_wait16(v1);
         __nv_bfloat16* o = out + (row0 + c) * ld;
         const int nj = rows - c < 16 ? rows - c : 16;
-        if (MODE == kGateUpSwiGLU) {
+        if (ph == 0) {
           if (f0 < cols) {
 #pragma unroll
             for (int j = 0; j < 16; ++j)
@@ -337,8 +355,15 @@ grouped_gemm_small_kernel(const __grid_constant__ CUtensorMap tmW_s,
         }
       }
       tc_fence_before();
+      if (ph == 0) {   // the group's activations, for the TMA loads of its down tiles
+        fence_proxy_async_global();
+        __threadfence();
+      }
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&acc_empty[acc]));
+      if (lane == 0) {
+        mbar_arrive(smem_u32(&acc_empty[acc]));
+        if (ph == 0) atomicAdd(a.sync + 1 + cu.g, 1);
+      }
     }
   }
 

@@ -72,6 +72,9 @@ __global__ void balance_loss_kernel(const int32_t* counts, const float* psum, in
 }
 
 constexpr int kKernelsPerForward = 6;
+// counters of the fused row copy and of the decode FFN kernel's groups (1 + G <= 2 + kMaxRouted)
+constexpr size_t kSyncBytes = 2048;
+static_assert(kSyncBytes >= 4 * (2 + kMaxRouted), "per-group counters");
 
 }  // namespace
 
@@ -97,7 +100,6 @@ struct moe_handle {
   // small-batch (decode) path: token counts <= n_tok, weights on the MMA's M dimension
   bool small = false;
   int n_tok = 0, small_stages = 0;
-  int small_grid2 = 0;     // CTAs of the small-batch down GEMM
   size_t small_smem = 0;
   int n_pad = 0, maxk = 16, maxc = 32;
   int router_stages = 0, router_kps = 1;
@@ -118,9 +120,10 @@ struct moe_handle {
   float *tile_psum = nullptr, *psum_total = nullptr;
   void *xp = nullptr, *hs = nullptr, *hr = nullptr, *ys = nullptr, *yr = nullptr;
   int* err = nullptr;
-  int* copy_done = nullptr;   // counter of the fused permute (paired bf16 path with a shared group)
+  int* copy_done = nullptr;   // counters of the fused row copy (paired bf16 path with a shared
+                              // group; decode FFN kernel: also one per group, see SmallGemmArgs)
   int32_t* row_tok = nullptr; // [rows_cap] token of each routed row (decode-sized path: the
-                              // scan places the rows, the gate/up GEMM's epilogue warps copy them)
+                              // scan places the rows, the decode FFN kernel's epilogue warps copy them)
   // e4m3 gate/up: quantised weights (interleaved rows), per-row scales, quantised tokens
   void *w8_gu_s = nullptr, *w8_gu_r = nullptr, *u8 = nullptr;
   float *sw_s = nullptr, *sw_r = nullptr, *su = nullptr, *su_p = nullptr;
@@ -135,8 +138,8 @@ struct moe_handle {
   int32_t *idx_dev = nullptr, *cnt_dev = nullptr;
   float *w_dev = nullptr, *aux_dev = nullptr;
   CUtensorMap tmE, tmXp, tmWguS, tmWguR, tmHs, tmHr, tmWdS, tmWdR;
-  CUtensorMap tmXpN, tmHsN, tmHrN;   // token operands of the small-batch GEMMs (n_tok rows)
-  CUtensorMap tmWguS64, tmWguR64;    // gate/up weights in 64-row boxes (small-batch gate/up GEMM)
+  CUtensorMap tmXpN, tmHsN, tmHrN;   // token operands of the decode FFN kernel (n_tok rows)
+  CUtensorMap tmWguS64, tmWguR64;    // gate/up weights in 64-row boxes (decode FFN kernel)
   // moe_forward_host_pipelined: copy-in / forward / copy-out streams, two staging slots
   struct PipeSlot {
     void *u = nullptr, *h = nullptr;
@@ -253,10 +256,10 @@ int32_t moe_abi_version(void) { return MOE_ABI_VERSION; }
 const char* moe_last_error(void) { return g_last_error.c_str(); }
 
 int32_t moe_kernels_per_forward(const moe_handle* handle) {
-  // six timing slots; the permute has no kernel when the gate/up GEMM copies the rows (on
-  // decode-sized layers after the scan has placed them), and e4m3 layers add the token
-  // quantisation
-  return handle ? kKernelsPerForward - (handle->fuse_permute || handle->small ? 1 : 0) +
+  // six timing slots; the permute has no kernel when the gate/up GEMM copies the rows, and
+  // decode-sized layers run both GEMMs (and the row copy, after the scan has placed the
+  // rows) in one kernel; e4m3 layers add the token quantisation
+  return handle ? kKernelsPerForward - (handle->small ? 2 : handle->fuse_permute ? 1 : 0) +
                       (handle->e4m3 ? 1 : 0) +
                       (handle->e4m3_down ? 1 + handle->has_shared : 0)
                 : 0;
@@ -395,8 +398,8 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
   MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->ts2), (size_t)(H->G + 1) * 4));
   MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->err), 256));
   MOE_CUDA(cudaMemsetAsync(H->err, 0, 256, st));
-  MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->copy_done), 256));
-  MOE_CUDA(cudaMemsetAsync(H->copy_done, 0, 256, st));
+  MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->copy_done), kSyncBytes));
+  MOE_CUDA(cudaMemsetAsync(H->copy_done, 0, kSyncBytes, st));
   const size_t rc = (size_t)H->rows_cap, tp = (size_t)H->T_pad;
   MOE_TRY(dalloc(H, &H->xp, rc * d * (H->e4m3 ? 1 : es)));   // e4m3 rows on that path
   if (H->small) MOE_TRY(dalloc(H, reinterpret_cast<void**>(&H->row_tok), rc * 4));
@@ -515,22 +518,14 @@ static moe_status create_impl(const moe_cfg* cfg, moe_handle* H) {
                                     (int)H->simt_router_smem));
       const int stages = small_stages(H->n_tok);
       H->small_stages = stages;
-      // The down GEMM's grid: the fewest CTAs that still give each the same work when every
-      // routed expert receives tokens (a tile of the shared group counts as n_shared routed
-      // tiles: its K is n_shared * inter), so that no CTA runs a last tile alone.
-      {
-        const int64_t mt = (d + 2 * kSmallBM - 1) / (2 * kSmallBM);   // 256 features per tile
-        const int64_t act = std::min<int64_t>((int64_t)nr, (int64_t)c.T * c.top_k);
-        const int64_t units = act * mt + (ks ? mt * (int64_t)ks : 0);
-        const int64_t per = (units + H->n_sms - 1) / H->n_sms;
-        const int64_t g2 = per > 0 ? (units + per - 1) / per : H->n_sms;
-        H->small_grid2 = (int)std::min<int64_t>(H->n_sms, std::max<int64_t>(1, g2));
-      }
       H->small_smem = small_smem_bytes(H->n_tok, stages);
-      MOE_CUDA(cudaFuncSetAttribute((const void*)grouped_gemm_small_kernel<kGateUpSwiGLU>,
+      MOE_CUDA(cudaFuncSetAttribute((const void*)decode_ffn_kernel,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)H->small_smem));
-      MOE_CUDA(cudaFuncSetAttribute((const void*)grouped_gemm_small_kernel<kDown>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)H->small_smem));
+      // the kernel's grid-wide waits need every CTA resident at once: one CTA per SM
+      int per_sm = 0;
+      MOE_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, (const void*)decode_ffn_kernel,
+                                                             kSmallThreads, H->small_smem));
+      if (per_sm < 1) return fail(MOE_ERR_UNSUPPORTED, "the decode FFN kernel does not fit on an SM");
       bool okn = encode_2d(&H->tmXpN, H->xp, d, rc, (uint32_t)H->n_tok) &&
            encode_2d(&H->tmHrN, H->hr, I, rc, (uint32_t)H->n_tok) &&
            encode_3d(&H->tmWguR64, H->w_gu_r, d, 2 * I, nr, 64);
@@ -595,7 +590,8 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
               H->psum_total,
               H->tile_base, H->grp_row, H->ts1, H->ts2,
               H->fuse_permute || H->small ? H->copy_done : nullptr, H->bwd ? H->ts3 : nullptr};
-  if (H->small) {   // the scan places the routed rows; the gate/up GEMM copies them
+  if (H->small) sa.n_sync = 1 + H->G;   // the decode FFN kernel's per-group counters too
+  if (H->small) {   // the scan places the routed rows; the decode FFN kernel copies them
     sa.topk_idx = topk_idx; sa.topk_rank = H->topk_rank;
     sa.slot_row = H->slot_row; sa.row_tok = H->row_tok;
     sa.top_k = K; sa.router_rows = H->router_rows; sa.rows_cap = (int)H->rows_cap; sa.err = H->err;
@@ -659,31 +655,23 @@ moe_status moe_forward(moe_handle* H, const void* u, void* h, int32_t* topk_idx,
     CUtensorMap tmUN;   // token rows of the shared group, n_tok per tile
     if (!encode_2d(&tmUN, u, d, T, (uint32_t)H->n_tok))
       return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed for u");
-    SmallGemmArgs s1{};
-    s1.grp_row = H->grp_row; s1.ts = H->ts1; s1.counts = expert_counts; s1.G = H->G;
-    s1.has_shared = H->has_shared; s1.T = T; s1.n_tok = H->n_tok; s1.stages = H->small_stages;
-    s1.kb_shared = d / 64; s1.kb_routed = d / 64;
-    s1.cols_shared = Is; s1.cols_routed = I;
-    s1.out_shared = static_cast<__nv_bfloat16*>(H->hs); s1.ld_shared = Is;
-    s1.out_routed = static_cast<__nv_bfloat16*>(H->hr); s1.ld_routed = I;
-    s1.err = H->err;
-    // the routed rows (placed by the scan) are copied by the gate/up GEMM's epilogue warps
-    s1.row_tok = H->row_tok; s1.u = static_cast<const __nv_bfloat16*>(u);
-    s1.xp = static_cast<__nv_bfloat16*>(H->xp); s1.n_rows = T * K; s1.copy_vecs = d / 8;
-    s1.copy_done = H->copy_done;
+    SmallGemmArgs s{};
+    s.grp_row = H->grp_row; s.counts = expert_counts; s.G = H->G;
+    s.has_shared = H->has_shared; s.T = T; s.n_tok = H->n_tok; s.stages = H->small_stages;
+    s.ph[0] = SmallPhase{H->ts1, d / 64, d / 64, Is, I, static_cast<__nv_bfloat16*>(H->hs), Is,
+                         static_cast<__nv_bfloat16*>(H->hr), I};
+    s.ph[1] = SmallPhase{H->ts2, Is / 64, I / 64, d, d, static_cast<__nv_bfloat16*>(H->ys), d,
+                         static_cast<__nv_bfloat16*>(H->yr), d};
+    s.err = H->err;
+    // the routed rows (placed by the scan) are copied by the kernel's epilogue warps
+    s.row_tok = H->row_tok; s.u = static_cast<const __nv_bfloat16*>(u);
+    s.xp = static_cast<__nv_bfloat16*>(H->xp); s.n_rows = T * K; s.copy_vecs = d / 8;
+    s.sync = H->copy_done;
     tick(H, stream, 3);
-    launch_pdl(grouped_gemm_small_kernel<kGateUpSwiGLU>, dim3(H->n_sms), dim3(kSmallThreads), H->small_smem, stream,  H->tmWguS64, H->tmWguR64, tmUN, H->tmXpN, s1);
+    launch_pdl(decode_ffn_kernel, dim3(H->n_sms), dim3(kSmallThreads), H->small_smem, stream, H->tmWguS64,
+               H->tmWguR64, tmUN, H->tmXpN, H->tmWdS, H->tmWdR, H->tmHsN, H->tmHrN, s);
     MOE_CUDA(cudaGetLastError());
-    SmallGemmArgs s2 = s1;
-    s2.copy_done = nullptr;   // no row copy: the activations are expert-contiguous rows
-    s2.ts = H->ts2;
-    s2.kb_shared = Is / 64; s2.kb_routed = I / 64;
-    s2.cols_shared = d; s2.cols_routed = d;
-    s2.out_shared = static_cast<__nv_bfloat16*>(H->ys); s2.ld_shared = d;
-    s2.out_routed = static_cast<__nv_bfloat16*>(H->yr); s2.ld_routed = d;
-    tick(H, stream, 4);
-    launch_pdl(grouped_gemm_small_kernel<kDown>, dim3(H->small_grid2), dim3(kSmallThreads), H->small_smem, stream,  H->tmWdS, H->tmWdR, H->tmHsN, H->tmHrN, s2);
-    MOE_CUDA(cudaGetLastError());
+    tick(H, stream, 4);   // (the down GEMM runs inside the same kernel)
   } else if (H->bf16) {
     GemmArgs g1{};
     g1.grp_row = H->grp_row; g1.ts = H->ts1; g1.G = H->G; g1.has_shared = H->has_shared;

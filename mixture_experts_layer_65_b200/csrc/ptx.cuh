@@ -21,6 +21,7 @@ enum DevErr : int {
   kErrWaitEpilogue = 0x103,   // epilogue gave up waiting for an accumulator
   kErrWaitDrain = 0x104,      // teardown gave up waiting for in-flight copies / MMAs
   kErrWaitCopy = 0x105,       // fused GEMM producer gave up waiting for the row copies
+  kErrWaitHidden = 0x106,     // decode FFN producer gave up waiting for a group's activations
   kErrRouteIndex = 0x201,     // routed index outside [0, n_routed)
   kErrPermuteRow = 0x202,     // destination row outside the permuted buffer
   kErrOutRow = 0x203,         // GEMM output row outside its buffer

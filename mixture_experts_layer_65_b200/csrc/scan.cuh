@@ -46,7 +46,7 @@ struct ScanArgs {
   int32_t* ts3;               // [G + 1] tile prefix of a GEMM with N = the group's
                               // intermediate width at bn2 columns per tile (the backward's
                               // dHmid GEMM), or nullptr
-  // Routed-row indices (decode-sized layers, whose gate/up GEMM copies the token rows
+  // Routed-row indices (decode-sized layers, whose decode FFN kernel copies the token rows
   // itself): with slot_row != nullptr the scan ends by placing every (token, slot) —
   // slot_row[t, k] = its destination row, row_tok[row] = t — as the permute would.
   const int32_t* topk_idx;    // [T, top_k]
@@ -55,6 +55,7 @@ struct ScanArgs {
   int32_t* row_tok;           // [rows_cap]
   int top_k, router_rows, rows_cap;
   int* err;
+  int n_sync;                 // counters at copy_done to zero (0: one)
 };
 
 struct ScanSmem {
@@ -84,7 +85,8 @@ __device__ void scan_tail(const ScanArgs& a, int tid, uint8_t* smem, Sync sync) 
   const bool active = seg < nseg;
   const int t0 = seg * seg_len;
   const int t1 = min(a.n_tiles, t0 + seg_len);
-  if (tid == 0 && a.copy_done) *a.copy_done = 0;
+  if (a.copy_done)
+    for (int i = tid; i < (a.n_sync > 1 ? a.n_sync : 1); i += kScanThreads) a.copy_done[i] = 0;
 
   // 1. per-segment sums, tiles in ascending order (loads batched, adds in order); a
   //    segment of at most kScanBatch tiles keeps its histogram entries for step 4

@@ -84,43 +84,16 @@ int main() {
       CHECK((long)T * p < (1L << 31), "T=%d parts=%d overflows the grid", T, p);
     }
   }
-  // small-batch GEMM schedule: the remap is a bijection of [0, total), each CTA's tiles
-  // stay increasing, and the heaviest CTA (shared tiles cost w, routed tiles 1) is never
-  // heavier than without it
-  for (int grid : {132, 148}) {
-    for (int total = 1; total <= 3 * grid + 7; ++total) {
-      for (int n_sh = 0; n_sh <= std::min(total, 40); ++n_sh) {
-        for (int w : {1, 2, 4}) {
-          const bool rb = small_rebalance(total, n_sh, grid, w > 1);
-          std::vector<int> seen(total, 0), cost(grid, 0), plain(grid, 0), last(grid, -1);
-          bool mono = true;
-          for (int p = 0; p < total; ++p) {
-            const int t = small_tile_at(p, total, n_sh, grid, rb);
-            if (t < 0 || t >= total) { mono = false; break; }
-            ++seen[t];
-            const int b = p % grid;
-            mono = mono && t > last[b];
-            last[b] = t;
-            cost[b] += t < n_sh ? w : 1;
-            plain[b] += p < n_sh ? w : 1;
-          }
-          bool bij = mono;
-          for (int t = 0; t < total && bij; ++t) bij = seen[t] == 1;
-          CHECK(bij, "grid=%d total=%d n_sh=%d w=%d: not a bijection or not increasing", grid, total, n_sh, w);
-          CHECK(*std::max_element(cost.begin(), cost.end()) <= *std::max_element(plain.begin(), plain.end()),
-                "grid=%d total=%d n_sh=%d w=%d: remap made the heaviest CTA heavier", grid, total, n_sh, w);
-          CHECK(w > 1 || !rb, "grid=%d total=%d n_sh=%d: remap without heavier shared tiles", grid, total, n_sh);
-        }
-      }
-    }
-  }
-  // small-batch GEMM: for every token width a ring of 2 .. kSmallMaxStages stages that fits
-  // the opt-in shared memory with the epilogue buffers and the control block
+  // decode FFN kernel: for every token width a ring of 2 .. kSmallMaxStages stages that fits
+  // the opt-in shared memory with the control block, and two accumulators of 2 n_tok
+  // columns that fit its TMEM allocation
   for (int nt = 16; nt <= kSmallMaxTok; nt += 16) {
     const int st = small_stages(nt);
     CHECK(st >= 2 && st <= kSmallMaxStages, "n_tok=%d stages=%d", nt, st);
     CHECK(small_smem_bytes(nt, st) <= kRouterSmemBudget, "n_tok=%d bytes=%zu", nt, small_smem_bytes(nt, st));
     CHECK(small_stage_bytes(nt) % 1024 == 0, "n_tok=%d stage %u", nt, small_stage_bytes(nt));
+    const uint32_t tc = small_tmem_cols(nt);
+    CHECK(tc >= 4u * nt && tc <= 512 && (tc & (tc - 1)) == 0, "n_tok=%d TMEM columns %u", nt, tc);
   }
   // the paired GEMM's ring and control block fit the opt-in shared memory
   CHECK(kGemmSmemBytes <= kRouterSmemBudget, "GEMM smem %zu", kGemmSmemBytes);

@@ -169,7 +169,7 @@ def test_full_size_intermediates_on_sampled_rows_of_every_expert(name):
 def test_per_kernel_timing_records_every_slot(name, spec):
     """moe_timing_begin / moe_timing_end (the benchmark's per-kernel slots) on every launch
     path: each slot of each recorded forward is recorded, whether or not a kernel runs in it
-    (the permute and, on decode-sized layers, the combine run inside other kernels)."""
+    (the permute and, on decode-sized layers, the down GEMM run inside other kernels)."""
     w = W.make_workload("16b_prefill", alpha1=0.001, **spec)
     layer = MoELayer.from_workload(w)
     u = to_device_tensor(w.u, "cuda")
@@ -182,5 +182,5 @@ def test_per_kernel_timing_records_every_slot(name, spec):
     layer.device_status()
     assert n == 3
     assert all(np.isfinite(v) and v >= 0.0 for v in ms.values()), ms
-    assert ms["gate_up_gemm"] > 0.0 and ms["down_gemm"] > 0.0
+    assert ms["gate_up_gemm"] > 0.0 and (name == "decode_sized" or ms["down_gemm"] > 0.0)
     layer.close()
