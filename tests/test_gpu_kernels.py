@@ -26,6 +26,10 @@ SPECS = [
     dict(T=333, d=256, n_shared=2, n_routed=16, inter=192, top_k=4),   # row copy in the GEMM
     dict(T=700, d=256, n_shared=0, n_routed=16, inter=128, top_k=2),   # permute kernel
     dict(T=96, d=256, n_shared=2, n_routed=16, inter=128, top_k=4),    # decode-sized: copy in the GEMM
+    # decode-sized with ragged weight tiles: the last gate/up tile holds 64 of its 128
+    # features (inter % 128 == 64) and the last down tile 128 of its 256 (d % 256 == 128)
+    dict(T=40, d=384, n_shared=1, n_routed=8, inter=192, top_k=2),
+    dict(T=17, d=128, n_shared=0, n_routed=8, inter=64, top_k=1),
 ]
 
 
