@@ -91,6 +91,23 @@ def peak_regime(clk: dict | None, timed_s: float) -> str:
 PEAK_KEY = {"burst": "bf16_tflops", "sustained": "bf16_tflops_sustained"}
 
 
+def choose_kernel_timing(regime: str, no_graph: bool, burst_kt, post_kt):
+    """The per-kernel timing pass held against the timed region's peak: the one measured in
+    the same clock regime.  burst_kt / post_kt = (summed ms per kernel, forwards, clocks) of
+    the pass before the timed region (after a pause) and of the pass right after it (or,
+    with no_graph, of the timed steps themselves).  Returns (ms, forwards, clocks, text)."""
+    ms, n, clk = post_kt
+    if no_graph:
+        return ms, n, clk, "CUDA events between the library's kernels over the timed steps"
+    if regime == "burst" and burst_kt is not None:
+        ms, n, clk = burst_kt
+        return ms, n, clk, (f"CUDA events between the library's kernels over {n} eager forwards "
+                            f"after a {KERNEL_REST_S:.0f} s pause before the timed region (burst "
+                            "clocks, as in the timed region)")
+    return ms, n, clk, (f"CUDA events between the library's kernels over {n} eager forwards "
+                        "right after the timed region (its clock regime)")
+
+
 def workload_desc(w, n_gpus: int) -> dict:
     return {"workload": f"{w.name}: T={w.T} d={w.d} shared={w.n_shared} routed={w.n_routed} "
                         f"inter={w.inter} top_k={w.top_k} {w.dtype}"
@@ -480,17 +497,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     # the kernel durations measured in that regime: the pass before the timed steps for a
     # short (burst-clock) region, the pass right after them for a power-capped one
     regime = peak_regime(clk, ms * 1e-3)
-    kernel_clk = clk
-    if args.no_graph:
-        timing_desc = "CUDA events between the library's kernels over the timed steps"
-    elif regime == "burst" and burst_kt is not None:
-        kernel_ms, n_rec, kernel_clk = burst_kt
-        timing_desc = (f"CUDA events between the library's kernels over {n_rec} eager forwards "
-                       f"after a {KERNEL_REST_S:.0f} s pause before the timed region (burst clocks, "
-                       "as in the timed region)")
-    else:
-        timing_desc = (f"CUDA events between the library's kernels over {n_rec} eager forwards "
-                       "right after the timed region (its clock regime)")
+    kernel_ms, n_rec, kernel_clk, timing_desc = choose_kernel_timing(
+        regime, args.no_graph, burst_kt, (kernel_ms, n_rec, clk))
     work = algorithmic_work(w, int((out.expert_counts > 0).sum().item()))
     per_kernel = {}
     # e4m3 gate/up variant: that GEMM's peak is the measured bf16 peak times the nominal

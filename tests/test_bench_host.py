@@ -167,3 +167,21 @@ def test_peak_regime_follows_the_sampled_clock():
     assert bench.peak_regime(capped, 0.04) == "burst"
     assert bench.peak_regime(None, 5.0) == "burst"
     assert bench.PEAK_KEY["burst"] == "bf16_tflops"
+
+
+def test_kernel_timing_follows_the_timed_regions_clock_regime():
+    """A burst-clock timed region takes the per-kernel pass measured before it (after a
+    pause); a power-capped one the pass right after it; eager runs their own timed steps."""
+    burst = ({"gate_up_gemm": 1.0}, 8, {"sm_mhz": 1965.0})
+    post = ({"gate_up_gemm": 2.0}, 100, {"sm_mhz": 1200.0})
+    ms, n, clk, text = bench.choose_kernel_timing("burst", False, burst, post)
+    assert (ms, n, clk) == burst and "before the timed region" in text
+    ms, n, clk, text = bench.choose_kernel_timing("sustained", False, burst, post)
+    assert (ms, n, clk) == post and "right after" in text
+    ms, n, clk, text = bench.choose_kernel_timing("burst", True, None, post)
+    assert (ms, n, clk) == post and "over the timed steps" in text
+    # the regime itself: power-capped only when timed long enough with the cap seen
+    capped = {"sm_mhz": 1200.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    assert bench.peak_regime(capped, 0.8) == "sustained"
+    assert bench.peak_regime(capped, 0.05) == "burst"
+    assert bench.peak_regime({"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}, 2.0) == "burst"
