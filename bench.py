@@ -61,6 +61,10 @@ def parse_args():
                    help="also time K forward + backward steps (input, router and weight "
                         "gradients) after the forward measurements and add a 'backward' "
                         "object to the line; bf16 prefill-sized layers only")
+    p.add_argument("--expert-parallel", action="store_true",
+                   help="time the expert-parallel forward instead (routed experts split over the "
+                        "ranks, token rows exchanged by all-to-all; one rank: local copies) and "
+                        "print its line; not the headline")
     p.add_argument("--dry-run", action="store_true",
                    help="CPU check of the multi-rank plumbing (gloo): rank discovery, the "
                         "global balance loss's exchange on synthetic per-rank statistics and "
@@ -302,6 +306,70 @@ def run_reference(args, rank: int, world: int):
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- expert parallel
+class _LocalComm:
+    """The expert-parallel forward's collectives for a single rank: the row exchange is a copy
+    and the sums over ranks are the rank's own values."""
+
+    def all_to_all_single(self, out, inp, out_splits=None, in_splits=None):
+        out.copy_(inp)
+
+    def all_reduce(self, t):
+        pass
+
+
+def run_expert_parallel(args, rank: int, world: int, local_rank: int):
+    """Tokens/s of the expert-parallel forward (`expert_parallel.ep_forward` over the library's
+    moe_ep_* calls): each rank holds n_routed / world routed experts and the shared ones and
+    routes its own T tokens; eager launches (the forward reads the exchange's split sizes on
+    the host), CUDA-event timing, max over ranks."""
+    import torch
+    import torch.distributed as dist
+
+    from mixture_experts_layer_65_b200 import workloads as W
+    from mixture_experts_layer_65_b200.expert_parallel import (DistComm, ep_forward,
+                                                              lib_backend_from_workload)
+    from mixture_experts_layer_65_b200.layer import to_device_tensor
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = W.make_workload(args.config, **({"T": args.tokens} if args.tokens else {}))
+    be = lib_backend_from_workload(w, rank, world, device=dev, recv_capacity=w.T * w.top_k * world)
+    u = torch.roll(to_device_tensor(w.u, dev), shifts=rank * 997, dims=0).contiguous()
+    comm = DistComm() if world > 1 else _LocalComm()
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(max(3, args.warmup)):
+        ep_forward(be, u, comm)
+    torch.cuda.synchronize()
+    be.device_status()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        ep_forward(be, u, comm)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    be.device_status()
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    be.close()
+    if rank != 0:
+        return
+    print(json.dumps({
+        "mode": "expert_parallel", "metric": METRIC, "value": world * w.T * args.steps / (ms * 1e-3),
+        "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup),
+        "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": dict(workload_desc(w, world), parallelism=f"ep{world}"),
+        "launch": "eager (the exchange's split sizes are read on the host each step)",
+        "collectives": "NCCL all_to_all_single / all_reduce" if world > 1 else "one rank: local copies"}),
+        flush=True)
 
 
 # --------------------------------------------------------------------------- our arm
@@ -754,7 +822,10 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=None)
     try:
-        run_ours(args, rank, world, local_rank)
+        if args.expert_parallel:
+            run_expert_parallel(args, rank, world, local_rank)
+        else:
+            run_ours(args, rank, world, local_rank)
     finally:
         if world > 1:
             dist.destroy_process_group()
