@@ -81,6 +81,22 @@ def test_gloo_two_ranks_match_the_full_batch(load):
         assert full.counts[e0:e0 + nl].sum() > 3 * full.counts[nl:].sum()
 
 
+def test_single_rank_with_local_copies_matches_the_full_batch():
+    """The benchmark's one-rank expert-parallel run (`bench.py --expert-parallel`): the
+    all-to-alls become local copies and the sums over ranks the rank's own values; with the
+    oracle-based rank it reproduces the full-batch oracle."""
+    import bench
+    spec, _ = LOADS["zipf"]
+    w = W.make_workload("16b_prefill", **spec)
+    out = ep_forward(OracleEPBackend(w, 0, w.T, 0, 1), None, bench._LocalComm())
+    full = O.moe_forward(w.u, w.centroids, w.w_gate, w.w_up, w.w_down, w.n_shared, w.top_k,
+                         w.alpha1, bias=w.logit_bias)
+    np.testing.assert_allclose(out.h.numpy(), full.h, rtol=0, atol=1e-12 * np.abs(full.h).max())
+    np.testing.assert_array_equal(out.topk_idx.numpy(), full.routing.topk_idx)
+    np.testing.assert_array_equal(out.expert_counts.numpy(), full.counts)
+    assert float(out.aux_loss[0]) == pytest.approx(full.aux, rel=2.0 ** -23)
+
+
 def test_expert_range_splits_evenly():
     assert expert_range(64, 8, 3) == (24, 8)
     with pytest.raises(ValueError):
