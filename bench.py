@@ -336,6 +336,11 @@ def run_expert_parallel(args, rank: int, world: int, local_rank: int):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     w = W.make_workload(args.config, **({"T": args.tokens} if args.tokens else {}))
+    if w.dtype != "bf16" or getattr(w, "gate_up_e4m3", False) or w.n_routed % world:
+        print(f"bench.py: --expert-parallel takes bf16 layers whose routed experts split evenly "
+              f"over the ranks ({w.name}: {w.dtype}, {w.n_routed} routed, {world} ranks)",
+              file=sys.stderr)
+        sys.exit(2)
     be = lib_backend_from_workload(w, rank, world, device=dev, recv_capacity=w.T * w.top_k * world)
     u = torch.roll(to_device_tensor(w.u, dev), shifts=rank * 997, dims=0).contiguous()
     comm = DistComm() if world > 1 else _LocalComm()
