@@ -303,41 +303,57 @@ __device__ __forceinline__ bool masked_row_valid(const MaskedTransposeArgs& a, i
 // (eight vectors each, coalesced) into shared memory, where each 128-byte row stores its
 // vectors XOR-permuted by (row / 8) mod 8, then write 64 destination rows of eight vectors,
 // each vector gathering one column of eight source rows; eight consecutive threads write one
-// destination row's 128 bytes, and the gathers of a warp hit distinct banks.  C and the
-// strides must be multiples of 8 elements (the library's widths are multiples of 64).
+// destination row's 128 bytes, and the gathers of a warp hit distinct banks.  A CTA takes
+// kMtColTiles column tiles of one row tile: the rows' validity (a binary search over the
+// groups per row) is looked up once, and each next tile's loads are in flight while the
+// current tile is stored.  C and the strides must be multiples of 8 elements (the library's
+// widths are multiples of 64).
 constexpr int kMtTile = 64;
+constexpr int kMtColTiles = 8;
 static __global__ void __launch_bounds__(256) masked_transpose_kernel(MaskedTransposeArgs a) {
   pdl_launch_dependents();
   pdl_wait();
   __shared__ __align__(16) __nv_bfloat16 tile[kMtTile][kMtTile];
   __shared__ bool valid[kMtTile];
-  const int c0 = blockIdx.x * kMtTile;
   const int64_t r0 = (int64_t)blockIdx.y * kMtTile;
   const int t = threadIdx.x;
   if (t < kMtTile) valid[t] = r0 + t < a.rows && masked_row_valid(a, r0 + t);
   __syncthreads();
+  auto load = [&](int c0, uint4 (&v)[2]) {   // this thread's two source vectors of tile c0
 #pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const int row = t / 8 + 32 * i, vec = t % 8;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (valid[row] && c0 + vec * 8 < a.C)
-      v = __ldg(reinterpret_cast<const uint4*>(a.src + (r0 + row) * a.ld_src + c0 + vec * 8));
-    *reinterpret_cast<uint4*>(&tile[row][(vec ^ ((row >> 3) & 7)) * 8]) = v;
-  }
-  __syncthreads();
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const int c = t / 8 + 32 * i, rv = t % 8;   // destination row c0 + c, vector rv
-    if (c0 + c >= a.C || r0 + rv * 8 >= a.rows) continue;
-    const int ch = ((c >> 3) ^ rv) * 8 + (c & 7);   // column c of source rows 8 rv .. 8 rv + 7
-    uint32_t w[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const __nv_bfloat16 lo = tile[rv * 8 + 2 * j][ch], hi = tile[rv * 8 + 2 * j + 1][ch];
-      w[j] = (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
+    for (int i = 0; i < 2; ++i) {
+      const int row = t / 8 + 32 * i, vec = t % 8;
+      v[i] = make_uint4(0u, 0u, 0u, 0u);
+      if (valid[row] && c0 + vec * 8 < a.C)
+        v[i] = __ldg(reinterpret_cast<const uint4*>(a.src + (r0 + row) * a.ld_src + c0 + vec * 8));
     }
-    *reinterpret_cast<uint4*>(a.dst + (int64_t)(c0 + c) * a.ld_dst + r0 + rv * 8) =
-        make_uint4(w[0], w[1], w[2], w[3]);
+  };
+  int c0 = (int)blockIdx.x * kMtColTiles * kMtTile;
+  uint4 v[2];
+  if (c0 < a.C) load(c0, v);
+  for (int ct = 0; ct < kMtColTiles && c0 < a.C; ++ct, c0 += kMtTile) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int row = t / 8 + 32 * i, vec = t % 8;
+      *reinterpret_cast<uint4*>(&tile[row][(vec ^ ((row >> 3) & 7)) * 8]) = v[i];
+    }
+    __syncthreads();
+    if (ct + 1 < kMtColTiles && c0 + kMtTile < a.C) load(c0 + kMtTile, v);   // next tile in flight
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int c = t / 8 + 32 * i, rv = t % 8;   // destination row c0 + c, vector rv
+      if (c0 + c >= a.C || r0 + rv * 8 >= a.rows) continue;
+      const int ch = ((c >> 3) ^ rv) * 8 + (c & 7);   // column c of source rows 8 rv .. 8 rv + 7
+      uint32_t w[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const __nv_bfloat16 lo = tile[rv * 8 + 2 * j][ch], hi = tile[rv * 8 + 2 * j + 1][ch];
+        w[j] = (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
+      }
+      *reinterpret_cast<uint4*>(a.dst + (int64_t)(c0 + c) * a.ld_dst + r0 + rv * 8) =
+          make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    __syncthreads();   // the tile buffer is refilled next turn
   }
 }
 

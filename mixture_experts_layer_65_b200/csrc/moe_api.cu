@@ -1067,7 +1067,7 @@ moe_status moe_backward(moe_handle* H, const void* u, const int32_t* topk_idx, c
     MaskedTransposeArgs ma{static_cast<const __nv_bfloat16*>(src), static_cast<__nv_bfloat16*>(dst), rows, C,
                            ld_src, ld_dst, routed ? H->grp_row + H->has_shared : nullptr, expert_counts,
                            nr, 0, T, routed ? rows : (int64_t)T};
-    launch_pdl(masked_transpose_kernel, dim3((unsigned)((C + kMtTile - 1) / kMtTile),
+    launch_pdl(masked_transpose_kernel, dim3((unsigned)((C + kMtTile * kMtColTiles - 1) / (kMtTile * kMtColTiles)),
                                              (unsigned)((rows + kMtTile - 1) / kMtTile)),
                dim3(256), 0, stream, ma);
     return cudaGetLastError();
